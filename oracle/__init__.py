@@ -1,0 +1,203 @@
+"""CPU oracle for the microscaling-quantized linear layer (TEST INFRASTRUCTURE).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+reference leg of ``bench.py`` may import this package.  The product path (the
+CUDA library and its binding) never touches it.
+
+This module is a thin ctypes wrapper over ``nvq_oracle.c``; every arithmetic
+step lives in that C file.  Arrays are numpy: BF16 tensors travel as their
+raw ``uint16`` bit patterns.
+"""
+import ctypes
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_i64 = ctypes.c_int64
+
+NVFP4_BLOCK = 16
+MXFP8_BLOCK = 32
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.oracle_e2m1_value.restype = ctypes.c_double
+        L.oracle_e2m1_value.argtypes = [ctypes.c_int]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_e4m3_value.argtypes = [ctypes.c_int]
+        L.oracle_e8m0_value.restype = ctypes.c_double
+        L.oracle_e8m0_value.argtypes = [ctypes.c_int]
+        L.oracle_e2m1_encode.restype = ctypes.c_int
+        L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        L.oracle_e4m3_encode.restype = ctypes.c_int
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_take_nan_flag.restype = ctypes.c_int
+        L.oracle_sf_bytes.restype = _i64
+        L.oracle_sf_bytes.argtypes = [_i64, _i64]
+        L.oracle_sf_offset.restype = _i64
+        L.oracle_sf_offset.argtypes = [_i64, _i64, _i64]
+        L.oracle_amax.restype = ctypes.c_float
+        L.oracle_amax.argtypes = [_u16p, _i64, _i64, _i64]
+        L.oracle_nvfp4_quantize.restype = None
+        L.oracle_nvfp4_quantize.argtypes = [_u16p, _i64, _i64, _i64, _f32p, _u8p, _u8p, _f32p]
+        L.oracle_nvfp4_dequantize.restype = None
+        L.oracle_nvfp4_dequantize.argtypes = [_u8p, _u8p, ctypes.c_float, _i64, _i64, _f64p]
+        L.oracle_mxfp8_quantize.restype = None
+        L.oracle_mxfp8_quantize.argtypes = [_u16p, _i64, _i64, _i64, _u8p, _u8p]
+        L.oracle_mxfp8_dequantize.restype = None
+        L.oracle_mxfp8_dequantize.argtypes = [_u8p, _u8p, _i64, _i64, _f64p]
+        L.oracle_gemm_rows.restype = None
+        L.oracle_gemm_rows.argtypes = [_f64p, _f64p, _i64, _i64, _i64p, _i64, _u16p, _f64p]
+        L.oracle_num_threads.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a, t):
+    return a.ctypes.data_as(t)
+
+
+def _bf16_bits(x):
+    """Accept a numpy uint16 array of BF16 bit patterns or a torch bf16 tensor."""
+    if hasattr(x, "dtype") and str(x.dtype) == "torch.bfloat16":
+        x = x.contiguous().view(dtype=__import__("torch").int16).numpy().view(np.uint16)
+    x = np.ascontiguousarray(x)
+    assert x.dtype == np.uint16 and x.ndim == 2
+    return x
+
+
+# --- element formats -------------------------------------------------------
+
+def e2m1_value(code):
+    return lib().oracle_e2m1_value(int(code))
+
+
+def e4m3_value(code):
+    return lib().oracle_e4m3_value(int(code))
+
+
+def e8m0_value(code):
+    return lib().oracle_e8m0_value(int(code))
+
+
+def e2m1_encode(v):
+    return lib().oracle_e2m1_encode(float(np.float32(v)))
+
+
+def e4m3_encode(v):
+    return lib().oracle_e4m3_encode(float(np.float32(v)))
+
+
+def take_nan_flag():
+    return bool(lib().oracle_take_nan_flag())
+
+
+# --- scale layout ----------------------------------------------------------
+
+def sf_bytes(rows, cols):
+    return int(lib().oracle_sf_bytes(rows, cols))
+
+
+def sf_offset(r, c, cols):
+    return int(lib().oracle_sf_offset(r, c, cols))
+
+
+# --- quantization ------------------------------------------------------------
+
+def amax(x_bits, ldx=None):
+    x = _bf16_bits(x_bits)
+    M, K = x.shape
+    return float(lib().oracle_amax(_ptr(x, _u16p), M, K, ldx or K))
+
+
+def nvfp4_quantize(x_bits, calib_amax=None):
+    """Returns (codes u8 [M, K/2], sf u8 [sf_bytes(M, K/16)], g_dec float32)."""
+    x = _bf16_bits(x_bits)
+    M, K = x.shape
+    assert K % NVFP4_BLOCK == 0
+    codes = np.zeros((M, K // 2), dtype=np.uint8)
+    sf = np.zeros(sf_bytes(M, K // NVFP4_BLOCK), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    ca = None
+    if calib_amax is not None:
+        ca_arr = np.array([calib_amax], dtype=np.float32)
+        ca = _ptr(ca_arr, _f32p)
+    lib().oracle_nvfp4_quantize(_ptr(x, _u16p), M, K, K, ca, _ptr(codes, _u8p), _ptr(sf, _u8p), _ptr(g, _f32p))
+    return codes, sf, np.float32(g[0])
+
+
+def nvfp4_dequantize(codes, sf, g_dec, rows, K):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    out = np.empty((rows, K), dtype=np.float64)
+    lib().oracle_nvfp4_dequantize(_ptr(codes, _u8p), _ptr(sf, _u8p), float(g_dec), rows, K, _ptr(out, _f64p))
+    return out
+
+
+def mxfp8_quantize(x_bits):
+    """Returns (codes u8 [M, K], sf u8 [sf_bytes(M, K/32)])."""
+    x = _bf16_bits(x_bits)
+    M, K = x.shape
+    assert K % MXFP8_BLOCK == 0
+    codes = np.zeros((M, K), dtype=np.uint8)
+    sf = np.zeros(sf_bytes(M, K // MXFP8_BLOCK), dtype=np.uint8)
+    lib().oracle_mxfp8_quantize(_ptr(x, _u16p), M, K, K, _ptr(codes, _u8p), _ptr(sf, _u8p))
+    return codes, sf
+
+
+def mxfp8_dequantize(codes, sf, rows, K):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    out = np.empty((rows, K), dtype=np.float64)
+    lib().oracle_mxfp8_dequantize(_ptr(codes, _u8p), _ptr(sf, _u8p), rows, K, _ptr(out, _f64p))
+    return out
+
+
+# --- GEMM ------------------------------------------------------------------------
+
+def gemm_rows(A_hat, B_hat, rows=None, bias_bits=None):
+    """out[i, n] = sum_k A_hat[rows[i], k] * B_hat[n, k] (+ bias[n]), binary64."""
+    A = np.ascontiguousarray(A_hat, dtype=np.float64)
+    B = np.ascontiguousarray(B_hat, dtype=np.float64)
+    N, K = B.shape
+    assert A.shape[1] == K
+    if rows is None:
+        rows = np.arange(A.shape[0], dtype=np.int64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.empty((rows.size, N), dtype=np.float64)
+    bp = None
+    if bias_bits is not None:
+        bias = np.ascontiguousarray(bias_bits, dtype=np.uint16).reshape(-1)
+        assert bias.size == N
+        bp = _ptr(bias, _u16p)
+    lib().oracle_gemm_rows(_ptr(A, _f64p), _ptr(B, _f64p), N, K, _ptr(rows, _i64p), rows.size, bp, _ptr(out, _f64p))
+    return out
+
+
+def num_threads():
+    return int(lib().oracle_num_threads())
+
+
+# --- acceptance rule --------------------------------------------------------------
+
+GEMM_TOL = 2e-3
+
+
+def gemm_row_errors(D, Y):
+    """Per-row max_n |D - Y| / ||Y[row, :]||_2 (all-zero reference rows: max |D|)."""
+    D = np.asarray(D, dtype=np.float64)
+    Y = np.asarray(Y, dtype=np.float64)
+    err = np.abs(D - Y).max(axis=1)
+    nrm = np.linalg.norm(Y, axis=1)
+    zero_row = np.where(err > 0, np.inf, 0.0)
+    return np.where(nrm > 0, err / np.where(nrm > 0, nrm, 1.0), zero_row)
