@@ -1,0 +1,446 @@
+"""Benchmark of the microscaling-quantized linear hot path on B200.
+
+One step = one FLUX-like NVFP4 W4A4 FF-up linear on a fresh activation batch:
+dynamic activation quantization (amax pass + quantize-and-pack) of BF16
+[4608, 3072], then the block-scaled tcgen05 GEMM against the pre-quantized
+weight [12288, 3072], writing BF16 [4608, 12288].  The weight is quantized
+once, outside the timed region (it is a load-time step).
+
+Metric: TFLOP/s of quant+GEMM (2*M*N*K per step / step time) and the
+activation quantizer's HBM GB/s (2 B read + 0.5625 B written per element).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+runs its own independent batch (weak scaling, no collective on the data path;
+the only collectives are the timing barrier and the max-over-ranks of the
+elapsed time).
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "NVFP4 quant+GEMM TFLOPS at 4608x3072x12288; act-quant HBM GB/s"
+WORKLOAD = "ffup"
+ROTATE = 4                    # input sets cycled through so a step's inputs are not L2-resident
+FP4_OVER_BF16 = 4.0           # nominal dense FP4 / BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
+ACT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # BF16 read, E2M1 codes + E4M3 scale written
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons of one GPU through NVML."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index, period=0.02):
+        self.samples = []
+        self.reasons = 0
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except Exception:
+                bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clock data rather than guess
+            self.err = repr(e)
+        self._period = period
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def start(self):
+        if self.ok:
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, device):
+    import microscaling_quantized_linear_b200 as nvq
+
+    w = workloads.WORKLOADS[WORKLOAD]
+    M, N, K = w.M, w.N, w.K
+    flops = 2.0 * M * N * K
+    stream = torch.cuda.current_stream(device)
+
+    # Inputs: ROTATE activation batches and ROTATE quantized weights (seeded per
+    # rank), resident in HBM before the timed region.
+    xs = [workloads.activation(WORKLOAD, seed=1000 * rank + i).to(device) for i in range(ROTATE)]
+    wq = []
+    for i in range(ROTATE):
+        wd = workloads.weight(WORKLOAD, seed=1000 * rank + 100 + i).to(device)
+        wq.append(nvq.quantize_weight("nvfp4", wd))
+        del wd
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty(nvq.scale_bytes("nvfp4", M, K), dtype=torch.uint8, device=device)
+    gscale = torch.empty(1, dtype=torch.float32, device=device)
+    ws = nvq.new_workspace(device)
+    outs = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(2)]
+
+    n_ev = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
+
+    def step(i, timed):
+        x = xs[i % ROTATE]
+        wc, wsf, wg = wq[i % ROTATE]
+        if timed:
+            ev[i][0].record(stream)
+        nvq.nvfp4_quantize(x, codes, scales, gscale, workspace=ws, stream=stream)
+        if timed:
+            ev[i][1].record(stream)
+        nvq.block_scaled_linear("nvfp4", codes, scales, gscale, wc, wsf, wg, M, N, K,
+                                out=outs[i % 2], stream=stream)
+        if timed:
+            ev[i][2].record(stream)
+
+    for i in range(args.warmup):
+        step(i, False)
+    torch.cuda.synchronize(device)
+    if nvq.device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    clocks = ClockSampler(device.index)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i, True)
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = t.item()
+    status = nvq.device_status()
+
+    quant_us = [ev[i][0].elapsed_time(ev[i][1]) * 1e3 for i in range(n_ev)]
+    gemm_us = [ev[i][1].elapsed_time(ev[i][2]) * 1e3 for i in range(n_ev)]
+    ms_per_step = elapsed_ms / args.steps
+    value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+
+    peaks = load_peaks()
+    sustained = elapsed_ms > 1000.0
+    bf16_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    fp4_peak = bf16_peak * FP4_OVER_BF16
+    gemm_mean = statistics.mean(gemm_us)
+    gemm_tflops = flops / (gemm_mean * 1e-6) / 1e12
+    act_bytes = M * K * ACT_BYTES_PER_ELEM + 4
+    quant_mean = statistics.mean(quant_us)
+    act_gbs = act_bytes / (quant_mean * 1e-6) / 1e9
+
+    e2e = run_e2e(nvq, args, device, stream, xs[0].cpu(), wq[0], M, N, K, flops, world)
+
+    res = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1",
+        "data": "synthetic",
+        "config": {
+            "workload": "NVFP4 W4A4 FF-up linear, FLUX-like: A BF16 [4608,3072] N(0,1) 0.5% x50 outliers, "
+                        "W BF16 [12288,3072] N(0,0.02), out BF16 [4608,12288]; dynamic per-tensor activation scale",
+            "M": M, "N": N, "K": K,
+            "parallelism": "replicas" if world > 1 else "single-gpu",
+            "l2": "inputs rotated over %d activation+weight sets (%.0f MB) plus a %.0f MB output write per step, "
+                  "all larger than the 126 MB L2" % (ROTATE, ROTATE * (M * K * 2 + N * K * 0.5625) / 1e6,
+                                                     M * N * 2 / 1e6),
+        },
+        "act_quant": {
+            "value": round(act_gbs, 1), "unit": "GB/s", "us_per_call": round(quant_mean, 3),
+            "bytes_per_call": int(act_bytes), "launches_per_call": 2,
+            "frac": round(act_gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"],
+            "peak_source": peaks["source"],
+        },
+        "roofline": {
+            "kernel": "bsgemm_kernel<NVFP4,256>",
+            "bound": "tensor",
+            "achieved": round(gemm_tflops, 1),
+            "peak": round(fp4_peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(gemm_tflops / fp4_peak, 4),
+            "traffic": None,
+            "peak_source": "%s bf16 %s x %.0f (nominal FP4/BF16 ratio)" % (
+                peaks["source"], "sustained" if sustained else "burst", FP4_OVER_BF16),
+            "us_per_launch": round(gemm_mean, 3),
+            "flops_per_launch": flops,
+        },
+        "kernel_share": {
+            "quantize(amax+pack)": round(quant_mean / (quant_mean + gemm_mean), 4),
+            "gemm": round(gemm_mean / (quant_mean + gemm_mean), 4),
+        },
+        "gpu_launches": 3 * args.steps,
+        "e2e": e2e,
+        "device_status": status,
+        "clocks": clocks.summary(),
+    }
+    if args.mxfp8:
+        res["mxfp8_ffdown"] = run_mxfp8_component(nvq, args, device, stream, peaks)
+    return res
+
+
+def run_e2e(nvq, args, device, stream, x_host_src, wq, M, N, K, flops, world):
+    """Same step through the public API with host buffers: H2D of the BF16
+    activation from pinned memory, quantize + GEMM, D2H of the BF16 output."""
+    x_host = x_host_src.pin_memory()
+    out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x_host, device=device)
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty(nvq.scale_bytes("nvfp4", M, K), dtype=torch.uint8, device=device)
+    g = torch.empty(1, dtype=torch.float32, device=device)
+    ws = nvq.new_workspace(device)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    wc, wsf, wg = wq
+    steps = max(3, min(args.steps, 20))
+
+    def step():
+        x_dev.copy_(x_host, non_blocking=True)
+        nvq.nvfp4_quantize(x_dev, codes, scales, g, workspace=ws, stream=stream)
+        nvq.block_scaled_linear("nvfp4", codes, scales, g, wc, wsf, wg, M, N, K, out=out, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = t.item()
+    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(out_host.numel() * 2),
+            "ms_per_step": round(ms, 4), "steps": steps}
+
+
+def run_mxfp8_component(nvq, args, device, stream, peaks):
+    """MXFP8 FF-down linear (A [4608,12288] GELU(N(0,1)), W [3072,12288]):
+    per-kernel times of the MXFP8 quantizer and the MXFP8 GEMM."""
+    w = workloads.WORKLOADS["ffdown"]
+    M, N, K = w.M, w.N, w.K
+    xs = [workloads.activation("ffdown", seed=i).to(device) for i in range(2)]
+    wc, wsf, _ = nvq.quantize_weight("mxfp8", workloads.weight("ffdown").to(device))
+    codes = torch.empty((M, K), dtype=torch.uint8, device=device)
+    scales = torch.empty(nvq.scale_bytes("mxfp8", M, K), dtype=torch.uint8, device=device)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    iters = 50
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+    for i in range(5 + iters):
+        timed = i >= 5
+        e = evs[i - 5] if timed else None
+        if timed:
+            e[0].record(stream)
+        nvq.mxfp8_quantize(xs[i % 2], codes, scales, stream=stream)
+        if timed:
+            e[1].record(stream)
+        nvq.block_scaled_linear("mxfp8", codes, scales, None, wc, wsf, None, M, N, K, out=out, stream=stream)
+        if timed:
+            e[2].record(stream)
+    torch.cuda.synchronize(device)
+    q_us = statistics.mean(e[0].elapsed_time(e[1]) * 1e3 for e in evs)
+    g_us = statistics.mean(e[1].elapsed_time(e[2]) * 1e3 for e in evs)
+    flops = 2.0 * M * N * K
+    fp8_peak = peaks["bf16_tflops"] * 2.0
+    qbytes = M * K * (2 + 1 + 1 / 32)
+    return {"workload": "MXFP8 FF-down 4608x3072x12288", "quant_us": round(q_us, 3),
+            "quant_gbs": round(qbytes / (q_us * 1e-6) / 1e9, 1),
+            "quant_frac_hbm": round(qbytes / (q_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+            "gemm_us": round(g_us, 3), "gemm_tflops": round(flops / (g_us * 1e-6) / 1e12, 1),
+            "gemm_frac_fp8": round(flops / (g_us * 1e-6) / 1e12 / fp8_peak, 4),
+            "fp8_peak": round(fp8_peak, 1), "l2": "2 activation batches (226 MB) alternate"}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def oracle_step_seconds(x, w_hat, rows):
+    """Oracle work on a bounded sample: amax of the whole activation, then
+    quantize + dequantize + FP64 GEMM of `rows` rows (calibrated with that
+    amax, which reproduces the dynamic result exactly).  Returns the time
+    extrapolated to the full M rows, and the measured seconds."""
+    import oracle
+
+    xb = x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    M, K = xb.shape
+    t0 = time.perf_counter()
+    amax = oracle.amax(xb)
+    t1 = time.perf_counter()
+    sub = xb[:rows]
+    c, s, g = oracle.nvfp4_quantize(sub, calib_amax=amax)
+    a_hat = oracle.nvfp4_dequantize(c, s, g, rows, K)
+    oracle.gemm_rows(a_hat, w_hat)
+    t2 = time.perf_counter()
+    return (t1 - t0) + (t2 - t1) * (M / rows), (t2 - t0)
+
+
+def cpu_baseline(budget_s=15.0):
+    import oracle
+
+    w = workloads.WORKLOADS[WORKLOAD]
+    M, N, K = w.M, w.N, w.K
+    x = workloads.activation(WORKLOAD)
+    wt = workloads.weight(WORKLOAD)
+    wb = wt.contiguous().view(torch.int16).numpy().view(np.uint16)
+    wc, wsf, wg = oracle.nvfp4_quantize(wb)
+    w_hat = oracle.nvfp4_dequantize(wc, wsf, wg, N, K)
+    full, measured = oracle_step_seconds(x, w_hat, 128)          # calibrate the rate
+    rows = int(max(128, min(M, 128 * round(budget_s / max(measured, 1e-3)))))
+    rows = max(128, rows // 128 * 128)
+    full, measured = oracle_step_seconds(x, w_hat, rows)
+    return {"value": round(2.0 * M * N * K / full / 1e12, 6), "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "activation amax over all 4608 rows, then NVFP4 quantize + FP64 dequantize + FP64 GEMM "
+                      "of the first %d rows against the full dequantized weight; time extrapolated to 4608 rows "
+                      "(%.1f s measured)" % (rows, measured),
+            "seconds_full_step_extrapolated": round(full, 2)}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on the host cores."""
+    import oracle
+
+    w = workloads.WORKLOADS[WORKLOAD]
+    M, N, K = w.M, w.N, w.K
+    x = workloads.activation(WORKLOAD)
+    wt = workloads.weight(WORKLOAD)
+    wb = wt.contiguous().view(torch.int16).numpy().view(np.uint16)
+    wc, wsf, wg = oracle.nvfp4_quantize(wb)
+    w_hat = oracle.nvfp4_dequantize(wc, wsf, wg, N, K)
+    total_budget = 150.0
+    _, probe = oracle_step_seconds(x, w_hat, 8)
+    per_step = total_budget / max(1, args.steps + args.warmup)
+    rows = int(max(1, min(M, 8 * per_step / max(probe, 1e-4))))
+    for _ in range(args.warmup):
+        oracle_step_seconds(x, w_hat, rows)
+    fulls = [oracle_step_seconds(x, w_hat, rows)[0] for _ in range(args.steps)]
+    full = statistics.mean(fulls)
+    value = 2.0 * M * N * K / full / 1e12
+    sample = ("per step: activation amax over all 4608 rows, then NVFP4 quantize + FP64 dequantize + FP64 GEMM "
+              "of the first %d rows against the full dequantized weight; time extrapolated to 4608 rows" % rows)
+    return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(full * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "NVFP4 W4A4 FF-up linear, FLUX-like, 4608x12288x3072 (CPU oracle)",
+                       "M": M, "N": N, "K": K},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# --------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-mxfp8", dest="mxfp8", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        res = run_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            res["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

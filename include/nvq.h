@@ -1,0 +1,209 @@
+/*
+ * nvq.h -- C ABI of the B200 (sm_100a) microscaling-quantized linear layer.
+ *
+ * The layer has two parts (page "NVIDIA量化推理：5步极速优化显存+成功率翻倍",
+ * section "MXFP8和NVFP4技术背景解析"; page "NVIDIA Blackwell平台FP4量化技术解析与
+ * 图像生成优化", section 3.1):
+ *   1. dynamic activation quantization, BF16 -> NVFP4 (E2M1 values in
+ *      16-element blocks, an E4M3 block scale, one FP32 per-tensor global
+ *      scale) or BF16 -> MXFP8 (E4M3 values in 32-element blocks, an E8M0
+ *      block scale);
+ *   2. the block-scaled GEMM that multiplies the quantized activations by
+ *      pre-quantized weights on the tensor cores and writes BF16.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All data pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or keeps them.  It allocates no device memory of
+ *    its own: the only library state on the device is one status word per
+ *    GPU (a static device variable), read by nvq_device_status().
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  The return value reports only host-side argument
+ *    checks and launch errors.  Errors found by the host launch nothing.
+ *  - Matrices are row-major.  BF16 tensors are [rows, K] with a row pitch
+ *    `ld` in elements.  Quantized codes are dense: an NVFP4 row is K/2 bytes
+ *    (element 2j in the low nibble of byte j, 2j+1 in the high nibble), an
+ *    MXFP8 row is K bytes of E4M3.
+ *  - Block scales form a logical matrix S[rows][K / block] of bytes (E4M3 for
+ *    NVFP4, E8M0 for MXFP8) stored in the 128x4 tile order the sm_100
+ *    block-scaled tensor-core instructions read: tiles of 128 rows x 4
+ *    scale columns, 512 bytes each, tile (r/128, c/4) at
+ *    ((r/128) * (C/4) + c/4) * 512, and inside a tile row r, column c at
+ *    (r%32)*16 + ((r%128)/32)*4 + (c%4), where C = K / block.
+ *  - Shape contract: rows (M, N) multiples of 128 ("block alignment must be
+ *    a multiple of 128", NVIDIA Blackwell平台FP4量化技术解析与图像生成优化,
+ *    section 5.2); K a positive multiple of 64 (NVFP4) or 128 (MXFP8) so
+ *    scale columns fill whole tiles; every BF16 pitch a multiple of 8
+ *    elements and >= K; all pointers 16-byte aligned; rows * K < 2^31.
+ *    Otherwise NVQ_ERR_SHAPE / NVQ_ERR_ALIGN, and nothing is launched.
+ *    M == 0 (an empty batch) is accepted and launches nothing.
+ *  - The device must be compute capability 10.0 (B200, sm_100a), else
+ *    NVQ_ERR_ARCH.
+ *  - Inputs must be finite.  A NaN or infinity in a tensor handed to
+ *    nvfp4_quantize sets NVQ_STATUS_NONFINITE in the device status word; the
+ *    codes written for such a tensor are unspecified.
+ */
+#ifndef NVQ_H
+#define NVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define NVQ_API __attribute__((visibility("default")))
+#else
+#define NVQ_API
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st* nvq_stream_t;
+
+typedef enum { NVQ_NVFP4 = 0, NVQ_MXFP8 = 1 } nvq_format;
+
+/* Return codes (host side). */
+enum {
+    NVQ_OK = 0,
+    NVQ_ERR_NULL = -1,      /* a required pointer is NULL */
+    NVQ_ERR_SHAPE = -2,     /* a size or pitch breaks the shape contract */
+    NVQ_ERR_ALIGN = -3,     /* a pointer is not 16-byte aligned */
+    NVQ_ERR_ARCH = -4,      /* current device is not compute capability 10.0 */
+    NVQ_ERR_CUDA = -5,      /* a CUDA runtime/driver call or launch failed */
+    NVQ_ERR_FORMAT = -7     /* unknown nvq_format value */
+};
+
+/* Bits of the device status word (nvq_device_status). */
+enum {
+    NVQ_STATUS_TIMEOUT = 1,     /* a GEMM pipeline wait gave up (bounded spin) */
+    NVQ_STATUS_NONFINITE = 2    /* nvfp4_quantize saw a NaN/Inf amax */
+};
+
+/* Bytes of the code buffer for a [rows, K] tensor: rows*K/2 (NVFP4), rows*K (MXFP8). */
+NVQ_API size_t nvq_codes_bytes(int format, int64_t rows, int64_t K);
+
+/* Bytes of the swizzled scale buffer: ceil(rows/128)*128 * ceil((K/block)/4)*4,
+ * block = 16 (NVFP4) or 32 (MXFP8). */
+NVQ_API size_t nvq_scale_bytes(int format, int64_t rows, int64_t K);
+
+/* Bytes of device scratch that nvfp4_quantize / quantize_weight(NVQ_NVFP4)
+ * need (per-CTA partial maxima of the tensor; fully rewritten by every call,
+ * so it needs no initialization).  Constant for the life of the library. */
+NVQ_API size_t nvq_workspace_bytes(void);
+
+/*
+ * nvfp4_quantize -- dynamic BF16 -> NVFP4 activation quantization.
+ * Page "NVIDIA Blackwell平台FP4量化技术解析与图像生成优化", section 3.1: the
+ * run-time quantizer turns a BF16 input into [FP4 data, FP8 block scales,
+ * FP32 global scale]; page "NVIDIA量化推理：5步极速优化显存+成功率翻倍",
+ * step 2: the per-tensor scale is computed from the live activation.
+ *
+ *   x            [M, K] BF16, row pitch ldx elements (read only)
+ *   codes        out, nvq_codes_bytes(NVQ_NVFP4, M, K) bytes
+ *   scales       out, nvq_scale_bytes(NVQ_NVFP4, M, K) bytes (E4M3, tile order)
+ *   global_scale out, one float: the decode scale g_dec = amax / 2688
+ *   calib_amax   NULL for the dynamic path (amax taken from x).  Otherwise a
+ *                device float holding a calibrated per-tensor amax (page
+ *                "FP8量化技术提升SD3.5...", section 校准): the amax pass is
+ *                skipped; elements beyond the calibrated range saturate.
+ *   workspace    device scratch of nvq_workspace_bytes(); must not be shared
+ *                by two calls that can run at the same time.
+ *
+ * Arithmetic, in FP32 round-to-nearest-even, bit-exact with the CPU oracle:
+ *   g_enc = 2688 / amax, g_dec = amax / 2688; per 16-block along K,
+ *   b = max|x|, sc = E4M3(b / 6 * g_enc), r = g_enc / sc, q = E2M1(x * r)
+ *   (round to nearest even, saturate, sign kept).  A block whose scale
+ *   rounds to zero gets zero codes.  amax < 2^-100 (zero included) gives
+ *   all-zero codes and scales and g_dec = 0.
+ */
+NVQ_API int nvfp4_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
+                   uint8_t* codes, uint8_t* scales, float* global_scale,
+                   const float* calib_amax, void* workspace, nvq_stream_t stream);
+
+/*
+ * mxfp8_quantize -- BF16 -> MXFP8 (E4M3 elements, E8M0 scale per 32-block).
+ * Page "NVIDIA量化推理：5步极速优化显存+成功率翻倍", section "MXFP8量化格式"
+ * (OCP 8-bit microscaling format).  Per 32-block along K: X = floor(log2(max
+ * |x|)) - 8 clamped to [-127, 127] (-127 for an all-zero block), scale byte
+ * X + 127, q = E4M3(x * 2^-X) rounded to nearest even and saturated at 448.
+ *
+ *   x       [M, K] BF16, row pitch ldx elements
+ *   codes   out, nvq_codes_bytes(NVQ_MXFP8, M, K) bytes
+ *   scales  out, nvq_scale_bytes(NVQ_MXFP8, M, K) bytes (E8M0, tile order)
+ */
+NVQ_API int mxfp8_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
+                   uint8_t* codes, uint8_t* scales, nvq_stream_t stream);
+
+/*
+ * quantize_weight -- offline weight quantization ("double quantization" of
+ * BF16 weights into FP4 data + FP8 scales, page "NVIDIA Blackwell平台FP4量化
+ * 技术解析与图像生成优化", section 3.1), run once at load time.  Same
+ * arithmetic as nvfp4_quantize / mxfp8_quantize applied to W [N, K]; for
+ * NVFP4 the global scale is the weight's own static g_dec.
+ *
+ *   global_scale  NVFP4: out, required.  MXFP8: ignored (may be NULL).
+ *   workspace     NVFP4: required (nvq_workspace_bytes()).  MXFP8: ignored.
+ */
+NVQ_API int quantize_weight(int format, const void* w, int64_t N, int64_t K, int64_t ldw,
+                    uint8_t* codes, uint8_t* scales, float* global_scale,
+                    void* workspace, nvq_stream_t stream);
+
+/*
+ * block_scaled_linear -- D = A * B^T on the block-scaled tensor cores
+ * (page "NVIDIA Blackwell平台FP4量化技术解析与图像生成优化", section 3.1: FP4
+ * operands with FP8 block scales consumed by the 5th-generation tensor
+ * cores; page "NVIDIA量化推理：5步极速优化显存+成功率翻倍": every nn.Linear of
+ * the transformer becomes a quantized linear).
+ *
+ *   D[m, n] = bf16( alpha * sum_k a(m,k) * sa(m, k/bs) * b(n,k) * sb(n, k/bs) + bias[n] )
+ *   with alpha = a_global[0] * b_global[0] for NVFP4 and 1 for MXFP8.
+ *
+ *   a_codes, a_scales   quantized activations [M, K] (nvfp4_quantize/mxfp8_quantize)
+ *   a_global            NVFP4: device float g_dec of A.  MXFP8: ignored.
+ *   b_codes, b_scales   quantized weights [N, K] (quantize_weight)
+ *   b_global            NVFP4: device float g_dec of B.  MXFP8: ignored.
+ *   bias                NULL or BF16 [N]
+ *   out                 BF16 [M, N], row pitch ldo elements (ldo >= N, multiple of 8)
+ *   M, N                multiples of 128; K a multiple of 256 (NVFP4) or 128 (MXFP8)
+ *
+ * Accumulation is FP32 in tensor memory; the order of the K sum is the
+ * hardware's.  Results match the FP64 sum over the dequantized operands to
+ * a relative error (normalised by the output row's L2 norm) of 2e-3.
+ * Pipeline waits inside the kernel are bounded; if one gives up, the kernel
+ * sets NVQ_STATUS_TIMEOUT, writes nothing further and exits.
+ */
+NVQ_API int block_scaled_linear(int format,
+                        const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                        const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global,
+                        const void* bias, void* out, int64_t ldo,
+                        int64_t M, int64_t N, int64_t K, nvq_stream_t stream);
+
+/*
+ * nvq_device_status -- synchronizes `stream`, then returns the current
+ * device's status word (NVQ_STATUS_* bits, 0 = clean) and clears it.
+ * Returns NVQ_ERR_CUDA (< 0) if the synchronization or the read fails.
+ */
+NVQ_API int nvq_device_status(nvq_stream_t stream);
+
+/* Human-readable name of a return code. */
+NVQ_API const char* nvq_status_string(int code);
+
+/*
+ * nvq_probe_convert -- conversion self-test (no counterpart on the pages).
+ * Runs the device's FP32 -> E2M1 and FP32 -> E4M3 round-to-nearest-even,
+ * saturating conversions that the quantize kernels use on n inputs, so
+ * tests can compare them with the CPU oracle on every tie and edge case.
+ *   in         n floats (device)
+ *   e2m1_out   n bytes (device), code in the low nibble
+ *   e4m3_out   n bytes (device)
+ */
+NVQ_API int nvq_probe_convert(const float* in, int64_t n, uint8_t* e2m1_out, uint8_t* e4m3_out,
+                      nvq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVQ_H */

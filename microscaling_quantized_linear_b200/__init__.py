@@ -1,0 +1,234 @@
+"""Python binding of ``libnvq.so``: the B200 microscaling-quantized linear layer.
+
+Argument marshalling only.  Every step of quantization and of the GEMM runs
+in the CUDA kernels behind the C ABI declared in ``include/nvq.h``; this
+module turns torch tensors into device pointers and the current CUDA stream,
+allocates output tensors with torch when the caller does not pass them, and
+raises ``NvqError`` on a non-zero return code.  There is no fallback: if the
+shared library is missing, importing this package fails.
+
+Names follow the C ABI: ``nvfp4_quantize``, ``mxfp8_quantize``,
+``quantize_weight``, ``block_scaled_linear``, plus the size helpers.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnvq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libnvq.so is not built (expected at %s); run "
+        "`python -m microscaling_quantized_linear_b200.build` or __graft_entry__.build()" % LIB_PATH)
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+NVFP4 = 0
+MXFP8 = 1
+_FORMATS = {"nvfp4": NVFP4, "mxfp8": MXFP8, NVFP4: NVFP4, MXFP8: MXFP8}
+
+NVQ_STATUS_TIMEOUT = 1
+NVQ_STATUS_NONFINITE = 2
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_sz = ctypes.c_size_t
+
+_lib.nvq_codes_bytes.restype = _sz
+_lib.nvq_codes_bytes.argtypes = [ctypes.c_int, _i64, _i64]
+_lib.nvq_scale_bytes.restype = _sz
+_lib.nvq_scale_bytes.argtypes = [ctypes.c_int, _i64, _i64]
+_lib.nvq_workspace_bytes.restype = _sz
+_lib.nvq_workspace_bytes.argtypes = []
+_lib.nvfp4_quantize.restype = ctypes.c_int
+_lib.nvfp4_quantize.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.mxfp8_quantize.restype = ctypes.c_int
+_lib.mxfp8_quantize.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp]
+_lib.quantize_weight.restype = ctypes.c_int
+_lib.quantize_weight.argtypes = [ctypes.c_int, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]
+_lib.block_scaled_linear.restype = ctypes.c_int
+_lib.block_scaled_linear.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
+                                     _i64, _i64, _i64, _vp]
+_lib.nvq_device_status.restype = ctypes.c_int
+_lib.nvq_device_status.argtypes = [_vp]
+_lib.nvq_status_string.restype = ctypes.c_char_p
+_lib.nvq_status_string.argtypes = [ctypes.c_int]
+_lib.nvq_probe_convert.restype = ctypes.c_int
+_lib.nvq_probe_convert.argtypes = [_vp, _i64, _vp, _vp, _vp]
+
+EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_quantize",
+            "mxfp8_quantize", "quantize_weight", "block_scaled_linear", "nvq_device_status",
+            "nvq_status_string", "nvq_probe_convert")
+
+
+class NvqError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__("%s failed: %s (%d)" % (what, status_string(code), code))
+
+
+def status_string(code):
+    return _lib.nvq_status_string(int(code)).decode()
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise NvqError(rc, what)
+
+
+def _fmt(f):
+    try:
+        return _FORMATS[f]
+    except KeyError:
+        raise ValueError("unknown format %r" % (f,)) from None
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _pitch(t):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit stride in the last dimension")
+    return t.stride(0)
+
+
+# --------------------------------------------------------------------------- sizes
+
+def codes_bytes(fmt, rows, K):
+    return int(_lib.nvq_codes_bytes(_fmt(fmt), rows, K))
+
+
+def scale_bytes(fmt, rows, K):
+    return int(_lib.nvq_scale_bytes(_fmt(fmt), rows, K))
+
+
+def workspace_bytes():
+    return int(_lib.nvq_workspace_bytes())
+
+
+def new_workspace(device="cuda"):
+    return torch.empty(workspace_bytes(), dtype=torch.uint8, device=device)
+
+
+# --------------------------------------------------------------------------- quantizers
+
+def nvfp4_quantize(x, codes=None, scales=None, global_scale=None, calib_amax=None, workspace=None,
+                   stream=None):
+    """BF16 [M, K] -> (codes u8 [M, K/2], scales u8 (tile order), global_scale f32 [1])."""
+    M, K = x.shape
+    dev = x.device
+    codes = codes if codes is not None else torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    scales = scales if scales is not None else torch.empty(scale_bytes(NVFP4, M, K), dtype=torch.uint8, device=dev)
+    global_scale = global_scale if global_scale is not None else torch.empty(1, dtype=torch.float32, device=dev)
+    if workspace is None and calib_amax is None:
+        workspace = new_workspace(dev)
+    _check(_lib.nvfp4_quantize(_ptr(x), M, K, _pitch(x), _ptr(codes), _ptr(scales), _ptr(global_scale),
+                               _ptr(calib_amax), _ptr(workspace), _stream(stream, dev)), "nvfp4_quantize")
+    return codes, scales, global_scale
+
+
+def mxfp8_quantize(x, codes=None, scales=None, stream=None):
+    """BF16 [M, K] -> (codes u8 [M, K] (E4M3), scales u8 (E8M0, tile order))."""
+    M, K = x.shape
+    dev = x.device
+    codes = codes if codes is not None else torch.empty((M, K), dtype=torch.uint8, device=dev)
+    scales = scales if scales is not None else torch.empty(scale_bytes(MXFP8, M, K), dtype=torch.uint8, device=dev)
+    _check(_lib.mxfp8_quantize(_ptr(x), M, K, _pitch(x), _ptr(codes), _ptr(scales), _stream(stream, dev)),
+           "mxfp8_quantize")
+    return codes, scales
+
+
+def quantize_weight(fmt, w, codes=None, scales=None, global_scale=None, workspace=None, stream=None):
+    """Offline weight quantization; returns (codes, scales, global_scale or None)."""
+    f = _fmt(fmt)
+    N, K = w.shape
+    dev = w.device
+    cols = K // 2 if f == NVFP4 else K
+    codes = codes if codes is not None else torch.empty((N, cols), dtype=torch.uint8, device=dev)
+    scales = scales if scales is not None else torch.empty(scale_bytes(f, N, K), dtype=torch.uint8, device=dev)
+    if f == NVFP4:
+        global_scale = global_scale if global_scale is not None else torch.empty(1, dtype=torch.float32, device=dev)
+        workspace = workspace if workspace is not None else new_workspace(dev)
+    _check(_lib.quantize_weight(f, _ptr(w), N, K, _pitch(w), _ptr(codes), _ptr(scales), _ptr(global_scale),
+                                _ptr(workspace), _stream(stream, dev)), "quantize_weight")
+    return codes, scales, global_scale
+
+
+# --------------------------------------------------------------------------- GEMM
+
+def block_scaled_linear(fmt, a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K,
+                        bias=None, out=None, stream=None):
+    """D = bf16(alpha * A . B^T + bias) on the block-scaled tensor cores; returns out [M, N]."""
+    f = _fmt(fmt)
+    dev = a_codes.device
+    out = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _check(_lib.block_scaled_linear(f, _ptr(a_codes), _ptr(a_scales), _ptr(a_global), _ptr(b_codes),
+                                    _ptr(b_scales), _ptr(b_global), _ptr(bias), _ptr(out), _pitch(out),
+                                    M, N, K, _stream(stream, dev)), "block_scaled_linear")
+    return out
+
+
+class QuantizedLinear:
+    """A linear layer whose weight is quantized once (offline) and whose
+    activations are quantized on every call, then multiplied on the
+    block-scaled tensor cores.  Holds device buffers only; each call is the
+    ABI sequence quantize -> block_scaled_linear on one stream."""
+
+    def __init__(self, weight, fmt="nvfp4", bias=None):
+        self.fmt = _fmt(fmt)
+        self.N, self.K = weight.shape
+        self.device = weight.device
+        self.w_codes, self.w_scales, self.w_global = quantize_weight(self.fmt, weight)
+        self.bias = bias
+        self._ws = new_workspace(self.device) if self.fmt == NVFP4 else None
+        self._bufs = {}
+
+    def _act_bufs(self, M):
+        b = self._bufs.get(M)
+        if b is None:
+            cols = self.K // 2 if self.fmt == NVFP4 else self.K
+            b = (torch.empty((M, cols), dtype=torch.uint8, device=self.device),
+                 torch.empty(scale_bytes(self.fmt, M, self.K), dtype=torch.uint8, device=self.device),
+                 torch.empty(1, dtype=torch.float32, device=self.device))
+            self._bufs[M] = b
+        return b
+
+    def __call__(self, x, out=None, stream=None):
+        M = x.shape[0]
+        codes, scales, g = self._act_bufs(M)
+        if self.fmt == NVFP4:
+            nvfp4_quantize(x, codes, scales, g, workspace=self._ws, stream=stream)
+        else:
+            mxfp8_quantize(x, codes, scales, stream=stream)
+            g = None
+        return block_scaled_linear(self.fmt, codes, scales, g, self.w_codes, self.w_scales, self.w_global,
+                                   M, self.N, self.K, bias=self.bias, out=out, stream=stream)
+
+
+# --------------------------------------------------------------------------- diagnostics
+
+def device_status(stream=None, device=None):
+    """Synchronize the stream; return and clear the device status word."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    rc = _lib.nvq_device_status(_stream(stream, dev))
+    if rc < 0:
+        raise NvqError(rc, "nvq_device_status")
+    return rc
+
+
+def probe_convert(values, stream=None):
+    """Device FP32 -> (E2M1 codes, E4M3 codes) with the quantizers' conversions."""
+    n = values.numel()
+    e2 = torch.empty(n, dtype=torch.uint8, device=values.device)
+    e4 = torch.empty(n, dtype=torch.uint8, device=values.device)
+    _check(_lib.nvq_probe_convert(_ptr(values), n, _ptr(e2), _ptr(e4), _stream(stream, values.device)),
+           "nvq_probe_convert")
+    return e2, e4

@@ -1,0 +1,46 @@
+"""Build the CUDA library ``libnvq.so`` in-tree for sm_100a (B200).
+
+One translation unit (``csrc/nvq.cu``) holds the C ABI and includes the
+kernels; the CUDA runtime is linked statically and the driver API is reached
+through ``cudaGetDriverEntryPoint``, so the library loads on a machine
+without a GPU driver (it then reports errors from its entry points).
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+LIB = os.path.join(HERE, "libnvq.so")
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+NVCC_FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-lineinfo", "-std=c++17",
+    "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+    "-cudart", "static",
+    # scale arithmetic must stay IEEE FP32 round-to-nearest in program order
+    "-fmad=false", "-ftz=false", "-prec-div=true", "-prec-sqrt=true",
+    "-I", os.path.join(ROOT, "include"),
+]
+
+
+def sources():
+    return [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cu", ".cuh"))]
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    deps = sources() + [os.path.join(ROOT, "include", "nvq.h"), __file__]
+    if not force and os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(d) for d in deps):
+        return LIB
+    tmp = LIB + ".tmp.%d" % os.getpid()
+    cmd = [NVCC, *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []),
+           os.path.join(CSRC, "nvq.cu"), "-o", tmp]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

@@ -1,0 +1,282 @@
+// gemm.cuh -- block-scaled GEMM on the sm_100a 5th-generation tensor cores.
+//
+//   D[M, N] = bf16( alpha * A[M, K] . B[N, K]^T + bias[N] )
+//
+// A and B are quantized operands (NVFP4: E2M1 codes + E4M3 scales per 16 of
+// K; MXFP8: E4M3 codes + E8M0 scales per 32 of K), both K-major ("TN").
+// The tensor core applies the block scales itself (tcgen05.mma
+// kind::mxf4nvf4 / kind::mxf8f6f4 with .block_scale), so no dequantized copy
+// of either operand ever exists (page "NVIDIA Blackwell平台FP4量化技术解析与图像
+// 生成优化", section 3.1: FP4 decoded to BF16 inside the SM).
+//
+// Structure: one persistent CTA per SM, 6 warps.
+//   warp 0  TMA producer: per pipeline stage one 128 x 128-byte tile of A,
+//           one BN x 128-byte tile of B (tensor maps, 128-byte swizzle), and
+//           the matching 512-byte scale tiles (plain bulk copies: the global
+//           128x4 tile order is exactly what tensor memory wants).
+//   warp 1  allocates tensor memory; one lane moves each stage's scale tiles
+//           to tensor memory (tcgen05.cp) and issues the MMAs into an FP32
+//           accumulator in tensor memory; tcgen05.commit frees the stage.
+//   warps 2-5  epilogue: tensor memory -> registers (tcgen05.ld), scale by
+//           alpha, add bias, round to BF16, store.
+// Every mbarrier wait is bounded in wall time; a wait that gives up sets the
+// status word and an abort flag that releases the other roles.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+
+namespace nvq {
+
+constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s per wait
+
+template <int FMT, int BN_>
+struct GemmCfg {
+    static constexpr int BM = 128;
+    static constexpr int BN = BN_;
+    static constexpr int KBYTES = 128;                       // bytes of K per stage (one swizzle atom)
+    static constexpr int BK = FMT == 0 ? 256 : 128;          // K elements per stage
+    static constexpr int MMA_K = FMT == 0 ? 64 : 32;         // K elements per instruction
+    static constexpr int KSTEPS = BK / MMA_K;                // 4 instructions per stage
+    static constexpr int MMA_K_BYTES = KBYTES / KSTEPS;      // 32
+    static constexpr int SF_BLOCK = FMT == 0 ? 16 : 32;
+    static constexpr int SF_ATOMS = BK / SF_BLOCK / 4;       // 128x4 scale tiles per 128 rows per stage
+    static constexpr int A_BYTES = BM * KBYTES;
+    static constexpr int B_BYTES = BN * KBYTES;
+    static constexpr int SFA_BYTES = SF_ATOMS * 512;
+    static constexpr int SFB_BYTES = (BN / 128) * SF_ATOMS * 512;
+    static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int STAGE_BYTES = (TX_BYTES + 1023) / 1024 * 1024;
+    static constexpr int STAGES = 4;
+    static constexpr int OFF_B = A_BYTES;
+    static constexpr int OFF_SFA = A_BYTES + B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
+    // tensor-memory columns: accumulator, then scale factors of A and B
+    static constexpr int TM_ACC = 0;
+    static constexpr int TM_SFA = BN;
+    static constexpr int SFA_COLS = FMT == 0 ? 4 * KSTEPS : 4;
+    static constexpr int TM_SFB = TM_SFA + SFA_COLS;
+    static constexpr int SFB_COLS_PER_MMA = 4 * (BN / 128);
+    static constexpr int SFB_COLS = FMT == 0 ? SFB_COLS_PER_MMA * KSTEPS : SFB_COLS_PER_MMA;
+    static constexpr int TM_USED = TM_SFB + SFB_COLS;
+    static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
+    static constexpr int THREADS = 192;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    // instruction descriptor: A/B format (E2M1 = 1 for mxf4nvf4, E4M3 = 0 for
+    // mxf8f6f4) in bits 7-9 / 10-12, K-major A and B, N >> 3 in bits 17-22,
+    // scale format (0 = UE4M3, 1 = UE8M0) in bit 23, M >> 4 in bits 24-28.
+    static constexpr uint32_t IDESC =
+        (FMT == 0 ? (1u << 7) | (1u << 10) : 0u) |
+        ((uint32_t)(BN >> 3) << 17) |
+        (FMT == 0 ? 0u : (1u << 23)) |
+        ((uint32_t)(BM >> 4) << 24);
+    static_assert(TM_USED <= 512, "tensor memory overflow");
+    static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
+};
+
+struct GemmParams {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const float* a_global;
+    const float* b_global;
+    const __nv_bfloat16* bias;
+    __nv_bfloat16* out;
+    unsigned int* status;
+    uint32_t ldo;
+    uint32_t num_m_blocks, num_n_blocks, num_k_tiles;
+    uint32_t sf_ctiles;          // (K / SF_BLOCK) / 4: scale tiles per 128 rows
+};
+
+template <int FMT, int BN>
+__global__ void __launch_bounds__(192, 1)
+bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+              const GemmParams p) {
+    using C = GemmCfg<FMT, BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    const uint32_t full0 = smem_u32(bars);
+    const uint32_t empty0 = full0 + 8 * C::STAGES;
+    const uint32_t tfull = empty0 + 8 * C::STAGES;
+    const uint32_t tempty = tfull + 8;
+    const uint32_t drain = tempty + 8;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 3);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    volatile int* never = abort_flag + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        mbar_init(tfull, 1);
+        mbar_init(tempty, 4);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        *never = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmap_a);
+        prefetch_tensormap(&tmap_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), C::TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const uint32_t num_tiles = p.num_m_blocks * p.num_n_blocks;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+                for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt) {
+                    const uint32_t s = it % C::STAGES, use = it / C::STAGES;
+                    if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint32_t fb = full0 + 8 * s;
+                    mbar_arrive_expect_tx(fb, C::TX_BYTES);
+                    tma_load_2d(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), (int32_t)(mb * C::BM));
+                    tma_load_2d(st + C::OFF_B, &tmap_b, fb, (int32_t)(kt * C::KBYTES), (int32_t)(nb * BN));
+                    bulk_load(st + C::OFF_SFA,
+                              p.sfa + ((size_t)mb * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
+                              C::SFA_BYTES, fb);
+#pragma unroll
+                    for (int h = 0; h < BN / 128; ++h)
+                        bulk_load(st + C::OFF_SFB + h * C::SF_ATOMS * 512,
+                                  p.sfb + ((size_t)(nb * (BN / 128) + h) * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
+                                  C::SF_ATOMS * 512, fb);
+                    ++it;
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+            }
+            // every load this thread issued must land before the CTA exits
+            for (uint32_t j = it > (uint32_t)C::STAGES ? it - C::STAGES : 0; j < it; ++j)
+                mbar_wait_bounded(full0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, t_local = 0;
+            bool ok = true;
+            for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t_local) {
+                if (t_local > 0 && !mbar_wait_bounded(tempty, (t_local - 1) & 1, abort_flag, kWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt, ++it) {
+                    const uint32_t s = it % C::STAGES, use = it / C::STAGES;
+                    if (!mbar_wait_bounded(full0 + 8 * s, use & 1, abort_flag, kWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
+                    // scale tiles: shared memory -> tensor memory (4 columns each)
+#pragma unroll
+                    for (int a = 0; a < C::SF_ATOMS; ++a)
+                        tc_cp_32x128b_warpx4(tmem + C::TM_SFA + 4 * a,
+                                             smem_desc(st + C::OFF_SFA + 512 * a, 16, 128, 0));
+#pragma unroll
+                    for (int h = 0; h < BN / 128; ++h)
+#pragma unroll
+                        for (int a = 0; a < C::SF_ATOMS; ++a)
+                            tc_cp_32x128b_warpx4(tmem + C::TM_SFB + C::SFB_COLS_PER_MMA * a + 4 * h,
+                                                 smem_desc(st + C::OFF_SFB + h * C::SF_ATOMS * 512 + 512 * a, 16, 128, 0));
+#pragma unroll
+                    for (int k = 0; k < C::KSTEPS; ++k) {
+                        const uint64_t adesc = smem_desc(st + k * C::MMA_K_BYTES, 16, 1024, 2);
+                        const uint64_t bdesc = smem_desc(st + C::OFF_B + k * C::MMA_K_BYTES, 16, 1024, 2);
+                        const uint32_t acc = (kt | (uint32_t)k) != 0;
+                        if (FMT == 0) {
+                            tc_mma_nvf4(tmem + C::TM_ACC, adesc, bdesc, C::IDESC,
+                                        tmem + C::TM_SFA + 4 * k,
+                                        tmem + C::TM_SFB + C::SFB_COLS_PER_MMA * k, acc);
+                        } else {
+                            const uint32_t id = C::IDESC | ((uint32_t)k << 29) | ((uint32_t)k << 4);
+                            tc_mma_mxf8(tmem + C::TM_ACC, adesc, bdesc, id,
+                                        (tmem + C::TM_SFA) | ((uint32_t)k << 30),
+                                        (tmem + C::TM_SFB) | ((uint32_t)k << 30), acc);
+                        }
+                    }
+                    tc_commit(empty0 + 8 * s);
+                }
+                if (!ok) break;
+                tc_commit(tfull);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+            }
+            tc_commit(drain);
+            mbar_wait_bounded(drain, 0, never, kWaitLimitNs);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int q = warp & 3;                       // tensor-memory lane quarter of this warp
+        const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
+        uint32_t t_local = 0;
+        for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t_local) {
+            const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+            if (!mbar_wait_bounded(tfull, t_local & 1, abort_flag, kWaitLimitNs)) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t row = mb * C::BM + 32 * q + lane;
+            __nv_bfloat16* orow = p.out + (size_t)row * p.ldo + (size_t)nb * BN;
+            const __nv_bfloat16* brow = p.bias ? p.bias + (size_t)nb * BN : nullptr;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                uint32_t r[32];
+                tc_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + C::TM_ACC + c, r);
+                tc_wait_ld();
+                uint32_t packed[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    float v0 = __fmul_rn(__uint_as_float(r[2 * j]), alpha);
+                    float v1 = __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha);
+                    if (brow) {
+                        const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(brow + c + 2 * j);
+                        v0 = __fadd_rn(v0, __bfloat162float(bb.x));
+                        v1 = __fadd_rn(v1, __bfloat162float(bb.y));
+                    }
+                    const __nv_bfloat162 o = __floats2bfloat162_rn(v0, v1);
+                    packed[j] = *reinterpret_cast<const uint32_t*>(&o);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TM_COLS);
+    }
+}
+
+}  // namespace nvq

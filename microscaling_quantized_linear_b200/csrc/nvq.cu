@@ -1,0 +1,320 @@
+// nvq.cu -- C ABI of the microscaling-quantized linear layer (see include/nvq.h).
+//
+// Host side only: argument checks (nothing is launched when one fails),
+// per-device capability and SM-count cache, TMA descriptor encoding through
+// the driver entry point (no link-time dependency on libcuda), kernel
+// launches on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/nvq.h"
+#include "gemm.cuh"
+#include "quantize.cuh"
+
+namespace nvq {
+
+// One status word per device (NVQ_STATUS_* bits), set by kernels, read and
+// cleared by nvq_device_status().
+__device__ unsigned int g_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool arch_ok = false;
+    int num_sms = 0;
+    unsigned int* status = nullptr;
+    bool gemm_attr[2][2] = {{false, false}, {false, false}};
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return NVQ_ERR_CUDA;
+        d.arch_ok = (major == 10 && minor == 0);
+        d.num_sms = sms;
+        if (d.arch_ok) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return NVQ_ERR_CUDA;
+            d.status = static_cast<unsigned int*>(p);
+        }
+        d.ready = true;
+    }
+    if (!d.arch_ok) return NVQ_ERR_ARCH;
+    *out = &d;
+    return NVQ_OK;
+}
+
+int get_encoder() {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_encode) return NVQ_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return NVQ_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    return NVQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int block_of(int format) { return format == NVQ_NVFP4 ? 16 : 32; }
+int k_multiple(int format) { return format == NVQ_NVFP4 ? 64 : 128; }
+
+// Checks shared by the quantizers: BF16 [rows, K] input with pitch ld.
+int check_quant_shape(int format, int64_t rows, int64_t K, int64_t ld) {
+    if (rows < 0 || K <= 0 || rows % 128 != 0 || K % k_multiple(format) != 0) return NVQ_ERR_SHAPE;
+    if (ld < K || ld % 8 != 0) return NVQ_ERR_SHAPE;
+    if (rows * K >= (int64_t(1) << 31) || rows * ld >= (int64_t(1) << 40) || ld >= (int64_t(1) << 31))
+        return NVQ_ERR_SHAPE;
+    return NVQ_OK;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? NVQ_OK : NVQ_ERR_CUDA; }
+
+int launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, uint32_t* partial, int num_sms,
+                cudaStream_t stream, uint32_t* npartial_out) {
+    const uint32_t vecs_per_row = (uint32_t)(K / 8), pitch_vecs = (uint32_t)(ld / 8);
+    const uint64_t total = (uint64_t)rows * vecs_per_row;
+    uint64_t want = (total + 4 * kAmaxThreads - 1) / (4 * kAmaxThreads);
+    uint32_t grid = (uint32_t)(want < 1 ? 1 : want);
+    const uint32_t cap = (uint32_t)num_sms * 4 < (uint32_t)kMaxAmaxPartials ? (uint32_t)num_sms * 4 : kMaxAmaxPartials;
+    if (grid > cap) grid = cap;
+    amax_partials_kernel<<<grid, kAmaxThreads, 0, stream>>>(static_cast<const uint4*>(x), (uint32_t)rows,
+                                                            vecs_per_row, pitch_vecs, partial);
+    *npartial_out = grid;
+    return launch_status();
+}
+
+uint32_t quant_grid(uint64_t units, int num_sms) {
+    uint64_t blocks = (units + kQuantThreads - 1) / kQuantThreads;
+    const uint64_t cap = (uint64_t)num_sms * 8;      // 8 resident 256-thread CTAs per SM
+    if (blocks > cap) blocks = cap;
+    return (uint32_t)(blocks < 1 ? 1 : blocks);
+}
+
+int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
+                        float* global_scale, const float* calib_amax, void* workspace, cudaStream_t stream) {
+    int rc = check_quant_shape(NVQ_NVFP4, M, K, ldx);
+    if (rc) return rc;
+    if (M == 0) return NVQ_OK;                       // empty batch: nothing to read or write
+    if (!x || !codes || !scales || !global_scale || (!workspace && !calib_amax)) return NVQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (workspace && !aligned16(workspace)))
+        return NVQ_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(global_scale) & 3u) return NVQ_ERR_ALIGN;
+    if (calib_amax && (reinterpret_cast<uintptr_t>(calib_amax) & 3u)) return NVQ_ERR_ALIGN;
+    DeviceInfo* d = nullptr;
+    if ((rc = device_info(&d))) return rc;
+    uint32_t npartial = 0;
+    uint32_t* partial = static_cast<uint32_t*>(workspace);
+    if (!calib_amax) {
+        if ((rc = launch_amax(x, M, K, ldx, partial, d->num_sms, stream, &npartial))) return rc;
+    }
+    const uint32_t nblk = (uint32_t)(K / 16);
+    const uint64_t units = (uint64_t)M * nblk;
+    nvfp4_quantize_kernel<<<quant_grid(units, d->num_sms), kQuantThreads, 0, stream>>>(
+        static_cast<const uint16_t*>(x), (uint32_t)M, nblk, (uint32_t)ldx, codes, scales, global_scale,
+        partial, npartial, calib_amax, d->status);
+    return launch_status();
+}
+
+int mxfp8_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
+                        cudaStream_t stream) {
+    int rc = check_quant_shape(NVQ_MXFP8, M, K, ldx);
+    if (rc) return rc;
+    if (M == 0) return NVQ_OK;
+    if (!x || !codes || !scales) return NVQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return NVQ_ERR_ALIGN;
+    DeviceInfo* d = nullptr;
+    if ((rc = device_info(&d))) return rc;
+    const uint32_t nblk = (uint32_t)(K / 32);
+    const uint64_t units = (uint64_t)M * nblk;
+    mxfp8_quantize_kernel<<<quant_grid(units, d->num_sms), kQuantThreads, 0, stream>>>(
+        static_cast<const uint16_t*>(x), (uint32_t)M, nblk, (uint32_t)ldx, codes, scales);
+    return launch_status();
+}
+
+int encode_codes_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t kbytes, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {(cuuint64_t)kbytes, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kbytes};
+    const cuuint32_t box[2] = {128u, box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVQ_OK : NVQ_ERR_CUDA;
+}
+
+template <int FMT, int BN>
+int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
+                void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    using C = GemmCfg<FMT, BN>;
+    const int64_t kbytes = FMT == 0 ? K / 2 : K;
+    CUtensorMap ma, mb;
+    int rc;
+    if ((rc = encode_codes_map(&ma, a_codes, M, kbytes, C::BM))) return rc;
+    if ((rc = encode_codes_map(&mb, b_codes, N, kbytes, BN))) return rc;
+    auto kern = bsgemm_kernel<FMT, BN>;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!d->gemm_attr[FMT][BN == 256]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+                cudaSuccess)
+                return NVQ_ERR_CUDA;
+            d->gemm_attr[FMT][BN == 256] = true;
+        }
+    }
+    GemmParams p;
+    p.sfa = a_scales;
+    p.sfb = b_scales;
+    p.a_global = a_global;
+    p.b_global = b_global;
+    p.bias = static_cast<const __nv_bfloat16*>(bias);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.status = d->status;
+    p.ldo = (uint32_t)ldo;
+    p.num_m_blocks = (uint32_t)(M / C::BM);
+    p.num_n_blocks = (uint32_t)(N / BN);
+    p.num_k_tiles = (uint32_t)(K / C::BK);
+    p.sf_ctiles = (uint32_t)(K / C::SF_BLOCK / 4);
+    const uint32_t tiles = p.num_m_blocks * p.num_n_blocks;
+    const uint32_t grid = tiles < (uint32_t)d->num_sms ? tiles : (uint32_t)d->num_sms;
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, p);
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace nvq
+
+using namespace nvq;
+
+extern "C" {
+
+size_t nvq_codes_bytes(int format, int64_t rows, int64_t K) {
+    if ((format != NVQ_NVFP4 && format != NVQ_MXFP8) || rows < 0 || K < 0) return 0;
+    return (size_t)(format == NVQ_NVFP4 ? rows * (K / 2) : rows * K);
+}
+
+size_t nvq_scale_bytes(int format, int64_t rows, int64_t K) {
+    if ((format != NVQ_NVFP4 && format != NVQ_MXFP8) || rows < 0 || K < 0) return 0;
+    const int64_t cols = K / block_of(format);
+    return (size_t)(((rows + 127) / 128) * 128 * ((cols + 3) / 4) * 4);
+}
+
+size_t nvq_workspace_bytes(void) { return (size_t)kMaxAmaxPartials * sizeof(uint32_t); }
+
+int nvfp4_quantize(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
+                   float* global_scale, const float* calib_amax, void* workspace, nvq_stream_t stream) {
+    return nvfp4_quantize_impl(x, M, K, ldx, codes, scales, global_scale, calib_amax, workspace,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mxfp8_quantize(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
+                   nvq_stream_t stream) {
+    return mxfp8_quantize_impl(x, M, K, ldx, codes, scales, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int quantize_weight(int format, const void* w, int64_t N, int64_t K, int64_t ldw, uint8_t* codes,
+                    uint8_t* scales, float* global_scale, void* workspace, nvq_stream_t stream) {
+    if (format == NVQ_NVFP4)
+        return nvfp4_quantize_impl(w, N, K, ldw, codes, scales, global_scale, nullptr, workspace,
+                                   reinterpret_cast<cudaStream_t>(stream));
+    if (format == NVQ_MXFP8)
+        return mxfp8_quantize_impl(w, N, K, ldw, codes, scales, reinterpret_cast<cudaStream_t>(stream));
+    return NVQ_ERR_FORMAT;
+}
+
+int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                        const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
+                        void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, nvq_stream_t stream) {
+    if (format != NVQ_NVFP4 && format != NVQ_MXFP8) return NVQ_ERR_FORMAT;
+    // the GEMM stages 256 (NVFP4) / 128 (MXFP8) elements of K at a time
+    const int64_t k_stage = format == NVQ_NVFP4 ? 256 : 128;
+    if (M < 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % k_stage) return NVQ_ERR_SHAPE;
+    if (ldo < N || ldo % 8 || M * ldo >= (int64_t(1) << 40) || ldo >= (int64_t(1) << 31)) return NVQ_ERR_SHAPE;
+    if (K >= (int64_t(1) << 24) || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVQ_ERR_SHAPE;
+    if (M == 0) return NVQ_OK;
+    if (!a_codes || !a_scales || !b_codes || !b_scales || !out) return NVQ_ERR_NULL;
+    if (format == NVQ_NVFP4 && (!a_global || !b_global)) return NVQ_ERR_NULL;
+    if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) ||
+        !aligned16(out) || (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+        return NVQ_ERR_ALIGN;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc) return rc;
+    if ((rc = get_encoder())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool wide = (N % 256) == 0;
+    if (format == NVQ_NVFP4)
+        return wide ? launch_gemm<0, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out,
+                                          ldo, M, N, K, s)
+                    : launch_gemm<0, 128>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out,
+                                          ldo, M, N, K, s);
+    return wide ? launch_gemm<1, 256>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M,
+                                      N, K, s)
+                : launch_gemm<1, 128>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M,
+                                      N, K, s);
+}
+
+int nvq_device_status(nvq_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NVQ_ERR_CUDA;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc) return rc;
+    unsigned int v = 0;
+    if (cudaMemcpy(&v, d->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return NVQ_ERR_CUDA;
+    const unsigned int zero = 0;
+    if (cudaMemcpy(d->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return NVQ_ERR_CUDA;
+    return (int)v;
+}
+
+const char* nvq_status_string(int code) {
+    switch (code) {
+        case NVQ_OK: return "ok";
+        case NVQ_ERR_NULL: return "null pointer";
+        case NVQ_ERR_SHAPE: return "shape or pitch breaks the contract";
+        case NVQ_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case NVQ_ERR_ARCH: return "device is not compute capability 10.0 (sm_100a)";
+        case NVQ_ERR_CUDA: return "CUDA error";
+        case NVQ_ERR_FORMAT: return "unknown format";
+        default: return "unknown status";
+    }
+}
+
+int nvq_probe_convert(const float* in, int64_t n, uint8_t* e2m1_out, uint8_t* e4m3_out, nvq_stream_t stream) {
+    if (!in || !e2m1_out || !e4m3_out) return NVQ_ERR_NULL;
+    if (n < 0 || n >= (int64_t(1) << 31)) return NVQ_ERR_SHAPE;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc) return rc;
+    if (n == 0) return NVQ_OK;
+    const uint32_t grid = quant_grid((uint64_t)n, d->num_sms);
+    probe_convert_kernel<<<grid, kQuantThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        in, (uint32_t)n, e2m1_out, e4m3_out);
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+"""Host-side checks of the C-ABI library that need no GPU.
+
+The library loads without a GPU driver, exports every entry point that
+include/nvq.h declares, and rejects bad arguments before touching the device
+(no kernel is launched and no pointer is dereferenced on these paths).
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import microscaling_quantized_linear_b200 as nvq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvq.h")
+
+NULL = None
+P16 = ctypes.c_void_p(0x10000)         # aligned, never dereferenced
+P_ODD = ctypes.c_void_p(0x10008)       # 8-byte aligned only
+L = nvq._lib
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^NVQ_API\s+[\w\s\*]*?\b(\w+)\s*\(", src, re.M)))
+
+
+def test_header_declarations_are_all_exported():
+    declared = declared_functions()
+    assert len(declared) >= 10
+    out = subprocess.run(["nm", "-D", "--defined-only", nvq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [f for f in declared if f not in exported]
+    assert not missing, missing
+    assert set(declared) == set(nvq.EXPORTED)
+
+
+def test_library_links_no_cuda_shared_objects():
+    out = subprocess.run(["ldd", nvq.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda" not in out and "libcudart" not in out
+
+
+def test_size_helpers():
+    assert nvq.codes_bytes("nvfp4", 4608, 3072) == 4608 * 1536
+    assert nvq.codes_bytes("mxfp8", 4608, 12288) == 4608 * 12288
+    assert nvq.scale_bytes("nvfp4", 4608, 3072) == 4608 * 192
+    assert nvq.scale_bytes("mxfp8", 4608, 12288) == 4608 * 384
+    assert nvq.scale_bytes("nvfp4", 130, 80) == 256 * 8          # padded to 128 rows x 4 columns
+    assert nvq.workspace_bytes() >= 4 * 148
+    assert L.nvq_codes_bytes(7, 128, 64) == 0
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5, -7):
+        assert nvq.status_string(code) and nvq.status_string(code) != "unknown status"
+
+
+def q4(x=P16, M=128, K=64, ld=64, codes=P16, scales=P16, g=P16, calib=NULL, ws=P16):
+    return L.nvfp4_quantize(x, M, K, ld, codes, scales, g, calib, ws, NULL)
+
+
+def test_nvfp4_quantize_rejects_bad_arguments():
+    assert q4(x=NULL) == -1
+    assert q4(codes=NULL) == -1
+    assert q4(g=NULL) == -1
+    assert q4(ws=NULL) == -1                 # dynamic path needs the workspace
+    assert q4(M=100) == -2                   # rows not a multiple of 128
+    assert q4(K=48, ld=48) == -2             # K not a multiple of 64
+    assert q4(ld=60) == -2                   # pitch < K
+    assert q4(ld=68) == -2                   # pitch not a multiple of 8
+    assert q4(M=-128) == -2
+    assert q4(M=1 << 20, K=1 << 12, ld=1 << 12) == -2   # rows * K >= 2^31
+    assert q4(x=P_ODD) == -3
+    assert q4(codes=P_ODD) == -3
+
+
+def test_mxfp8_quantize_rejects_bad_arguments():
+    assert L.mxfp8_quantize(NULL, 128, 128, 128, P16, P16, NULL) == -1
+    assert L.mxfp8_quantize(P16, 128, 64, 64, P16, P16, NULL) == -2      # K not a multiple of 128
+    assert L.mxfp8_quantize(P16, 128, 128, 128, P_ODD, P16, NULL) == -3
+
+
+def test_quantize_weight_rejects_bad_format():
+    assert L.quantize_weight(5, P16, 128, 64, 64, P16, P16, P16, P16, NULL) == -7
+
+
+def gemm(fmt=0, a=P16, sa=P16, ga=P16, b=P16, sb=P16, gb=P16, bias=NULL, out=P16, ldo=128, M=128, N=128, K=256):
+    return L.block_scaled_linear(fmt, a, sa, ga, b, sb, gb, bias, out, ldo, M, N, K, NULL)
+
+
+def test_block_scaled_linear_rejects_bad_arguments():
+    assert gemm(fmt=3) == -7
+    assert gemm(a=NULL) == -1
+    assert gemm(ga=NULL) == -1                # NVFP4 needs both global scales
+    assert gemm(out=NULL) == -1
+    assert gemm(N=64, ldo=64) == -2
+    assert gemm(M=96) == -2
+    assert gemm(K=96) == -2
+    assert gemm(K=192) == -2                  # NVFP4 GEMM K must be a multiple of 256
+    assert gemm(fmt=1, ga=NULL, gb=NULL, K=64) == -2     # MXFP8 K must be a multiple of 128
+    assert gemm(ldo=120) == -2
+    assert gemm(ldo=132) == -2
+    assert gemm(a=P_ODD) == -3
+    assert gemm(out=P_ODD) == -3
+
+
+def test_valid_arguments_without_gpu_report_cuda_error():
+    # Arguments pass the host checks; with no device the library reports a
+    # CUDA error instead of launching.
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert q4() == -5
+    assert gemm() == -5

@@ -1,0 +1,120 @@
+"""GPU parity of the block-scaled GEMM (tcgen05) against the oracle's FP64
+sum over the oracle-dequantized operands.  Acceptance: for every checked row
+max_n |D - Y| / ||Y[row, :]||_2 <= 2e-3.  Small shapes compare every output;
+the full-size workloads compare sampled rows (first and last row of 128-row
+tiles plus random rows) in the same launch configuration the benchmark uses."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_common import act, bits, check_gemm, sample_rows, wgt
+
+pytestmark = pytest.mark.gpu
+
+nvq = pytest.importorskip("microscaling_quantized_linear_b200")
+
+
+def gpu_linear(fmt, x, w, bias=None, ldo=None):
+    M, K = x.shape
+    N = w.shape[0]
+    xd, wd = x.cuda(), w.cuda()
+    wc, ws, wg = nvq.quantize_weight(fmt, wd)
+    if fmt == "nvfp4":
+        ac, as_, ag = nvq.nvfp4_quantize(xd)
+    else:
+        ac, as_ = nvq.mxfp8_quantize(xd)
+        ag = None
+    out = None
+    if ldo is not None:
+        out = torch.full((M, ldo), 7.0, dtype=torch.bfloat16, device="cuda")[:, :N]
+    bd = bias.cuda() if bias is not None else None
+    D = nvq.block_scaled_linear(fmt, ac, as_, ag, wc, ws, wg, M, N, K, bias=bd, out=out)
+    assert nvq.device_status() == 0
+    return D
+
+
+def oracle_linear(fmt, x, w, rows=None, bias=None):
+    M, K = x.shape
+    N = w.shape[0]
+    if fmt == "nvfp4":
+        ac, as_, ag = oracle.nvfp4_quantize(bits(x))
+        wc, ws, wg = oracle.nvfp4_quantize(bits(w))
+        A = oracle.nvfp4_dequantize(ac, as_, ag, M, K)
+        B = oracle.nvfp4_dequantize(wc, ws, wg, N, K)
+    else:
+        ac, as_ = oracle.mxfp8_quantize(bits(x))
+        wc, ws = oracle.mxfp8_quantize(bits(w))
+        A = oracle.mxfp8_dequantize(ac, as_, M, K)
+        B = oracle.mxfp8_dequantize(wc, ws, N, K)
+    return oracle.gemm_rows(A, B, rows, bias_bits=None if bias is None else bits(bias.reshape(1, -1)))
+
+
+SMALL = [
+    # fmt, M, N, K  (N % 256 != 0 takes the 128-wide tile)
+    ("nvfp4", 128, 128, 256),
+    ("nvfp4", 256, 384, 512),
+    ("nvfp4", 384, 512, 768),
+    ("mxfp8", 128, 128, 128),
+    ("mxfp8", 256, 384, 384),
+    ("mxfp8", 384, 512, 640),
+]
+
+
+def test_tiny_workload_full_output():
+    x, w = act("tiny"), workloads.weight("tiny")
+    D = gpu_linear("nvfp4", x, w).float().cpu().numpy()
+    Y = oracle_linear("nvfp4", x, w)
+    check_gemm(D, Y)
+
+
+@pytest.mark.parametrize("fmt,M,N,K", SMALL)
+def test_small_shapes_full_output(fmt, M, N, K):
+    x = workloads.normal(M, K, seed=40 + M)
+    w = workloads.normal(N, K, seed=41 + N, std=0.05)
+    D = gpu_linear(fmt, x, w).float().cpu().numpy()
+    check_gemm(D, oracle_linear(fmt, x, w))
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp8"])
+def test_bias_and_output_pitch(fmt):
+    M, N, K = 256, 512, 512
+    x = workloads.normal(M, K, seed=50)
+    w = workloads.normal(N, K, seed=51, std=0.05)
+    b = workloads.bias(N)
+    D = gpu_linear(fmt, x, w, bias=b, ldo=N + 64)
+    full = D.as_strided((M, N + 64), (N + 64, 1))
+    assert (full[:, N:] == 7.0).all(), "padding columns of the output were written"
+    check_gemm(D.float().cpu().numpy(), oracle_linear(fmt, x, w, bias=b))
+
+
+def test_zero_activation_gives_zero_output():
+    x = torch.zeros(128, 256, dtype=torch.bfloat16)
+    w = workloads.weight("tiny")
+    D = gpu_linear("nvfp4", x, w)
+    assert (D == 0).all()
+
+
+def test_gemm_deterministic():
+    x, w = act("tiny"), workloads.weight("tiny")
+    a = gpu_linear("nvfp4", x, w)
+    b = gpu_linear("nvfp4", x, w)
+    assert torch.equal(a, b)
+
+
+FULL = [
+    ("ffup", "nvfp4", 1),
+    ("ffdown", "mxfp8", 1),
+    ("qkv4", "nvfp4", 8),
+]
+
+
+@pytest.mark.parametrize("name,fmt,every", FULL, ids=[f[0] for f in FULL])
+def test_full_size_workloads_sampled_rows(name, fmt, every):
+    x, w = act(name), wgt(name)
+    rows = sample_rows(x.shape[0], per_tile_every=every)
+    D = gpu_linear(fmt, x, w)
+    Dr = D[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    Y = oracle_linear(fmt, x, w, rows=rows)
+    check_gemm(Dr, Y)

@@ -1,0 +1,205 @@
+"""GPU parity of the quantize kernels against the CPU oracle: bit-exact codes,
+block scales and global scale, on every workload's tensors, on ragged and
+pitched shapes, and on the special cases."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_common import act, bits, sf_matrix, wgt
+
+pytestmark = pytest.mark.gpu
+
+nvq = pytest.importorskip("microscaling_quantized_linear_b200")
+
+
+def cuda(t):
+    return t.to("cuda")
+
+
+def run_nvfp4(x_cpu, ld=None, calib=None):
+    M, K = x_cpu.shape
+    if ld is not None and ld != K:
+        buf = torch.zeros(M, ld, dtype=torch.bfloat16)
+        buf[:, :K] = x_cpu
+        xd = cuda(buf)[:, :K]
+    else:
+        xd = cuda(x_cpu)
+    ca = None if calib is None else torch.tensor([calib], dtype=torch.float32, device="cuda")
+    codes, sf, g = nvq.nvfp4_quantize(xd, calib_amax=ca)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), sf.cpu().numpy(), np.float32(g.cpu().item())
+
+
+def run_mxfp8(x_cpu):
+    codes, sf = nvq.mxfp8_quantize(cuda(x_cpu))
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), sf.cpu().numpy()
+
+
+def assert_nvfp4_equal(got, want, M, K):
+    gc, gs, gg = got
+    wc, ws, wg = want
+    if not np.array_equal(gc, wc):
+        bad = np.argwhere(gc != wc)
+        r, b = bad[0]
+        raise AssertionError("%d code bytes differ; first at row %d byte %d: gpu %02x oracle %02x"
+                             % (len(bad), r, b, gc[r, b], wc[r, b]))
+    assert np.array_equal(gs, ws), "%d scale bytes differ" % int((gs != ws).sum())
+    assert np.float32(gg).tobytes() == np.float32(wg).tobytes(), (gg, wg)
+
+
+# ------------------------------------------------------------------ conversion probe
+
+def probe_inputs():
+    vals = []
+    e4 = [oracle.e4m3_value(c) for c in range(0x7F)]
+    e2 = [oracle.e2m1_value(c) for c in range(8)]
+    for table in (e4, e2):
+        for lo, hi in zip(table[:-1], table[1:]):
+            mid = np.float32((lo + hi) / 2)
+            vals += [mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(1e30)),
+                     np.float32(lo), np.float32(hi)]
+    vals += [0.0, 6.0, 6.5, 7.0, 8.0, 448.0, 464.0, 465.0, 480.0, 1e6, 3e38, 1e-30, 1e-45, 2 ** -10,
+             2 ** -9 * 0.5, 2 ** -9 * 0.5001]
+    rng = np.random.default_rng(0)
+    vals += list((np.float32(2.0) ** rng.uniform(-16, 10, 200000)).astype(np.float32))
+    v = np.array(vals, dtype=np.float32)
+    return np.concatenate([v, -v])
+
+
+def test_device_conversions_match_oracle_encoders():
+    v = probe_inputs()
+    e2, e4 = nvq.probe_convert(torch.from_numpy(v).cuda())
+    e2 = e2.cpu().numpy()
+    e4 = e4.cpu().numpy()
+    want2 = np.array([oracle.e2m1_encode(x) for x in v])
+    want4 = np.array([oracle.e4m3_encode(x) for x in v])
+    bad2 = np.flatnonzero(e2 != want2)
+    bad4 = np.flatnonzero(e4 != want4)
+    assert bad2.size == 0, "E2M1 differs at %r: gpu %r oracle %r" % (v[bad2[:5]], e2[bad2[:5]], want2[bad2[:5]])
+    assert bad4.size == 0, "E4M3 differs at %r: gpu %r oracle %r" % (v[bad4[:5]], e4[bad4[:5]], want4[bad4[:5]])
+
+
+# ------------------------------------------------------------------ NVFP4
+
+NVFP4_CASES = [
+    ("tiny_act", lambda: act("tiny")),
+    ("tiny_w", lambda: workloads.weight("tiny")),
+    ("ragged_384x320", lambda: workloads.normal(384, 320, seed=21)),      # 20 blocks per row, 3 row tiles
+    ("actq_4608x3072", lambda: act("actq")),
+    ("ffup_act", lambda: act("ffup")),
+    ("ffup_w_12288x3072", lambda: wgt("ffup")),
+    ("qkv4_act_18432x3072", lambda: act("qkv4")),
+]
+
+
+@pytest.mark.parametrize("name,make", NVFP4_CASES, ids=[c[0] for c in NVFP4_CASES])
+def test_nvfp4_quantize_bit_exact(name, make):
+    x = make()
+    M, K = x.shape
+    assert_nvfp4_equal(run_nvfp4(x), oracle.nvfp4_quantize(bits(x)), M, K)
+
+
+def test_nvfp4_quantize_pitched_input():
+    x = workloads.normal(256, 448, seed=22)
+    assert_nvfp4_equal(run_nvfp4(x, ld=520), oracle.nvfp4_quantize(bits(x)), 256, 448)
+
+
+def test_nvfp4_calibrated_amax():
+    x = act("tiny")
+    a = oracle.amax(bits(x))
+    for calib in (a, a / 3, a * 5):
+        assert_nvfp4_equal(run_nvfp4(x, calib=calib), oracle.nvfp4_quantize(bits(x), calib_amax=calib), 128, 256)
+
+
+def test_nvfp4_special_tensors():
+    cases = {
+        "zero": torch.zeros(128, 128, dtype=torch.bfloat16),
+        "below_floor": torch.full((128, 64), 2.0 ** -110).to(torch.bfloat16),
+        "subnormal_bf16": torch.full((128, 64), 2.0 ** -130).to(torch.bfloat16),
+        "neg_zero": torch.full((128, 64), -0.0).to(torch.bfloat16),
+        "one_hot": torch.zeros(128, 64).index_put_((torch.tensor([77]), torch.tensor([5])),
+                                                   torch.tensor([3.0e38])).to(torch.bfloat16),
+    }
+    x = workloads.normal(128, 128, seed=23)
+    x[3, 16:32] = 0
+    x[9, 32:48] = 1e-6        # scale underflows E4M3 -> zero codes
+    x[10, 0:16] = -x[10, 0:16].abs()
+    cases["mixed_blocks"] = x
+    for name, t in cases.items():
+        M, K = t.shape
+        assert_nvfp4_equal(run_nvfp4(t), oracle.nvfp4_quantize(bits(t)), M, K)
+
+
+def test_nvfp4_deterministic_and_no_overwrite():
+    x = act("ffup")
+    M, K = x.shape
+    xd = x.cuda()
+    guard = 4096
+    codes = torch.full((M * K // 2 + 2 * guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    sfb = nvq.scale_bytes("nvfp4", M, K)
+    sf = torch.full((sfb + 2 * guard,), 0x5A, dtype=torch.uint8, device="cuda")
+    g = torch.zeros(4, dtype=torch.float32, device="cuda")
+    c_view = codes[guard:guard + M * K // 2].view(M, K // 2)
+    s_view = sf[guard:guard + sfb]
+    nvq.nvfp4_quantize(xd, c_view, s_view, g[1:2])
+    first = (c_view.clone(), s_view.clone(), g.clone())
+    nvq.nvfp4_quantize(xd, c_view, s_view, g[1:2])
+    torch.cuda.synchronize()
+    assert torch.equal(first[0], c_view) and torch.equal(first[1], s_view) and torch.equal(first[2], g)
+    assert (codes[:guard] == 0xA5).all() and (codes[-guard:] == 0xA5).all()
+    assert (sf[:guard] == 0x5A).all() and (sf[-guard:] == 0x5A).all()
+    assert g[0].item() == 0 and g[2].item() == 0
+    assert nvq.device_status() == 0
+
+
+def test_nvfp4_nonfinite_input_sets_status():
+    nvq.device_status()
+    x = workloads.normal(128, 64, seed=3)
+    x[7, 7] = float("inf")
+    run_nvfp4(x)
+    assert nvq.device_status() & nvq.NVQ_STATUS_NONFINITE
+    assert nvq.device_status() == 0
+
+
+def test_empty_batch_launches_nothing():
+    x = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    codes, sf, g = nvq.nvfp4_quantize(x)
+    c8, s8 = nvq.mxfp8_quantize(x)
+    assert codes.numel() == 0 and c8.numel() == 0
+
+
+# ------------------------------------------------------------------ MXFP8
+
+MXFP8_CASES = [
+    ("tiny_act", lambda: act("tiny")),
+    ("ragged_256x384", lambda: workloads.normal(256, 384, seed=31)),
+    ("ffdown_act_4608x12288", lambda: act("ffdown")),
+    ("ffdown_w_3072x12288", lambda: wgt("ffdown")),
+    ("qkv4_act", lambda: act("qkv4")),
+]
+
+
+@pytest.mark.parametrize("name,make", MXFP8_CASES, ids=[c[0] for c in MXFP8_CASES])
+def test_mxfp8_quantize_bit_exact(name, make):
+    x = make()
+    gc, gs = run_mxfp8(x)
+    wc, ws = oracle.mxfp8_quantize(bits(x))
+    assert np.array_equal(gc, wc), "%d code bytes differ" % int((gc != wc).sum())
+    assert np.array_equal(gs, ws), "%d scale bytes differ" % int((gs != ws).sum())
+
+
+def test_mxfp8_special_tensors():
+    x = workloads.normal(128, 256, seed=33)
+    x[0, 0:32] = 0
+    x[1, 32:64] = 2.0 ** -130            # BF16 subnormals: X clamps to -127
+    x[2, 64:96] = 1.8984375              # floor-rule saturation
+    x[3, 96:128] = 3.0e38                # largest exponents
+    x[4, :] = -0.0
+    gc, gs = run_mxfp8(x)
+    wc, ws = oracle.mxfp8_quantize(bits(x))
+    assert np.array_equal(gc, wc) and np.array_equal(gs, ws)
+    S = sf_matrix(gs, 128, 8)
+    assert S[0, 0] == 0 and S[2, 2] == 119
