@@ -9,7 +9,7 @@
 // of either operand ever exists (page "NVIDIA Blackwell平台FP4量化技术解析与图像
 // 生成优化", section 3.1: FP4 decoded to BF16 inside the SM).
 //
-// Structure: one persistent CTA per SM, 6 warps.
+// Structure: one persistent CTA per SM, 6 warps, output tiles 128 x BN.
 //   warp 0  TMA producer: per pipeline stage one 128 x 128-byte tile of A,
 //           one BN x 128-byte tile of B (tensor maps, 128-byte swizzle), and
 //           the matching 512-byte scale tiles (plain bulk copies: the global
@@ -17,8 +17,11 @@
 //   warp 1  allocates tensor memory; one lane moves each stage's scale tiles
 //           to tensor memory (tcgen05.cp) and issues the MMAs into an FP32
 //           accumulator in tensor memory; tcgen05.commit frees the stage.
+//           With two accumulators (BN = 128 or 192) the MMAs of tile i+1 run
+//           while the epilogue drains tile i.
 //   warps 2-5  epilogue: tensor memory -> registers (tcgen05.ld), scale by
-//           alpha, add bias, round to BF16, store.
+//           alpha, add bias, round to BF16, stage 32 x 32 sub-tiles in
+//           64-byte-swizzled shared memory and write them with TMA stores.
 // Every mbarrier wait is bounded in wall time; a wait that gives up sets the
 // status word and an abort flag that releases the other roles.
 #pragma once
@@ -41,27 +44,35 @@ struct GemmCfg {
     static constexpr int MMA_K_BYTES = KBYTES / KSTEPS;      // 32
     static constexpr int SF_BLOCK = FMT == 0 ? 16 : 32;
     static constexpr int SF_ATOMS = BK / SF_BLOCK / 4;       // 128x4 scale tiles per 128 rows per stage
+    static constexpr int SFB_H = BN == 128 ? 1 : 2;          // 128-row scale tiles spanned by a B tile
     static constexpr int A_BYTES = BM * KBYTES;
     static constexpr int B_BYTES = BN * KBYTES;
     static constexpr int SFA_BYTES = SF_ATOMS * 512;
-    static constexpr int SFB_BYTES = (BN / 128) * SF_ATOMS * 512;
+    static constexpr int SFB_BYTES = SFB_H * SF_ATOMS * 512;
     static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr int STAGE_BYTES = (TX_BYTES + 1023) / 1024 * 1024;
-    static constexpr int STAGES = 4;
     static constexpr int OFF_B = A_BYTES;
     static constexpr int OFF_SFA = A_BYTES + B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
-    // tensor-memory columns: accumulator, then scale factors of A and B
-    static constexpr int TM_ACC = 0;
-    static constexpr int TM_SFA = BN;
+    // epilogue staging: 4 warps x 2 buffers x (32 rows x 64 bytes)
+    static constexpr int EPI_BUF_BYTES = 32 * 64;
+    static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
+    static constexpr int SMEM_LIMIT = 232448;
+    static constexpr int FIXED_BYTES = 1024 /*align*/ + 256 /*barriers*/ + EPI_BYTES;
+    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+    static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
+    // tensor-memory columns: accumulator(s), then scale factors of A and B
     static constexpr int SFA_COLS = FMT == 0 ? 4 * KSTEPS : 4;
-    static constexpr int TM_SFB = TM_SFA + SFA_COLS;
-    static constexpr int SFB_COLS_PER_MMA = 4 * (BN / 128);
+    static constexpr int SFB_COLS_PER_MMA = 4 * SFB_H;
     static constexpr int SFB_COLS = FMT == 0 ? SFB_COLS_PER_MMA * KSTEPS : SFB_COLS_PER_MMA;
+    static constexpr int ACC_BUFS = (2 * BN + SFA_COLS + SFB_COLS <= 512) ? 2 : 1;
+    static constexpr int TM_SFA = ACC_BUFS * BN;
+    static constexpr int TM_SFB = TM_SFA + SFA_COLS;
     static constexpr int TM_USED = TM_SFB + SFB_COLS;
     static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
     static constexpr int THREADS = 192;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
     // instruction descriptor: A/B format (E2M1 = 1 for mxf4nvf4, E4M3 = 0 for
     // mxf8f6f4) in bits 7-9 / 10-12, K-major A and B, N >> 3 in bits 17-22,
     // scale format (0 = UE4M3, 1 = UE8M0) in bit 23, M >> 4 in bits 24-28.
@@ -70,8 +81,10 @@ struct GemmCfg {
         ((uint32_t)(BN >> 3) << 17) |
         (FMT == 0 ? 0u : (1u << 23)) |
         ((uint32_t)(BM >> 4) << 24);
+    static_assert(BN == 128 || BN == 192 || BN == 256, "tile width");
     static_assert(TM_USED <= 512, "tensor memory overflow");
-    static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
+    static_assert(STAGES >= 2, "shared memory too small for two stages");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory overflow");
 };
 
 struct GemmParams {
@@ -80,9 +93,7 @@ struct GemmParams {
     const float* a_global;
     const float* b_global;
     const __nv_bfloat16* bias;
-    __nv_bfloat16* out;
     unsigned int* status;
-    uint32_t ldo;
     uint32_t num_m_blocks, num_n_blocks, num_k_tiles;
     uint32_t sf_ctiles;          // (K / SF_BLOCK) / 4: scale tiles per 128 rows
 };
@@ -90,17 +101,17 @@ struct GemmParams {
 template <int FMT, int BN>
 __global__ void __launch_bounds__(192, 1)
 bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-              const GemmParams p) {
+              const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
     using C = GemmCfg<FMT, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
     const uint32_t full0 = smem_u32(bars);
     const uint32_t empty0 = full0 + 8 * C::STAGES;
-    const uint32_t tfull = empty0 + 8 * C::STAGES;
-    const uint32_t tempty = tfull + 8;
-    const uint32_t drain = tempty + 8;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 3);
+    const uint32_t tfull0 = empty0 + 8 * C::STAGES;     // [ACC_BUFS]
+    const uint32_t tempty0 = tfull0 + 8 * 2;            // [ACC_BUFS]
+    const uint32_t drain = tempty0 + 8 * 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* never = abort_flag + 1;
 
@@ -110,8 +121,10 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
         }
-        mbar_init(tfull, 1);
-        mbar_init(tempty, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull0 + 8 * b, 1);
+            mbar_init(tempty0 + 8 * b, 4);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         *never = 0;
@@ -120,6 +133,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmap_a);
         prefetch_tensormap(&tmap_b);
+        prefetch_tensormap(&tmap_d);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), C::TM_COLS);
@@ -138,6 +152,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             bool ok = true;
             for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+                const uint32_t a0 = (nb * BN) / 128;             // first 128-row scale tile of B
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt) {
                     const uint32_t s = it % C::STAGES, use = it / C::STAGES;
                     if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
@@ -153,9 +168,9 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                               p.sfa + ((size_t)mb * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
                               C::SFA_BYTES, fb);
 #pragma unroll
-                    for (int h = 0; h < BN / 128; ++h)
+                    for (int h = 0; h < C::SFB_H; ++h)
                         bulk_load(st + C::OFF_SFB + h * C::SF_ATOMS * 512,
-                                  p.sfb + ((size_t)(nb * (BN / 128) + h) * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
+                                  p.sfb + ((size_t)(a0 + h) * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
                                   C::SF_ATOMS * 512, fb);
                     ++it;
                 }
@@ -174,14 +189,19 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             uint32_t it = 0, t_local = 0;
             bool ok = true;
             for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t_local) {
-                if (t_local > 0 && !mbar_wait_bounded(tempty, (t_local - 1) & 1, abort_flag, kWaitLimitNs)) {
+                const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
+                const uint32_t use = C::ACC_BUFS == 2 ? (t_local >> 1) : t_local;
+                if (use > 0 && !mbar_wait_bounded(tempty0 + 8 * buf, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t nb = tile / p.num_m_blocks;
+                const uint32_t sfb_shift = ((nb * BN) % 128) / 32;   // B tile starting mid scale tile (BN = 192)
+                const uint32_t d_tmem = tmem + buf * BN;
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt, ++it) {
-                    const uint32_t s = it % C::STAGES, use = it / C::STAGES;
-                    if (!mbar_wait_bounded(full0 + 8 * s, use & 1, abort_flag, kWaitLimitNs)) {
+                    const uint32_t s = it % C::STAGES, su = it / C::STAGES;
+                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
@@ -193,7 +213,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                         tc_cp_32x128b_warpx4(tmem + C::TM_SFA + 4 * a,
                                              smem_desc(st + C::OFF_SFA + 512 * a, 16, 128, 0));
 #pragma unroll
-                    for (int h = 0; h < BN / 128; ++h)
+                    for (int h = 0; h < C::SFB_H; ++h)
 #pragma unroll
                         for (int a = 0; a < C::SF_ATOMS; ++a)
                             tc_cp_32x128b_warpx4(tmem + C::TM_SFB + C::SFB_COLS_PER_MMA * a + 4 * h,
@@ -204,20 +224,20 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                         const uint64_t bdesc = smem_desc(st + C::OFF_B + k * C::MMA_K_BYTES, 16, 1024, 2);
                         const uint32_t acc = (kt | (uint32_t)k) != 0;
                         if (FMT == 0) {
-                            tc_mma_nvf4(tmem + C::TM_ACC, adesc, bdesc, C::IDESC,
+                            tc_mma_nvf4(d_tmem, adesc, bdesc, C::IDESC,
                                         tmem + C::TM_SFA + 4 * k,
-                                        tmem + C::TM_SFB + C::SFB_COLS_PER_MMA * k, acc);
+                                        tmem + C::TM_SFB + C::SFB_COLS_PER_MMA * k + sfb_shift, acc);
                         } else {
                             const uint32_t id = C::IDESC | ((uint32_t)k << 29) | ((uint32_t)k << 4);
-                            tc_mma_mxf8(tmem + C::TM_ACC, adesc, bdesc, id,
+                            tc_mma_mxf8(d_tmem, adesc, bdesc, id,
                                         (tmem + C::TM_SFA) | ((uint32_t)k << 30),
-                                        (tmem + C::TM_SFB) | ((uint32_t)k << 30), acc);
+                                        (tmem + C::TM_SFB + sfb_shift) | ((uint32_t)k << 30), acc);
                         }
                     }
                     tc_commit(empty0 + 8 * s);
                 }
                 if (!ok) break;
-                tc_commit(tfull);
+                tc_commit(tfull0 + 8 * buf);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -230,23 +250,32 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         // ---------------------------------------------------------- epilogue
         const int q = warp & 3;                       // tensor-memory lane quarter of this warp
         const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
-        uint32_t t_local = 0;
+        uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * 2 * C::EPI_BUF_BYTES;
+        const uint32_t swz = (uint32_t)((lane >> 1) & 3);     // 64-byte swizzle of this thread's row
+        uint32_t t_local = 0, nstore = 0;
         for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t_local) {
             const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
-            if (!mbar_wait_bounded(tfull, t_local & 1, abort_flag, kWaitLimitNs)) {
+            const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
+            const uint32_t use = C::ACC_BUFS == 2 ? (t_local >> 1) : t_local;
+            if (!mbar_wait_bounded(tfull0 + 8 * buf, use & 1, abort_flag, kWaitLimitNs)) {
                 *abort_flag = 1;
                 atomicOr(p.status, 1u);
                 break;
             }
             tc_fence_after();
-            const uint32_t row = mb * C::BM + 32 * q + lane;
-            __nv_bfloat16* orow = p.out + (size_t)row * p.ldo + (size_t)nb * BN;
-            const __nv_bfloat16* brow = p.bias ? p.bias + (size_t)nb * BN : nullptr;
+            const int32_t row0 = (int32_t)(mb * C::BM + 32 * q);
+            const uint32_t n0 = nb * BN;
+            const __nv_bfloat16* brow = p.bias ? p.bias + n0 : nullptr;
 #pragma unroll 1
             for (int c = 0; c < BN; c += 32) {
                 uint32_t r[32];
-                tc_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + C::TM_ACC + c, r);
+                tc_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + buf * BN + c, r);
                 tc_wait_ld();
+                if (c + 32 == BN) {                   // accumulator fully read: hand it back to the MMA warp
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
+                }
                 uint32_t packed[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
@@ -260,15 +289,24 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     const __nv_bfloat162 o = __floats2bfloat162_rn(v0, v1);
                     packed[j] = *reinterpret_cast<const uint32_t*>(&o);
                 }
-                uint4* dst = reinterpret_cast<uint4*>(orow + c);
+                uint8_t* sb = staging + (nstore & 1) * C::EPI_BUF_BYTES;
+                if (lane == 0) bulk_wait_group_read<1>();   // the store that last used this buffer has read it
+                __syncwarp();
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                    *reinterpret_cast<uint4*>(sb + lane * 64 + 16 * ((uint32_t)j ^ swz)) =
+                        make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmap_d, smem_u32(sb), (int32_t)(n0 + c), row0);
+                    bulk_commit_group();
+                }
+                ++nstore;
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty);
         }
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
 
     tc_fence_before();

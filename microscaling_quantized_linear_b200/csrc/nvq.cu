@@ -30,7 +30,7 @@ struct DeviceInfo {
     bool arch_ok = false;
     int num_sms = 0;
     unsigned int* status = nullptr;
-    bool gemm_attr[2][2] = {{false, false}, {false, false}};
+    bool gemm_attr[2][3] = {{false, false, false}, {false, false, false}};
 };
 
 std::mutex g_mu;
@@ -167,24 +167,37 @@ int encode_codes_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t 
     return r == CUDA_SUCCESS ? NVQ_OK : NVQ_ERR_CUDA;
 }
 
+int encode_out_map(CUtensorMap* map, const void* out, int64_t rows, int64_t cols, int64_t ldo) {
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)ldo * 2};
+    const cuuint32_t box[2] = {32u, 32u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(out), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVQ_OK : NVQ_ERR_CUDA;
+}
+
 template <int FMT, int BN>
 int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                 const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
                 void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
     using C = GemmCfg<FMT, BN>;
     const int64_t kbytes = FMT == 0 ? K / 2 : K;
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, md;
     int rc;
     if ((rc = encode_codes_map(&ma, a_codes, M, kbytes, C::BM))) return rc;
     if ((rc = encode_codes_map(&mb, b_codes, N, kbytes, BN))) return rc;
+    if ((rc = encode_out_map(&md, out, M, N, ldo))) return rc;
     auto kern = bsgemm_kernel<FMT, BN>;
+    const int wi = BN / 64 - 2;                      // 128 -> 0, 192 -> 1, 256 -> 2
     {
         std::lock_guard<std::mutex> lock(g_mu);
-        if (!d->gemm_attr[FMT][BN == 256]) {
+        if (!d->gemm_attr[FMT][wi]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
                 cudaSuccess)
                 return NVQ_ERR_CUDA;
-            d->gemm_attr[FMT][BN == 256] = true;
+            d->gemm_attr[FMT][wi] = true;
         }
     }
     GemmParams p;
@@ -193,16 +206,14 @@ int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, 
     p.a_global = a_global;
     p.b_global = b_global;
     p.bias = static_cast<const __nv_bfloat16*>(bias);
-    p.out = static_cast<__nv_bfloat16*>(out);
     p.status = d->status;
-    p.ldo = (uint32_t)ldo;
     p.num_m_blocks = (uint32_t)(M / C::BM);
     p.num_n_blocks = (uint32_t)(N / BN);
     p.num_k_tiles = (uint32_t)(K / C::BK);
     p.sf_ctiles = (uint32_t)(K / C::SF_BLOCK / 4);
     const uint32_t tiles = p.num_m_blocks * p.num_n_blocks;
     const uint32_t grid = tiles < (uint32_t)d->num_sms ? tiles : (uint32_t)d->num_sms;
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, p);
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, md, p);
     return launch_status();
 }
 
@@ -267,16 +278,27 @@ int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_sca
     if (rc) return rc;
     if ((rc = get_encoder())) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const bool wide = (N % 256) == 0;
-    if (format == NVQ_NVFP4)
-        return wide ? launch_gemm<0, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out,
-                                          ldo, M, N, K, s)
-                    : launch_gemm<0, 128>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out,
-                                          ldo, M, N, K, s);
-    return wide ? launch_gemm<1, 256>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M,
-                                      N, K, s)
-                : launch_gemm<1, 128>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M,
-                                      N, K, s);
+    // Tile width: 192 (two tensor-memory accumulators, epilogue overlapped)
+    // when N allows it, else 256 (one accumulator), else 128 (two).
+    const int bn = (N % 384 == 0) ? 192 : (N % 256 == 0) ? 256 : 128;
+    if (format == NVQ_NVFP4) {
+        if (bn == 192)
+            return launch_gemm<0, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
+                                       M, N, K, s);
+        if (bn == 256)
+            return launch_gemm<0, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
+                                       M, N, K, s);
+        return launch_gemm<0, 128>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M,
+                                   N, K, s);
+    }
+    if (bn == 192)
+        return launch_gemm<1, 192>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M, N,
+                                   K, s);
+    if (bn == 256)
+        return launch_gemm<1, 256>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M, N,
+                                   K, s);
+    return launch_gemm<1, 128>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M, N, K,
+                               s);
 }
 
 int nvq_device_status(nvq_stream_t stream) {

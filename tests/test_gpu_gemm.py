@@ -56,6 +56,7 @@ SMALL = [
     ("nvfp4", 128, 128, 256),
     ("nvfp4", 256, 384, 512),
     ("nvfp4", 384, 512, 768),
+    ("nvfp4", 1024, 768, 512),
     ("mxfp8", 128, 128, 128),
     ("mxfp8", 256, 384, 384),
     ("mxfp8", 384, 512, 640),
@@ -87,6 +88,28 @@ def test_bias_and_output_pitch(fmt):
     full = D.as_strided((M, N + 64), (N + 64, 1))
     assert (full[:, N:] == 7.0).all(), "padding columns of the output were written"
     check_gemm(D.float().cpu().numpy(), oracle_linear(fmt, x, w, bias=b))
+
+
+MANY_TILES = [
+    # several output tiles per persistent CTA: both tensor-memory accumulators,
+    # barrier phase wrap-around, and (BN = 192) tiles that start mid scale tile
+    ("nvfp4", 128 * 48, 384 * 4, 256),     # BN 192, 384 tiles
+    ("nvfp4", 128 * 40, 256 * 3, 512),     # BN 256 (one accumulator), 240 tiles
+    ("mxfp8", 128 * 40, 640, 256),         # BN 128, 200 tiles
+    ("mxfp8", 128 * 36, 384 * 3, 384),     # BN 192, 216 tiles
+]
+
+
+@pytest.mark.parametrize("fmt,M,N,K", MANY_TILES)
+def test_many_tiles_per_cta(fmt, M, N, K):
+    x = workloads.normal(M, K, seed=60 + M % 97)
+    w = workloads.normal(N, K, seed=61 + N % 89, std=0.05)
+    rows = sample_rows(M)
+    D = gpu_linear(fmt, x, w)
+    Dr = D[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    check_gemm(Dr, oracle_linear(fmt, x, w, rows=rows))
+    # every column tile of every sampled row was written (no stale tile)
+    assert torch.isfinite(D).all()
 
 
 def test_zero_activation_gives_zero_output():
