@@ -7,11 +7,15 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <unistd.h>
+
+#include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
-#include "../../include/nvq.h"
+#include "nvq.h"
 #include "gemm.cuh"
 #include "quantize.cuh"
 
@@ -31,6 +35,7 @@ struct DeviceInfo {
     int num_sms = 0;
     unsigned int* status = nullptr;
     bool gemm_attr[2][3] = {{false, false, false}, {false, false, false}};
+    bool fused_attr = false;
 };
 
 std::mutex g_mu;
@@ -98,9 +103,9 @@ int launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, uint32_t* pa
                 cudaStream_t stream, uint32_t* npartial_out) {
     const uint32_t vecs_per_row = (uint32_t)(K / 8), pitch_vecs = (uint32_t)(ld / 8);
     const uint64_t total = (uint64_t)rows * vecs_per_row;
-    uint64_t want = (total + 4 * kAmaxThreads - 1) / (4 * kAmaxThreads);
+    uint64_t want = (total + 8 * kAmaxThreads - 1) / (8 * kAmaxThreads);
     uint32_t grid = (uint32_t)(want < 1 ? 1 : want);
-    const uint32_t cap = (uint32_t)num_sms * 4 < (uint32_t)kMaxAmaxPartials ? (uint32_t)num_sms * 4 : kMaxAmaxPartials;
+    const uint32_t cap = (uint32_t)num_sms * 8 < (uint32_t)kMaxAmaxPartials ? (uint32_t)num_sms * 8 : kMaxAmaxPartials;
     if (grid > cap) grid = cap;
     amax_partials_kernel<<<grid, kAmaxThreads, 0, stream>>>(static_cast<const uint4*>(x), (uint32_t)rows,
                                                             vecs_per_row, pitch_vecs, partial);
@@ -115,6 +120,23 @@ uint32_t quant_grid(uint64_t units, int num_sms) {
     return (uint32_t)(blocks < 1 ? 1 : blocks);
 }
 
+// Epoch tags of the one-pass quantizer's workspace slots: process-wide,
+// monotonic, started at a per-process random value so that slots left in
+// reused memory by another process cannot match.
+std::atomic<uint32_t> g_epoch{0};
+std::once_flag g_epoch_once;
+
+uint32_t next_epoch() {
+    std::call_once(g_epoch_once, [] {
+        const uint64_t t = (uint64_t)std::chrono::steady_clock::now().time_since_epoch().count();
+        g_epoch.store((uint32_t)(t ^ (t >> 32) ^ ((uint64_t)getpid() << 16)));
+    });
+    uint32_t e = g_epoch.fetch_add(1) + 1;
+    return e;
+}
+
+constexpr size_t kFusedSmemMax = 220 * 1024;
+
 int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
                         float* global_scale, const float* calib_amax, void* workspace, cudaStream_t stream) {
     int rc = check_quant_shape(NVQ_NVFP4, M, K, ldx);
@@ -127,12 +149,42 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     if (calib_amax && (reinterpret_cast<uintptr_t>(calib_amax) & 3u)) return NVQ_ERR_ALIGN;
     DeviceInfo* d = nullptr;
     if ((rc = device_info(&d))) return rc;
+    const uint32_t nblk = (uint32_t)(K / 16);
+    if (!calib_amax) {
+        // One pass when every CTA's rows fit in shared memory (one CTA per SM).
+        const int64_t rows_per_cta = (M + d->num_sms - 1) / d->num_sms;
+        const size_t smem = (size_t)rows_per_cta * (size_t)K * 2 + 128;
+        if (smem <= kFusedSmemMax) {
+            {
+                std::lock_guard<std::mutex> lock(g_mu);
+                if (!d->fused_attr) {
+                    if (cudaFuncSetAttribute(nvfp4_quantize_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kFusedSmemMax + 128) != cudaSuccess)
+                        return NVQ_ERR_CUDA;
+                    d->fused_attr = true;
+                }
+            }
+            const uint32_t grid = (uint32_t)((M + rows_per_cta - 1) / rows_per_cta);
+            const uint16_t* xp = static_cast<const uint16_t*>(x);
+            uint32_t rows32 = (uint32_t)M, k32 = (uint32_t)K, ld32 = (uint32_t)ldx, rpc = (uint32_t)rows_per_cta;
+            unsigned long long* slots = reinterpret_cast<unsigned long long*>(
+                static_cast<uint8_t*>(workspace) + kWorkspaceSlotsOffset);
+            uint32_t epoch = next_epoch();
+            unsigned int* status = d->status;
+            void* args[] = {&xp, &rows32, &k32, &ld32, &rpc, &codes, &scales, &global_scale, &slots, &epoch, &status};
+            if (cudaLaunchCooperativeKernel((const void*)nvfp4_quantize_fused_kernel, dim3(grid),
+                                            dim3(kFusedThreads), args, smem, stream) != cudaSuccess) {
+                cudaGetLastError();
+                return NVQ_ERR_CUDA;
+            }
+            return NVQ_OK;
+        }
+    }
     uint32_t npartial = 0;
-    uint32_t* partial = static_cast<uint32_t*>(workspace);
+    uint32_t* partial = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + kWorkspacePartialsOffset);
     if (!calib_amax) {
         if ((rc = launch_amax(x, M, K, ldx, partial, d->num_sms, stream, &npartial))) return rc;
     }
-    const uint32_t nblk = (uint32_t)(K / 16);
     const uint64_t units = (uint64_t)M * nblk;
     nvfp4_quantize_kernel<<<quant_grid(units, d->num_sms), kQuantThreads, 0, stream>>>(
         static_cast<const uint16_t*>(x), (uint32_t)M, nblk, (uint32_t)ldx, codes, scales, global_scale,
@@ -235,7 +287,7 @@ size_t nvq_scale_bytes(int format, int64_t rows, int64_t K) {
     return (size_t)(((rows + 127) / 128) * 128 * ((cols + 3) / 4) * 4);
 }
 
-size_t nvq_workspace_bytes(void) { return (size_t)kMaxAmaxPartials * sizeof(uint32_t); }
+size_t nvq_workspace_bytes(void) { return kWorkspaceBytes; }
 
 int nvfp4_quantize(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
                    float* global_scale, const float* calib_amax, void* workspace, nvq_stream_t stream) {

@@ -155,6 +155,22 @@ def test_nvfp4_deterministic_and_no_overwrite():
     assert nvq.device_status() == 0
 
 
+def test_nvfp4_workspace_reuse_across_calls():
+    # One workspace for a sequence of different tensors (one-pass and two-pass
+    # paths, a zero tensor right after a large one): every result must be the
+    # oracle's, so no partial maximum of an earlier call can leak into a later one.
+    ws = nvq.new_workspace()
+    seq = [act("actq"), torch.zeros(4608, 3072, dtype=torch.bfloat16), act("ffup"),
+           act("qkv4"), workloads.normal(4608, 3072, seed=77, std=1e-3), act("tiny")]
+    for x in seq:
+        codes, sf, g = nvq.nvfp4_quantize(x.cuda(), workspace=ws)
+        torch.cuda.synchronize()
+        M, K = x.shape
+        assert_nvfp4_equal((codes.cpu().numpy(), sf.cpu().numpy(), np.float32(g.item())),
+                           oracle.nvfp4_quantize(bits(x)), M, K)
+    assert nvq.device_status() == 0
+
+
 def test_nvfp4_nonfinite_input_sets_status():
     nvq.device_status()
     x = workloads.normal(128, 64, seed=3)
