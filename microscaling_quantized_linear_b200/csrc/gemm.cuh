@@ -67,10 +67,13 @@ struct GemmCfg {
     static constexpr int SFA_COLS = FMT == 0 ? 4 * KSTEPS : 4;
     static constexpr int SFB_COLS_PER_MMA = 4 * SFB_H;
     static constexpr int SFB_COLS = FMT == 0 ? SFB_COLS_PER_MMA * KSTEPS : SFB_COLS_PER_MMA;
-    static constexpr int ACC_BUFS = (2 * BN + SFA_COLS + SFB_COLS <= 512) ? 2 : 1;
-    static constexpr int TM_SFA = ACC_BUFS * BN;
+    // Scale factors are double-buffered by stage parity, so the copies of
+    // stage s+1 never overwrite columns the MMAs of stage s still read.
+    static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
+    static constexpr int ACC_BUFS = (2 * BN + 2 * SF_COLS <= 512) ? 2 : 1;
+    static constexpr int TM_SFA = ACC_BUFS * BN;           // + (stage parity) * SF_COLS
     static constexpr int TM_SFB = TM_SFA + SFA_COLS;
-    static constexpr int TM_USED = TM_SFB + SFB_COLS;
+    static constexpr int TM_USED = ACC_BUFS * BN + 2 * SF_COLS;
     static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
     static constexpr int THREADS = 192;
     // instruction descriptor: A/B format (E2M1 = 1 for mxf4nvf4, E4M3 = 0 for
@@ -207,16 +210,17 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint32_t sfa_t = tmem + C::TM_SFA + (it & 1) * C::SF_COLS;
+                    const uint32_t sfb_t = sfa_t + C::SFA_COLS;
                     // scale tiles: shared memory -> tensor memory (4 columns each)
 #pragma unroll
                     for (int a = 0; a < C::SF_ATOMS; ++a)
-                        tc_cp_32x128b_warpx4(tmem + C::TM_SFA + 4 * a,
-                                             smem_desc(st + C::OFF_SFA + 512 * a, 16, 128, 0));
+                        tc_cp_32x128b_warpx4(sfa_t + 4 * a, smem_desc(st + C::OFF_SFA + 512 * a, 16, 128, 0));
 #pragma unroll
                     for (int h = 0; h < C::SFB_H; ++h)
 #pragma unroll
                         for (int a = 0; a < C::SF_ATOMS; ++a)
-                            tc_cp_32x128b_warpx4(tmem + C::TM_SFB + C::SFB_COLS_PER_MMA * a + 4 * h,
+                            tc_cp_32x128b_warpx4(sfb_t + C::SFB_COLS_PER_MMA * a + 4 * h,
                                                  smem_desc(st + C::OFF_SFB + h * C::SF_ATOMS * 512 + 512 * a, 16, 128, 0));
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k) {
@@ -224,14 +228,12 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                         const uint64_t bdesc = smem_desc(st + C::OFF_B + k * C::MMA_K_BYTES, 16, 1024, 2);
                         const uint32_t acc = (kt | (uint32_t)k) != 0;
                         if (FMT == 0) {
-                            tc_mma_nvf4(d_tmem, adesc, bdesc, C::IDESC,
-                                        tmem + C::TM_SFA + 4 * k,
-                                        tmem + C::TM_SFB + C::SFB_COLS_PER_MMA * k + sfb_shift, acc);
+                            tc_mma_nvf4(d_tmem, adesc, bdesc, C::IDESC, sfa_t + 4 * k,
+                                        sfb_t + C::SFB_COLS_PER_MMA * k + sfb_shift, acc);
                         } else {
                             const uint32_t id = C::IDESC | ((uint32_t)k << 29) | ((uint32_t)k << 4);
-                            tc_mma_mxf8(d_tmem, adesc, bdesc, id,
-                                        (tmem + C::TM_SFA) | ((uint32_t)k << 30),
-                                        (tmem + C::TM_SFB + sfb_shift) | ((uint32_t)k << 30), acc);
+                            tc_mma_mxf8(d_tmem, adesc, bdesc, id, sfa_t | ((uint32_t)k << 30),
+                                        (sfb_t + sfb_shift) | ((uint32_t)k << 30), acc);
                         }
                     }
                     tc_commit(empty0 + 8 * s);
