@@ -153,7 +153,7 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     if (!calib_amax) {
         // One pass when every CTA's rows fit in shared memory (one CTA per SM).
         const int64_t rows_per_cta = (M + d->num_sms - 1) / d->num_sms;
-        const size_t smem = (size_t)rows_per_cta * (size_t)K * 2 + 128;
+        const size_t smem = fused_smem_bytes((size_t)rows_per_cta, (size_t)K);
         if (smem <= kFusedSmemMax) {
             {
                 std::lock_guard<std::mutex> lock(g_mu);
@@ -330,9 +330,9 @@ int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_sca
     if (rc) return rc;
     if ((rc = get_encoder())) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // Tile width: 192 (two tensor-memory accumulators, epilogue overlapped)
-    // when N allows it, else 256 (one accumulator), else 128 (two).
-    const int bn = (N % 384 == 0) ? 192 : (N % 256 == 0) ? 256 : 128;
+    // Tile width: 256 when N allows it (fewest scale-factor copies per MMA),
+    // else 192 (two tensor-memory accumulators), else 128 (two).
+    const int bn = (N % 256 == 0) ? 256 : (N % 384 == 0) ? 192 : 128;
     if (format == NVQ_NVFP4) {
         if (bn == 192)
             return launch_gemm<0, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,

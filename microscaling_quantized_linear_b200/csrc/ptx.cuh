@@ -214,6 +214,51 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
     return out;
 }
 
+// Eight FP32 -> eight E2M1 codes in one word; a0 lands in bits 3:0, a7 in
+// bits 31:28 (element order = nibble order, low nibble first).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, float a3,
+                                               float a4, float a5, float a6, float a7) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+        : "=r"(out)
+        : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+    return out;
+}
+
+// Four FP32 -> four E4M3 codes in one word, a0 in bits 7:0.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float a0, float a1, float a2, float a3) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .b16 h0, h1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h1, %4, %3;\n\t"
+        "mov.b32 %0, {h0, h1};\n\t}"
+        : "=r"(out) : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+    return out;
+}
+
+// The two BF16 values packed in w, as FP32, each multiplied by m (FP32
+// round-to-nearest-even; one packed f32x2 multiply).
+__device__ __forceinline__ float2 bf16x2_mul(uint32_t w, float m) {
+    float2 c;
+    asm volatile(
+        "{\n\t.reg .b32 lo, hi;\n\t.reg .b64 x, y, z;\n\t"
+        "shl.b32 lo, %2, 16;\n\t"
+        "and.b32 hi, %2, 0xFFFF0000;\n\t"
+        "mov.b64 x, {lo, hi};\n\t"
+        "mov.b64 y, {%3, %3};\n\t"
+        "mul.rn.f32x2 z, x, y;\n\t"
+        "mov.b64 {%0, %1}, z;\n\t}"
+        : "=f"(c.x), "=f"(c.y) : "r"(w), "f"(m));
+    return c;
+}
+
 // Two FP32 -> two E4M3 codes in 16 bits (hi -> bits 15:8, lo -> bits 7:0),
 // round to nearest even, saturating to +-448.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {

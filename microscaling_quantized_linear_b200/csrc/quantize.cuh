@@ -1,20 +1,26 @@
 // quantize.cuh -- BF16 -> NVFP4 / MXFP8 quantize-and-pack kernels.
 //
 // NVFP4 (page "NVIDIA量化推理：5步极速优化显存+成功率翻倍", section NVFP4量化格式;
-// page "NVIDIA Blackwell平台FP4量化技术解析与图像生成优化", section 3.1):
-//   pass 1  amax_partials_kernel: per-CTA max|x| -> workspace[cta]
-//   pass 2  nvfp4_quantize_kernel: every CTA reduces the partials to the
-//           tensor amax (a few KB, L2-resident), derives g_enc / g_dec, then
-//           quantizes one 16-element block per thread: block amax -> E4M3
-//           scale -> E2M1 codes, 8 code bytes per thread, the 4 scale bytes
-//           of 4 neighbouring blocks gathered into one 32-bit store in the
-//           128x4 tile order.
+// page "NVIDIA Blackwell平台FP4量化技术解析与图像生成优化", section 3.1), per
+// 16-element block along K, in FP32 round-to-nearest-even:
+//   s = (b / 6) * g_enc, sc = E4M3(s), r = g_enc / E4M3(sc), q_i = E2M1(x_i * r)
+// with b the block's max |x| and g_enc = 2688 / amax of the tensor.
+//   one pass   nvfp4_quantize_fused_kernel (cooperative; rows fit on chip)
+//   two pass   amax_partials_kernel, then nvfp4_quantize_kernel
+//   calibrated nvfp4_quantize_kernel alone, amax given by the caller
 // MXFP8 (page "NVIDIA量化推理：5步极速优化显存+成功率翻倍", section MXFP8量化格式):
 //   mxfp8_quantize_kernel: one 32-element block per thread, E8M0 exponent
 //   from the block maximum's exponent bits, E4M3 codes of x * 2^-X.
 //
-// All scale arithmetic is FP32 round-to-nearest-even in a fixed order, with
-// no contraction, so results are bit-identical to the CPU oracle.
+// Exactness with fewer instructions: both divisions of the NVFP4 rule come
+// from small per-CTA tables that hold correctly rounded quotients.
+//   b / 6:       b = M * 2^(E-134) with M the 8-bit BF16 significand, so
+//                fl(b/6) = fl(M/6) * 2^(E-134) exactly whenever the result
+//                is a normal float (E >= 8); smaller E divides directly.
+//   g_enc / sc:  sc takes one of 127 values, so r comes from a 127-entry
+//                table computed once per CTA with a correctly rounded divide.
+// Products use packed f32x2 multiplies (IEEE round-to-nearest-even, like the
+// scalar ones); every result is bit-identical to the CPU oracle.
 #pragma once
 #include <cstdint>
 #include "ptx.cuh"
@@ -30,10 +36,6 @@ constexpr size_t kWorkspaceBytes = kWorkspacePartialsOffset + kMaxAmaxPartials *
 constexpr int kQuantThreads = 256;
 constexpr float kAmaxFloor = 0x1p-100f;       // below this the tensor quantizes to zero
 
-// bf16 bits (low 16 of u) -> float
-__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
-
 // max over the two 16-bit magnitudes packed in u
 __device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t u) {
     return __vmaxu2(acc, u & 0x7FFF7FFFu);
@@ -41,6 +43,14 @@ __device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t u) {
 
 __device__ __forceinline__ uint32_t fold2(uint32_t m2) {
     return max(m2 & 0xFFFFu, m2 >> 16);
+}
+
+// BF16 magnitude bits of the largest |x| among the 16 values in w[0..7].
+__device__ __forceinline__ uint32_t block16_max(const uint32_t (&w)[8]) {
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m2 = absmax2(m2, w[i]);
+    return fold2(m2);
 }
 
 // Block-wide max of one value per thread; result valid in every thread.
@@ -67,27 +77,47 @@ __device__ __forceinline__ float e4m3_decode_pos(uint32_t c) {
     return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0x1p-9f;
 }
 
-// Quantize one 16-element block (w[0..7] = 16 BF16 values) with the given
-// global encode scale; returns the E4M3 scale code, writes the 8 code bytes.
-__device__ __forceinline__ uint32_t nvfp4_block(const uint32_t (&w)[8], float g_enc, uint32_t& lo, uint32_t& hi) {
-    uint32_t m2 = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m2 = absmax2(m2, w[i]);
-    const float bmax = __uint_as_float(fold2(m2) << 16);
-    const float s = __fmul_rn(__fdiv_rn(bmax, 6.0f), g_enc);
+// ------------------------------------------------------------------ NVFP4 block
+// Per-CTA tables: d6[t] = fl((128 + t) / 6); rtab[c] = fl(g_enc / E4M3(c)).
+__device__ __forceinline__ void init_d6(float* d6) {
+    if (threadIdx.x < 128) d6[threadIdx.x] = __fdiv_rn((float)(128 + threadIdx.x), 6.0f);
+}
+
+__device__ __forceinline__ void init_rtab(float* rtab, float g_enc) {
+    if (threadIdx.x < 128)
+        rtab[threadIdx.x] = threadIdx.x ? __fdiv_rn(g_enc, e4m3_decode_pos(threadIdx.x)) : 0.0f;
+}
+
+// fl32(b / 6) for b given by its BF16 magnitude bits mb.
+__device__ __forceinline__ float div6(uint32_t mb, const float* d6) {
+    const uint32_t E = mb >> 7;
+    if (E >= 8) return __fmul_rn(d6[mb & 0x7Fu], __uint_as_float((E - 7u) << 23));
+    return __fdiv_rn(__uint_as_float(mb << 16), 6.0f);
+}
+
+// One 16-element block: block max bits mb, the 16 BF16 values in w[0..7].
+// Returns the E4M3 scale code; lo/hi receive the 16 E2M1 codes.  g_enc == 0
+// (a zero tensor) gives scale 0 and zero codes.
+__device__ __forceinline__ uint32_t nvfp4_block(uint32_t mb, const uint32_t (&w)[8], float g_enc,
+                                                const float* d6, const float* rtab, uint32_t& lo, uint32_t& hi) {
+    const float s = __fmul_rn(div6(mb, d6), g_enc);
     const uint32_t sc = cvt_e4m3x2(0.0f, s) & 0xFFu;
-    const float scv = e4m3_decode_pos(sc);
-    lo = hi = 0;
-    if (scv != 0.0f) {
-        const float rr = __fdiv_rn(g_enc, scv);
-        uint32_t q[8];
+    const float r = rtab[sc];
+    float2 p[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            q[i] = cvt_e2m1x2(__fmul_rn(bf16hi(w[i]), rr), __fmul_rn(bf16lo(w[i]), rr));
-        lo = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
-        hi = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
-    }
+    for (int i = 0; i < 8; ++i) p[i] = bf16x2_mul(w[i], r);
+    lo = cvt_e2m1x8(p[0].x, p[0].y, p[1].x, p[1].y, p[2].x, p[2].y, p[3].x, p[3].y);
+    hi = cvt_e2m1x8(p[4].x, p[4].y, p[5].x, p[5].y, p[6].x, p[6].y, p[7].x, p[7].y);
+    if (sc == 0) lo = hi = 0;                         // scale rounded to zero: zero codes (no -0)
     return sc;
+}
+
+__device__ __forceinline__ float encode_scale(float amax) {
+    return amax >= kAmaxFloor ? __fdiv_rn(2688.0f, amax) : 0.0f;
+}
+
+__device__ __forceinline__ float decode_scale(float amax) {
+    return amax >= kAmaxFloor ? __fdiv_rn(amax, 2688.0f) : 0.0f;
 }
 
 // ------------------------------------------------------------------ amax
@@ -126,25 +156,30 @@ amax_partials_kernel(const uint4* __restrict__ x, uint32_t rows, uint32_t vecs_p
     if (threadIdx.x == 0) partial[blockIdx.x] = m;
 }
 
-// ------------------------------------------------------------------ NVFP4
-// One thread = one 16-element block.  Block b of the tensor is (row b / nblk,
-// column b % nblk) with nblk = K / 16; its codes are bytes [8b, 8b + 8).
+// ------------------------------------------------------------------ NVFP4, streaming
+// One thread = one 16-element block per iteration.  Block b is (row b / nblk,
+// column b % nblk), nblk = K / 16; its codes are bytes [8b, 8b + 8).  The amax
+// is the reduction of the two-pass partials, or *calib_amax.
 __global__ void __launch_bounds__(kQuantThreads, 8)
 nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nblk, uint32_t ldx,
                       uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ g_dec_out,
                       const uint32_t* __restrict__ partial, uint32_t npartial,
                       const float* __restrict__ calib_amax, unsigned int* __restrict__ status) {
     __shared__ uint32_t red[kQuantThreads / 32];
+    __shared__ float d6[128], rtab[128];
     const uint32_t total = rows * nblk;
-    // the first block's loads do not depend on the amax: issue them first
+    const uint32_t stride = gridDim.x * kQuantThreads;
+    const uint32_t qs = stride / nblk, rs = stride - qs * nblk;
     uint32_t b = blockIdx.x * kQuantThreads + threadIdx.x;
-    uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
+    uint32_t r = b / nblk, c = b - r * nblk;
+    // the first block's loads do not depend on the amax: issue them first
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
     if (b < total) {
-        const uint32_t r = b / nblk, c = b - r * nblk;
         const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
-        p0 = __ldg(src);
-        p1 = __ldg(src + 1);
+        v0 = __ldg(src);
+        v1 = __ldg(src + 1);
     }
+    init_d6(d6);
     float amax;
     if (calib_amax != nullptr) {
         amax = *calib_amax;
@@ -155,27 +190,22 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
         if (m >= 0x7F80u && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, 2u);
         amax = __uint_as_float(m << 16);
     }
-    const bool zero_tensor = !(amax >= kAmaxFloor);
-    const float g_enc = __fdiv_rn(2688.0f, amax);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *g_dec_out = zero_tensor ? 0.0f : __fdiv_rn(amax, 2688.0f);
+    const float g_enc = encode_scale(amax);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *g_dec_out = decode_scale(amax);
+    init_rtab(rtab, g_enc);
+    __syncthreads();
 
     const uint32_t ctiles = nblk >> 2;
-    for (bool first = true; b - threadIdx.x < total; b += gridDim.x * kQuantThreads, first = false) {
+    for (bool first = true; b - threadIdx.x < total; first = false) {
         const bool active = b < total;       // whole warps stay in the loop for the shuffles
-        uint32_t r = 0, c = 0;
-        uint4 v0 = p0, v1 = p1;
-        if (active) {
-            r = b / nblk;
-            c = b - r * nblk;
-            if (!first) {
-                const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
-                v0 = __ldg(src);
-                v1 = __ldg(src + 1);
-            }
+        if (active && !first) {
+            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
+            v0 = __ldg(src);
+            v1 = __ldg(src + 1);
         }
         const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        uint32_t sc = 0, lo = 0, hi = 0;
-        if (!zero_tensor) sc = nvfp4_block(w, g_enc, lo, hi);
+        uint32_t lo, hi;
+        const uint32_t sc = nvfp4_block(block16_max(w), w, g_enc, d6, rtab, lo, hi);
         // gather the scales of 4 neighbouring blocks (c % 4 == 0..3, same row)
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
@@ -186,6 +216,13 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
                 *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r, c, ctiles)) =
                     sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
         }
+        b += stride;
+        r += qs;
+        c += rs;
+        if (c >= nblk) {
+            c -= nblk;
+            ++r;
+        }
     }
 }
 
@@ -193,10 +230,11 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
 // For tensors whose rows fit in the shared memory of one CTA per SM: every
 // CTA copies its rows into shared memory once (bulk copies, 4 chunks with
 // their own mbarriers so the block maxima are taken while later chunks are
-// still landing), publishes its partial amax in an epoch-tagged 64-bit slot
-// of the workspace, waits (bounded) until every CTA's slot carries this
-// call's epoch, and quantizes from shared memory.  HBM sees exactly one read
-// of the activation.  Must be launched cooperatively (all CTAs co-resident).
+// still landing, and kept in shared memory), publishes its partial amax in an
+// epoch-tagged 64-bit slot of the workspace, waits (bounded) until every
+// CTA's slot carries this call's epoch, and quantizes from shared memory.
+// HBM sees exactly one read of the activation.  Must be launched
+// cooperatively (all CTAs co-resident).
 constexpr int kFusedThreads = 1024;
 constexpr int kFusedChunks = 4;
 constexpr uint64_t kFusedWaitNs = 2000000000ull;   // 2 s
@@ -223,6 +261,11 @@ __device__ __forceinline__ void lds_block32(const uint8_t* base, uint32_t b, uin
     v1 = sw ? first : second;
 }
 
+// Shared memory the one-pass kernel needs for rows_per_cta rows of K.
+__host__ __device__ constexpr size_t fused_smem_bytes(size_t rows_per_cta, size_t K) {
+    return 128 /*align*/ + rows_per_cta * K * 2 /*tile*/ + rows_per_cta * (K / 16) * 2 /*block maxima*/;
+}
+
 __global__ void __launch_bounds__(kFusedThreads, 1)
 nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t K, uint32_t ldx,
                             uint32_t rows_per_cta, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
@@ -230,13 +273,15 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
                             uint32_t epoch, unsigned int* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const uint32_t nblk = K >> 4;
+    uint16_t* bmax = reinterpret_cast<uint16_t*>(tile + (size_t)rows_per_cta * K * 2);
     __shared__ __align__(8) uint64_t bars[kFusedChunks];
     __shared__ uint32_t red[kFusedThreads / 32];
+    __shared__ float d6[128], rtab[128];
     __shared__ int s_timeout;
 
     const uint32_t r0 = blockIdx.x * rows_per_cta;
     const uint32_t nr = min(rows_per_cta, rows - r0);
-    const uint32_t nblk = K >> 4;
     const uint32_t row_bytes = K * 2;
     const uint32_t rows_per_chunk = (nr + kFusedChunks - 1) / kFusedChunks;
     if (threadIdx.x == 0) {
@@ -257,10 +302,11 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
             }
         }
     }
+    init_d6(d6);
     __syncthreads();
 
-    // partial amax, chunk by chunk as the copies land
-    uint32_t m2 = 0;
+    // block maxima, chunk by chunk as the copies land
+    uint32_t m = 0;
     for (int c = 0; c < kFusedChunks; ++c) {
         const uint32_t ra = min(nr, c * rows_per_chunk), rb = min(nr, (c + 1) * rows_per_chunk);
         if (!mbar_wait_bounded(smem_u32(&bars[c]), 0, &s_timeout, kFusedWaitNs)) s_timeout = 1;
@@ -268,16 +314,18 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
         for (uint32_t b = ra * nblk + threadIdx.x; b < rb * nblk; b += kFusedThreads) {
             uint4 v0, v1;
             lds_block32(tile, b, v0, v1);
-            m2 = absmax2(absmax2(absmax2(absmax2(m2, v0.x), v0.y), v0.z), v0.w);
-            m2 = absmax2(absmax2(absmax2(absmax2(m2, v1.x), v1.y), v1.z), v1.w);
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            const uint32_t mb = block16_max(w);
+            bmax[b] = (uint16_t)mb;
+            m = max(m, mb);
         }
     }
-    const uint32_t cta_max = block_max_u32<kFusedThreads>(fold2(m2), red);
+    const uint32_t cta_max = block_max_u32<kFusedThreads>(m, red);
     if (threadIdx.x == 0)
         st_release_u64(slots + blockIdx.x, ((unsigned long long)epoch << 32) | cta_max);
 
     // every CTA's partial, tagged with this call's epoch
-    uint32_t m = 0;
+    m = 0;
     if (threadIdx.x < gridDim.x) {
         const unsigned long long* slot = slots + threadIdx.x;
         unsigned long long v = ld_acquire_u64(slot);
@@ -294,10 +342,9 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
     }
     const uint32_t amax_bits = block_max_u32<kFusedThreads>(m, red);
     if (s_timeout) {                                  // a copy or a peer never arrived: write nothing
-        if (threadIdx.x == 0) atomicOr(status, 1u);
-        // let every issued copy land before the CTA exits
         if (threadIdx.x == 0) {
-            int never = 0;
+            atomicOr(status, 1u);
+            int never = 0;                            // let every issued copy land before the CTA exits
             for (int c = 0; c < kFusedChunks; ++c) mbar_wait_bounded(smem_u32(&bars[c]), 0, &never, kFusedWaitNs);
         }
         __syncthreads();
@@ -305,29 +352,42 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
     }
     if (amax_bits >= 0x7F80u && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, 2u);
     const float amax = __uint_as_float(amax_bits << 16);
-    const bool zero_tensor = !(amax >= kAmaxFloor);
-    const float g_enc = __fdiv_rn(2688.0f, amax);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *g_dec_out = zero_tensor ? 0.0f : __fdiv_rn(amax, 2688.0f);
+    const float g_enc = encode_scale(amax);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *g_dec_out = decode_scale(amax);
+    init_rtab(rtab, g_enc);
+    __syncthreads();
 
     const uint32_t total = nr * nblk;
     const uint32_t ctiles = nblk >> 2;
+    const uint32_t qs = kFusedThreads / nblk, rs = kFusedThreads - qs * nblk;
+    uint32_t rl = threadIdx.x / nblk, c = threadIdx.x - rl * nblk;
+    const size_t code_base = (size_t)r0 * nblk * 8;
     for (uint32_t base = 0; base < total; base += kFusedThreads) {
         const uint32_t b = base + threadIdx.x;
         const bool active = b < total;
         uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-        if (active) lds_block32(tile, b, v0, v1);
+        uint32_t mb = 0;
+        if (active) {
+            lds_block32(tile, b, v0, v1);
+            mb = bmax[b];
+        }
         const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        uint32_t lo = 0, hi = 0, sc = 0;
-        if (!zero_tensor) sc = nvfp4_block(w, g_enc, lo, hi);
+        uint32_t lo, hi;
+        const uint32_t sc = nvfp4_block(mb, w, g_enc, d6, rtab, lo, hi);
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
         const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
         if (active) {
-            const uint32_t rl = b / nblk, c = b - rl * nblk, r = r0 + rl;
-            *reinterpret_cast<uint2*>(codes + (size_t)r * (K >> 1) + (size_t)c * 8) = make_uint2(lo, hi);
+            *reinterpret_cast<uint2*>(codes + code_base + (size_t)b * 8) = make_uint2(lo, hi);
             if ((c & 3u) == 0)
-                *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r, c, ctiles)) =
+                *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r0 + rl, c, ctiles)) =
                     sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        }
+        rl += qs;
+        c += rs;
+        if (c >= nblk) {
+            c -= nblk;
+            ++rl;
         }
     }
 }
@@ -340,16 +400,16 @@ mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
                       uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
     const uint32_t total = rows * nblk;
     const uint32_t ctiles = nblk >> 2;
-    for (uint32_t b = blockIdx.x * kQuantThreads + threadIdx.x; b - threadIdx.x < total;
-         b += gridDim.x * kQuantThreads) {
+    const uint32_t stride = gridDim.x * kQuantThreads;
+    const uint32_t qs = stride / nblk, rs = stride - qs * nblk;
+    uint32_t b = blockIdx.x * kQuantThreads + threadIdx.x;
+    uint32_t r = b / nblk, c = b - r * nblk;
+    for (; b - threadIdx.x < total; b += stride) {
         const bool active = b < total;
-        uint32_t r = 0, c = 0;
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) w[i] = 0;
         if (active) {
-            r = b / nblk;
-            c = b - r * nblk;
             const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 32);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -374,9 +434,9 @@ mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
         uint32_t q[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const uint32_t p0 = cvt_e4m3x2(__fmul_rn(bf16hi(w[2 * i]), mult), __fmul_rn(bf16lo(w[2 * i]), mult));
-            const uint32_t p1 = cvt_e4m3x2(__fmul_rn(bf16hi(w[2 * i + 1]), mult), __fmul_rn(bf16lo(w[2 * i + 1]), mult));
-            q[i] = p0 | (p1 << 16);
+            const float2 p0 = bf16x2_mul(w[2 * i], mult);
+            const float2 p1 = bf16x2_mul(w[2 * i + 1], mult);
+            q[i] = cvt_e4m3x4(p0.x, p0.y, p1.x, p1.y);
         }
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
@@ -388,6 +448,12 @@ mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
             if ((c & 3u) == 0)
                 *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r, c, ctiles)) =
                     sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        }
+        r += qs;
+        c += rs;
+        if (c >= nblk) {
+            c -= nblk;
+            ++r;
         }
     }
 }
