@@ -1,0 +1,300 @@
+// gemm_pair.cuh -- block-scaled GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+// Same product as gemm.cuh, D = bf16(alpha * A . B^T + bias), on output tiles
+// of 256 x BN computed by a cluster of two CTAs on two SMs:
+//   CTA r (r = 0, 1) stages rows [128r, 128r + 128) of the A tile and rows
+//   [r BN/2, (r+1) BN/2) of the B tile in its own shared memory, holds the
+//   scale tiles of its 128 A rows and of all BN B rows, and owns accumulator
+//   rows [128r, 128r + 128) in its own tensor memory.
+//   The leader (r = 0) alone issues tcgen05.cp (both CTAs' scales into both
+//   tensor memories) and the 256 x BN x K MMAs; its commits arrive on the
+//   barriers of both CTAs (.multicast::cluster on the commit).
+//   Both CTAs' tile loads complete on the leader's full barrier
+//   (.cta_group::2 tensor loads; no load multicast anywhere).
+//   Each CTA drains its own accumulator half; the peer's epilogue warps
+//   arrive remotely on the leader's accumulator-empty barrier.
+// Per SM this halves the B bytes staged from L2 and the tensor-core
+// instructions issued for the same work, compared with one 128 x BN tile
+// per SM.  All waits are bounded (status word + abort flag), as in gemm.cuh.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace nvq {
+
+template <int FMT, int BN_>
+struct PairCfg {
+    static constexpr int BM = 256;                           // rows per pair; 128 per CTA
+    static constexpr int BN = BN_;
+    static constexpr int BN_HALF = BN / 2;                   // B rows staged per CTA
+    static constexpr int KBYTES = 128;
+    static constexpr int BK = FMT == 0 ? 256 : 128;
+    static constexpr int MMA_K = FMT == 0 ? 64 : 32;
+    static constexpr int KSTEPS = BK / MMA_K;
+    static constexpr int MMA_K_BYTES = KBYTES / KSTEPS;
+    static constexpr int SF_BLOCK = FMT == 0 ? 16 : 32;
+    static constexpr int SF_ATOMS = BK / SF_BLOCK / 4;
+    static constexpr int SF_CHUNK = SF_ATOMS * 512;          // scale bytes per 128 rows per stage
+    static constexpr int SFB_H = BN / 128;                   // 128-row scale tiles of the B tile
+    static constexpr int A_BYTES = 128 * KBYTES;
+    static constexpr int B_BYTES = BN_HALF * KBYTES;
+    static constexpr int SFA_BYTES = SF_CHUNK;
+    static constexpr int SFB_BYTES = SFB_H * SF_CHUNK;
+    static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // per CTA per stage
+    static constexpr int STAGE_BYTES = (TX_BYTES + 1023) / 1024 * 1024;
+    static constexpr int OFF_B = A_BYTES;
+    static constexpr int OFF_SFA = A_BYTES + B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
+    static constexpr int EPI_BUF_BYTES = 32 * 64;
+    static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
+    static constexpr int SMEM_LIMIT = 232448;
+    static constexpr int FIXED_BYTES = 1024 + 256 + EPI_BYTES;
+    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+    static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
+    static constexpr int SFA_COLS = FMT == 0 ? 4 * KSTEPS : 4;
+    static constexpr int SFB_COLS_PER_MMA = 4 * SFB_H;
+    static constexpr int SFB_COLS = FMT == 0 ? SFB_COLS_PER_MMA * KSTEPS : SFB_COLS_PER_MMA;
+    static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
+    static constexpr int ACC_BUFS = (2 * BN + 2 * SF_COLS <= 512) ? 2 : 1;
+    static constexpr int TM_SFA = ACC_BUFS * BN;
+    static constexpr int TM_USED = ACC_BUFS * BN + 2 * SF_COLS;
+    static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
+    static constexpr int THREADS = 192;
+    static constexpr uint32_t IDESC =
+        (FMT == 0 ? (1u << 7) | (1u << 10) : 0u) |
+        ((uint32_t)(BN >> 3) << 17) |
+        (FMT == 0 ? 0u : (1u << 23)) |
+        ((uint32_t)(BM >> 4) << 24);
+    static_assert(BN == 256, "pair tiles are 256 x 256");
+    static_assert(TM_USED <= 512, "tensor memory overflow");
+    static_assert(STAGES >= 2, "shared memory too small");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory overflow");
+};
+
+template <int FMT, int BN>
+__global__ void __launch_bounds__(192, 1)
+bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                   const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                   const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
+    using C = PairCfg<FMT, BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
+    const uint32_t full0 = smem_u32(bars);
+    const uint32_t empty0 = full0 + 8 * C::STAGES;
+    const uint32_t tfull0 = empty0 + 8 * C::STAGES;
+    const uint32_t tempty0 = tfull0 + 8 * 2;
+    const uint32_t drain = tempty0 + 8 * 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    volatile int* never = abort_flag + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();               // 0 = leader
+    const uint32_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull0 + 8 * b, 1);
+            mbar_init(tempty0 + 8 * b, 8);                 // 4 epilogue warps in each CTA
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        *never = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmap_a);
+        prefetch_tensormap(&tmap_b);
+        prefetch_tensormap(&tmap_sfa);
+        prefetch_tensormap(&tmap_sfb);
+        prefetch_tensormap(&tmap_d);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(tmem_holder), C::TM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();                                        // barriers of both CTAs initialised
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const uint32_t num_tiles = p.num_m_blocks * p.num_n_blocks;   // 256 x BN tiles
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer (both CTAs)
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (uint32_t tile = pair; tile < num_tiles && ok; tile += npairs) {
+                const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+                const int32_t arow = (int32_t)(mb * 256 + 128 * rank);
+                const int32_t brow = (int32_t)(nb * BN + C::BN_HALF * rank);
+                const uint32_t sfa_atom = mb * 2 + rank;              // this CTA's 128 A rows
+                const uint32_t sfb_atom = nb * (BN / 128);
+                for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt) {
+                    const uint32_t s = it % C::STAGES, use = it / C::STAGES;
+                    if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint32_t fb = mapa_shared(full0 + 8 * s, 0);   // the leader's full barrier
+                    if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * C::TX_BYTES);
+                    tma_load_2d_pair(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), arow);
+                    tma_load_2d_pair(st + C::OFF_B, &tmap_b, fb, (int32_t)(kt * C::KBYTES), brow);
+                    // scale tiles: the tensors are viewed as rows of 256 bytes
+                    tma_load_2d_pair(st + C::OFF_SFA, &tmap_sfa, fb, 0,
+                                     (int32_t)(((size_t)sfa_atom * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 2));
+#pragma unroll
+                    for (int h = 0; h < C::SFB_H; ++h)
+                        tma_load_2d_pair(st + C::OFF_SFB + h * C::SF_CHUNK, &tmap_sfb, fb, 0,
+                                         (int32_t)(((size_t)(sfb_atom + h) * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 2));
+                    ++it;
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+            }
+            if (rank == 0)      // the leader's barriers count both CTAs' bytes: wait for the last stages
+                for (uint32_t j = it > (uint32_t)C::STAGES ? it - C::STAGES : 0; j < it; ++j)
+                    mbar_wait_bounded(full0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer (leader only)
+        if (lane == 0 && rank == 0) {
+            uint32_t it = 0, t_local = 0;
+            bool ok = true;
+            for (uint32_t tile = pair; tile < num_tiles && ok; tile += npairs, ++t_local) {
+                const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
+                const uint32_t use = C::ACC_BUFS == 2 ? (t_local >> 1) : t_local;
+                if (use > 0 && !mbar_wait_bounded(tempty0 + 8 * buf, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + buf * BN;
+                for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt, ++it) {
+                    const uint32_t s = it % C::STAGES, su = it / C::STAGES;
+                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint32_t sfa_t = tmem + C::TM_SFA + (it & 1) * C::SF_COLS;
+                    const uint32_t sfb_t = sfa_t + C::SFA_COLS;
+#pragma unroll
+                    for (int a = 0; a < C::SF_ATOMS; ++a)
+                        tc_cp_pair_32x128b_warpx4(sfa_t + 4 * a, smem_desc(st + C::OFF_SFA + 512 * a, 16, 128, 0));
+#pragma unroll
+                    for (int h = 0; h < C::SFB_H; ++h)
+#pragma unroll
+                        for (int a = 0; a < C::SF_ATOMS; ++a)
+                            tc_cp_pair_32x128b_warpx4(sfb_t + C::SFB_COLS_PER_MMA * a + 4 * h,
+                                                      smem_desc(st + C::OFF_SFB + h * C::SF_CHUNK + 512 * a, 16, 128, 0));
+#pragma unroll
+                    for (int k = 0; k < C::KSTEPS; ++k) {
+                        const uint64_t adesc = smem_desc(st + k * C::MMA_K_BYTES, 16, 1024, 2);
+                        const uint64_t bdesc = smem_desc(st + C::OFF_B + k * C::MMA_K_BYTES, 16, 1024, 2);
+                        const uint32_t acc = (kt | (uint32_t)k) != 0;
+                        if (FMT == 0) {
+                            tc_mma_nvf4_pair(d_tmem, adesc, bdesc, C::IDESC, sfa_t + 4 * k,
+                                             sfb_t + C::SFB_COLS_PER_MMA * k, acc);
+                        } else {
+                            const uint32_t id = C::IDESC | ((uint32_t)k << 29) | ((uint32_t)k << 4);
+                            tc_mma_mxf8_pair(d_tmem, adesc, bdesc, id, sfa_t | ((uint32_t)k << 30),
+                                             sfb_t | ((uint32_t)k << 30), acc);
+                        }
+                    }
+                    tc_commit_pair_mc(empty0 + 8 * s, 0x3);     // frees the stage in both CTAs
+                }
+                if (!ok) break;
+                tc_commit_pair_mc(tfull0 + 8 * buf, 0x3);       // accumulator ready in both CTAs
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+            }
+            tc_commit_pair(drain);
+            mbar_wait_bounded(drain, 0, never, kWaitLimitNs);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue (both CTAs)
+        const int q = warp & 3;
+        const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
+        uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * 2 * C::EPI_BUF_BYTES;
+        const uint32_t swz = (uint32_t)((lane >> 1) & 3);
+        uint32_t t_local = 0, nstore = 0;
+        for (uint32_t tile = pair; tile < num_tiles; tile += npairs, ++t_local) {
+            const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+            const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
+            const uint32_t use = C::ACC_BUFS == 2 ? (t_local >> 1) : t_local;
+            if (!mbar_wait_bounded(tfull0 + 8 * buf, use & 1, abort_flag, kWaitLimitNs)) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+                break;
+            }
+            tc_fence_after();
+            const int32_t row0 = (int32_t)(mb * 256 + 128 * rank + 32 * q);
+            const uint32_t n0 = nb * BN;
+            const __nv_bfloat16* brow = p.bias ? p.bias + n0 : nullptr;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                uint32_t r[32];
+                tc_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + buf * BN + c, r);
+                tc_wait_ld();
+                if (c + 32 == BN) {                        // accumulator half read: release it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty0 + 8 * buf, 0));
+                }
+                uint32_t packed[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    float v0 = __fmul_rn(__uint_as_float(r[2 * j]), alpha);
+                    float v1 = __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha);
+                    if (brow) {
+                        const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(brow + c + 2 * j);
+                        v0 = __fadd_rn(v0, __bfloat162float(bb.x));
+                        v1 = __fadd_rn(v1, __bfloat162float(bb.y));
+                    }
+                    const __nv_bfloat162 o = __floats2bfloat162_rn(v0, v1);
+                    packed[j] = *reinterpret_cast<const uint32_t*>(&o);
+                }
+                uint8_t* sb = staging + (nstore & 1) * C::EPI_BUF_BYTES;
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    *reinterpret_cast<uint4*>(sb + lane * 64 + 16 * ((uint32_t)j ^ swz)) =
+                        make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmap_d, smem_u32(sb), (int32_t)(n0 + c), row0);
+                    bulk_commit_group();
+                }
+                ++nstore;
+            }
+        }
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    cluster_sync();                                        // both CTAs done with the pair's resources
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, C::TM_COLS);
+    }
+}
+
+}  // namespace nvq

@@ -12,11 +12,13 @@
 #include <atomic>
 #include <chrono>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
 #include "nvq.h"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "quantize.cuh"
 
 namespace nvq {
@@ -35,6 +37,7 @@ struct DeviceInfo {
     int num_sms = 0;
     unsigned int* status = nullptr;
     bool gemm_attr[2][3] = {{false, false, false}, {false, false, false}};
+    bool pair_attr[2] = {false, false};
     bool fused_attr = false;
 };
 
@@ -137,6 +140,13 @@ uint32_t next_epoch() {
 
 constexpr size_t kFusedSmemMax = 220 * 1024;
 
+// NVQ_GEMM_PAIRS=0 in the environment selects the one-CTA GEMM for every
+// shape (the test suite runs both kernels on the same shapes).
+const bool g_use_pairs = [] {
+    const char* e = getenv("NVQ_GEMM_PAIRS");
+    return !(e && e[0] == '0');
+}();
+
 int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
                         float* global_scale, const float* calib_amax, void* workspace, cudaStream_t stream) {
     int rc = check_quant_shape(NVQ_NVFP4, M, K, ldx);
@@ -228,6 +238,77 @@ int encode_out_map(CUtensorMap* map, const void* out, int64_t rows, int64_t cols
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? NVQ_OK : NVQ_ERR_CUDA;
+}
+
+// Scale buffer viewed as rows of 256 bytes; a box of box_rows rows is one
+// stage's scale chunk for 128 rows (2 KB NVFP4, 512 B MXFP8).
+int encode_scale_map(CUtensorMap* map, const void* scales, size_t bytes, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {256u, (cuuint64_t)(bytes / 256)};
+    const cuuint64_t strides[1] = {256u};
+    const cuuint32_t box[2] = {256u, box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(scales), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVQ_OK : NVQ_ERR_CUDA;
+}
+
+// 256 x 256 tiles on CTA pairs (M % 256 == 0, N % 256 == 0).
+template <int FMT>
+int launch_gemm_pair(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                     const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
+                     void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    using C = PairCfg<FMT, 256>;
+    const int64_t kbytes = FMT == 0 ? K / 2 : K;
+    const int fmt = FMT == 0 ? NVQ_NVFP4 : NVQ_MXFP8;
+    CUtensorMap ma, mb, msa, msb, md;
+    int rc;
+    if ((rc = encode_codes_map(&ma, a_codes, M, kbytes, 128))) return rc;
+    if ((rc = encode_codes_map(&mb, b_codes, N, kbytes, C::BN_HALF))) return rc;
+    if ((rc = encode_scale_map(&msa, a_scales, nvq_scale_bytes(fmt, M, K), C::SF_CHUNK / 256))) return rc;
+    if ((rc = encode_scale_map(&msb, b_scales, nvq_scale_bytes(fmt, N, K), C::SF_CHUNK / 256))) return rc;
+    if ((rc = encode_out_map(&md, out, M, N, ldo))) return rc;
+    auto kern = bsgemm_pair_kernel<FMT, 256>;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!d->pair_attr[FMT]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+                cudaSuccess)
+                return NVQ_ERR_CUDA;
+            d->pair_attr[FMT] = true;
+        }
+    }
+    GemmParams p;
+    p.sfa = a_scales;
+    p.sfb = b_scales;
+    p.a_global = a_global;
+    p.b_global = b_global;
+    p.bias = static_cast<const __nv_bfloat16*>(bias);
+    p.status = d->status;
+    p.num_m_blocks = (uint32_t)(M / 256);
+    p.num_n_blocks = (uint32_t)(N / 256);
+    p.num_k_tiles = (uint32_t)(K / C::BK);
+    p.sf_ctiles = (uint32_t)(K / C::SF_BLOCK / 4);
+    const uint32_t tiles = p.num_m_blocks * p.num_n_blocks;
+    const uint32_t pairs = (uint32_t)d->num_sms / 2;
+    const uint32_t grid = 2 * (tiles < pairs ? tiles : pairs);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, md, p) != cudaSuccess) {
+        cudaGetLastError();
+        return NVQ_ERR_CUDA;
+    }
+    return NVQ_OK;
 }
 
 template <int FMT, int BN>
@@ -333,6 +414,14 @@ int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_sca
     // Tile width: 256 when N allows it (fewest scale-factor copies per MMA),
     // else 192 (two tensor-memory accumulators), else 128 (two).
     const int bn = (N % 256 == 0) ? 256 : (N % 384 == 0) ? 192 : 128;
+    // CTA pairs (256 x 256 tiles) when both M and N allow them.
+    const bool pair = g_use_pairs && (M % 256 == 0) && (N % 256 == 0);
+    if (pair)
+        return format == NVQ_NVFP4
+                   ? launch_gemm_pair<0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
+                                         M, N, K, s)
+                   : launch_gemm_pair<1>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo,
+                                         M, N, K, s);
     if (format == NVQ_NVFP4) {
         if (bn == 192)
             return launch_gemm<0, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,

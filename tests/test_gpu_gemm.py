@@ -52,7 +52,8 @@ def oracle_linear(fmt, x, w, rows=None, bias=None):
 
 
 SMALL = [
-    # fmt, M, N, K  (N % 256 != 0 takes the 128-wide tile)
+    # fmt, M, N, K.  M % 256 == 0 and N % 256 == 0 run on CTA pairs (256 x 256
+    # tiles); otherwise one CTA per tile, 256 wide if N allows, else 192 or 128.
     ("nvfp4", 128, 128, 256),
     ("nvfp4", 256, 384, 512),
     ("nvfp4", 384, 512, 768),
@@ -60,6 +61,8 @@ SMALL = [
     ("mxfp8", 128, 128, 128),
     ("mxfp8", 256, 384, 384),
     ("mxfp8", 384, 512, 640),
+    ("mxfp8", 512, 512, 384),          # CTA-pair kernel
+    ("mxfp8", 256, 256, 128),          # CTA-pair kernel, one K stage
 ]
 
 
@@ -140,3 +143,37 @@ def test_full_size_workloads_sampled_rows(name, fmt, every):
     Dr = D[torch.from_numpy(rows).cuda()].float().cpu().numpy()
     Y = oracle_linear(fmt, x, w, rows=rows)
     check_gemm(Dr, Y)
+
+
+SINGLE_CTA_SCRIPT = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, %r)
+sys.path.insert(0, %r)
+import test_gpu_gemm as t
+from gpu_common import check_gemm, sample_rows
+import workloads
+for fmt, M, N, K in [("nvfp4", 1024, 768, 512), ("mxfp8", 512, 512, 384), ("nvfp4", 4608, 12288, 3072)]:
+    x = workloads.normal(M, K, seed=90 + M % 13)
+    w = workloads.normal(N, K, seed=91 + N % 11, std=0.05)
+    rows = sample_rows(M, per_tile_every=4)
+    D = t.gpu_linear(fmt, x, w)
+    Dr = D[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    err = check_gemm(Dr, t.oracle_linear(fmt, x, w, rows=rows))
+    print(fmt, M, N, K, "max row err %.2e" % err)
+print("OK")
+"""
+
+
+def test_single_cta_kernel_on_pair_shapes():
+    # The library picks CTA pairs for these shapes; NVQ_GEMM_PAIRS=0 (read
+    # when the library loads, hence a fresh process) forces the one-CTA
+    # kernel, which must give the same answers.
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    env = dict(os.environ, NVQ_GEMM_PAIRS="0")
+    out = subprocess.run([sys.executable, "-c", SINGLE_CTA_SCRIPT % (root, here)], env=env,
+                         capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0 and out.stdout.strip().endswith("OK"), out.stdout + out.stderr
