@@ -125,6 +125,9 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
     cluster_sync();                                        // barriers of both CTAs initialised
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // everything above overlaps the previous grid; no global data is
+    // touched before it has completed
+    griddep_wait();
     const uint32_t num_tiles = p.num_m_blocks * p.num_n_blocks;   // 256 x BN tiles
 
     if (warp == 0) {

@@ -140,6 +140,14 @@ uint32_t next_epoch() {
 
 constexpr size_t kFusedSmemMax = 220 * 1024;
 
+// Dynamic NVFP4 quantization: two passes (amax, then quantize with
+// programmatic dependent launch) unless NVQ_QUANT_ONE_PASS=1 selects the
+// cooperative one-pass kernel for tensors that fit on chip.
+const bool g_quant_one_pass = [] {
+    const char* e = getenv("NVQ_QUANT_ONE_PASS");
+    return e && e[0] == '1';
+}();
+
 // NVQ_GEMM_PAIRS=0 in the environment selects the one-CTA GEMM for every
 // shape (the test suite runs both kernels on the same shapes).
 const bool g_use_pairs = [] {
@@ -160,7 +168,7 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     DeviceInfo* d = nullptr;
     if ((rc = device_info(&d))) return rc;
     const uint32_t nblk = (uint32_t)(K / 16);
-    if (!calib_amax) {
+    if (!calib_amax && g_quant_one_pass) {
         // One pass when every CTA's rows fit in shared memory (one CTA per SM).
         const int64_t rows_per_cta = (M + d->num_sms - 1) / d->num_sms;
         const size_t smem = fused_smem_bytes((size_t)rows_per_cta, (size_t)K);
@@ -191,15 +199,29 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
         }
     }
     uint32_t npartial = 0;
-    uint32_t* partial = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + kWorkspacePartialsOffset);
+    uint32_t* partial = calib_amax ? nullptr
+                                   : reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + kWorkspacePartialsOffset);
     if (!calib_amax) {
         if ((rc = launch_amax(x, M, K, ldx, partial, d->num_sms, stream, &npartial))) return rc;
     }
     const uint64_t units = (uint64_t)M * nblk;
-    nvfp4_quantize_kernel<<<quant_grid(units, d->num_sms), kQuantThreads, 0, stream>>>(
-        static_cast<const uint16_t*>(x), (uint32_t)M, nblk, (uint32_t)ldx, codes, scales, global_scale,
-        partial, npartial, calib_amax, d->status);
-    return launch_status();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(quant_grid(units, d->num_sms));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = calib_amax ? 0 : 1;   // overlap only with our own amax pass
+    const uint16_t* xp = static_cast<const uint16_t*>(x);
+    const uint32_t* pp = partial;
+    if (cudaLaunchKernelEx(&cfg, nvfp4_quantize_kernel, xp, (uint32_t)M, nblk, (uint32_t)ldx, codes, scales,
+                           global_scale, pp, npartial, calib_amax, d->status) != cudaSuccess) {
+        cudaGetLastError();
+        return NVQ_ERR_CUDA;
+    }
+    return NVQ_OK;
 }
 
 int mxfp8_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
@@ -297,13 +319,15 @@ int launch_gemm_pair(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_sca
     cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, md, p) != cudaSuccess) {
         cudaGetLastError();
         return NVQ_ERR_CUDA;
@@ -346,8 +370,21 @@ int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, 
     p.sf_ctiles = (uint32_t)(K / C::SF_BLOCK / 4);
     const uint32_t tiles = p.num_m_blocks * p.num_n_blocks;
     const uint32_t grid = tiles < (uint32_t)d->num_sms ? tiles : (uint32_t)d->num_sms;
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, md, p);
-    return launch_status();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ma, mb, md, p) != cudaSuccess) {
+        cudaGetLastError();
+        return NVQ_ERR_CUDA;
+    }
+    return NVQ_OK;
 }
 
 }  // namespace

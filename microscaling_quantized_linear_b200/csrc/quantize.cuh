@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(kAmaxThreads)
 amax_partials_kernel(const uint4* __restrict__ x, uint32_t rows, uint32_t vecs_per_row,
                      uint32_t pitch_vecs, uint32_t* __restrict__ partial) {
     __shared__ uint32_t red[kAmaxThreads / 32];
+    griddep_launch();                     // the quantize pass may start its prologue
     uint32_t m2 = 0;
     const uint32_t total = rows * vecs_per_row;
     const uint32_t stride = gridDim.x * kAmaxThreads;
@@ -180,6 +181,10 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
         v1 = __ldg(src + 1);
     }
     init_d6(d6);
+    // x is final (the amax pass that may still be running only reads it);
+    // the partial maxima and every output are touched only after this wait.
+    griddep_wait();
+    griddep_launch();
     float amax;
     if (calib_amax != nullptr) {
         amax = *calib_amax;

@@ -147,8 +147,8 @@ def test_full_size_workloads_sampled_rows(name, fmt, every):
 
 SINGLE_CTA_SCRIPT = r"""
 import sys, numpy as np, torch
-sys.path.insert(0, %r)
-sys.path.insert(0, %r)
+sys.path.insert(0, ROOT_DIR)
+sys.path.insert(0, TEST_DIR)
 import test_gpu_gemm as t
 from gpu_common import check_gemm, sample_rows
 import workloads
@@ -174,6 +174,7 @@ def test_single_cta_kernel_on_pair_shapes():
     here = os.path.dirname(os.path.abspath(__file__))
     root = os.path.dirname(here)
     env = dict(os.environ, NVQ_GEMM_PAIRS="0")
-    out = subprocess.run([sys.executable, "-c", SINGLE_CTA_SCRIPT % (root, here)], env=env,
+    script = SINGLE_CTA_SCRIPT.replace("ROOT_DIR", repr(root)).replace("TEST_DIR", repr(here))
+    out = subprocess.run([sys.executable, "-c", script], env=env,
                          capture_output=True, text=True, timeout=600)
     assert out.returncode == 0 and out.stdout.strip().endswith("OK"), out.stdout + out.stderr
