@@ -9,16 +9,20 @@
 // of either operand ever exists (page "NVIDIA Blackwell平台FP4量化技术解析与图像
 // 生成优化", section 3.1: FP4 decoded to BF16 inside the SM).
 //
-// Structure: one persistent CTA per SM, 6 warps, output tiles 128 x BN.
+// Structure: one persistent CTA per SM, 7-9 warps, output tiles 128 x BN.
 //   warp 0  TMA producer: per pipeline stage one 128 x 128-byte tile of A,
 //           one BN x 128-byte tile of B (tensor maps, 128-byte swizzle), and
 //           the matching 512-byte scale tiles (plain bulk copies: the global
 //           128x4 tile order is exactly what tensor memory wants).
-//   warp 1  allocates tensor memory; one lane moves each stage's scale tiles
-//           to tensor memory (tcgen05.cp) and issues the MMAs into an FP32
+//   warp 1  allocates tensor memory; one lane issues the MMAs into an FP32
 //           accumulator in tensor memory; tcgen05.commit frees the stage.
 //           With two accumulators (BN = 128 or 192) the MMAs of tile i+1 run
 //           while the epilogue drains tile i.
+//   warps 6+  scale-factor copy warps, one per 128-row block of scales of a
+//           stage (A, then B): tcgen05.cp into a tensor-memory scale slot.
+//           Each copy instruction occupies its issuing thread for ~100
+//           cycles while the MMA warp's instructions run in parallel, so the
+//           copies are spread over several warps and kept off the MMA warp.
 //   warps 2-5  epilogue: tensor memory -> registers (tcgen05.ld), scale by
 //           alpha, add bias, round to BF16, stage 32 x 32 sub-tiles in
 //           64-byte-swizzled shared memory and write them with TMA stores.
@@ -58,7 +62,7 @@ struct GemmCfg {
     static constexpr int EPI_BUF_BYTES = 32 * 64;
     static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
     static constexpr int SMEM_LIMIT = 232448;
-    static constexpr int FIXED_BYTES = 1024 /*align*/ + 256 /*barriers*/ + EPI_BYTES;
+    static constexpr int FIXED_BYTES = 1024 /*align*/ + 512 /*barriers*/ + EPI_BYTES;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
     static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
@@ -67,15 +71,20 @@ struct GemmCfg {
     static constexpr int SFA_COLS = FMT == 0 ? 4 * KSTEPS : 4;
     static constexpr int SFB_COLS_PER_MMA = 4 * SFB_H;
     static constexpr int SFB_COLS = FMT == 0 ? SFB_COLS_PER_MMA * KSTEPS : SFB_COLS_PER_MMA;
-    // Scale factors are double-buffered by stage parity, so the copies of
-    // stage s+1 never overwrite columns the MMAs of stage s still read.
+    // Scale factors live in SF_SLOTS tensor-memory slots (SF_COLS columns
+    // each), filled by dedicated copy warps ahead of the MMAs.
     static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
     static constexpr int ACC_BUFS = (2 * BN + 2 * SF_COLS <= 512) ? 2 : 1;
-    static constexpr int TM_SFA = ACC_BUFS * BN;           // + (stage parity) * SF_COLS
-    static constexpr int TM_SFB = TM_SFA + SFA_COLS;
-    static constexpr int TM_USED = ACC_BUFS * BN + 2 * SF_COLS;
+    static constexpr int SF_SLOTS_FIT = (512 - ACC_BUFS * BN) / SF_COLS;
+    static constexpr int SF_SLOTS = SF_SLOTS_FIT < STAGES ? SF_SLOTS_FIT : STAGES;
+    static constexpr int TM_SF = ACC_BUFS * BN;            // slot j at TM_SF + j * SF_COLS
+    static constexpr int TM_USED = ACC_BUFS * BN + SF_SLOTS * SF_COLS;
     static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
-    static constexpr int THREADS = 192;
+    // copy jobs per stage: the A scales, then each 128-row block of B scales;
+    // one warp per job (a tcgen05.cp takes ~100 cycles to issue, so the jobs
+    // run in parallel warps, off the MMA warp's path)
+    static constexpr int SF_WARPS = 1 + SFB_H;
+    static constexpr int THREADS = 32 * (6 + SF_WARPS);
     // instruction descriptor: A/B format (E2M1 = 1 for mxf4nvf4, E4M3 = 0 for
     // mxf8f6f4) in bits 7-9 / 10-12, K-major A and B, N >> 3 in bits 17-22,
     // scale format (0 = UE4M3, 1 = UE8M0) in bit 23, M >> 4 in bits 24-28.
@@ -86,6 +95,7 @@ struct GemmCfg {
         ((uint32_t)(BM >> 4) << 24);
     static_assert(BN == 128 || BN == 192 || BN == 256, "tile width");
     static_assert(TM_USED <= 512, "tensor memory overflow");
+    static_assert(SF_SLOTS >= 2, "tensor memory too small for two scale slots");
     static_assert(STAGES >= 2, "shared memory too small for two stages");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory overflow");
 };
@@ -101,20 +111,46 @@ struct GemmParams {
     uint32_t sf_ctiles;          // (K / SF_BLOCK) / 4: scale tiles per 128 rows
 };
 
+// Scale-factor copy warp `job` (0: A scales, 1..SFB_H: B scale row block
+// job-1) for one pipeline stage: shared memory -> tensor-memory slot.
+template <typename C, bool PAIR>
+__device__ __forceinline__ void sf_copy_job(int job, uint32_t st, uint32_t sf_slot) {
+    if (job == 0) {
+#pragma unroll
+        for (int a = 0; a < C::SF_ATOMS; ++a) {
+            const uint64_t d = smem_desc(st + C::OFF_SFA + 512 * a, 16, 128, 0);
+            if (PAIR) tc_cp_pair_32x128b_warpx4(sf_slot + 4 * a, d);
+            else tc_cp_32x128b_warpx4(sf_slot + 4 * a, d);
+        }
+    } else {
+        const int h = job - 1;
+#pragma unroll
+        for (int a = 0; a < C::SF_ATOMS; ++a) {
+            const uint64_t d = smem_desc(st + C::OFF_SFB + h * C::SF_ATOMS * 512 + 512 * a, 16, 128, 0);
+            const uint32_t t = sf_slot + C::SFA_COLS + C::SFB_COLS_PER_MMA * a + 4 * h;
+            if (PAIR) tc_cp_pair_32x128b_warpx4(t, d);
+            else tc_cp_32x128b_warpx4(t, d);
+        }
+    }
+}
+
 template <int FMT, int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(GemmCfg<FMT, BN>::THREADS, 1)
 bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
               const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
     using C = GemmCfg<FMT, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
-    const uint32_t full0 = smem_u32(bars);
-    const uint32_t empty0 = full0 + 8 * C::STAGES;
-    const uint32_t tfull0 = empty0 + 8 * C::STAGES;     // [ACC_BUFS]
-    const uint32_t tempty0 = tfull0 + 8 * 2;            // [ACC_BUFS]
-    const uint32_t drain = tempty0 + 8 * 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+    const uint32_t full0 = smem_u32(bars);                 // [STAGES]  TMA -> copy warps, MMA
+    const uint32_t empty0 = full0 + 8 * C::STAGES;         // [STAGES]  MMA -> TMA
+    const uint32_t sffull0 = empty0 + 8 * C::STAGES;       // [SF_SLOTS] copy warps -> MMA
+    const uint32_t sfempty0 = sffull0 + 8 * C::SF_SLOTS;   // [SF_SLOTS] MMA -> copy warps
+    const uint32_t tfull0 = sfempty0 + 8 * C::SF_SLOTS;    // [2]  MMA -> epilogue
+    const uint32_t tempty0 = tfull0 + 8 * 2;               // [2]  epilogue -> MMA
+    const uint32_t drain = tempty0 + 8 * 2;                // MMA warp's own completion
+    const uint32_t sfdrain = drain + 8;                    // copy warps' own completion
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 2 * C::SF_SLOTS + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* never = abort_flag + 1;
 
@@ -124,11 +160,16 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
         }
+        for (int j = 0; j < C::SF_SLOTS; ++j) {
+            mbar_init(sffull0 + 8 * j, C::SF_WARPS);
+            mbar_init(sfempty0 + 8 * j, 1);
+        }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
             mbar_init(tempty0 + 8 * b, 4);
         }
         mbar_init(drain, 1);
+        mbar_init(sfdrain, C::SF_WARPS);
         *abort_flag = 0;
         *never = 0;
         fence_mbarrier_init();
@@ -150,6 +191,8 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     // touched before it has completed
     griddep_wait();
     const uint32_t num_tiles = p.num_m_blocks * p.num_n_blocks;
+    const uint32_t total_iters = ((num_tiles > blockIdx.x) ? (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0)
+                                 * p.num_k_tiles;
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
@@ -207,24 +250,16 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 const uint32_t d_tmem = tmem + buf * BN;
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt, ++it) {
                     const uint32_t s = it % C::STAGES, su = it / C::STAGES;
-                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
+                    const uint32_t slot = it % C::SF_SLOTS, sv = it / C::SF_SLOTS;
+                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs) ||
+                        !mbar_wait_bounded(sffull0 + 8 * slot, sv & 1, abort_flag, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
-                    const uint32_t sfa_t = tmem + C::TM_SFA + (it & 1) * C::SF_COLS;
+                    const uint32_t sfa_t = tmem + C::TM_SF + slot * C::SF_COLS;
                     const uint32_t sfb_t = sfa_t + C::SFA_COLS;
-                    // scale tiles: shared memory -> tensor memory (4 columns each)
-#pragma unroll
-                    for (int a = 0; a < C::SF_ATOMS; ++a)
-                        tc_cp_32x128b_warpx4(sfa_t + 4 * a, smem_desc(st + C::OFF_SFA + 512 * a, 16, 128, 0));
-#pragma unroll
-                    for (int h = 0; h < C::SFB_H; ++h)
-#pragma unroll
-                        for (int a = 0; a < C::SF_ATOMS; ++a)
-                            tc_cp_32x128b_warpx4(sfb_t + C::SFB_COLS_PER_MMA * a + 4 * h,
-                                                 smem_desc(st + C::OFF_SFB + h * C::SF_ATOMS * 512 + 512 * a, 16, 128, 0));
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k) {
                         const uint64_t adesc = smem_desc(st + k * C::MMA_K_BYTES, 16, 1024, 2);
@@ -239,7 +274,8 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                                         (sfb_t + sfb_shift) | ((uint32_t)k << 30), acc);
                         }
                     }
-                    tc_commit(empty0 + 8 * s);
+                    tc_commit(empty0 + 8 * s);        // shared-memory stage free
+                    tc_commit(sfempty0 + 8 * slot);   // scale slot free
                 }
                 if (!ok) break;
                 tc_commit(tfull0 + 8 * buf);
@@ -251,8 +287,32 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             tc_commit(drain);
             mbar_wait_bounded(drain, 0, never, kWaitLimitNs);
         }
+    } else if (warp >= 6) {
+        // ---------------------------------------------------------- scale-factor copy warps
+        if (lane == 0) {
+            const int job = warp - 6;
+            bool ok = true;
+            for (uint32_t it = 0; it < total_iters; ++it) {
+                const uint32_t s = it % C::STAGES, su = it / C::STAGES;
+                const uint32_t slot = it % C::SF_SLOTS, sv = it / C::SF_SLOTS;
+                if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs) ||
+                    (sv > 0 && !mbar_wait_bounded(sfempty0 + 8 * slot, (sv - 1) & 1, abort_flag, kWaitLimitNs))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                sf_copy_job<C, false>(job, smem_u32(smem + s * C::STAGE_BYTES), tmem + C::TM_SF + slot * C::SF_COLS);
+                tc_commit(sffull0 + 8 * slot);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+            }
+            tc_commit(sfdrain);
+            mbar_wait_bounded(sfdrain, 0, never, kWaitLimitNs);
+        }
     } else {
-        // ---------------------------------------------------------- epilogue
+        // ---------------------------------------------------------- epilogue (warps 2-5)
         const int q = warp & 3;                       // tensor-memory lane quarter of this warp
         const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
         uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * 2 * C::EPI_BUF_BYTES;

@@ -7,8 +7,9 @@
 //   scale tiles of its 128 A rows and of all BN B rows, and owns accumulator
 //   rows [128r, 128r + 128) in its own tensor memory.
 //   The leader (r = 0) alone issues tcgen05.cp (both CTAs' scales into both
-//   tensor memories) and the 256 x BN x K MMAs; its commits arrive on the
-//   barriers of both CTAs (.multicast::cluster on the commit).
+//   tensor memories, from its scale-copy warps) and the 256 x BN x K MMAs
+//   (from its MMA warp); the MMA commits arrive on the barriers of both CTAs
+//   (.multicast::cluster on the commit).
 //   Both CTAs' tile loads complete on the leader's full barrier
 //   (.cta_group::2 tensor loads; no load multicast anywhere).
 //   Each CTA drains its own accumulator half; the peer's epilogue warps
@@ -50,7 +51,7 @@ struct PairCfg {
     static constexpr int EPI_BUF_BYTES = 32 * 64;
     static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
     static constexpr int SMEM_LIMIT = 232448;
-    static constexpr int FIXED_BYTES = 1024 + 256 + EPI_BYTES;
+    static constexpr int FIXED_BYTES = 1024 + 512 + EPI_BYTES;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
     static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
@@ -60,10 +61,13 @@ struct PairCfg {
     static constexpr int SFB_COLS = FMT == 0 ? SFB_COLS_PER_MMA * KSTEPS : SFB_COLS_PER_MMA;
     static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
     static constexpr int ACC_BUFS = (2 * BN + 2 * SF_COLS <= 512) ? 2 : 1;
-    static constexpr int TM_SFA = ACC_BUFS * BN;
-    static constexpr int TM_USED = ACC_BUFS * BN + 2 * SF_COLS;
+    static constexpr int SF_SLOTS_FIT = (512 - ACC_BUFS * BN) / SF_COLS;
+    static constexpr int SF_SLOTS = SF_SLOTS_FIT < STAGES ? SF_SLOTS_FIT : STAGES;
+    static constexpr int TM_SF = ACC_BUFS * BN;
+    static constexpr int TM_USED = ACC_BUFS * BN + SF_SLOTS * SF_COLS;
     static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
-    static constexpr int THREADS = 192;
+    static constexpr int SF_WARPS = 1 + SFB_H;             // copy warps (used in the leader)
+    static constexpr int THREADS = 32 * (6 + SF_WARPS);
     static constexpr uint32_t IDESC =
         (FMT == 0 ? (1u << 7) | (1u << 10) : 0u) |
         ((uint32_t)(BN >> 3) << 17) |
@@ -71,12 +75,13 @@ struct PairCfg {
         ((uint32_t)(BM >> 4) << 24);
     static_assert(BN == 256, "pair tiles are 256 x 256");
     static_assert(TM_USED <= 512, "tensor memory overflow");
+    static_assert(SF_SLOTS >= 2, "tensor memory too small for two scale slots");
     static_assert(STAGES >= 2, "shared memory too small");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory overflow");
 };
 
 template <int FMT, int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(PairCfg<FMT, BN>::THREADS, 1)
 bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                    const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
@@ -86,10 +91,13 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
     const uint32_t full0 = smem_u32(bars);
     const uint32_t empty0 = full0 + 8 * C::STAGES;
-    const uint32_t tfull0 = empty0 + 8 * C::STAGES;
+    const uint32_t sffull0 = empty0 + 8 * C::STAGES;
+    const uint32_t sfempty0 = sffull0 + 8 * C::SF_SLOTS;
+    const uint32_t tfull0 = sfempty0 + 8 * C::SF_SLOTS;
     const uint32_t tempty0 = tfull0 + 8 * 2;
     const uint32_t drain = tempty0 + 8 * 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+    const uint32_t sfdrain = drain + 8;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 2 * C::SF_SLOTS + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* never = abort_flag + 1;
 
@@ -101,11 +109,16 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
         }
+        for (int j = 0; j < C::SF_SLOTS; ++j) {
+            mbar_init(sffull0 + 8 * j, C::SF_WARPS);
+            mbar_init(sfempty0 + 8 * j, 1);
+        }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
             mbar_init(tempty0 + 8 * b, 8);                 // 4 epilogue warps in each CTA
         }
         mbar_init(drain, 1);
+        mbar_init(sfdrain, C::SF_WARPS);
         *abort_flag = 0;
         *never = 0;
         fence_mbarrier_init();
@@ -129,6 +142,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
     // touched before it has completed
     griddep_wait();
     const uint32_t num_tiles = p.num_m_blocks * p.num_n_blocks;   // 256 x BN tiles
+    const uint32_t total_iters = ((num_tiles > pair) ? (num_tiles - pair + npairs - 1) / npairs : 0) * p.num_k_tiles;
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer (both CTAs)
@@ -186,23 +200,16 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 const uint32_t d_tmem = tmem + buf * BN;
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt, ++it) {
                     const uint32_t s = it % C::STAGES, su = it / C::STAGES;
-                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
+                    const uint32_t slot = it % C::SF_SLOTS, sv = it / C::SF_SLOTS;
+                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs) ||
+                        !mbar_wait_bounded(sffull0 + 8 * slot, sv & 1, abort_flag, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
-                    const uint32_t sfa_t = tmem + C::TM_SFA + (it & 1) * C::SF_COLS;
+                    const uint32_t sfa_t = tmem + C::TM_SF + slot * C::SF_COLS;
                     const uint32_t sfb_t = sfa_t + C::SFA_COLS;
-#pragma unroll
-                    for (int a = 0; a < C::SF_ATOMS; ++a)
-                        tc_cp_pair_32x128b_warpx4(sfa_t + 4 * a, smem_desc(st + C::OFF_SFA + 512 * a, 16, 128, 0));
-#pragma unroll
-                    for (int h = 0; h < C::SFB_H; ++h)
-#pragma unroll
-                        for (int a = 0; a < C::SF_ATOMS; ++a)
-                            tc_cp_pair_32x128b_warpx4(sfb_t + C::SFB_COLS_PER_MMA * a + 4 * h,
-                                                      smem_desc(st + C::OFF_SFB + h * C::SF_CHUNK + 512 * a, 16, 128, 0));
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k) {
                         const uint64_t adesc = smem_desc(st + k * C::MMA_K_BYTES, 16, 1024, 2);
@@ -218,6 +225,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                         }
                     }
                     tc_commit_pair_mc(empty0 + 8 * s, 0x3);     // frees the stage in both CTAs
+                    tc_commit_pair(sfempty0 + 8 * slot);         // scale slot free
                 }
                 if (!ok) break;
                 tc_commit_pair_mc(tfull0 + 8 * buf, 0x3);       // accumulator ready in both CTAs
@@ -228,6 +236,30 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             }
             tc_commit_pair(drain);
             mbar_wait_bounded(drain, 0, never, kWaitLimitNs);
+        }
+    } else if (warp >= 6) {
+        // ---------------------------------------------------------- scale-factor copy warps (leader)
+        if (lane == 0 && rank == 0) {
+            const int job = warp - 6;
+            bool ok = true;
+            for (uint32_t it = 0; it < total_iters; ++it) {
+                const uint32_t s = it % C::STAGES, su = it / C::STAGES;
+                const uint32_t slot = it % C::SF_SLOTS, sv = it / C::SF_SLOTS;
+                if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs) ||
+                    (sv > 0 && !mbar_wait_bounded(sfempty0 + 8 * slot, (sv - 1) & 1, abort_flag, kWaitLimitNs))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                sf_copy_job<C, true>(job, smem_u32(smem + s * C::STAGE_BYTES), tmem + C::TM_SF + slot * C::SF_COLS);
+                tc_commit_pair(sffull0 + 8 * slot);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+            }
+            tc_commit_pair(sfdrain);
+            mbar_wait_bounded(sfdrain, 0, never, kWaitLimitNs);
         }
     } else {
         // ---------------------------------------------------------- epilogue (both CTAs)
