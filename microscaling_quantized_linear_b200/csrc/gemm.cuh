@@ -9,7 +9,7 @@
 // of either operand ever exists (page "NVIDIA Blackwell平台FP4量化技术解析与图像
 // 生成优化", section 3.1: FP4 decoded to BF16 inside the SM).
 //
-// Structure: one persistent CTA per SM, 7-9 warps, output tiles 128 x BN.
+// Structure: one persistent CTA per SM, 12-13 warps, output tiles 128 x BN.
 //   warp 0  TMA producer: per pipeline stage one 128 x 128-byte tile of A,
 //           one BN x 128-byte tile of B (tensor maps, 128-byte swizzle), and
 //           the matching 512-byte scale tiles (plain bulk copies: the global
@@ -18,14 +18,15 @@
 //           accumulator in tensor memory; tcgen05.commit frees the stage.
 //           With two accumulators (BN = 128 or 192) the MMAs of tile i+1 run
 //           while the epilogue drains tile i.
-//   warps 6+  scale-factor copy warps, one per 128-row block of scales of a
+//   warps 10+ scale-factor copy warps, one per 128-row block of scales of a
 //           stage (A, then B): tcgen05.cp into a tensor-memory scale slot.
 //           Each copy instruction occupies its issuing thread for ~100
 //           cycles while the MMA warp's instructions run in parallel, so the
 //           copies are spread over several warps and kept off the MMA warp.
-//   warps 2-5  epilogue: tensor memory -> registers (tcgen05.ld), scale by
-//           alpha, add bias, round to BF16, stage 32 x 32 sub-tiles in
-//           64-byte-swizzled shared memory and write them with TMA stores.
+//   warps 2-9  epilogue, two warps per tensor-memory lane quarter: tensor
+//           memory -> registers (tcgen05.ld), scale by alpha, add bias,
+//           round to BF16, release the accumulator, then stage 32 x 32
+//           sub-tiles in 64-byte-swizzled shared memory for TMA stores.
 // Every mbarrier wait is bounded in wall time; a wait that gives up sets the
 // status word and an abort flag that releases the other roles.
 #pragma once
@@ -36,6 +37,72 @@
 namespace nvq {
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s per wait
+// Warp roles: 0 TMA producer, 1 MMA issuer, 2..9 epilogue (two warps per
+// tensor-memory lane quarter, each owning half of the tile's columns),
+// 10.. scale-factor copy warps.
+constexpr int kEpiWarps = 8;
+constexpr int kFirstSfWarp = 2 + kEpiWarps;
+
+// Drains one 32-row x BN/2-column share of an accumulator: all its tensor-
+// memory chunks are read (and rounded to BF16) first, then the accumulator
+// is released through release_bar, then the BF16 sub-tiles are written via
+// the warp's 64-byte-swizzled staging buffer and TMA stores.
+template <int BN>
+__device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half, int lane, float alpha,
+                                                  const __nv_bfloat16* bias_tile, uint8_t* staging,
+                                                  const CUtensorMap* tmap_d, int32_t row0, uint32_t n0,
+                                                  uint32_t release_bar, bool release_remote) {
+    constexpr int NC = BN / 64;                          // 32-column chunks per warp
+    const int c0 = half * (BN / 2);
+    uint32_t packed[NC][16];
+#pragma unroll
+    for (int j = 0; j < NC; j += 2) {
+        uint32_t r0[32], r1[32];
+        tc_ld_32x32b_x32(tmem_acc_q + c0 + 32 * j, r0);
+        if (j + 1 < NC) tc_ld_32x32b_x32(tmem_acc_q + c0 + 32 * (j + 1), r1);
+        tc_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (j + u >= NC) break;
+            const uint32_t* r = u ? r1 : r0;
+            const int c = c0 + 32 * (j + u);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                float v0 = __fmul_rn(__uint_as_float(r[2 * e]), alpha);
+                float v1 = __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha);
+                if (bias_tile) {
+                    const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(bias_tile + c + 2 * e);
+                    v0 = __fadd_rn(v0, __bfloat162float(bb.x));
+                    v1 = __fadd_rn(v1, __bfloat162float(bb.y));
+                }
+                const __nv_bfloat162 o = __floats2bfloat162_rn(v0, v1);
+                packed[j + u][e] = *reinterpret_cast<const uint32_t*>(&o);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+        if (release_remote) mbar_arrive_cluster(release_bar);
+        else mbar_arrive(release_bar);
+    }
+    const uint32_t swz = (uint32_t)((lane >> 1) & 3);     // 64-byte swizzle of this thread's row
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+        if (lane == 0) bulk_wait_group_read<0>();         // the previous store has read the buffer
+        __syncwarp();
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4*>(staging + lane * 64 + 16 * ((uint32_t)v ^ swz)) =
+                make_uint4(packed[j][4 * v], packed[j][4 * v + 1], packed[j][4 * v + 2], packed[j][4 * v + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmap_d, smem_u32(staging), (int32_t)(n0 + c0 + 32 * j), row0);
+            bulk_commit_group();
+        }
+    }
+}
 
 template <int FMT, int BN_>
 struct GemmCfg {
@@ -58,9 +125,9 @@ struct GemmCfg {
     static constexpr int OFF_B = A_BYTES;
     static constexpr int OFF_SFA = A_BYTES + B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
-    // epilogue staging: 4 warps x 2 buffers x (32 rows x 64 bytes)
+    // epilogue staging: 8 warps x (32 rows x 64 bytes)
     static constexpr int EPI_BUF_BYTES = 32 * 64;
-    static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
+    static constexpr int EPI_BYTES = kEpiWarps * EPI_BUF_BYTES;
     static constexpr int SMEM_LIMIT = 232448;
     static constexpr int FIXED_BYTES = 1024 /*align*/ + 512 /*barriers*/ + EPI_BYTES;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
@@ -84,7 +151,7 @@ struct GemmCfg {
     // one warp per job (a tcgen05.cp takes ~100 cycles to issue, so the jobs
     // run in parallel warps, off the MMA warp's path)
     static constexpr int SF_WARPS = 1 + SFB_H;
-    static constexpr int THREADS = 32 * (6 + SF_WARPS);
+    static constexpr int THREADS = 32 * (kFirstSfWarp + SF_WARPS);
     // instruction descriptor: A/B format (E2M1 = 1 for mxf4nvf4, E4M3 = 0 for
     // mxf8f6f4) in bits 7-9 / 10-12, K-major A and B, N >> 3 in bits 17-22,
     // scale format (0 = UE4M3, 1 = UE8M0) in bit 23, M >> 4 in bits 24-28.
@@ -166,7 +233,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
-            mbar_init(tempty0 + 8 * b, 4);
+            mbar_init(tempty0 + 8 * b, kEpiWarps);
         }
         mbar_init(drain, 1);
         mbar_init(sfdrain, C::SF_WARPS);
@@ -287,10 +354,10 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             tc_commit(drain);
             mbar_wait_bounded(drain, 0, never, kWaitLimitNs);
         }
-    } else if (warp >= 6) {
+    } else if (warp >= kFirstSfWarp) {
         // ---------------------------------------------------------- scale-factor copy warps
         if (lane == 0) {
-            const int job = warp - 6;
+            const int job = warp - kFirstSfWarp;
             bool ok = true;
             for (uint32_t it = 0; it < total_iters; ++it) {
                 const uint32_t s = it % C::STAGES, su = it / C::STAGES;
@@ -312,12 +379,12 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             mbar_wait_bounded(sfdrain, 0, never, kWaitLimitNs);
         }
     } else {
-        // ---------------------------------------------------------- epilogue (warps 2-5)
+        // ---------------------------------------------------------- epilogue (warps 2-9)
         const int q = warp & 3;                       // tensor-memory lane quarter of this warp
+        const int half = (warp - 2) >> 2;             // which half of the tile's columns
         const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
-        uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * 2 * C::EPI_BUF_BYTES;
-        const uint32_t swz = (uint32_t)((lane >> 1) & 3);     // 64-byte swizzle of this thread's row
-        uint32_t t_local = 0, nstore = 0;
+        uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * C::EPI_BUF_BYTES;
+        uint32_t t_local = 0;
         for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t_local) {
             const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
             const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
@@ -328,47 +395,10 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 break;
             }
             tc_fence_after();
-            const int32_t row0 = (int32_t)(mb * C::BM + 32 * q);
             const uint32_t n0 = nb * BN;
-            const __nv_bfloat16* brow = p.bias ? p.bias + n0 : nullptr;
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
-                uint32_t r[32];
-                tc_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + buf * BN + c, r);
-                tc_wait_ld();
-                if (c + 32 == BN) {                   // accumulator fully read: hand it back to the MMA warp
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
-                }
-                uint32_t packed[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float v0 = __fmul_rn(__uint_as_float(r[2 * j]), alpha);
-                    float v1 = __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha);
-                    if (brow) {
-                        const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(brow + c + 2 * j);
-                        v0 = __fadd_rn(v0, __bfloat162float(bb.x));
-                        v1 = __fadd_rn(v1, __bfloat162float(bb.y));
-                    }
-                    const __nv_bfloat162 o = __floats2bfloat162_rn(v0, v1);
-                    packed[j] = *reinterpret_cast<const uint32_t*>(&o);
-                }
-                uint8_t* sb = staging + (nstore & 1) * C::EPI_BUF_BYTES;
-                if (lane == 0) bulk_wait_group_read<1>();   // the store that last used this buffer has read it
-                __syncwarp();
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    *reinterpret_cast<uint4*>(sb + lane * 64 + 16 * ((uint32_t)j ^ swz)) =
-                        make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmap_d, smem_u32(sb), (int32_t)(n0 + c), row0);
-                    bulk_commit_group();
-                }
-                ++nstore;
-            }
+            drain_accumulator<BN>(tmem + ((uint32_t)(32 * q) << 16) + buf * BN, half, lane, alpha,
+                                  p.bias ? p.bias + n0 : nullptr, staging, &tmap_d,
+                                  (int32_t)(mb * C::BM + 32 * q), n0, tempty0 + 8 * buf, false);
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();

@@ -49,7 +49,7 @@ struct PairCfg {
     static constexpr int OFF_SFA = A_BYTES + B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
     static constexpr int EPI_BUF_BYTES = 32 * 64;
-    static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
+    static constexpr int EPI_BYTES = kEpiWarps * EPI_BUF_BYTES;
     static constexpr int SMEM_LIMIT = 232448;
     static constexpr int FIXED_BYTES = 1024 + 512 + EPI_BYTES;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
@@ -67,7 +67,7 @@ struct PairCfg {
     static constexpr int TM_USED = ACC_BUFS * BN + SF_SLOTS * SF_COLS;
     static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
     static constexpr int SF_WARPS = 1 + SFB_H;             // copy warps (used in the leader)
-    static constexpr int THREADS = 32 * (6 + SF_WARPS);
+    static constexpr int THREADS = 32 * (kFirstSfWarp + SF_WARPS);
     static constexpr uint32_t IDESC =
         (FMT == 0 ? (1u << 7) | (1u << 10) : 0u) |
         ((uint32_t)(BN >> 3) << 17) |
@@ -115,7 +115,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
-            mbar_init(tempty0 + 8 * b, 8);                 // 4 epilogue warps in each CTA
+            mbar_init(tempty0 + 8 * b, 2 * kEpiWarps);     // the epilogue warps of both CTAs
         }
         mbar_init(drain, 1);
         mbar_init(sfdrain, C::SF_WARPS);
@@ -237,10 +237,10 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             tc_commit_pair(drain);
             mbar_wait_bounded(drain, 0, never, kWaitLimitNs);
         }
-    } else if (warp >= 6) {
+    } else if (warp >= kFirstSfWarp) {
         // ---------------------------------------------------------- scale-factor copy warps (leader)
         if (lane == 0 && rank == 0) {
-            const int job = warp - 6;
+            const int job = warp - kFirstSfWarp;
             bool ok = true;
             for (uint32_t it = 0; it < total_iters; ++it) {
                 const uint32_t s = it % C::STAGES, su = it / C::STAGES;
@@ -262,12 +262,12 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             mbar_wait_bounded(sfdrain, 0, never, kWaitLimitNs);
         }
     } else {
-        // ---------------------------------------------------------- epilogue (both CTAs)
+        // ---------------------------------------------------------- epilogue (both CTAs, warps 2-9)
         const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
         const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
-        uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * 2 * C::EPI_BUF_BYTES;
-        const uint32_t swz = (uint32_t)((lane >> 1) & 3);
-        uint32_t t_local = 0, nstore = 0;
+        uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * C::EPI_BUF_BYTES;
+        uint32_t t_local = 0;
         for (uint32_t tile = pair; tile < num_tiles; tile += npairs, ++t_local) {
             const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
             const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
@@ -278,47 +278,11 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 break;
             }
             tc_fence_after();
-            const int32_t row0 = (int32_t)(mb * 256 + 128 * rank + 32 * q);
             const uint32_t n0 = nb * BN;
-            const __nv_bfloat16* brow = p.bias ? p.bias + n0 : nullptr;
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
-                uint32_t r[32];
-                tc_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + buf * BN + c, r);
-                tc_wait_ld();
-                if (c + 32 == BN) {                        // accumulator half read: release it
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty0 + 8 * buf, 0));
-                }
-                uint32_t packed[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float v0 = __fmul_rn(__uint_as_float(r[2 * j]), alpha);
-                    float v1 = __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha);
-                    if (brow) {
-                        const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(brow + c + 2 * j);
-                        v0 = __fadd_rn(v0, __bfloat162float(bb.x));
-                        v1 = __fadd_rn(v1, __bfloat162float(bb.y));
-                    }
-                    const __nv_bfloat162 o = __floats2bfloat162_rn(v0, v1);
-                    packed[j] = *reinterpret_cast<const uint32_t*>(&o);
-                }
-                uint8_t* sb = staging + (nstore & 1) * C::EPI_BUF_BYTES;
-                if (lane == 0) bulk_wait_group_read<1>();
-                __syncwarp();
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    *reinterpret_cast<uint4*>(sb + lane * 64 + 16 * ((uint32_t)j ^ swz)) =
-                        make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmap_d, smem_u32(sb), (int32_t)(n0 + c), row0);
-                    bulk_commit_group();
-                }
-                ++nstore;
-            }
+            drain_accumulator<BN>(tmem + ((uint32_t)(32 * q) << 16) + buf * BN, half, lane, alpha,
+                                  p.bias ? p.bias + n0 : nullptr, staging, &tmap_d,
+                                  (int32_t)(mb * 256 + 128 * rank + 32 * q), n0,
+                                  mapa_shared(tempty0 + 8 * buf, 0), true);
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();
