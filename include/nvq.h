@@ -191,6 +191,41 @@ NVQ_API int nvq_device_status(nvq_stream_t stream);
 NVQ_API const char* nvq_status_string(int code);
 
 /*
+ * nvfp4_quantize_noalloc -- nvfp4_quantize for callers that cannot allocate
+ * device memory.  The paper has no counterpart to this entry point.
+ *
+ * Some callers cannot call cudaMalloc, nor hand the library a workspace:
+ * code that runs inside a host framework which owns all device memory and
+ * offers its plug-ins neither an allocator nor a scratch buffer, or code on
+ * a latency-critical path where a device allocation (and the synchronisation
+ * it can imply) is not acceptable.  This variant takes the same inputs and
+ * outputs as nvfp4_quantize on the dynamic path (no calibrated amax) and
+ * needs no workspace: its scratch -- the amax pass's partial maxima, at most
+ * NVQ_NOALLOC_MAX_PARTIALS 32-bit words (4 KB) -- is a static array inside
+ * the library, resident on every GPU that loads the library until the
+ * process exits.  It allocates nothing and calls no allocating routine.
+ *
+ *   Same arguments, layouts, arithmetic and results as nvfp4_quantize with
+ *   calib_amax == NULL (bit-identical codes, scales and global scale).
+ *   The first call on a device (the current device) looks up the scratch
+ *   array's device address; make that first call before any stream capture.
+ *   Every call on a device shares the one scratch array: two calls whose
+ *   work can overlap on the GPU (different streams, no ordering between
+ *   them) race on it and may produce wrong results.  Calls ordered on one
+ *   stream are safe.  The scratch keeps the last call's contents; nothing in
+ *   it needs to start at zero, because every call rewrites every partial it
+ *   reads.
+ *   Returns NVQ_ERR_SHAPE, launching nothing, if the amax pass would need
+ *   more partial maxima than the scratch holds (it never launches more than
+ *   NVQ_NOALLOC_MAX_PARTIALS CTAs, so this only guards the limit), plus the
+ *   errors of nvfp4_quantize.
+ */
+#define NVQ_NOALLOC_MAX_PARTIALS 1024
+NVQ_API int nvfp4_quantize_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                   uint8_t* codes, uint8_t* scales, float* global_scale,
+                                   nvq_stream_t stream);
+
+/*
  * nvq_probe_convert -- conversion self-test (no counterpart on the pages).
  * Runs the device's FP32 -> E2M1 and FP32 -> E4M3 round-to-nearest-even,
  * saturating conversions that the quantize kernels use on n inputs, so

@@ -57,10 +57,14 @@ _lib.nvq_status_string.restype = ctypes.c_char_p
 _lib.nvq_status_string.argtypes = [ctypes.c_int]
 _lib.nvq_probe_convert.restype = ctypes.c_int
 _lib.nvq_probe_convert.argtypes = [_vp, _i64, _vp, _vp, _vp]
+_lib.nvfp4_quantize_noalloc.restype = ctypes.c_int
+_lib.nvfp4_quantize_noalloc.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]
 
 EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_quantize",
             "mxfp8_quantize", "quantize_weight", "block_scaled_linear", "nvq_device_status",
-            "nvq_status_string", "nvq_probe_convert")
+            "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc")
+
+NOALLOC_MAX_PARTIALS = 1024
 
 
 class NvqError(RuntimeError):
@@ -132,6 +136,16 @@ def nvfp4_quantize(x, codes=None, scales=None, global_scale=None, calib_amax=Non
         workspace = new_workspace(dev)
     _check(_lib.nvfp4_quantize(_ptr(x), M, K, _pitch(x), _ptr(codes), _ptr(scales), _ptr(global_scale),
                                _ptr(calib_amax), _ptr(workspace), _stream(stream, dev)), "nvfp4_quantize")
+    return codes, scales, global_scale
+
+
+def nvfp4_quantize_noalloc(x, codes, scales, global_scale, stream=None):
+    """nvfp4_quantize (dynamic amax) through the entry point that needs no
+    workspace and allocates nothing: its scratch is a static array inside the
+    library.  The outputs must be given (this call allocates nothing)."""
+    M, K = x.shape
+    _check(_lib.nvfp4_quantize_noalloc(_ptr(x), M, K, _pitch(x), _ptr(codes), _ptr(scales), _ptr(global_scale),
+                                       _stream(stream, x.device)), "nvfp4_quantize_noalloc")
     return codes, scales, global_scale
 
 

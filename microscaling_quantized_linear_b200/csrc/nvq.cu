@@ -27,6 +27,13 @@ namespace nvq {
 // cleared by nvq_device_status().
 __device__ unsigned int g_status;
 
+// Scratch of nvfp4_quantize_noalloc: the amax pass's partial maxima.  A
+// static device array, so the entry point never allocates; its device
+// address is looked up by the entry point's first call on each device.
+// Shared by every call on a device; fully rewritten by each call's amax pass
+// before it is read.
+static __device__ __align__(256) uint32_t g_noalloc_partials[NVQ_NOALLOC_MAX_PARTIALS];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -515,6 +522,62 @@ int nvq_probe_convert(const float* in, int64_t n, uint8_t* e2m1_out, uint8_t* e4
     probe_convert_kernel<<<grid, kQuantThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         in, (uint32_t)n, e2m1_out, e4m3_out);
     return launch_status();
+}
+
+int nvfp4_quantize_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
+                           float* global_scale, nvq_stream_t stream) {
+    // Device address of the static scratch array, looked up on this entry
+    // point's first call on each device (with that device current).
+    static uint32_t* scratch[kMaxDevices] = {};
+    int rc = check_quant_shape(NVQ_NVFP4, M, K, ldx);
+    if (rc) return rc;
+    if (M == 0) return NVQ_OK;
+    if (!x || !codes || !scales || !global_scale) return NVQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return NVQ_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(global_scale) & 3u) return NVQ_ERR_ALIGN;
+    DeviceInfo* d = nullptr;
+    if ((rc = device_info(&d))) return rc;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVQ_ERR_CUDA;
+    uint32_t* partials = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!scratch[dev]) {
+            void* ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_noalloc_partials) != cudaSuccess) return NVQ_ERR_CUDA;
+            scratch[dev] = static_cast<uint32_t*>(ptr);
+        }
+        partials = scratch[dev];
+    }
+    // the amax pass writes one partial per CTA: it must fit the static scratch
+    const uint64_t vectors = (uint64_t)M * (uint64_t)(K / 8);
+    uint64_t grid = (vectors + 8 * kAmaxThreads - 1) / (8 * kAmaxThreads);
+    const uint64_t cap = (uint64_t)d->num_sms * 8 < (uint64_t)kMaxAmaxPartials ? (uint64_t)d->num_sms * 8
+                                                                               : (uint64_t)kMaxAmaxPartials;
+    if (grid > cap) grid = cap;
+    if (grid > NVQ_NOALLOC_MAX_PARTIALS) return NVQ_ERR_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t npartial = 0;
+    if ((rc = launch_amax(x, M, K, ldx, partials, d->num_sms, s, &npartial))) return rc;
+    const uint32_t nblk = (uint32_t)(K / 16);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(quant_grid((uint64_t)M * nblk, d->num_sms));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const uint16_t* xp = static_cast<const uint16_t*>(x);
+    const uint32_t* pp = partials;
+    const float* no_calib = nullptr;
+    if (cudaLaunchKernelEx(&cfg, nvfp4_quantize_kernel, xp, (uint32_t)M, nblk, (uint32_t)ldx, codes, scales,
+                           global_scale, pp, npartial, no_calib, d->status) != cudaSuccess) {
+        cudaGetLastError();
+        return NVQ_ERR_CUDA;
+    }
+    return NVQ_OK;
 }
 
 }  // extern "C"

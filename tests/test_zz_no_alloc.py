@@ -1,0 +1,80 @@
+"""The quantizer entry point that allocates nothing (nvfp4_quantize_noalloc).
+
+Some callers cannot call cudaMalloc or hand the library a workspace: code
+inside a host framework that owns all device memory and gives its plug-ins
+no allocator or scratch buffer, or code on a latency-critical path that must
+not allocate.  For them the library offers a variant of the dynamic NVFP4
+quantizer whose scratch (the amax pass's partial maxima) is a static array
+inside the library.  Its results must be those of nvfp4_quantize with a
+workspace, bit for bit, call after call: the shared scratch keeps the last
+call's contents, so two calls in a row on different tensors also check that
+nothing stale leaks from one call into the next.
+
+This file is named to be collected last, and it works both on its own in a
+fresh process (its first call is the first on the device) and after the
+rest of the suite.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+nvq = pytest.importorskip("microscaling_quantized_linear_b200")
+
+
+def quantize_noalloc_cabi(x):
+    """Calls the C entry point directly with caller-allocated outputs."""
+    M, K = x.shape
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty(nvq.scale_bytes("nvfp4", M, K), dtype=torch.uint8, device="cuda")
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = nvq._lib.nvfp4_quantize_noalloc(ctypes.c_void_p(x.data_ptr()), M, K, x.stride(0),
+                                         ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                                         ctypes.c_void_p(g.data_ptr()), stream)
+    assert rc == 0, nvq.status_string(rc)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy(), g.cpu().numpy()
+
+
+def quantize_with_workspace(x):
+    codes, scales, g = nvq.nvfp4_quantize(x, workspace=nvq.new_workspace())
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy(), g.cpu().numpy()
+
+
+def assert_same(a, b):
+    # codes, scales and global scale are integers / exactly rounded: bit-exact
+    for u, v, name in zip(a, b, ("codes", "scales", "global scale")):
+        assert u.shape == v.shape and np.array_equal(u.view(np.uint8), v.view(np.uint8)), name
+
+
+def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
+    # A large-amax tensor, then a small-amax one, then the first again: each
+    # call of the no-alloc entry point must reproduce the workspace entry point.
+    tensors = [workloads.activation("ffup").cuda(),                 # outliers x50
+               workloads.normal(4608, 3072, seed=5, std=1e-3).cuda(),
+               workloads.activation("tiny").cuda()]
+    tensors.append(tensors[0])
+    for x in tensors:
+        first = quantize_noalloc_cabi(x)
+        second = quantize_noalloc_cabi(x)
+        want = quantize_with_workspace(x)
+        assert_same(first, want)
+        assert_same(second, want)
+    assert nvq.device_status() == 0
+
+
+def test_noalloc_rejects_bad_arguments_without_launching():
+    x = workloads.activation("tiny").cuda()
+    M, K = x.shape
+    null = ctypes.c_void_p(0)
+    rc = nvq._lib.nvfp4_quantize_noalloc(ctypes.c_void_p(x.data_ptr()), M - 1, K, K, null, null, null, null)
+    assert rc == -2                      # rows not a multiple of 128
+    rc = nvq._lib.nvfp4_quantize_noalloc(ctypes.c_void_p(x.data_ptr()), M, K, K, null, null, null, null)
+    assert rc == -1                      # outputs must be given
