@@ -125,7 +125,7 @@ int launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, uint32_t* pa
 
 uint32_t quant_grid(uint64_t units, int num_sms) {
     uint64_t blocks = (units + kQuantThreads - 1) / kQuantThreads;
-    const uint64_t cap = (uint64_t)num_sms * 8;      // 8 resident 256-thread CTAs per SM
+    const uint64_t cap = (uint64_t)num_sms * 6;      // 6 resident 256-thread CTAs per SM
     if (blocks > cap) blocks = cap;
     return (uint32_t)(blocks < 1 ? 1 : blocks);
 }

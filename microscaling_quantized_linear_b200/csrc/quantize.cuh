@@ -133,18 +133,17 @@ amax_partials_kernel(const uint4* __restrict__ x, uint32_t rows, uint32_t vecs_p
     const uint32_t stride = gridDim.x * kAmaxThreads;
     uint32_t i = blockIdx.x * kAmaxThreads + threadIdx.x;
     if (pitch_vecs == vecs_per_row) {
-        // contiguous: 8 independent 16-byte loads in flight per thread
-        for (; i + 7 * stride < total; i += 8 * stride) {
+        // contiguous: batches of 8 independent 16-byte loads, all issued
+        // before any is used (predicated at the tail, so a thread with fewer
+        // than 8 vectors still has all of them in flight at once)
+        for (; i < total; i += 8 * stride) {
             uint4 v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = __ldg(x + i + u * stride);
+            for (int u = 0; u < 8; ++u)
+                v[u] = (i + u * stride < total) ? __ldg(x + i + u * stride) : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 m2 = absmax2(absmax2(absmax2(absmax2(m2, v[u].x), v[u].y), v[u].z), v[u].w);
-        }
-        for (; i < total; i += stride) {
-            uint4 v = __ldg(x + i);
-            m2 = absmax2(absmax2(absmax2(absmax2(m2, v.x), v.y), v.z), v.w);
         }
     } else {
         for (; i < total; i += stride) {
@@ -158,10 +157,11 @@ amax_partials_kernel(const uint4* __restrict__ x, uint32_t rows, uint32_t vecs_p
 }
 
 // ------------------------------------------------------------------ NVFP4, streaming
-// One thread = one 16-element block per iteration.  Block b is (row b / nblk,
-// column b % nblk), nblk = K / 16; its codes are bytes [8b, 8b + 8).  The amax
-// is the reduction of the two-pass partials, or *calib_amax.
-__global__ void __launch_bounds__(kQuantThreads, 8)
+// One thread = two 16-element blocks per iteration (b and b + stride, both
+// loaded before either is computed).  Block b is (row b / nblk, column
+// b % nblk), nblk = K / 16; its codes are bytes [8b, 8b + 8).  The amax is the
+// reduction of the two-pass partials, or *calib_amax.
+__global__ void __launch_bounds__(kQuantThreads, 6)
 nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nblk, uint32_t ldx,
                       uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ g_dec_out,
                       const uint32_t* __restrict__ partial, uint32_t npartial,
@@ -173,12 +173,22 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
     const uint32_t qs = stride / nblk, rs = stride - qs * nblk;
     uint32_t b = blockIdx.x * kQuantThreads + threadIdx.x;
     uint32_t r = b / nblk, c = b - r * nblk;
-    // the first block's loads do not depend on the amax: issue them first
-    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-    if (b < total) {
-        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
-        v0 = __ldg(src);
-        v1 = __ldg(src + 1);
+    // Each iteration handles blocks b and b + stride; (r1, c1) is the second.
+    uint32_t r1 = r + qs, c1 = c + rs;
+    if (c1 >= nblk) {
+        c1 -= nblk;
+        ++r1;
+    }
+    // the first iteration's loads do not depend on the amax: issue them first
+    uint4 v[4];
+    const uint4 zero4 = make_uint4(0, 0, 0, 0);
+    {
+        const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
+        const uint4* s1 = reinterpret_cast<const uint4*>(x + (size_t)r1 * ldx + (size_t)c1 * 16);
+        v[0] = b < total ? __ldg(s0) : zero4;
+        v[1] = b < total ? __ldg(s0 + 1) : zero4;
+        v[2] = b + stride < total ? __ldg(s1) : zero4;
+        v[3] = b + stride < total ? __ldg(s1 + 1) : zero4;
     }
     init_d6(d6);
     // x is final (the amax pass that may still be running only reads it);
@@ -201,32 +211,47 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
     __syncthreads();
 
     const uint32_t ctiles = nblk >> 2;
+    const uint32_t stride2 = 2 * stride, qs2 = stride2 / nblk, rs2 = stride2 - qs2 * nblk;
     for (bool first = true; b - threadIdx.x < total; first = false) {
-        const bool active = b < total;       // whole warps stay in the loop for the shuffles
-        if (active && !first) {
-            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
-            v0 = __ldg(src);
-            v1 = __ldg(src + 1);
+        if (!first) {
+            const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
+            const uint4* s1 = reinterpret_cast<const uint4*>(x + (size_t)r1 * ldx + (size_t)c1 * 16);
+            v[0] = b < total ? __ldg(s0) : zero4;
+            v[1] = b < total ? __ldg(s0 + 1) : zero4;
+            v[2] = b + stride < total ? __ldg(s1) : zero4;
+            v[3] = b + stride < total ? __ldg(s1 + 1) : zero4;
         }
-        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        uint32_t lo, hi;
-        const uint32_t sc = nvfp4_block(block16_max(w), w, g_enc, d6, rtab, lo, hi);
-        // gather the scales of 4 neighbouring blocks (c % 4 == 0..3, same row)
-        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
-        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
-        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
-        if (active) {
-            *reinterpret_cast<uint2*>(codes + (size_t)b * 8) = make_uint2(lo, hi);
-            if ((c & 3u) == 0)
-                *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r, c, ctiles)) =
-                    sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const uint32_t bu = b + u * stride, ru = u ? r1 : r, cu = u ? c1 : c;
+            const bool active = bu < total;   // whole warps stay in the loop for the shuffles
+            const uint4 p0 = v[2 * u], p1 = v[2 * u + 1];
+            const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            uint32_t lo, hi;
+            const uint32_t sc = nvfp4_block(block16_max(w), w, g_enc, d6, rtab, lo, hi);
+            // gather the scales of 4 neighbouring blocks (c % 4 == 0..3, same row)
+            const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
+            const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
+            const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
+            if (active) {
+                *reinterpret_cast<uint2*>(codes + (size_t)bu * 8) = make_uint2(lo, hi);
+                if ((cu & 3u) == 0)
+                    *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(ru, cu, ctiles)) =
+                        sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            }
         }
-        b += stride;
-        r += qs;
-        c += rs;
+        b += stride2;
+        r += qs2;
+        c += rs2;
         if (c >= nblk) {
             c -= nblk;
             ++r;
+        }
+        r1 += qs2;
+        c1 += rs2;
+        if (c1 >= nblk) {
+            c1 -= nblk;
+            ++r1;
         }
     }
 }
