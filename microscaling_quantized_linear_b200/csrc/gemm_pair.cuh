@@ -1,7 +1,9 @@
 // gemm_pair.cuh -- block-scaled GEMM on CTA pairs (tcgen05 cta_group::2).
 //
 // Same product as gemm.cuh, D = bf16(alpha * A . B^T + bias), on output tiles
-// of 256 x BN computed by a cluster of two CTAs on two SMs:
+// of 256 x BN (BN = 256, or 192 with two tensor-memory accumulators so the
+// epilogue of one tile overlaps the MMAs of the next) computed by a cluster
+// of two CTAs on two SMs:
 //   CTA r (r = 0, 1) stages rows [128r, 128r + 128) of the A tile and rows
 //   [r BN/2, (r+1) BN/2) of the B tile in its own shared memory, holds the
 //   scale tiles of its 128 A rows and of all BN B rows, and owns accumulator
@@ -38,7 +40,7 @@ struct PairCfg {
     static constexpr int SF_BLOCK = FMT == 0 ? 16 : 32;
     static constexpr int SF_ATOMS = BK / SF_BLOCK / 4;
     static constexpr int SF_CHUNK = SF_ATOMS * 512;          // scale bytes per 128 rows per stage
-    static constexpr int SFB_H = BN / 128;                   // 128-row scale tiles of the B tile
+    static constexpr int SFB_H = 2;                          // 128-row scale tiles spanned by the B tile
     static constexpr int A_BYTES = 128 * KBYTES;
     static constexpr int B_BYTES = BN_HALF * KBYTES;
     static constexpr int SFA_BYTES = SF_CHUNK;
@@ -73,7 +75,7 @@ struct PairCfg {
         ((uint32_t)(BN >> 3) << 17) |
         (FMT == 0 ? 0u : (1u << 23)) |
         ((uint32_t)(BM >> 4) << 24);
-    static_assert(BN == 256, "pair tiles are 256 x 256");
+    static_assert(BN == 256 || BN == 192, "pair tiles are 256 x 256 or 256 x 192");
     static_assert(TM_USED <= 512, "tensor memory overflow");
     static_assert(SF_SLOTS >= 2, "tensor memory too small for two scale slots");
     static_assert(STAGES >= 2, "shared memory too small");
@@ -154,7 +156,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 const int32_t arow = (int32_t)(mb * 256 + 128 * rank);
                 const int32_t brow = (int32_t)(nb * BN + C::BN_HALF * rank);
                 const uint32_t sfa_atom = mb * 2 + rank;              // this CTA's 128 A rows
-                const uint32_t sfb_atom = nb * (BN / 128);
+                const uint32_t sfb_atom = (nb * BN) / 128;            // first scale tile of the B tile
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt) {
                     const uint32_t s = it % C::STAGES, use = it / C::STAGES;
                     if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
@@ -198,6 +200,8 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + buf * BN;
+                // a 192-wide B tile may start half-way through a 128-row scale tile
+                const uint32_t sfb_shift = (((tile / p.num_m_blocks) * BN) % 128) / 32;
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt, ++it) {
                     const uint32_t s = it % C::STAGES, su = it / C::STAGES;
                     const uint32_t slot = it % C::SF_SLOTS, sv = it / C::SF_SLOTS;
@@ -217,11 +221,11 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                         const uint32_t acc = (kt | (uint32_t)k) != 0;
                         if (FMT == 0) {
                             tc_mma_nvf4_pair(d_tmem, adesc, bdesc, C::IDESC, sfa_t + 4 * k,
-                                             sfb_t + C::SFB_COLS_PER_MMA * k, acc);
+                                             sfb_t + C::SFB_COLS_PER_MMA * k + sfb_shift, acc);
                         } else {
                             const uint32_t id = C::IDESC | ((uint32_t)k << 29) | ((uint32_t)k << 4);
                             tc_mma_mxf8_pair(d_tmem, adesc, bdesc, id, sfa_t | ((uint32_t)k << 30),
-                                             sfb_t | ((uint32_t)k << 30), acc);
+                                             (sfb_t + sfb_shift) | ((uint32_t)k << 30), acc);
                         }
                     }
                     tc_commit_pair_mc(empty0 + 8 * s, 0x3);     // frees the stage in both CTAs

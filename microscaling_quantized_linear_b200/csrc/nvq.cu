@@ -44,7 +44,7 @@ struct DeviceInfo {
     int num_sms = 0;
     unsigned int* status = nullptr;
     bool gemm_attr[2][3] = {{false, false, false}, {false, false, false}};
-    bool pair_attr[2] = {false, false};
+    bool pair_attr[2][2] = {{false, false}, {false, false}};
     bool fused_attr = false;
 };
 
@@ -282,12 +282,12 @@ int encode_scale_map(CUtensorMap* map, const void* scales, size_t bytes, uint32_
     return r == CUDA_SUCCESS ? NVQ_OK : NVQ_ERR_CUDA;
 }
 
-// 256 x 256 tiles on CTA pairs (M % 256 == 0, N % 256 == 0).
-template <int FMT>
+// 256 x BN tiles on CTA pairs (M % 256 == 0, N % BN == 0).
+template <int FMT, int BN>
 int launch_gemm_pair(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                      const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
                      void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
-    using C = PairCfg<FMT, 256>;
+    using C = PairCfg<FMT, BN>;
     const int64_t kbytes = FMT == 0 ? K / 2 : K;
     const int fmt = FMT == 0 ? NVQ_NVFP4 : NVQ_MXFP8;
     CUtensorMap ma, mb, msa, msb, md;
@@ -297,14 +297,14 @@ int launch_gemm_pair(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_sca
     if ((rc = encode_scale_map(&msa, a_scales, nvq_scale_bytes(fmt, M, K), C::SF_CHUNK / 256))) return rc;
     if ((rc = encode_scale_map(&msb, b_scales, nvq_scale_bytes(fmt, N, K), C::SF_CHUNK / 256))) return rc;
     if ((rc = encode_out_map(&md, out, M, N, ldo))) return rc;
-    auto kern = bsgemm_pair_kernel<FMT, 256>;
+    auto kern = bsgemm_pair_kernel<FMT, BN>;
     {
         std::lock_guard<std::mutex> lock(g_mu);
-        if (!d->pair_attr[FMT]) {
+        if (!d->pair_attr[FMT][BN == 256]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
                 cudaSuccess)
                 return NVQ_ERR_CUDA;
-            d->pair_attr[FMT] = true;
+            d->pair_attr[FMT][BN == 256] = true;
         }
     }
     GemmParams p;
@@ -315,7 +315,7 @@ int launch_gemm_pair(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_sca
     p.bias = static_cast<const __nv_bfloat16*>(bias);
     p.status = d->status;
     p.num_m_blocks = (uint32_t)(M / 256);
-    p.num_n_blocks = (uint32_t)(N / 256);
+    p.num_n_blocks = (uint32_t)(N / BN);
     p.num_k_tiles = (uint32_t)(K / C::BK);
     p.sf_ctiles = (uint32_t)(K / C::SF_BLOCK / 4);
     const uint32_t tiles = p.num_m_blocks * p.num_n_blocks;
@@ -458,14 +458,23 @@ int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_sca
     // Tile width: 256 when N allows it (fewest scale-factor copies per MMA),
     // else 192 (two tensor-memory accumulators), else 128 (two).
     const int bn = (N % 256 == 0) ? 256 : (N % 384 == 0) ? 192 : 128;
-    // CTA pairs (256 x 256 tiles) when both M and N allow them.
-    const bool pair = g_use_pairs && (M % 256 == 0) && (N % 256 == 0);
-    if (pair)
-        return format == NVQ_NVFP4
-                   ? launch_gemm_pair<0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
-                                         M, N, K, s)
-                   : launch_gemm_pair<1>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo,
-                                         M, N, K, s);
+    // CTA pairs when M allows them: 256 x 256 tiles, else 256 x 192 (two
+    // accumulators) when N is a multiple of 384 only.  Measured on the FF-up
+    // shape, 256 x 256 with one accumulator is faster than 256 x 192 with two.
+    if (g_use_pairs && M % 256 == 0) {
+        if (N % 256 == 0)
+            return format == NVQ_NVFP4
+                       ? launch_gemm_pair<0, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
+                                                  out, ldo, M, N, K, s)
+                       : launch_gemm_pair<1, 256>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias,
+                                                  out, ldo, M, N, K, s);
+        if (N % 384 == 0)
+            return format == NVQ_NVFP4
+                       ? launch_gemm_pair<0, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
+                                                  out, ldo, M, N, K, s)
+                       : launch_gemm_pair<1, 192>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias,
+                                                  out, ldo, M, N, K, s);
+    }
     if (format == NVQ_NVFP4) {
         if (bn == 192)
             return launch_gemm<0, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
