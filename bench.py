@@ -38,6 +38,42 @@ FP4_OVER_BF16 = 4.0           # nominal dense FP4 / BF16 tensor throughput on B2
 ACT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # BF16 read, E2M1 codes + E4M3 scale written
 
 
+# DRAM traffic of the roofline kernel per launch on this workload, from one
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum).  It holds for
+# the kernel sources it was taken on; once they change the figure is stale
+# and is reported as null.
+GEMM_TRAFFIC = {"kernel": None, "bytes_per_launch": None, "sources_sha256": None}
+KERNEL_SOURCES = ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh")
+
+
+def kernel_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "microscaling_quantized_linear_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gemm_kernel_name(fmt, M, N):
+    """The GEMM kernel block_scaled_linear launches for this shape (the
+    library's tile choice: CTA pairs on 256-row tiles when M allows them)."""
+    f = 0 if fmt == "nvfp4" else 1
+    pairs = os.environ.get("NVQ_GEMM_PAIRS", "1") != "0"
+    if pairs and M % 256 == 0 and (N % 256 == 0 or N % 384 == 0):
+        return "bsgemm_pair_kernel<%d, %d>" % (f, 256 if N % 256 == 0 else 192)
+    bn = 256 if N % 256 == 0 else 192 if N % 384 == 0 else 128
+    return "bsgemm_kernel<%d, %d>" % (f, bn)
+
+
+def gemm_traffic(kernel):
+    if GEMM_TRAFFIC["kernel"] != kernel or GEMM_TRAFFIC["bytes_per_launch"] is None:
+        return None
+    if kernel_sources_sha256() != GEMM_TRAFFIC["sources_sha256"]:
+        return None
+    return GEMM_TRAFFIC["bytes_per_launch"]
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -193,6 +229,7 @@ def run_ours(args, rank, world, device):
     act_gbs = act_bytes / (quant_mean * 1e-6) / 1e9
 
     e2e = run_e2e(nvq, args, device, stream, xs[0].cpu(), wq[0], M, N, K, flops, world)
+    kernel = gemm_kernel_name("nvfp4", M, N)
 
     res = {
         "metric": METRIC,
@@ -223,13 +260,15 @@ def run_ours(args, rank, world, device):
             "peak_source": peaks["source"],
         },
         "roofline": {
-            "kernel": "bsgemm_kernel<NVFP4,256>",
+            "kernel": kernel,
             "bound": "tensor",
             "achieved": round(gemm_tflops, 1),
             "peak": round(fp4_peak, 1),
             "unit": "TFLOP/s",
             "frac": round(gemm_tflops / fp4_peak, 4),
-            "traffic": None,
+            "traffic": gemm_traffic(kernel),
+            "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+            "algorithmic_bytes": int(M * K * 0.5625 + N * K * 0.5625 + M * N * 2),
             "peak_source": "%s bf16 %s x %.0f (nominal FP4/BF16 ratio)" % (
                 peaks["source"], "sustained" if sustained else "burst", FP4_OVER_BF16),
             "us_per_launch": round(gemm_mean, 3),
