@@ -42,7 +42,11 @@ ACT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # BF16 read, E2M1 codes + E4M3 scale
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum).  It holds for
 # the kernel sources it was taken on; once they change the figure is stale
 # and is reported as null.
-GEMM_TRAFFIC = {"kernel": None, "bytes_per_launch": None, "sources_sha256": None}
+# Taken on the FF-up workload; the summary is in
+# profiles/bsgemm_pair_kernel_nvfp4_ffup.md.
+GEMM_TRAFFIC = {"kernel": "bsgemm_pair_kernel<0, 256>",
+                "bytes_per_launch": 29262080 + 62670080,
+                "sources_sha256": "4970e14821728a6b1ac7b85cdcc351648eba55cd5496d684d2b5e663626f4e1a"}
 KERNEL_SOURCES = ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh")
 
 
