@@ -179,7 +179,7 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
         // One pass when every CTA's rows fit in shared memory (one CTA per SM).
         const int64_t rows_per_cta = (M + d->num_sms - 1) / d->num_sms;
         const size_t smem = fused_smem_bytes((size_t)rows_per_cta, (size_t)K);
-        if (smem <= kFusedSmemMax) {
+        if (smem <= kFusedSmemMax && (M + rows_per_cta - 1) / rows_per_cta <= kMaxFusedCtas) {
             {
                 std::lock_guard<std::mutex> lock(g_mu);
                 if (!d->fused_attr) {

@@ -29,9 +29,10 @@ namespace nvq {
 
 constexpr int kAmaxThreads = 256;
 constexpr int kMaxAmaxPartials = 1024;        // u32 partial maxima of the two-pass path
-constexpr int kMaxFusedCtas = 1024;           // u64 epoch-tagged slots of the one-pass path
+constexpr int kMaxFusedCtas = 256;            // epoch-tagged slots of the one-pass path
+constexpr int kFusedSlotStride = 16;          // u64 per slot: one 128-byte line each, so polls spread over L2
 constexpr size_t kWorkspaceSlotsOffset = 0;
-constexpr size_t kWorkspacePartialsOffset = kMaxFusedCtas * 8;
+constexpr size_t kWorkspacePartialsOffset = (size_t)kMaxFusedCtas * kFusedSlotStride * 8;
 constexpr size_t kWorkspaceBytes = kWorkspacePartialsOffset + kMaxAmaxPartials * 4;
 constexpr int kQuantThreads = 256;
 constexpr float kAmaxFloor = 0x1p-100f;       // below this the tensor quantizes to zero
@@ -269,13 +270,15 @@ constexpr int kFusedThreads = 1024;
 constexpr int kFusedChunks = 4;
 constexpr uint64_t kFusedWaitNs = 2000000000ull;   // 2 s
 
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
+// The slot word carries its epoch and its value together, so relaxed
+// single-copy-atomic 64-bit accesses suffice: nothing else is published.
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
     unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 
@@ -352,25 +355,38 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
     }
     const uint32_t cta_max = block_max_u32<kFusedThreads>(m, red);
     if (threadIdx.x == 0)
-        st_release_u64(slots + blockIdx.x, ((unsigned long long)epoch << 32) | cta_max);
+        st_relaxed_u64(slots + (size_t)blockIdx.x * kFusedSlotStride, ((unsigned long long)epoch << 32) | cta_max);
 
-    // every CTA's partial, tagged with this call's epoch
-    m = 0;
-    if (threadIdx.x < gridDim.x) {
-        const unsigned long long* slot = slots + threadIdx.x;
-        unsigned long long v = ld_acquire_u64(slot);
-        if ((uint32_t)(v >> 32) != epoch) {
-            const uint64_t t0 = globaltimer_ns();
-            while ((uint32_t)((v = ld_acquire_u64(slot)) >> 32) != epoch) {
-                if (s_timeout || globaltimer_ns() - t0 > kFusedWaitNs) {
-                    s_timeout = 1;
-                    break;
+    // Every CTA's partial, tagged with this call's epoch.  One warp polls
+    // (lane l watches slots l, l + 32, ...); the other warps wait at the
+    // barrier below, so the poll traffic is one load per slot per CTA.
+    __shared__ uint32_t s_amax;
+    if (threadIdx.x < 32) {
+        uint32_t mine = 0, pending = 0;
+        for (uint32_t j = threadIdx.x, bit = 0; j < gridDim.x; j += 32, ++bit) pending |= 1u << bit;
+        const uint64_t t0 = globaltimer_ns();
+        while (true) {
+            for (uint32_t j = threadIdx.x, bit = 0; j < gridDim.x; j += 32, ++bit) {
+                if (!(pending & (1u << bit))) continue;
+                const unsigned long long v = ld_relaxed_u64(slots + (size_t)j * kFusedSlotStride);
+                if ((uint32_t)(v >> 32) == epoch) {
+                    mine = max(mine, (uint32_t)(v & 0xFFFFFFFFull));
+                    pending &= ~(1u << bit);
                 }
             }
+            if (!__any_sync(0xFFFFFFFFu, pending != 0)) break;
+            int give_up = 0;                          // decided by lane 0 so the warp leaves together
+            if (threadIdx.x == 0) give_up = s_timeout || globaltimer_ns() - t0 > kFusedWaitNs;
+            if (__shfl_sync(0xFFFFFFFFu, give_up, 0)) {
+                if (threadIdx.x == 0) s_timeout = 1;
+                break;
+            }
         }
-        m = (uint32_t)(v & 0xFFFFFFFFull);
+        mine = __reduce_max_sync(0xFFFFFFFFu, mine);
+        if (threadIdx.x == 0) s_amax = mine;
     }
-    const uint32_t amax_bits = block_max_u32<kFusedThreads>(m, red);
+    __syncthreads();
+    const uint32_t amax_bits = s_amax;
     if (s_timeout) {                                  // a copy or a peer never arrived: write nothing
         if (threadIdx.x == 0) {
             atomicOr(status, 1u);

@@ -156,9 +156,10 @@ def test_nvfp4_deterministic_and_no_overwrite():
 
 
 def test_nvfp4_workspace_reuse_across_calls():
-    # One workspace for a sequence of different tensors (one-pass and two-pass
-    # paths, a zero tensor right after a large one): every result must be the
-    # oracle's, so no partial maximum of an earlier call can leak into a later one.
+    # One workspace for a sequence of different tensors (a zero tensor right
+    # after a large one, shapes of different grid sizes): every result must be
+    # the oracle's, so no partial maximum of an earlier call can leak into a
+    # later one.
     ws = nvq.new_workspace()
     seq = [act("actq"), torch.zeros(4608, 3072, dtype=torch.bfloat16), act("ffup"),
            act("qkv4"), workloads.normal(4608, 3072, seed=77, std=1e-3), act("tiny")]
@@ -185,6 +186,46 @@ def test_empty_batch_launches_nothing():
     codes, sf, g = nvq.nvfp4_quantize(x)
     c8, s8 = nvq.mxfp8_quantize(x)
     assert codes.numel() == 0 and c8.numel() == 0
+
+
+ONE_PASS_SCRIPT = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, ROOT_DIR)
+sys.path.insert(0, TEST_DIR)
+import test_gpu_quantize as t
+import oracle, workloads
+import microscaling_quantized_linear_b200 as nvq
+from gpu_common import act, bits
+ws = nvq.new_workspace()
+cases = [act("actq"), act("ffup"), torch.zeros(4608, 3072, dtype=torch.bfloat16),
+         workloads.normal(4608, 3072, seed=78, std=1e-3), act("tiny"), workloads.normal(256, 384, seed=31),
+         workloads.normal(1152, 6144, seed=79)]
+for x in cases:
+    codes, sf, g = nvq.nvfp4_quantize(x.cuda(), workspace=ws)
+    torch.cuda.synchronize()
+    M, K = x.shape
+    t.assert_nvfp4_equal((codes.cpu().numpy(), sf.cpu().numpy(), np.float32(g.item())),
+                         oracle.nvfp4_quantize(bits(x)), M, K)
+    print(M, K, "ok")
+assert nvq.device_status() == 0
+print("OK")
+"""
+
+
+def test_nvfp4_one_pass_path():
+    # NVQ_QUANT_ONE_PASS=1 (read when the library loads, hence a fresh
+    # process) routes the dynamic NVFP4 quantizer through the cooperative
+    # one-pass kernel wherever the rows fit in shared memory; its results must
+    # be the oracle's, call after call on one workspace.
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    env = dict(os.environ, NVQ_QUANT_ONE_PASS="1")
+    script = ONE_PASS_SCRIPT.replace("ROOT_DIR", repr(root)).replace("TEST_DIR", repr(here))
+    out = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0 and out.stdout.strip().endswith("OK"), out.stdout + out.stderr
 
 
 # ------------------------------------------------------------------ MXFP8
