@@ -12,8 +12,14 @@
 //   tensor memories, from its scale-copy warps) and the 256 x BN x K MMAs
 //   (from its MMA warp); the MMA commits arrive on the barriers of both CTAs
 //   (.multicast::cluster on the commit).
-//   Both CTAs' tile loads complete on the leader's full barrier
-//   (.cta_group::2 tensor loads; no load multicast anywhere).
+//   Both CTAs' tile loads complete on the leader's barriers (.cta_group::2
+//   tensor loads; no load multicast anywhere): the scale tiles on sfdata[s],
+//   which only the copy warps wait for, and the A and B tiles on full[s],
+//   which also counts the copy warps' commits.  The MMA lane therefore waits
+//   once per stage: it issues the MMAs one after another (the tensor pipe
+//   holds little more than one in flight), so every barrier check in its
+//   loop is time the pipe stands idle.  Stage s owns scale slot s in tensor
+//   memory, and one commit per stage frees both.
 //   Each CTA drains its own accumulator half; the peer's epilogue warps
 //   arrive remotely on the leader's accumulator-empty barrier.
 // Per SM this halves the B bytes staged from L2 and the tensor-core
@@ -45,8 +51,9 @@ struct PairCfg {
     static constexpr int B_BYTES = BN_HALF * KBYTES;
     static constexpr int SFA_BYTES = SF_CHUNK;
     static constexpr int SFB_BYTES = SFB_H * SF_CHUNK;
-    static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // per CTA per stage
-    static constexpr int STAGE_BYTES = (TX_BYTES + 1023) / 1024 * 1024;
+    static constexpr int AB_BYTES = A_BYTES + B_BYTES;                    // per CTA per stage
+    static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;                  // per CTA per stage
+    static constexpr int STAGE_BYTES = (AB_BYTES + SF_BYTES + 1023) / 1024 * 1024;
     static constexpr int OFF_B = A_BYTES;
     static constexpr int OFF_SFA = A_BYTES + B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
@@ -54,19 +61,22 @@ struct PairCfg {
     static constexpr int EPI_BYTES = kEpiWarps * EPI_BUF_BYTES;
     static constexpr int SMEM_LIMIT = 232448;
     static constexpr int FIXED_BYTES = 1024 + 512 + EPI_BYTES;
-    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-    static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
     static constexpr int SFA_COLS = FMT == 0 ? 4 * KSTEPS : 4;
     static constexpr int SFB_COLS_PER_MMA = 4 * SFB_H;
     static constexpr int SFB_COLS = FMT == 0 ? SFB_COLS_PER_MMA * KSTEPS : SFB_COLS_PER_MMA;
     static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
-    static constexpr int ACC_BUFS = (2 * BN + 2 * SF_COLS <= 512) ? 2 : 1;
-    static constexpr int SF_SLOTS_FIT = (512 - ACC_BUFS * BN) / SF_COLS;
-    static constexpr int SF_SLOTS = SF_SLOTS_FIT < STAGES ? SF_SLOTS_FIT : STAGES;
+    // Each pipeline stage owns one tensor-memory scale slot, so the stage
+    // count is bounded by shared memory and by the columns left beside the
+    // accumulator(s).  Two accumulators only when at least 4 slots remain.
+    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
+    static constexpr int ACC_BUFS = (512 - 2 * BN) / SF_COLS >= 4 ? 2 : 1;
+    static constexpr int SLOTS_FIT = (512 - ACC_BUFS * BN) / SF_COLS;
+    static constexpr int STAGES_MIN2 = STAGES_FIT < SLOTS_FIT ? STAGES_FIT : SLOTS_FIT;
+    static constexpr int STAGES = STAGES_MIN2 > 8 ? 8 : STAGES_MIN2;
+    static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
     static constexpr int TM_SF = ACC_BUFS * BN;
-    static constexpr int TM_USED = ACC_BUFS * BN + SF_SLOTS * SF_COLS;
+    static constexpr int TM_USED = ACC_BUFS * BN + STAGES * SF_COLS;
     static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
     static constexpr int SF_WARPS = 1 + SFB_H;             // copy warps (used in the leader)
     static constexpr int THREADS = 32 * (kFirstSfWarp + SF_WARPS);
@@ -77,8 +87,7 @@ struct PairCfg {
         ((uint32_t)(BM >> 4) << 24);
     static_assert(BN == 256 || BN == 192, "pair tiles are 256 x 256 or 256 x 192");
     static_assert(TM_USED <= 512, "tensor memory overflow");
-    static_assert(SF_SLOTS >= 2, "tensor memory too small for two scale slots");
-    static_assert(STAGES >= 2, "shared memory too small");
+    static_assert(STAGES >= 4, "too few pipeline stages");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory overflow");
 };
 
@@ -91,15 +100,20 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
+    // full[s]:   A and B tiles of both CTAs landed (tx) + the scale copies
+    //            into slot s committed (one arrival per copy warp): the MMA
+    //            warp's single wait per stage
+    // sfdata[s]: both CTAs' scale tiles landed (tx): the copy warps' wait
+    // empty[s]:  the stage's MMAs completed (commit multicast to both CTAs):
+    //            frees shared-memory stage s and tensor-memory scale slot s
     const uint32_t full0 = smem_u32(bars);
     const uint32_t empty0 = full0 + 8 * C::STAGES;
-    const uint32_t sffull0 = empty0 + 8 * C::STAGES;
-    const uint32_t sfempty0 = sffull0 + 8 * C::SF_SLOTS;
-    const uint32_t tfull0 = sfempty0 + 8 * C::SF_SLOTS;
+    const uint32_t sfdata0 = empty0 + 8 * C::STAGES;
+    const uint32_t tfull0 = sfdata0 + 8 * C::STAGES;
     const uint32_t tempty0 = tfull0 + 8 * 2;
     const uint32_t drain = tempty0 + 8 * 2;
     const uint32_t sfdrain = drain + 8;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 2 * C::SF_SLOTS + 6);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* never = abort_flag + 1;
 
@@ -108,12 +122,9 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
     const uint32_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(full0 + 8 * s, 1);
+            mbar_init(full0 + 8 * s, 1 + C::SF_WARPS);
             mbar_init(empty0 + 8 * s, 1);
-        }
-        for (int j = 0; j < C::SF_SLOTS; ++j) {
-            mbar_init(sffull0 + 8 * j, C::SF_WARPS);
-            mbar_init(sfempty0 + 8 * j, 1);
+            mbar_init(sfdata0 + 8 * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
@@ -164,17 +175,22 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                         break;
                     }
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
-                    const uint32_t fb = mapa_shared(full0 + 8 * s, 0);   // the leader's full barrier
-                    if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * C::TX_BYTES);
-                    tma_load_2d_pair(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), arow);
-                    tma_load_2d_pair(st + C::OFF_B, &tmap_b, fb, (int32_t)(kt * C::KBYTES), brow);
-                    // scale tiles: the tensors are viewed as rows of 256 bytes
-                    tma_load_2d_pair(st + C::OFF_SFA, &tmap_sfa, fb, 0,
+                    const uint32_t fb = mapa_shared(full0 + 8 * s, 0);     // the leader's barriers
+                    const uint32_t sb = mapa_shared(sfdata0 + 8 * s, 0);
+                    if (rank == 0) {
+                        mbar_arrive_expect_tx(sfdata0 + 8 * s, 2 * C::SF_BYTES);
+                        mbar_arrive_expect_tx(full0 + 8 * s, 2 * C::AB_BYTES);
+                    }
+                    // scale tiles first (the copy warps need them before the
+                    // MMAs can run); the tensors are viewed as rows of 256 bytes
+                    tma_load_2d_pair(st + C::OFF_SFA, &tmap_sfa, sb, 0,
                                      (int32_t)(((size_t)sfa_atom * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 2));
 #pragma unroll
                     for (int h = 0; h < C::SFB_H; ++h)
-                        tma_load_2d_pair(st + C::OFF_SFB + h * C::SF_CHUNK, &tmap_sfb, fb, 0,
+                        tma_load_2d_pair(st + C::OFF_SFB + h * C::SF_CHUNK, &tmap_sfb, sb, 0,
                                          (int32_t)(((size_t)(sfb_atom + h) * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 2));
+                    tma_load_2d_pair(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), arow);
+                    tma_load_2d_pair(st + C::OFF_B, &tmap_b, fb, (int32_t)(kt * C::KBYTES), brow);
                     ++it;
                 }
             }
@@ -183,8 +199,10 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 atomicOr(p.status, 1u);
             }
             if (rank == 0)      // the leader's barriers count both CTAs' bytes: wait for the last stages
-                for (uint32_t j = it > (uint32_t)C::STAGES ? it - C::STAGES : 0; j < it; ++j)
+                for (uint32_t j = it > (uint32_t)C::STAGES ? it - C::STAGES : 0; j < it; ++j) {
+                    mbar_wait_bounded(sfdata0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
                     mbar_wait_bounded(full0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
+                }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer (leader only)
@@ -204,15 +222,13 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 const uint32_t sfb_shift = (((tile / p.num_m_blocks) * BN) % 128) / 32;
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt, ++it) {
                     const uint32_t s = it % C::STAGES, su = it / C::STAGES;
-                    const uint32_t slot = it % C::SF_SLOTS, sv = it / C::SF_SLOTS;
-                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs) ||
-                        !mbar_wait_bounded(sffull0 + 8 * slot, sv & 1, abort_flag, kWaitLimitNs)) {
+                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
-                    const uint32_t sfa_t = tmem + C::TM_SF + slot * C::SF_COLS;
+                    const uint32_t sfa_t = tmem + C::TM_SF + s * C::SF_COLS;
                     const uint32_t sfb_t = sfa_t + C::SFA_COLS;
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k) {
@@ -228,8 +244,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                                              (sfb_t + sfb_shift) | ((uint32_t)k << 30), acc);
                         }
                     }
-                    tc_commit_pair_mc(empty0 + 8 * s, 0x3);     // frees the stage in both CTAs
-                    tc_commit_pair(sfempty0 + 8 * slot);         // scale slot free
+                    tc_commit_pair_mc(empty0 + 8 * s, 0x3);     // frees stage and scale slot in both CTAs
                 }
                 if (!ok) break;
                 tc_commit_pair_mc(tfull0 + 8 * buf, 0x3);       // accumulator ready in both CTAs
@@ -248,15 +263,16 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             bool ok = true;
             for (uint32_t it = 0; it < total_iters; ++it) {
                 const uint32_t s = it % C::STAGES, su = it / C::STAGES;
-                const uint32_t slot = it % C::SF_SLOTS, sv = it / C::SF_SLOTS;
-                if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs) ||
-                    (sv > 0 && !mbar_wait_bounded(sfempty0 + 8 * slot, (sv - 1) & 1, abort_flag, kWaitLimitNs))) {
+                // slot s is free once the MMAs of its previous use completed
+                // (the same commit that freed the shared-memory stage)
+                if ((su > 0 && !mbar_wait_bounded(empty0 + 8 * s, (su - 1) & 1, abort_flag, kWaitLimitNs)) ||
+                    !mbar_wait_bounded(sfdata0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                sf_copy_job<C, true>(job, smem_u32(smem + s * C::STAGE_BYTES), tmem + C::TM_SF + slot * C::SF_COLS);
-                tc_commit_pair(sffull0 + 8 * slot);
+                sf_copy_job<C, true>(job, smem_u32(smem + s * C::STAGE_BYTES), tmem + C::TM_SF + s * C::SF_COLS);
+                tc_commit_pair(full0 + 8 * s);               // the copies' share of the MMA's wait
             }
             if (!ok) {
                 *abort_flag = 1;
