@@ -80,11 +80,16 @@ __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half,
             }
         }
     }
+    // The release signal carries no data: tcgen05.wait::ld has returned, so
+    // every load of this share has read the accumulator before the arrive
+    // executes, and the MMA lane only has to be ordered after that (its
+    // tcgen05.fence::after_thread_sync).  Hence a relaxed arrive; a release
+    // arrive at cluster scope stalled the warp for about 1,700 cycles.
     tc_fence_before();
     __syncwarp();
     if (lane == 0) {
-        if (release_remote) mbar_arrive_cluster(release_bar);
-        else mbar_arrive(release_bar);
+        if (release_remote) mbar_arrive_relaxed_cluster(release_bar);
+        else mbar_arrive_relaxed(release_bar);
     }
     const uint32_t swz = (uint32_t)((lane >> 1) & 3);     // 64-byte swizzle of this thread's row
 #pragma unroll
