@@ -43,53 +43,67 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s per wait
 constexpr int kEpiWarps = 8;
 constexpr int kFirstSfWarp = 2 + kEpiWarps;
 
-// Drains one 32-row x BN/2-column share of an accumulator: all its tensor-
-// memory chunks are read (and rounded to BF16) first, then the accumulator
-// is released through release_bar, then the BF16 sub-tiles are written via
-// the warp's 64-byte-swizzled staging buffer and TMA stores.
+// alpha * acc + bias for 32 accumulator columns (c .. c+31 of the tile),
+// rounded to BF16 pairs; products as packed f32x2 multiplies (RNE per lane).
+__device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], float alpha, const __nv_bfloat16* bias_tile,
+                                               int c, uint32_t (&packed)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        float2 v = f32x2_mul(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), alpha);
+        if (bias_tile) {
+            const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(bias_tile + c + 2 * e);
+            v.x = __fadd_rn(v.x, __bfloat162float(bb.x));
+            v.y = __fadd_rn(v.y, __bfloat162float(bb.y));
+        }
+        const __nv_bfloat162 o = __floats2bfloat162_rn(v.x, v.y);
+        packed[e] = *reinterpret_cast<const uint32_t*>(&o);
+    }
+}
+
+// Drains one 32-row x BN/2-column share of an accumulator.  Tensor-memory
+// chunks are read two at a time; every pair but the last is converted to
+// BF16 before the next is read, and the accumulator is released as soon as
+// the last pair is in registers (its conversion follows the release), so the
+// MMAs of the next tile wait for the loads and one conversion only.  The
+// BF16 sub-tiles are then written via the warp's 64-byte-swizzled staging
+// buffer and TMA stores.
 template <int BN>
 __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half, int lane, float alpha,
                                                   const __nv_bfloat16* bias_tile, uint8_t* staging,
                                                   const CUtensorMap* tmap_d, int32_t row0, uint32_t n0,
                                                   uint32_t release_bar, bool release_remote) {
     constexpr int NC = BN / 64;                          // 32-column chunks per warp
+    constexpr int JL = (NC - 1) & ~1;                    // first chunk of the last pair
     const int c0 = half * (BN / 2);
     uint32_t packed[NC][16];
 #pragma unroll
-    for (int j = 0; j < NC; j += 2) {
+    for (int j = 0; j < JL; j += 2) {
         uint32_t r0[32], r1[32];
         tc_ld_32x32b_x32(tmem_acc_q + c0 + 32 * j, r0);
-        if (j + 1 < NC) tc_ld_32x32b_x32(tmem_acc_q + c0 + 32 * (j + 1), r1);
+        tc_ld_32x32b_x32(tmem_acc_q + c0 + 32 * (j + 1), r1);
         tc_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (j + u >= NC) break;
-            const uint32_t* r = u ? r1 : r0;
-            const int c = c0 + 32 * (j + u);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                float v0 = __fmul_rn(__uint_as_float(r[2 * e]), alpha);
-                float v1 = __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha);
-                if (bias_tile) {
-                    const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(bias_tile + c + 2 * e);
-                    v0 = __fadd_rn(v0, __bfloat162float(bb.x));
-                    v1 = __fadd_rn(v1, __bfloat162float(bb.y));
-                }
-                const __nv_bfloat162 o = __floats2bfloat162_rn(v0, v1);
-                packed[j + u][e] = *reinterpret_cast<const uint32_t*>(&o);
-            }
-        }
+        epilogue_chunk(r0, alpha, bias_tile, c0 + 32 * j, packed[j]);
+        epilogue_chunk(r1, alpha, bias_tile, c0 + 32 * (j + 1), packed[j + 1]);
     }
-    // The release signal carries no data: tcgen05.wait::ld has returned, so
-    // every load of this share has read the accumulator before the arrive
-    // executes, and the MMA lane only has to be ordered after that (its
-    // tcgen05.fence::after_thread_sync).  Hence a relaxed arrive; a release
-    // arrive at cluster scope stalled the warp for about 1,700 cycles.
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) {
-        if (release_remote) mbar_arrive_relaxed_cluster(release_bar);
-        else mbar_arrive_relaxed(release_bar);
+    {
+        uint32_t r0[32], r1[32];
+        tc_ld_32x32b_x32(tmem_acc_q + c0 + 32 * JL, r0);
+        if (JL + 1 < NC) tc_ld_32x32b_x32(tmem_acc_q + c0 + 32 * (JL + 1), r1);
+        tc_wait_ld();
+        // The release signal carries no data: tcgen05.wait::ld has returned,
+        // so every load of this share has read the accumulator before the
+        // arrive executes, and the MMA lane only has to be ordered after that
+        // (its tcgen05.fence::after_thread_sync).  Hence a relaxed arrive; a
+        // release arrive at cluster scope stalled the warp for about 1,700
+        // cycles.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            if (release_remote) mbar_arrive_relaxed_cluster(release_bar);
+            else mbar_arrive_relaxed(release_bar);
+        }
+        epilogue_chunk(r0, alpha, bias_tile, c0 + 32 * JL, packed[JL]);
+        if (JL + 1 < NC) epilogue_chunk(r1, alpha, bias_tile, c0 + 32 * (JL + 1), packed[JL + 1 < NC ? JL + 1 : JL]);
     }
     const uint32_t swz = (uint32_t)((lane >> 1) & 3);     // 64-byte swizzle of this thread's row
 #pragma unroll

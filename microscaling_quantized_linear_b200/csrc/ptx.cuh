@@ -377,6 +377,18 @@ __device__ __forceinline__ float2 bf16x2_mul(uint32_t w, float m) {
     return c;
 }
 
+// (a * m, b * m) as one packed f32x2 multiply (round to nearest even per lane).
+__device__ __forceinline__ float2 f32x2_mul(float a, float b, float m) {
+    float2 c;
+    asm("{\n\t.reg .b64 x, y, z;\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mov.b64 y, {%4, %4};\n\t"
+        "mul.rn.f32x2 z, x, y;\n\t"
+        "mov.b64 {%0, %1}, z;\n\t}"
+        : "=f"(c.x), "=f"(c.y) : "f"(a), "f"(b), "f"(m));
+    return c;
+}
+
 // Two FP32 -> two E4M3 codes in 16 bits (hi -> bits 15:8, lo -> bits 7:0),
 // round to nearest even, saturating to +-448.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
