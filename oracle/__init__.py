@@ -56,6 +56,14 @@ def lib():
         L.oracle_mxfp8_quantize.argtypes = [_u16p, _i64, _i64, _i64, _u8p, _u8p]
         L.oracle_mxfp8_dequantize.restype = None
         L.oracle_mxfp8_dequantize.argtypes = [_u8p, _u8p, _i64, _i64, _f64p]
+        L.oracle_mxfp8_quantize_ex.restype = None
+        L.oracle_mxfp8_quantize_ex.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int, _u8p, _u8p]
+        L.oracle_mxfp8_dequantize_ex.restype = None
+        L.oracle_mxfp8_dequantize_ex.argtypes = [_u8p, _u8p, _i64, _i64, ctypes.c_int, _f64p]
+        L.oracle_e5m2_value.restype = ctypes.c_double
+        L.oracle_e5m2_value.argtypes = [ctypes.c_int]
+        L.oracle_e5m2_encode.restype = ctypes.c_int
+        L.oracle_e5m2_encode.argtypes = [ctypes.c_float]
         L.oracle_gemm_rows.restype = None
         L.oracle_gemm_rows.argtypes = [_f64p, _f64p, _i64, _i64, _i64p, _i64, _u16p, _f64p]
         L.oracle_num_threads.restype = ctypes.c_int
@@ -84,6 +92,14 @@ def e2m1_value(code):
 
 def e4m3_value(code):
     return lib().oracle_e4m3_value(int(code))
+
+
+def e5m2_value(code):
+    return lib().oracle_e5m2_value(int(code))
+
+
+def e5m2_encode(v):
+    return lib().oracle_e5m2_encode(float(np.float32(v)))
 
 
 def e8m0_value(code):
@@ -144,22 +160,28 @@ def nvfp4_dequantize(codes, sf, g_dec, rows, K):
     return out
 
 
-def mxfp8_quantize(x_bits):
-    """Returns (codes u8 [M, K], sf u8 [sf_bytes(M, K/32)])."""
+ELEMS = {"e4m3": 0, "e5m2": 1}
+RULES = {"floor": 0, "ceil": 1}
+
+
+def mxfp8_quantize(x_bits, elem="e4m3", rule="floor"):
+    """Returns (codes u8 [M, K], sf u8 [sf_bytes(M, K/32)]).
+    elem: "e4m3" or "e5m2" elements; rule: "floor" (OCP) or "ceil" block exponent."""
     x = _bf16_bits(x_bits)
     M, K = x.shape
     assert K % MXFP8_BLOCK == 0
     codes = np.zeros((M, K), dtype=np.uint8)
     sf = np.zeros(sf_bytes(M, K // MXFP8_BLOCK), dtype=np.uint8)
-    lib().oracle_mxfp8_quantize(_ptr(x, _u16p), M, K, K, _ptr(codes, _u8p), _ptr(sf, _u8p))
+    lib().oracle_mxfp8_quantize_ex(_ptr(x, _u16p), M, K, K, ELEMS[elem], RULES[rule], _ptr(codes, _u8p),
+                                   _ptr(sf, _u8p))
     return codes, sf
 
 
-def mxfp8_dequantize(codes, sf, rows, K):
+def mxfp8_dequantize(codes, sf, rows, K, elem="e4m3"):
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     sf = np.ascontiguousarray(sf, dtype=np.uint8)
     out = np.empty((rows, K), dtype=np.float64)
-    lib().oracle_mxfp8_dequantize(_ptr(codes, _u8p), _ptr(sf, _u8p), rows, K, _ptr(out, _f64p))
+    lib().oracle_mxfp8_dequantize_ex(_ptr(codes, _u8p), _ptr(sf, _u8p), rows, K, ELEMS[elem], _ptr(out, _f64p))
     return out
 
 

@@ -37,7 +37,14 @@
  *     scale), in exactly the order written below, with no fused multiply-add.
  *   - A tensor whose amax_t is below 2^-100 (zero included) quantizes to all
  *     zero codes and scales with g_dec = 0.
- *   - MXFP8 block scale: OCP MX rule X = floor(log2(block amax)) - 8.
+ *   - MXFP8 block scale: OCP MX rule X = floor(log2(block amax)) - emax, emax
+ *     the exponent of the element type's largest normal (8 for E4M3, 15 for
+ *     E5M2); the "ceil" variant takes the smallest X with block amax <=
+ *     max_elem * 2^X instead, so no element saturates.
+ *   - E5M2 is the IEEE-like variant: s.eeeee.mm, bias 15, max finite 57344,
+ *     S.11111.00 = infinity, S.11111.xx = NaN; encoding saturates at 57344.
+ *   - Ragged row counts: codes are dense over the M rows; the scale tiles
+ *     are padded to a multiple of 128 rows with zero bytes.
  *   - Scale bytes are stored in the 128x4 tensor-core tile order (see
  *     oracle_sf_offset).
  *   - Codes are K-contiguous; two E2M1 codes per byte, even element in the
@@ -69,6 +76,16 @@ ORACLE_EXPORT double oracle_e4m3_value(int code) {
     int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
     if (e == 15 && m == 7) return NAN;
     double mag = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* E5M2 ([P1] "MXFP8量化格式" names E4M3 and E5M2): s.eeeee.mm, bias 15;
+ * e == 0 is subnormal (m * 2^-16); e == 31 is infinity (m == 0) or NaN. */
+ORACLE_EXPORT double oracle_e5m2_value(int code) {
+    int s = (code >> 7) & 1, e = (code >> 2) & 31, m = code & 3;
+    double mag;
+    if (e == 31) mag = (m == 0) ? INFINITY : NAN;
+    else mag = (e == 0) ? ldexp((double)m, -16) : ldexp(1.0 + m / 4.0, e - 15);
     return s ? -mag : mag;
 }
 
@@ -115,6 +132,13 @@ ORACLE_EXPORT int oracle_e4m3_encode(float v) {
     if (isnan(v)) { g_nan_seen = 1; return 0x7F; }
     int sign = signbit(v) ? 0x80 : 0x00;
     return sign | round_to_table(fabs((double)v), 0x7E, oracle_e4m3_value);
+}
+
+/* E5M2 encode of an FP32 value: RNE, saturate to 57344 (code 0x7B), sign kept. */
+ORACLE_EXPORT int oracle_e5m2_encode(float v) {
+    if (isnan(v)) { g_nan_seen = 1; return 0x7F; }
+    int sign = signbit(v) ? 0x80 : 0x00;
+    return sign | round_to_table(fabs((double)v), 0x7B, oracle_e5m2_value);
 }
 
 /* Returns 1 if any NaN input reached an encoder since the last call. */
@@ -253,17 +277,52 @@ static int floor_log2(double b) {
     return e - 1;
 }
 
+/* The element types of MXFP8: code -> value, value -> code, the largest
+ * finite value and the exponent emax of that value. */
+typedef struct {
+    double (*value)(int);
+    int (*encode)(float);
+    double max_value;
+    int emax;
+} mx_elem;
+
+static mx_elem mx_element(int elem) {
+    mx_elem e;
+    if (elem == 1) { e.value = oracle_e5m2_value; e.encode = oracle_e5m2_encode; e.max_value = 57344.0; e.emax = 15; }
+    else { e.value = oracle_e4m3_value; e.encode = oracle_e4m3_encode; e.max_value = 448.0; e.emax = 8; }
+    return e;
+}
+
+/* Shared block exponent X for block amax b > 0.
+ *   rule 0 (OCP "floor"): X = floor(log2 b) - emax.
+ *   rule 1 ("ceil"): the smallest X with b <= max_value * 2^X, found by
+ *   stepping from the floor value (so that the definition is what runs).
+ * Clamped to [-127, 127]; b == 0 gives -127. */
+static int mx_block_exponent(float b, const mx_elem* e, int rule) {
+    if (b == 0.0f) return -127;
+    int X = floor_log2((double)b) - e->emax;
+    if (rule == 1) {
+        while ((double)b > ldexp(e->max_value, X)) ++X;
+        while ((double)b <= ldexp(e->max_value, X - 1)) --X;
+    }
+    if (X < -127) X = -127;
+    if (X > 127) X = 127;
+    return X;
+}
+
 /*
- * Quantize one BF16 tensor to MXFP8 (E4M3 elements).
+ * Quantize one BF16 tensor to MXFP8.
+ *   elem:  0 = E4M3 elements, 1 = E5M2 elements.
+ *   rule:  0 = floor block exponent (OCP), 1 = ceil (no saturation).
  *   codes: rows M, K bytes per row (dense).
- *   sf:    oracle_sf_bytes(M, K/32) bytes of E8M0, 128x4 tile order.
- * Per 32-block along K: b = max |x_i|; X = floor(log2 b) - 8 clamped to
- * [-127, 127] (X = -127 when b == 0); scale byte = X + 127;
- * q_i = E4M3(x_i * 2^-X)  (FP32 multiply by a power of two).
+ *   sf:    oracle_sf_bytes(M, K/32) bytes of E8M0, 128x4 tile order, zero padding.
+ * Per 32-block along K: b = max |x_i|; X as in mx_block_exponent; scale
+ * byte = X + 127; q_i = ELEM(x_i * 2^-X)  (FP32 multiply by a power of two).
  */
-ORACLE_EXPORT void oracle_mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
-                                         uint8_t* codes, uint8_t* sf) {
+ORACLE_EXPORT void oracle_mxfp8_quantize_ex(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                            int elem, int rule, uint8_t* codes, uint8_t* sf) {
     const int64_t nblk = K / MXFP8_BLOCK;
+    const mx_elem e = mx_element(elem);
     memset(sf, 0, (size_t)oracle_sf_bytes(M, nblk));
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m) {
@@ -274,29 +333,39 @@ ORACLE_EXPORT void oracle_mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K
                 float a = fabsf(bf16_to_float(blk[i]));
                 if (a > b) b = a;
             }
-            int X = (b == 0.0f) ? -127 : floor_log2((double)b) - 8;
-            if (X < -127) X = -127;
-            if (X > 127) X = 127;
+            int X = mx_block_exponent(b, &e, rule);
             sf[oracle_sf_offset(m, j, nblk)] = (uint8_t)(X + 127);
             float mult = (float)ldexp(1.0, -X);   /* exact: 2^-X fits FP32 */
             for (int i = 0; i < MXFP8_BLOCK; ++i) {
                 float v = bf16_to_float(blk[i]) * mult;
-                codes[m * K + j * MXFP8_BLOCK + i] = (uint8_t)oracle_e4m3_encode(v);
+                codes[m * K + j * MXFP8_BLOCK + i] = (uint8_t)e.encode(v);
             }
         }
     }
 }
 
-/* x_hat = E4M3(q) * 2^X, binary64, row-major [rows][K]. */
-ORACLE_EXPORT void oracle_mxfp8_dequantize(const uint8_t* codes, const uint8_t* sf,
-                                           int64_t rows, int64_t K, double* out) {
+/* The default MXFP8 quantizer: E4M3 elements, floor block exponent. */
+ORACLE_EXPORT void oracle_mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                         uint8_t* codes, uint8_t* sf) {
+    oracle_mxfp8_quantize_ex(x, M, K, ldx, 0, 0, codes, sf);
+}
+
+/* x_hat = ELEM(q) * 2^X, binary64, row-major [rows][K]. */
+ORACLE_EXPORT void oracle_mxfp8_dequantize_ex(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t K,
+                                              int elem, double* out) {
     const int64_t nblk = K / MXFP8_BLOCK;
+    const mx_elem e = mx_element(elem);
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < rows; ++m)
         for (int64_t k = 0; k < K; ++k) {
             double s = oracle_e8m0_value(sf[oracle_sf_offset(m, k / MXFP8_BLOCK, nblk)]);
-            out[m * K + k] = oracle_e4m3_value(codes[m * K + k]) * s;
+            out[m * K + k] = e.value(codes[m * K + k]) * s;
         }
+}
+
+ORACLE_EXPORT void oracle_mxfp8_dequantize(const uint8_t* codes, const uint8_t* sf,
+                                           int64_t rows, int64_t K, double* out) {
+    oracle_mxfp8_dequantize_ex(codes, sf, rows, K, 0, out);
 }
 
 /* ------------------------------------------------------------------ */

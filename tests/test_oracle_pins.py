@@ -438,3 +438,146 @@ def test_acceptance_rule():
     assert abs(oracle.gemm_row_errors(D, Y)[0] - 0.001) < 1e-15
     D = Y + np.array([[0.0, 0.0], [1e-30, 0.0]])
     assert np.isinf(oracle.gemm_row_errors(D, Y)[1])
+
+
+# --------------------------------------------------------------------------
+# MXFP8 with E5M2 elements and the ceil block exponent; ragged row counts
+# --------------------------------------------------------------------------
+
+def test_e5m2_decode_matches_torch_all_256_codes():
+    lib_vals = torch.arange(256, dtype=torch.uint8).view(torch.float8_e5m2).double().numpy()
+    ours = np.array([oracle.e5m2_value(c) for c in range(256)])
+    assert np.array_equal(np.isnan(ours), np.isnan(lib_vals))
+    fin = ~np.isnan(lib_vals)
+    assert np.array_equal(ours[fin], lib_vals[fin])
+    assert np.array_equal(np.signbit(ours[fin]), np.signbit(lib_vals[fin]))
+    assert ours[0x7B] == 57344.0 and np.isinf(ours[0x7C]) and ours[0x01] == 2.0 ** -16
+
+
+def test_e5m2_encode_matches_torch_below_the_maximum():
+    # torch's float8_e5m2 cast rounds to nearest even and overflows to inf
+    # past the top, so compare at every midpoint +-1 ulp below 57344 and on
+    # random values; saturation is checked separately.
+    vals = [oracle.e5m2_value(c) for c in range(0x7C)]
+    probes = []
+    for lo, hi in zip(vals[:-1], vals[1:]):
+        mid = np.float32((lo + hi) / 2)
+        probes += [mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(1e9))]
+    rng = np.random.default_rng(7)
+    probes += list((rng.standard_normal(20000) * np.exp2(rng.integers(-18, 15, 20000))).astype(np.float32))
+    probes = np.array([p for p in probes if abs(p) < 57344], dtype=np.float32)
+    probes = np.concatenate([probes, -probes])
+    want = torch.tensor(probes).to(torch.float8_e5m2).view(torch.uint8).numpy().astype(np.int64)
+    got = np.array([oracle.e5m2_encode(p) for p in probes])
+    assert np.array_equal(got, want)
+    for c in range(256):
+        if (c & 0x7F) >= 0x7C:
+            continue
+        assert oracle.e5m2_encode(oracle.e5m2_value(c)) == c, hex(c)
+    assert oracle.e5m2_encode(60000.0) == 0x7B and oracle.e5m2_encode(-1e30) == 0xFB
+
+
+@pytest.mark.parametrize("case", ["e4m3/floor", "e4m3/ceil", "e5m2/floor", "e5m2/ceil"])
+def test_mxfp8_element_and_rule_hand_worked_blocks(golden_dir, case):
+    g = json.load(open(os.path.join(golden_dir, "mxfp8_elem_rule_blocks.json")))
+    vals = np.zeros(g["K"], dtype=np.float32)
+    for k, v in g["x_block0"].items():
+        vals[int(k)] = v
+    for k, v in g["x_block1"].items():
+        vals[32 + int(k)] = v
+    x = bf16(vals.tolist(), (1, g["K"]))
+    assert torch.equal(x.float()[0], torch.tensor(vals))          # the inputs are exact BF16
+    elem, rule = case.split("/")
+    codes, sf = oracle.mxfp8_quantize(bits(x), elem=elem, rule=rule)
+    want = g["cases"][case]
+    assert [int(sf[oracle.sf_offset(0, j, 2)]) for j in range(2)] == want["scale_codes"]
+    for key, c in want["codes"].items():
+        b, i = map(int, key.split(":"))
+        assert int(codes[0, 32 * b + i]) == c, (key, hex(int(codes[0, 32 * b + i])), hex(c))
+
+
+@pytest.mark.parametrize("elem,maxv", [("e4m3", 448.0), ("e5m2", 57344.0)])
+def test_mxfp8_block_exponent_rules_by_brute_force(elem, maxv):
+    # floor rule: X = floor(log2 b) - emax, from the exact binary exponent;
+    # ceil rule: the smallest integer X with b <= max * 2^X, by search over X.
+    emax = 8 if elem == "e4m3" else 15
+    x = workloads.normal(64, 256, seed=23, std=3.0)
+    x[3, :32] *= 1e-30
+    xb = x.float().numpy()
+    for rule in ("floor", "ceil"):
+        _, sf = oracle.mxfp8_quantize(bits(x), elem=elem, rule=rule)
+        for r in range(64):
+            for j in range(8):
+                b = float(np.abs(xb[r, 32 * j:32 * j + 32]).max())
+                if rule == "floor":
+                    m, e = np.frexp(b)                 # exact: b = m * 2^e, m in [0.5, 1)
+                    X = (e - 1) - emax if b > 0 else -127
+                else:
+                    X = next(X for X in range(-200, 200) if b <= maxv * 2.0 ** X) if b > 0 else -127
+                X = min(max(X, -127), 127)
+                assert int(sf[oracle.sf_offset(r, j, 8)]) == X + 127, (rule, r, j, b)
+
+
+@pytest.mark.parametrize("elem", ["e4m3", "e5m2"])
+def test_mxfp8_ceil_rule_never_saturates_and_matches_torch_cast(elem):
+    # Under the ceil rule every |x| <= max * 2^X, so no element clips and each
+    # code is exactly torch's round-to-nearest-even cast of x * 2^-X.
+    maxv = 448.0 if elem == "e4m3" else 57344.0
+    tdt = torch.float8_e4m3fn if elem == "e4m3" else torch.float8_e5m2
+    x = workloads.normal(128, 512, seed=29)
+    x[9, 64:96] *= 1.75 / x[9, 64:96].float().abs().max()     # a block whose max is exactly 1.75 * 2^e
+    codes, sf = oracle.mxfp8_quantize(bits(x), elem=elem, rule="ceil")
+    xb = x.float().numpy()
+    X = np.array([[int(sf[oracle.sf_offset(r, j, 16)]) - 127 for j in range(16)] for r in range(128)])
+    Xe = np.repeat(X, 32, axis=1).astype(np.float64)
+    assert np.all(np.abs(xb) <= maxv * np.exp2(Xe))
+    scaled = torch.from_numpy((xb * np.exp2(-Xe)).astype(np.float32))   # exact: power-of-two scaling
+    want = scaled.to(tdt).view(torch.uint8).numpy()
+    assert np.array_equal(codes, want)
+    codes_f, _ = oracle.mxfp8_quantize(bits(x), elem=elem, rule="floor")
+    top = 0x7E if elem == "e4m3" else 0x7B
+    assert ((codes_f & 0x7F) == top).sum() > ((codes & 0x7F) == top).sum()   # the floor rule clips some
+
+
+@pytest.mark.parametrize("elem,rule", [("e5m2", "floor"), ("e5m2", "ceil"), ("e4m3", "ceil")])
+@pytest.mark.parametrize("k", [-3, 5])
+def test_mxfp8_variants_power_of_two_equivariance(elem, rule, k):
+    x = workloads.normal(128, 256, seed=31)
+    c0, s0 = oracle.mxfp8_quantize(bits(x), elem=elem, rule=rule)
+    c1, s1 = oracle.mxfp8_quantize(bits((x.float() * 2.0 ** k).to(torch.bfloat16)), elem=elem, rule=rule)
+    assert np.array_equal(c0, c1)
+    nz = s0 != 0
+    assert np.array_equal(s1[nz].astype(int), s0[nz].astype(int) + k)
+
+
+def test_mxfp8_e5m2_dequantize_matches_library_decode():
+    x = workloads.normal(128, 256, seed=37)
+    codes, sf = oracle.mxfp8_quantize(bits(x), elem="e5m2")
+    got = oracle.mxfp8_dequantize(codes, sf, 128, 256, elem="e5m2")
+    vals = torch.from_numpy(codes).view(torch.float8_e5m2).double().numpy()
+    scale = np.array([[torch.tensor([sf[oracle.sf_offset(r, k // 32, 8)]], dtype=torch.uint8)
+                       .view(torch.float8_e8m0fnu).double().item() for k in range(256)] for r in range(128)])
+    assert np.array_equal(got, vals * scale)
+
+
+@pytest.mark.parametrize("M", [1, 100, 129])
+def test_ragged_rows_equal_the_zero_padded_tensor(M):
+    # A ragged row count quantizes its rows exactly as the zero-padded tensor
+    # does (zero rows change neither amax nor any other row), and the scale
+    # rows past M are zero.
+    K = 256
+    x = workloads.normal(M, K, seed=41 + M)
+    Mp = (M + 127) // 128 * 128
+    xp = torch.zeros(Mp, K, dtype=torch.bfloat16)
+    xp[:M] = x
+    c, s, g = oracle.nvfp4_quantize(bits(x))
+    cp, sp, gp = oracle.nvfp4_quantize(bits(xp))
+    assert g == gp and np.array_equal(c, cp[:M]) and np.array_equal(s, sp)
+    for elem, rule in (("e4m3", "floor"), ("e5m2", "ceil")):
+        c8, s8 = oracle.mxfp8_quantize(bits(x), elem=elem, rule=rule)
+        c8p, s8p = oracle.mxfp8_quantize(bits(xp), elem=elem, rule=rule)
+        assert np.array_equal(c8, c8p[:M])
+        # padded rows: zero blocks give scale byte 0 (X = -127), the same as the zero padding
+        assert np.array_equal(s8, s8p)
+    nblk = K // 16
+    assert all(s[oracle.sf_offset(r, j, nblk)] == 0 for r in range(M, Mp) for j in range(nblk))
