@@ -23,18 +23,20 @@
  *  - Matrices are row-major.  BF16 tensors are [rows, K] with a row pitch
  *    `ld` in elements.  Quantized codes are dense: an NVFP4 row is K/2 bytes
  *    (element 2j in the low nibble of byte j, 2j+1 in the high nibble), an
- *    MXFP8 row is K bytes of E4M3.
+ *    MXFP8 row is K bytes of E4M3 (or E5M2, format NVQ_MXFP8_E5M2).
  *  - Block scales form a logical matrix S[rows][K / block] of bytes (E4M3 for
  *    NVFP4, E8M0 for MXFP8) stored in the 128x4 tile order the sm_100
  *    block-scaled tensor-core instructions read: tiles of 128 rows x 4
  *    scale columns, 512 bytes each, tile (r/128, c/4) at
  *    ((r/128) * (C/4) + c/4) * 512, and inside a tile row r, column c at
- *    (r%32)*16 + ((r%128)/32)*4 + (c%4), where C = K / block.
- *  - Shape contract: rows (M, N) multiples of 128 ("block alignment must be
- *    a multiple of 128", NVIDIA Blackwell平台FP4量化技术解析与图像生成优化,
- *    section 5.2); K a positive multiple of 64 (NVFP4) or 128 (MXFP8) so
- *    scale columns fill whole tiles; every BF16 pitch a multiple of 8
- *    elements and >= K; all pointers 16-byte aligned; rows * K < 2^31.
+ *    (r%32)*16 + ((r%128)/32)*4 + (c%4), where C = K / block.  The tiles
+ *    cover the rows rounded up to 128 ("block alignment must be a multiple
+ *    of 128", NVIDIA Blackwell平台FP4量化技术解析与图像生成优化, section 5.2);
+ *    the quantizers write zero into the rows past the tensor's last row.
+ *  - Shape contract: any row count (M, N >= 0; a ragged count is padded
+ *    only in the scale tiles); K a positive multiple of 64 (NVFP4) or 128
+ *    (MXFP8) so scale columns fill whole tiles; every BF16 pitch a multiple
+ *    of 8 elements and >= K; all pointers 16-byte aligned; rows * K < 2^31.
  *    Otherwise NVQ_ERR_SHAPE / NVQ_ERR_ALIGN, and nothing is launched.
  *    M == 0 (an empty batch) is accepted and launches nothing.
  *  - The device must be compute capability 10.0 (B200, sm_100a), else
@@ -62,7 +64,15 @@ extern "C" {
 /* Same type as cudaStream_t; declared here so the header needs no CUDA headers. */
 typedef struct CUstream_st* nvq_stream_t;
 
-typedef enum { NVQ_NVFP4 = 0, NVQ_MXFP8 = 1 } nvq_format;
+/* NVQ_MXFP8_E5M2: MXFP8 with E5M2 elements (page "NVIDIA量化推理：5步极速优化显存+
+ * 成功率翻倍", section MXFP8量化格式, names E4M3 and E5M2 as the element types). */
+typedef enum { NVQ_NVFP4 = 0, NVQ_MXFP8 = 1, NVQ_MXFP8_E5M2 = 2 } nvq_format;
+
+/* MXFP8 block-exponent rule (mxfp8_quantize_ex).  FLOOR is the OCP rule
+ * X = floor(log2(block max)) - emax (elements in [max, 2*max) * 2^X
+ * saturate); CEIL takes the smallest X with block max <= max * 2^X, so no
+ * element saturates.  emax = 8 (E4M3, max 448), 15 (E5M2, max 57344). */
+enum { NVQ_SCALE_FLOOR = 0, NVQ_SCALE_CEIL = 1 };
 
 /* Return codes (host side). */
 enum {
@@ -81,7 +91,7 @@ enum {
     NVQ_STATUS_NONFINITE = 2    /* nvfp4_quantize saw a NaN/Inf amax */
 };
 
-/* Bytes of the code buffer for a [rows, K] tensor: rows*K/2 (NVFP4), rows*K (MXFP8). */
+/* Bytes of the code buffer for a [rows, K] tensor: rows*K/2 (NVFP4), rows*K (MXFP8, either element). */
 NVQ_API size_t nvq_codes_bytes(int format, int64_t rows, int64_t K);
 
 /* Bytes of the swizzled scale buffer: ceil(rows/128)*128 * ceil((K/block)/4)*4,
@@ -137,12 +147,31 @@ NVQ_API int mxfp8_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
                    uint8_t* codes, uint8_t* scales, nvq_stream_t stream);
 
 /*
+ * mxfp8_quantize_ex -- mxfp8_quantize with a choice of element type and
+ * block-exponent rule (page "NVIDIA量化推理：5步极速优化显存+成功率翻倍",
+ * section MXFP8量化格式: E4M3 or E5M2 elements under one 8-bit shared
+ * exponent per 32 values).
+ *
+ *   elem_format  NVQ_MXFP8 (E4M3 elements) or NVQ_MXFP8_E5M2 (E5M2: 1 sign,
+ *                5 exponent, 2 mantissa bits, bias 15, largest 57344)
+ *   scale_rule   NVQ_SCALE_FLOOR or NVQ_SCALE_CEIL (see above)
+ * Per 32-block: X from the rule, clamped to [-127, 127] (-127 for an
+ * all-zero block), scale byte X + 127, q = ELEM(x * 2^-X) rounded to nearest
+ * even and saturated.  Other arguments and errors as mxfp8_quantize; an
+ * unknown elem_format or scale_rule gives NVQ_ERR_FORMAT.
+ */
+NVQ_API int mxfp8_quantize_ex(const void* x, int64_t M, int64_t K, int64_t ldx,
+                      uint8_t* codes, uint8_t* scales, int elem_format, int scale_rule,
+                      nvq_stream_t stream);
+
+/*
  * quantize_weight -- offline weight quantization ("double quantization" of
  * BF16 weights into FP4 data + FP8 scales, page "NVIDIA Blackwell平台FP4量化
  * 技术解析与图像生成优化", section 3.1), run once at load time.  Same
  * arithmetic as nvfp4_quantize / mxfp8_quantize applied to W [N, K]; for
  * NVFP4 the global scale is the weight's own static g_dec.
  *
+ *   format        NVQ_NVFP4, NVQ_MXFP8 or NVQ_MXFP8_E5M2 (floor block exponent)
  *   global_scale  NVFP4: out, required.  MXFP8: ignored (may be NULL).
  *   workspace     NVFP4: required (nvq_workspace_bytes()).  MXFP8: ignored.
  */
@@ -165,8 +194,12 @@ NVQ_API int quantize_weight(int format, const void* w, int64_t N, int64_t K, int
  *   b_codes, b_scales   quantized weights [N, K] (quantize_weight)
  *   b_global            NVFP4: device float g_dec of B.  MXFP8: ignored.
  *   bias                NULL or BF16 [N]
+ *   format              NVQ_NVFP4, NVQ_MXFP8 (E4M3 x E4M3) or NVQ_MXFP8_E5M2 (E5M2 x E5M2)
  *   out                 BF16 [M, N], row pitch ldo elements (ldo >= N, multiple of 8)
- *   M, N                multiples of 128; K a multiple of 256 (NVFP4) or 128 (MXFP8)
+ *   M, N                M any, N a multiple of 8 (ragged tiles read zeros past the
+ *                       end and store nothing there; bias is read only for n < N;
+ *                       the store of a row's last chunk is clipped at 16 bytes);
+ *                       K a multiple of 256 (NVFP4) or 128 (MXFP8)
  *
  * Accumulation is FP32 in tensor memory; the order of the K sum is the
  * hardware's.  Results match the FP64 sum over the dequantized operands to

@@ -27,7 +27,13 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 NVFP4 = 0
 MXFP8 = 1
-_FORMATS = {"nvfp4": NVFP4, "mxfp8": MXFP8, NVFP4: NVFP4, MXFP8: MXFP8}
+MXFP8_E5M2 = 2
+_FORMATS = {"nvfp4": NVFP4, "mxfp8": MXFP8, "mxfp8_e5m2": MXFP8_E5M2,
+            NVFP4: NVFP4, MXFP8: MXFP8, MXFP8_E5M2: MXFP8_E5M2}
+SCALE_FLOOR = 0
+SCALE_CEIL = 1
+_ELEMS = {"e4m3": MXFP8, "e5m2": MXFP8_E5M2}
+_RULES = {"floor": SCALE_FLOOR, "ceil": SCALE_CEIL}
 
 NVQ_STATUS_TIMEOUT = 1
 NVQ_STATUS_NONFINITE = 2
@@ -46,6 +52,8 @@ _lib.nvfp4_quantize.restype = ctypes.c_int
 _lib.nvfp4_quantize.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.mxfp8_quantize.restype = ctypes.c_int
 _lib.mxfp8_quantize.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp]
+_lib.mxfp8_quantize_ex.restype = ctypes.c_int
+_lib.mxfp8_quantize_ex.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, ctypes.c_int, ctypes.c_int, _vp]
 _lib.quantize_weight.restype = ctypes.c_int
 _lib.quantize_weight.argtypes = [ctypes.c_int, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]
 _lib.block_scaled_linear.restype = ctypes.c_int
@@ -61,8 +69,8 @@ _lib.nvfp4_quantize_noalloc.restype = ctypes.c_int
 _lib.nvfp4_quantize_noalloc.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]
 
 EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_quantize",
-            "mxfp8_quantize", "quantize_weight", "block_scaled_linear", "nvq_device_status",
-            "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc")
+            "mxfp8_quantize", "mxfp8_quantize_ex", "quantize_weight", "block_scaled_linear",
+            "nvq_device_status", "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc")
 
 NOALLOC_MAX_PARTIALS = 1024
 
@@ -149,14 +157,21 @@ def nvfp4_quantize_noalloc(x, codes, scales, global_scale, stream=None):
     return codes, scales, global_scale
 
 
-def mxfp8_quantize(x, codes=None, scales=None, stream=None):
-    """BF16 [M, K] -> (codes u8 [M, K] (E4M3), scales u8 (E8M0, tile order))."""
+def mxfp8_quantize(x, codes=None, scales=None, stream=None, elem="e4m3", rule="floor"):
+    """BF16 [M, K] -> (codes u8 [M, K] (E4M3 or E5M2), scales u8 (E8M0, tile order)).
+    elem "e4m3" | "e5m2"; rule "floor" (OCP) | "ceil" (no element saturates)."""
     M, K = x.shape
     dev = x.device
     codes = codes if codes is not None else torch.empty((M, K), dtype=torch.uint8, device=dev)
     scales = scales if scales is not None else torch.empty(scale_bytes(MXFP8, M, K), dtype=torch.uint8, device=dev)
-    _check(_lib.mxfp8_quantize(_ptr(x), M, K, _pitch(x), _ptr(codes), _ptr(scales), _stream(stream, dev)),
-           "mxfp8_quantize")
+    if elem == "e4m3" and rule == "floor":
+        rc = _lib.mxfp8_quantize(_ptr(x), M, K, _pitch(x), _ptr(codes), _ptr(scales), _stream(stream, dev))
+    else:
+        if elem not in _ELEMS or rule not in _RULES:
+            raise ValueError("unknown element type %r or rule %r" % (elem, rule))
+        rc = _lib.mxfp8_quantize_ex(_ptr(x), M, K, _pitch(x), _ptr(codes), _ptr(scales), _ELEMS[elem],
+                                    _RULES[rule], _stream(stream, dev))
+    _check(rc, "mxfp8_quantize")
     return codes, scales
 
 
@@ -165,7 +180,7 @@ def quantize_weight(fmt, w, codes=None, scales=None, global_scale=None, workspac
     f = _fmt(fmt)
     N, K = w.shape
     dev = w.device
-    cols = K // 2 if f == NVFP4 else K
+    cols = K // 2 if f == NVFP4 else K     # MXFP8 (either element type): one byte per value
     codes = codes if codes is not None else torch.empty((N, cols), dtype=torch.uint8, device=dev)
     scales = scales if scales is not None else torch.empty(scale_bytes(f, N, K), dtype=torch.uint8, device=dev)
     if f == NVFP4:

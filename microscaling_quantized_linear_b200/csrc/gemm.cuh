@@ -45,15 +45,21 @@ constexpr int kFirstSfWarp = 2 + kEpiWarps;
 
 // alpha * acc + bias for 32 accumulator columns (c .. c+31 of the tile),
 // rounded to BF16 pairs; products as packed f32x2 multiplies (RNE per lane).
+// Bias entries at tile columns >= nlim (past N) are not read.
 __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], float alpha, const __nv_bfloat16* bias_tile,
-                                               int c, uint32_t (&packed)[16]) {
+                                               int c, int nlim, uint32_t (&packed)[16]) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         float2 v = f32x2_mul(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), alpha);
         if (bias_tile) {
-            const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(bias_tile + c + 2 * e);
-            v.x = __fadd_rn(v.x, __bfloat162float(bb.x));
-            v.y = __fadd_rn(v.y, __bfloat162float(bb.y));
+            const int n = c + 2 * e;
+            if (n + 1 < nlim) {
+                const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(bias_tile + n);
+                v.x = __fadd_rn(v.x, __bfloat162float(bb.x));
+                v.y = __fadd_rn(v.y, __bfloat162float(bb.y));
+            } else if (n < nlim) {
+                v.x = __fadd_rn(v.x, __bfloat162float(bias_tile[n]));
+            }
         }
         const __nv_bfloat162 o = __floats2bfloat162_rn(v.x, v.y);
         packed[e] = *reinterpret_cast<const uint32_t*>(&o);
@@ -71,7 +77,7 @@ template <int BN>
 __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half, int lane, float alpha,
                                                   const __nv_bfloat16* bias_tile, uint8_t* staging,
                                                   const CUtensorMap* tmap_d, int32_t row0, uint32_t n0,
-                                                  uint32_t release_bar, bool release_remote) {
+                                                  int nlim, uint32_t release_bar, bool release_remote) {
     constexpr int NC = BN / 64;                          // 32-column chunks per warp
     constexpr int JL = (NC - 1) & ~1;                    // first chunk of the last pair
     const int c0 = half * (BN / 2);
@@ -82,8 +88,8 @@ __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half,
         tc_ld_32x32b_x32(tmem_acc_q + c0 + 32 * j, r0);
         tc_ld_32x32b_x32(tmem_acc_q + c0 + 32 * (j + 1), r1);
         tc_wait_ld();
-        epilogue_chunk(r0, alpha, bias_tile, c0 + 32 * j, packed[j]);
-        epilogue_chunk(r1, alpha, bias_tile, c0 + 32 * (j + 1), packed[j + 1]);
+        epilogue_chunk(r0, alpha, bias_tile, c0 + 32 * j, nlim, packed[j]);
+        epilogue_chunk(r1, alpha, bias_tile, c0 + 32 * (j + 1), nlim, packed[j + 1]);
     }
     {
         uint32_t r0[32], r1[32];
@@ -102,8 +108,8 @@ __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half,
             if (release_remote) mbar_arrive_relaxed_cluster(release_bar);
             else mbar_arrive_relaxed(release_bar);
         }
-        epilogue_chunk(r0, alpha, bias_tile, c0 + 32 * JL, packed[JL]);
-        if (JL + 1 < NC) epilogue_chunk(r1, alpha, bias_tile, c0 + 32 * (JL + 1), packed[JL + 1 < NC ? JL + 1 : JL]);
+        epilogue_chunk(r0, alpha, bias_tile, c0 + 32 * JL, nlim, packed[JL]);
+        if (JL + 1 < NC) epilogue_chunk(r1, alpha, bias_tile, c0 + 32 * (JL + 1), nlim, packed[JL + 1 < NC ? JL + 1 : JL]);
     }
     const uint32_t swz = (uint32_t)((lane >> 1) & 3);     // 64-byte swizzle of this thread's row
 #pragma unroll
@@ -175,7 +181,7 @@ struct GemmCfg {
     // mxf8f6f4) in bits 7-9 / 10-12, K-major A and B, N >> 3 in bits 17-22,
     // scale format (0 = UE4M3, 1 = UE8M0) in bit 23, M >> 4 in bits 24-28.
     static constexpr uint32_t IDESC =
-        (FMT == 0 ? (1u << 7) | (1u << 10) : 0u) |
+        (FMT != 1 ? (1u << 7) | (1u << 10) : 0u) |   // A, B type: E2M1 (NVFP4) / E5M2 (FMT 2); 0 = E4M3
         ((uint32_t)(BN >> 3) << 17) |
         (FMT == 0 ? 0u : (1u << 23)) |
         ((uint32_t)(BM >> 4) << 24);
@@ -195,6 +201,8 @@ struct GemmParams {
     unsigned int* status;
     uint32_t num_m_blocks, num_n_blocks, num_k_tiles;
     uint32_t sf_ctiles;          // (K / SF_BLOCK) / 4: scale tiles per 128 rows
+    uint32_t n_total;            // N: output columns past it are neither stored nor biased
+    uint32_t sfa_rtiles, sfb_rtiles;   // 128-row scale tiles in the A and B scale buffers
 };
 
 // Scale-factor copy warp `job` (0: A scales, 1..SFB_H: B scale row block
@@ -299,14 +307,18 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     mbar_arrive_expect_tx(fb, C::TX_BYTES);
                     tma_load_2d(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), (int32_t)(mb * C::BM));
                     tma_load_2d(st + C::OFF_B, &tmap_b, fb, (int32_t)(kt * C::KBYTES), (int32_t)(nb * BN));
+                    // plain bulk copies have no out-of-range fill: a B tile that
+                    // runs past N (its rows are not stored) reads the last scale tile
                     bulk_load(st + C::OFF_SFA,
                               p.sfa + ((size_t)mb * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
                               C::SFA_BYTES, fb);
 #pragma unroll
-                    for (int h = 0; h < C::SFB_H; ++h)
+                    for (int h = 0; h < C::SFB_H; ++h) {
+                        const uint32_t bt = min(a0 + h, p.sfb_rtiles - 1);
                         bulk_load(st + C::OFF_SFB + h * C::SF_ATOMS * 512,
-                                  p.sfb + ((size_t)(a0 + h) * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
+                                  p.sfb + ((size_t)bt * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
                                   C::SF_ATOMS * 512, fb);
+                    }
                     ++it;
                 }
             }
@@ -417,7 +429,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             const uint32_t n0 = nb * BN;
             drain_accumulator<BN>(tmem + ((uint32_t)(32 * q) << 16) + buf * BN, half, lane, alpha,
                                   p.bias ? p.bias + n0 : nullptr, staging, &tmap_d,
-                                  (int32_t)(mb * C::BM + 32 * q), n0, tempty0 + 8 * buf, false);
+                                  (int32_t)(mb * C::BM + 32 * q), n0, (int)(p.n_total - n0), tempty0 + 8 * buf, false);
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();

@@ -81,7 +81,7 @@ struct PairCfg {
     static constexpr int SF_WARPS = 1 + SFB_H;             // copy warps (used in the leader)
     static constexpr int THREADS = 32 * (kFirstSfWarp + SF_WARPS);
     static constexpr uint32_t IDESC =
-        (FMT == 0 ? (1u << 7) | (1u << 10) : 0u) |
+        (FMT != 1 ? (1u << 7) | (1u << 10) : 0u) |   // A, B type: E2M1 (NVFP4) / E5M2 (FMT 2); 0 = E4M3
         ((uint32_t)(BN >> 3) << 17) |
         (FMT == 0 ? 0u : (1u << 23)) |
         ((uint32_t)(BM >> 4) << 24);
@@ -301,7 +301,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             const uint32_t n0 = nb * BN;
             drain_accumulator<BN>(tmem + ((uint32_t)(32 * q) << 16) + buf * BN, half, lane, alpha,
                                   p.bias ? p.bias + n0 : nullptr, staging, &tmap_d,
-                                  (int32_t)(mb * 256 + 128 * rank + 32 * q), n0,
+                                  (int32_t)(mb * 256 + 128 * rank + 32 * q), n0, (int)(p.n_total - n0),
                                   mapa_shared(tempty0 + 8 * buf, 0), true);
         }
         if (lane == 0) bulk_wait_group_all();

@@ -43,8 +43,8 @@ struct DeviceInfo {
     bool arch_ok = false;
     int num_sms = 0;
     unsigned int* status = nullptr;
-    bool gemm_attr[2][3] = {{false, false, false}, {false, false, false}};
-    bool pair_attr[2][2] = {{false, false}, {false, false}};
+    bool gemm_attr[3][3] = {};
+    bool pair_attr[3][2] = {};
     bool fused_attr = false;
 };
 
@@ -98,9 +98,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int block_of(int format) { return format == NVQ_NVFP4 ? 16 : 32; }
 int k_multiple(int format) { return format == NVQ_NVFP4 ? 64 : 128; }
 
+bool is_mxfp8(int format) { return format == NVQ_MXFP8 || format == NVQ_MXFP8_E5M2; }
+
 // Checks shared by the quantizers: BF16 [rows, K] input with pitch ld.
 int check_quant_shape(int format, int64_t rows, int64_t K, int64_t ld) {
-    if (rows < 0 || K <= 0 || rows % 128 != 0 || K % k_multiple(format) != 0) return NVQ_ERR_SHAPE;
+    if (rows < 0 || K <= 0 || K % k_multiple(format) != 0) return NVQ_ERR_SHAPE;
     if (ld < K || ld % 8 != 0) return NVQ_ERR_SHAPE;
     if (rows * K >= (int64_t(1) << 31) || rows * ld >= (int64_t(1) << 40) || ld >= (int64_t(1) << 31))
         return NVQ_ERR_SHAPE;
@@ -232,7 +234,8 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
 }
 
 int mxfp8_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
-                        cudaStream_t stream) {
+                        int elem, int rule, cudaStream_t stream) {
+    if (!is_mxfp8(elem) || (rule != NVQ_SCALE_FLOOR && rule != NVQ_SCALE_CEIL)) return NVQ_ERR_FORMAT;
     int rc = check_quant_shape(NVQ_MXFP8, M, K, ldx);
     if (rc) return rc;
     if (M == 0) return NVQ_OK;
@@ -241,9 +244,12 @@ int mxfp8_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     DeviceInfo* d = nullptr;
     if ((rc = device_info(&d))) return rc;
     const uint32_t nblk = (uint32_t)(K / 32);
-    const uint64_t units = (uint64_t)M * nblk;
-    mxfp8_quantize_kernel<<<quant_grid(units, d->num_sms), kQuantThreads, 0, stream>>>(
-        static_cast<const uint16_t*>(x), (uint32_t)M, nblk, (uint32_t)ldx, codes, scales);
+    const uint32_t grid = quant_grid((uint64_t)M * nblk, d->num_sms);
+    const uint16_t* xp = static_cast<const uint16_t*>(x);
+    const bool e5 = elem == NVQ_MXFP8_E5M2, ceil_rule = rule == NVQ_SCALE_CEIL;
+    auto kern = e5 ? (ceil_rule ? mxfp8_quantize_kernel<1, 1> : mxfp8_quantize_kernel<1, 0>)
+                   : (ceil_rule ? mxfp8_quantize_kernel<0, 1> : mxfp8_quantize_kernel<0, 0>);
+    kern<<<grid, kQuantThreads, 0, stream>>>(xp, (uint32_t)M, nblk, (uint32_t)ldx, codes, scales);
     return launch_status();
 }
 
@@ -289,7 +295,7 @@ int launch_gemm_pair(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_sca
                      void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
     using C = PairCfg<FMT, BN>;
     const int64_t kbytes = FMT == 0 ? K / 2 : K;
-    const int fmt = FMT == 0 ? NVQ_NVFP4 : NVQ_MXFP8;
+    const int fmt = FMT == 0 ? NVQ_NVFP4 : NVQ_MXFP8;   // scale geometry only
     CUtensorMap ma, mb, msa, msb, md;
     int rc;
     if ((rc = encode_codes_map(&ma, a_codes, M, kbytes, 128))) return rc;
@@ -314,8 +320,11 @@ int launch_gemm_pair(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_sca
     p.b_global = b_global;
     p.bias = static_cast<const __nv_bfloat16*>(bias);
     p.status = d->status;
-    p.num_m_blocks = (uint32_t)(M / 256);
-    p.num_n_blocks = (uint32_t)(N / BN);
+    p.num_m_blocks = (uint32_t)((M + 255) / 256);
+    p.num_n_blocks = (uint32_t)((N + BN - 1) / BN);
+    p.n_total = (uint32_t)N;
+    p.sfa_rtiles = (uint32_t)((M + 127) / 128);
+    p.sfb_rtiles = (uint32_t)((N + 127) / 128);
     p.num_k_tiles = (uint32_t)(K / C::BK);
     p.sf_ctiles = (uint32_t)(K / C::SF_BLOCK / 4);
     const uint32_t tiles = p.num_m_blocks * p.num_n_blocks;
@@ -371,8 +380,11 @@ int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, 
     p.b_global = b_global;
     p.bias = static_cast<const __nv_bfloat16*>(bias);
     p.status = d->status;
-    p.num_m_blocks = (uint32_t)(M / C::BM);
-    p.num_n_blocks = (uint32_t)(N / BN);
+    p.num_m_blocks = (uint32_t)((M + C::BM - 1) / C::BM);
+    p.num_n_blocks = (uint32_t)((N + BN - 1) / BN);
+    p.n_total = (uint32_t)N;
+    p.sfa_rtiles = (uint32_t)((M + 127) / 128);
+    p.sfb_rtiles = (uint32_t)((N + 127) / 128);
     p.num_k_tiles = (uint32_t)(K / C::BK);
     p.sf_ctiles = (uint32_t)(K / C::SF_BLOCK / 4);
     const uint32_t tiles = p.num_m_blocks * p.num_n_blocks;
@@ -395,6 +407,34 @@ int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, 
 }
 
 }  // namespace
+// One launch per (format, tile shape); FMT 0 = NVFP4, 1 = MXFP8 (E4M3), 2 = MXFP8 (E5M2).
+template <int FMT>
+int launch_for_format(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                      const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
+                      void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, cudaStream_t s) {
+    // CTA pairs (256-row tiles) unless M fits one 128-row tile: 256 x 256
+    // tiles, or 256 x 192 (two accumulators for MXFP8) when N is a multiple of
+    // 384 but not of 256.  Measured on the FF-up shape, 256 x 256 with one
+    // accumulator is faster than 256 x 192 with two.  A ragged N takes 256.
+    if (g_use_pairs && M > 128) {
+        if (N % 384 == 0 && N % 256 != 0)
+            return launch_gemm_pair<FMT, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out,
+                                              ldo, M, N, K, s);
+        return launch_gemm_pair<FMT, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
+                                          M, N, K, s);
+    }
+    // One CTA per tile: width 256 when N allows it (fewest scale-factor copies
+    // per MMA), else 192 (two tensor-memory accumulators), else 128 (two).
+    if (N % 256 == 0)
+        return launch_gemm<FMT, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M,
+                                     N, K, s);
+    if (N % 384 == 0)
+        return launch_gemm<FMT, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M,
+                                     N, K, s);
+    return launch_gemm<FMT, 128>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M, N,
+                                 K, s);
+}
+
 }  // namespace nvq
 
 using namespace nvq;
@@ -402,12 +442,12 @@ using namespace nvq;
 extern "C" {
 
 size_t nvq_codes_bytes(int format, int64_t rows, int64_t K) {
-    if ((format != NVQ_NVFP4 && format != NVQ_MXFP8) || rows < 0 || K < 0) return 0;
+    if ((format != NVQ_NVFP4 && !is_mxfp8(format)) || rows < 0 || K < 0) return 0;
     return (size_t)(format == NVQ_NVFP4 ? rows * (K / 2) : rows * K);
 }
 
 size_t nvq_scale_bytes(int format, int64_t rows, int64_t K) {
-    if ((format != NVQ_NVFP4 && format != NVQ_MXFP8) || rows < 0 || K < 0) return 0;
+    if ((format != NVQ_NVFP4 && !is_mxfp8(format)) || rows < 0 || K < 0) return 0;
     const int64_t cols = K / block_of(format);
     return (size_t)(((rows + 127) / 128) * 128 * ((cols + 3) / 4) * 4);
 }
@@ -422,7 +462,14 @@ int nvfp4_quantize(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* co
 
 int mxfp8_quantize(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
                    nvq_stream_t stream) {
-    return mxfp8_quantize_impl(x, M, K, ldx, codes, scales, reinterpret_cast<cudaStream_t>(stream));
+    return mxfp8_quantize_impl(x, M, K, ldx, codes, scales, NVQ_MXFP8, NVQ_SCALE_FLOOR,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mxfp8_quantize_ex(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
+                      int elem_format, int scale_rule, nvq_stream_t stream) {
+    return mxfp8_quantize_impl(x, M, K, ldx, codes, scales, elem_format, scale_rule,
+                               reinterpret_cast<cudaStream_t>(stream));
 }
 
 int quantize_weight(int format, const void* w, int64_t N, int64_t K, int64_t ldw, uint8_t* codes,
@@ -430,18 +477,23 @@ int quantize_weight(int format, const void* w, int64_t N, int64_t K, int64_t ldw
     if (format == NVQ_NVFP4)
         return nvfp4_quantize_impl(w, N, K, ldw, codes, scales, global_scale, nullptr, workspace,
                                    reinterpret_cast<cudaStream_t>(stream));
-    if (format == NVQ_MXFP8)
-        return mxfp8_quantize_impl(w, N, K, ldw, codes, scales, reinterpret_cast<cudaStream_t>(stream));
+    if (is_mxfp8(format))
+        return mxfp8_quantize_impl(w, N, K, ldw, codes, scales, format, NVQ_SCALE_FLOOR,
+                                   reinterpret_cast<cudaStream_t>(stream));
     return NVQ_ERR_FORMAT;
 }
 
 int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                         const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
                         void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, nvq_stream_t stream) {
-    if (format != NVQ_NVFP4 && format != NVQ_MXFP8) return NVQ_ERR_FORMAT;
-    // the GEMM stages 256 (NVFP4) / 128 (MXFP8) elements of K at a time
+    if (format != NVQ_NVFP4 && !is_mxfp8(format)) return NVQ_ERR_FORMAT;
+    // the GEMM stages 256 (NVFP4) / 128 (MXFP8) elements of K at a time;
+    // M and N may be ragged (tensor-map loads fill past the end with zeros,
+    // stores are clipped)
     const int64_t k_stage = format == NVQ_NVFP4 ? 256 : 128;
-    if (M < 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % k_stage) return NVQ_ERR_SHAPE;
+    // N a multiple of 8: the tensor-map store of the last column chunk clips
+    // at 16-byte granularity, so a BF16 row must end on a 16-byte boundary
+    if (M < 0 || N <= 0 || N % 8 || K <= 0 || K % k_stage) return NVQ_ERR_SHAPE;
     if (ldo < N || ldo % 8 || M * ldo >= (int64_t(1) << 40) || ldo >= (int64_t(1) << 31)) return NVQ_ERR_SHAPE;
     if (K >= (int64_t(1) << 24) || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVQ_ERR_SHAPE;
     if (M == 0) return NVQ_OK;
@@ -455,44 +507,14 @@ int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_sca
     if (rc) return rc;
     if ((rc = get_encoder())) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // Tile width: 256 when N allows it (fewest scale-factor copies per MMA),
-    // else 192 (two tensor-memory accumulators), else 128 (two).
-    const int bn = (N % 256 == 0) ? 256 : (N % 384 == 0) ? 192 : 128;
-    // CTA pairs when M allows them: 256 x 256 tiles, else 256 x 192 (two
-    // accumulators) when N is a multiple of 384 only.  Measured on the FF-up
-    // shape, 256 x 256 with one accumulator is faster than 256 x 192 with two.
-    if (g_use_pairs && M % 256 == 0) {
-        if (N % 256 == 0)
-            return format == NVQ_NVFP4
-                       ? launch_gemm_pair<0, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
-                                                  out, ldo, M, N, K, s)
-                       : launch_gemm_pair<1, 256>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias,
-                                                  out, ldo, M, N, K, s);
-        if (N % 384 == 0)
-            return format == NVQ_NVFP4
-                       ? launch_gemm_pair<0, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
-                                                  out, ldo, M, N, K, s)
-                       : launch_gemm_pair<1, 192>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias,
-                                                  out, ldo, M, N, K, s);
-    }
-    if (format == NVQ_NVFP4) {
-        if (bn == 192)
-            return launch_gemm<0, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
-                                       M, N, K, s);
-        if (bn == 256)
-            return launch_gemm<0, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
-                                       M, N, K, s);
-        return launch_gemm<0, 128>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M,
-                                   N, K, s);
-    }
-    if (bn == 192)
-        return launch_gemm<1, 192>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M, N,
-                                   K, s);
-    if (bn == 256)
-        return launch_gemm<1, 256>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M, N,
-                                   K, s);
-    return launch_gemm<1, 128>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M, N, K,
-                               s);
+    if (format == NVQ_NVFP4)
+        return launch_for_format<0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M, N,
+                                    K, s);
+    if (format == NVQ_MXFP8)
+        return launch_for_format<1>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M, N,
+                                    K, s);
+    return launch_for_format<2>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M, N, K,
+                                s);
 }
 
 int nvq_device_status(nvq_stream_t stream) {

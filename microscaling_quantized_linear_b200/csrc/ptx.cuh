@@ -377,6 +377,19 @@ __device__ __forceinline__ float2 bf16x2_mul(uint32_t w, float m) {
     return c;
 }
 
+// Four FP32 -> four E5M2 codes in one word (a0 in bits 7:0), round to nearest
+// even, saturating to +-57344.
+__device__ __forceinline__ uint32_t cvt_e5m2x4(float a0, float a1, float a2, float a3) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .b16 h0, h1;\n\t"
+        "cvt.rn.satfinite.e5m2x2.f32 h0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e5m2x2.f32 h1, %4, %3;\n\t"
+        "mov.b32 %0, {h0, h1};\n\t}"
+        : "=r"(out) : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+    return out;
+}
+
 // (a * m, b * m) as one packed f32x2 multiply (round to nearest even per lane).
 __device__ __forceinline__ float2 f32x2_mul(float a, float b, float m) {
     float2 c;

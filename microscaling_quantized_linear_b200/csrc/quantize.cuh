@@ -72,6 +72,18 @@ __device__ __forceinline__ uint32_t sf_tile_offset(uint32_t r, uint32_t c, uint3
     return ((r >> 7) * ctiles + (c >> 2)) * 512u + (r & 31u) * 16u + ((r & 127u) >> 5) * 4u + (c & 3u);
 }
 
+// Scale rows past `rows`, up to the next multiple of 128, are zero (the
+// tensor-core tile holds 128 rows).  One 32-bit word = the 4 scale bytes of
+// one row in one column tile; thread `t` of `nthreads` writes its share.
+__device__ __forceinline__ void zero_pad_scale_rows(uint8_t* sf, uint32_t rows, uint32_t ctiles, uint32_t t,
+                                                    uint32_t nthreads) {
+    const uint32_t pad_rows = ((rows + 127u) & ~127u) - rows;
+    for (uint32_t i = t; i < pad_rows * ctiles; i += nthreads) {
+        const uint32_t r = rows + i / ctiles, ct = i - (i / ctiles) * ctiles;
+        *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r, 4 * ct, ctiles)) = 0u;
+    }
+}
+
 // E4M3 (non-negative) code -> float, exact.
 __device__ __forceinline__ float e4m3_decode_pos(uint32_t c) {
     const uint32_t e = (c >> 3) & 15u, m = c & 7u;
@@ -255,6 +267,7 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
             ++r1;
         }
     }
+    zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kQuantThreads + threadIdx.x, stride);
 }
 
 // ------------------------------------------------------------------ NVFP4, one pass
@@ -436,14 +449,22 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
             ++rl;
         }
     }
+    zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kFusedThreads + threadIdx.x, gridDim.x * kFusedThreads);
 }
 
 // ------------------------------------------------------------------ MXFP8
 // One thread = one 32-element block.  Block b is (row b / nblk, column
 // b % nblk), nblk = K / 32; its codes are bytes [32b, 32b + 32).
+// ELEM 0: E4M3 elements (largest 448 = 1.75 * 2^8); ELEM 1: E5M2 (largest
+// 57344 = 1.75 * 2^15).  RULE 0: X = floor(log2 b) - emax (OCP); RULE 1:
+// the smallest X with b <= largest * 2^X, i.e. one more than the floor
+// value when b's significand exceeds 1.75 (both largest values are
+// 1.75 * 2^emax), so no element saturates.
+template <int ELEM, int RULE>
 __global__ void __launch_bounds__(kQuantThreads)
 mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nblk, uint32_t ldx,
                       uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+    constexpr int EMAX = ELEM == 0 ? 8 : 15;
     const uint32_t total = rows * nblk;
     const uint32_t ctiles = nblk >> 2;
     const uint32_t stride = gridDim.x * kQuantThreads;
@@ -472,17 +493,21 @@ mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
             X = -127;
         } else {
             const int E = (int)(mb >> 7);
-            const int e = E ? E - 127 : (31 - __clz((int)(mb & 0x7F))) - 133;
-            X = min(max(e - 8, -127), 127);
+            const uint32_t mant = mb & 0x7Fu;
+            const int p = 31 - __clz((int)mant);      // subnormal: leading one of the mantissa
+            const int e = E ? E - 127 : p - 133;
+            int up = 0;
+            if (RULE == 1) up = E ? (mant > 96u) : (4u * mant > (7u << p));   // significand > 1.75
+            X = min(max(e - EMAX + up, -127), 127);
         }
         const uint32_t sc = (uint32_t)(X + 127);
-        const float mult = __uint_as_float((uint32_t)(127 - X) << 23);   // 2^-X, X <= 119
+        const float mult = __uint_as_float((uint32_t)(127 - X) << 23);   // 2^-X, -127 <= X <= 121
         uint32_t q[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const float2 p0 = bf16x2_mul(w[2 * i], mult);
             const float2 p1 = bf16x2_mul(w[2 * i + 1], mult);
-            q[i] = cvt_e4m3x4(p0.x, p0.y, p1.x, p1.y);
+            q[i] = ELEM == 0 ? cvt_e4m3x4(p0.x, p0.y, p1.x, p1.y) : cvt_e5m2x4(p0.x, p0.y, p1.x, p1.y);
         }
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
@@ -502,6 +527,7 @@ mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
             ++r;
         }
     }
+    zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kQuantThreads + threadIdx.x, stride);
 }
 
 // ------------------------------------------------------------------ probe

@@ -49,6 +49,8 @@ def test_size_helpers():
     assert nvq.scale_bytes("nvfp4", 4608, 3072) == 4608 * 192
     assert nvq.scale_bytes("mxfp8", 4608, 12288) == 4608 * 384
     assert nvq.scale_bytes("nvfp4", 130, 80) == 256 * 8          # padded to 128 rows x 4 columns
+    assert nvq.scale_bytes("mxfp8_e5m2", 100, 256) == nvq.scale_bytes("mxfp8", 100, 256) == 128 * 8
+    assert nvq.codes_bytes("mxfp8_e5m2", 100, 256) == 100 * 256
     assert nvq.workspace_bytes() >= 4 * 148
     assert L.nvq_codes_bytes(7, 128, 64) == 0
 
@@ -67,7 +69,6 @@ def test_nvfp4_quantize_rejects_bad_arguments():
     assert q4(codes=NULL) == -1
     assert q4(g=NULL) == -1
     assert q4(ws=NULL) == -1                 # dynamic path needs the workspace
-    assert q4(M=100) == -2                   # rows not a multiple of 128
     assert q4(K=48, ld=48) == -2             # K not a multiple of 64
     assert q4(ld=60) == -2                   # pitch < K
     assert q4(ld=68) == -2                   # pitch not a multiple of 8
@@ -83,6 +84,17 @@ def test_mxfp8_quantize_rejects_bad_arguments():
     assert L.mxfp8_quantize(P16, 128, 128, 128, P_ODD, P16, NULL) == -3
 
 
+def test_mxfp8_quantize_ex_rejects_bad_arguments():
+    def qx(elem=1, rule=0, x=P16, M=128, K=128, codes=P16):
+        return L.mxfp8_quantize_ex(x, M, K, K, codes, P16, elem, rule, NULL)
+    assert qx(elem=0) == -7                   # NVFP4 is not an MXFP8 element type
+    assert qx(elem=3) == -7
+    assert qx(rule=2) == -7
+    assert qx(x=NULL) == -1
+    assert qx(K=64) == -2
+    assert qx(codes=P_ODD) == -3
+
+
 def test_quantize_weight_rejects_bad_format():
     assert L.quantize_weight(5, P16, 128, 64, 64, P16, P16, P16, P16, NULL) == -7
 
@@ -93,11 +105,12 @@ def gemm(fmt=0, a=P16, sa=P16, ga=P16, b=P16, sb=P16, gb=P16, bias=NULL, out=P16
 
 def test_block_scaled_linear_rejects_bad_arguments():
     assert gemm(fmt=3) == -7
+    assert gemm(M=-1) == -2
     assert gemm(a=NULL) == -1
     assert gemm(ga=NULL) == -1                # NVFP4 needs both global scales
     assert gemm(out=NULL) == -1
-    assert gemm(N=64, ldo=64) == -2
-    assert gemm(M=96) == -2
+    assert gemm(N=0, ldo=8) == -2
+    assert gemm(N=130, ldo=136) == -2          # N must be a multiple of 8
     assert gemm(K=96) == -2
     assert gemm(K=192) == -2                  # NVFP4 GEMM K must be a multiple of 256
     assert gemm(fmt=1, ga=NULL, gb=NULL, K=64) == -2     # MXFP8 K must be a multiple of 128
@@ -115,3 +128,8 @@ def test_valid_arguments_without_gpu_report_cuda_error():
         pytest.skip("a GPU is present")
     assert q4() == -5
     assert gemm() == -5
+    # ragged row counts pass the host checks (the scale tiles are padded)
+    assert q4(M=100) == -5
+    assert gemm(M=96, N=64, ldo=64) == -5
+    assert gemm(fmt=2, ga=NULL, gb=NULL, K=128) == -5
+    assert L.mxfp8_quantize_ex(P16, 100, 128, 128, P16, P16, 2, 1, NULL) == -5

@@ -16,7 +16,10 @@ pytestmark = pytest.mark.gpu
 nvq = pytest.importorskip("microscaling_quantized_linear_b200")
 
 
-def gpu_linear(fmt, x, w, bias=None, ldo=None):
+ELEM = {"mxfp8": "e4m3", "mxfp8_e5m2": "e5m2"}
+
+
+def gpu_linear(fmt, x, w, bias=None, ldo=None, guard_rows=0):
     M, K = x.shape
     N = w.shape[0]
     xd, wd = x.cuda(), w.cuda()
@@ -24,11 +27,11 @@ def gpu_linear(fmt, x, w, bias=None, ldo=None):
     if fmt == "nvfp4":
         ac, as_, ag = nvq.nvfp4_quantize(xd)
     else:
-        ac, as_ = nvq.mxfp8_quantize(xd)
+        ac, as_ = nvq.mxfp8_quantize(xd, elem=ELEM[fmt])
         ag = None
-    # NaN-filled output (and padding columns): any tile the kernel fails to
-    # write, or any column it writes by mistake, shows up
-    out = torch.full((M, ldo or N), float("nan"), dtype=torch.bfloat16, device="cuda")[:, :N]
+    # NaN-filled output (and padding columns, and guard rows past M): any tile
+    # the kernel fails to write, or any element it writes by mistake, shows up
+    out = torch.full((M + guard_rows, ldo or N), float("nan"), dtype=torch.bfloat16, device="cuda")[:M, :N]
     bd = bias.cuda() if bias is not None else None
     D = nvq.block_scaled_linear(fmt, ac, as_, ag, wc, ws, wg, M, N, K, bias=bd, out=out)
     assert nvq.device_status() == 0
@@ -44,10 +47,11 @@ def oracle_linear(fmt, x, w, rows=None, bias=None):
         A = oracle.nvfp4_dequantize(ac, as_, ag, M, K)
         B = oracle.nvfp4_dequantize(wc, ws, wg, N, K)
     else:
-        ac, as_ = oracle.mxfp8_quantize(bits(x))
-        wc, ws = oracle.mxfp8_quantize(bits(w))
-        A = oracle.mxfp8_dequantize(ac, as_, M, K)
-        B = oracle.mxfp8_dequantize(wc, ws, N, K)
+        e = ELEM[fmt]
+        ac, as_ = oracle.mxfp8_quantize(bits(x), elem=e)
+        wc, ws = oracle.mxfp8_quantize(bits(w), elem=e)
+        A = oracle.mxfp8_dequantize(ac, as_, M, K, elem=e)
+        B = oracle.mxfp8_dequantize(wc, ws, N, K, elem=e)
     return oracle.gemm_rows(A, B, rows, bias_bits=None if bias is None else bits(bias.reshape(1, -1)))
 
 
@@ -63,6 +67,9 @@ SMALL = [
     ("mxfp8", 384, 512, 640),
     ("mxfp8", 512, 512, 384),          # CTA-pair kernel
     ("mxfp8", 256, 256, 128),          # CTA-pair kernel, one K stage
+    ("mxfp8_e5m2", 128, 128, 128),     # E5M2 x E5M2, one CTA
+    ("mxfp8_e5m2", 512, 512, 384),     # E5M2, CTA pairs
+    ("mxfp8_e5m2", 256, 384, 256),     # E5M2, 256 x 192 pair tiles (two accumulators)
 ]
 
 
@@ -90,6 +97,31 @@ def test_bias_and_output_pitch(fmt):
     D = gpu_linear(fmt, x, w, bias=b, ldo=N + 64)
     full = D.as_strided((M, N + 64), (N + 64, 1))
     assert torch.isnan(full[:, N:]).all(), "padding columns of the output were written"
+    check_gemm(D.float().cpu().numpy(), oracle_linear(fmt, x, w, bias=b))
+
+
+RAGGED = [
+    # row counts that are not multiples of 128 (N a multiple of 8): tensor-map
+    # loads read zeros past the end, stores are clipped, bias is read only for n < N
+    ("nvfp4", 1, 256, 256),
+    ("nvfp4", 100, 200, 256),
+    ("nvfp4", 300, 520, 512),          # CTA pairs, last pair tile mostly empty
+    ("mxfp8", 129, 136, 384),
+    ("mxfp8", 1000, 1000, 256),
+    ("mxfp8_e5m2", 700, 336, 256),
+]
+
+
+@pytest.mark.parametrize("fmt,M,N,K", RAGGED)
+def test_ragged_shapes_with_bias(fmt, M, N, K):
+    x = workloads.normal(M, K, seed=70 + M % 97)
+    w = workloads.normal(N, K, seed=71 + N % 89, std=0.05)
+    b = workloads.bias(N)
+    ldo = (N + 7) // 8 * 8 + 8
+    D = gpu_linear(fmt, x, w, bias=b, ldo=ldo, guard_rows=3)
+    full = D.as_strided((M + 3, ldo), (ldo, 1))
+    assert torch.isnan(full[:M, N:]).all(), "columns past N were written"
+    assert torch.isnan(full[M:]).all(), "rows past M were written"
     check_gemm(D.float().cpu().numpy(), oracle_linear(fmt, x, w, bias=b))
 
 
@@ -152,7 +184,8 @@ sys.path.insert(0, TEST_DIR)
 import test_gpu_gemm as t
 from gpu_common import check_gemm, sample_rows
 import workloads
-for fmt, M, N, K in [("nvfp4", 1024, 768, 512), ("mxfp8", 512, 512, 384), ("nvfp4", 4608, 12288, 3072)]:
+for fmt, M, N, K in [("nvfp4", 1024, 768, 512), ("mxfp8", 512, 512, 384), ("nvfp4", 4608, 12288, 3072),
+                     ("nvfp4", 300, 520, 512), ("mxfp8_e5m2", 700, 336, 256)]:
     x = workloads.normal(M, K, seed=90 + M % 13)
     w = workloads.normal(N, K, seed=91 + N % 11, std=0.05)
     rows = sample_rows(M, per_tile_every=4)

@@ -199,7 +199,8 @@ from gpu_common import act, bits
 ws = nvq.new_workspace()
 cases = [act("actq"), act("ffup"), torch.zeros(4608, 3072, dtype=torch.bfloat16),
          workloads.normal(4608, 3072, seed=78, std=1e-3), act("tiny"), workloads.normal(256, 384, seed=31),
-         workloads.normal(1152, 6144, seed=79)]
+         workloads.normal(1152, 6144, seed=79), workloads.normal(100, 3072, seed=81),
+         workloads.normal(1000, 1536, seed=82)]
 for x in cases:
     codes, sf, g = nvq.nvfp4_quantize(x.cuda(), workspace=ws)
     torch.cuda.synchronize()
@@ -226,6 +227,72 @@ def test_nvfp4_one_pass_path():
     script = ONE_PASS_SCRIPT.replace("ROOT_DIR", repr(root)).replace("TEST_DIR", repr(here))
     out = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True, timeout=600)
     assert out.returncode == 0 and out.stdout.strip().endswith("OK"), out.stdout + out.stderr
+
+
+# ------------------------------------------------------------------ ragged rows
+
+@pytest.mark.parametrize("M,K", [(1, 256), (100, 3072), (129, 512), (1000, 1536)])
+def test_nvfp4_ragged_rows_bit_exact_with_zero_scale_padding(M, K):
+    x = workloads.normal(M, K, seed=80 + M)
+    codes = torch.full((M, K // 2), 0xA5, dtype=torch.uint8, device="cuda")
+    sf = torch.full((nvq.scale_bytes("nvfp4", M, K),), 0xA5, dtype=torch.uint8, device="cuda")
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    nvq.nvfp4_quantize(x.cuda(), codes, sf, g)
+    torch.cuda.synchronize()
+    assert_nvfp4_equal((codes.cpu().numpy(), sf.cpu().numpy(), np.float32(g.item())),
+                       oracle.nvfp4_quantize(bits(x)), M, K)
+    # the calibrated path writes the same padding
+    sf2 = torch.full_like(sf, 0x5A)
+    ca = torch.tensor([oracle.amax(bits(x))], dtype=torch.float32, device="cuda")
+    nvq.nvfp4_quantize(x.cuda(), codes, sf2, g, calib_amax=ca)
+    torch.cuda.synchronize()
+    assert torch.equal(sf2, sf)
+    assert nvq.device_status() == 0
+
+
+# ------------------------------------------------------------------ MXFP8 variants
+
+def special_mxfp8_tensor():
+    """Blocks whose max is exactly 1.75 * 2^e (the rules agree), just above it
+    (the ceil rule steps up), BF16 subnormals, values near the BF16 maximum,
+    zeros and mixed signs; 128 x 512."""
+    x = workloads.normal(128, 512, seed=91).float()
+    x[0, :32] *= 1.75 / x[0, :32].abs().max()
+    x[1, :32] *= 1.7578125 / x[1, :32].abs().max()
+    x[2, 32:64] = x[2, 32:64] * 2.0 ** -130
+    x[3, :32] = 3.0e38 * torch.sign(x[3, :32])
+    x[4, :64] = 0.0
+    x[5, :32] = -x[5, :32].abs()
+    x[6, :32] = 57344.0 * 2.0 ** -10
+    return x.to(torch.bfloat16)
+
+
+MXFP8_VARIANTS = [(e, r) for e in ("e4m3", "e5m2") for r in ("floor", "ceil")]
+MXFP8_VARIANT_INPUTS = [
+    ("tiny_act", lambda: act("tiny")),
+    ("ragged_100x384", lambda: workloads.normal(100, 384, seed=33)),
+    ("special", special_mxfp8_tensor),
+    ("ffdown_act_4608x12288", lambda: act("ffdown")),
+]
+
+
+@pytest.mark.parametrize("elem,rule", MXFP8_VARIANTS, ids=["%s-%s" % v for v in MXFP8_VARIANTS])
+@pytest.mark.parametrize("name,make", MXFP8_VARIANT_INPUTS, ids=[c[0] for c in MXFP8_VARIANT_INPUTS])
+def test_mxfp8_element_and_rule_variants_bit_exact(elem, rule, name, make):
+    x = make()
+    M, K = x.shape
+    codes = torch.full((M, K), 0xA5, dtype=torch.uint8, device="cuda")
+    sf = torch.full((nvq.scale_bytes("mxfp8", M, K),), 0xA5, dtype=torch.uint8, device="cuda")
+    nvq.mxfp8_quantize(x.cuda(), codes, sf, elem=elem, rule=rule)
+    torch.cuda.synchronize()
+    wc, ws = oracle.mxfp8_quantize(bits(x), elem=elem, rule=rule)
+    gc = codes.cpu().numpy()
+    if not np.array_equal(gc, wc):
+        bad = np.argwhere(gc != wc)
+        r, k = bad[0]
+        raise AssertionError("%d code bytes differ; first at (%d, %d): gpu %02x oracle %02x"
+                             % (len(bad), r, k, gc[r, k], wc[r, k]))
+    assert np.array_equal(sf.cpu().numpy(), ws), "scale bytes (or their zero padding) differ"
 
 
 # ------------------------------------------------------------------ MXFP8

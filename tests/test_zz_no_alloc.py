@@ -74,7 +74,7 @@ def test_noalloc_rejects_bad_arguments_without_launching():
     x = workloads.activation("tiny").cuda()
     M, K = x.shape
     null = ctypes.c_void_p(0)
-    rc = nvq._lib.nvfp4_quantize_noalloc(ctypes.c_void_p(x.data_ptr()), M - 1, K, K, null, null, null, null)
-    assert rc == -2                      # rows not a multiple of 128
+    rc = nvq._lib.nvfp4_quantize_noalloc(ctypes.c_void_p(x.data_ptr()), M, K - 16, K, null, null, null, null)
+    assert rc == -2                      # K not a multiple of 64
     rc = nvq._lib.nvfp4_quantize_noalloc(ctypes.c_void_p(x.data_ptr()), M, K, K, null, null, null, null)
     assert rc == -1                      # outputs must be given
