@@ -145,8 +145,9 @@ struct GemmCfg {
     static constexpr int B_BYTES = BN * KBYTES;
     static constexpr int SFA_BYTES = SF_ATOMS * 512;
     static constexpr int SFB_BYTES = SFB_H * SF_ATOMS * 512;
-    static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-    static constexpr int STAGE_BYTES = (TX_BYTES + 1023) / 1024 * 1024;
+    static constexpr int AB_BYTES = A_BYTES + B_BYTES;       // per stage, on full[s]
+    static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;   // per stage, on sfdata[s]
+    static constexpr int STAGE_BYTES = (AB_BYTES + SF_BYTES + 1023) / 1024 * 1024;
     static constexpr int OFF_B = A_BYTES;
     static constexpr int OFF_SFA = A_BYTES + B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
@@ -155,22 +156,24 @@ struct GemmCfg {
     static constexpr int EPI_BYTES = kEpiWarps * EPI_BUF_BYTES;
     static constexpr int SMEM_LIMIT = 232448;
     static constexpr int FIXED_BYTES = 1024 /*align*/ + 512 /*barriers*/ + EPI_BYTES;
-    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-    static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
     // tensor-memory columns: accumulator(s), then scale factors of A and B
     static constexpr int SFA_COLS = FMT == 0 ? 4 * KSTEPS : 4;
     static constexpr int SFB_COLS_PER_MMA = 4 * SFB_H;
     static constexpr int SFB_COLS = FMT == 0 ? SFB_COLS_PER_MMA * KSTEPS : SFB_COLS_PER_MMA;
-    // Scale factors live in SF_SLOTS tensor-memory slots (SF_COLS columns
-    // each), filled by dedicated copy warps ahead of the MMAs.
+    // Each pipeline stage owns one tensor-memory scale slot (SF_COLS columns,
+    // filled by the copy warps ahead of the MMAs), so the stage count is
+    // bounded by shared memory and by the columns left beside the
+    // accumulator(s); two accumulators only when at least 4 slots remain.
     static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
-    static constexpr int ACC_BUFS = (2 * BN + 2 * SF_COLS <= 512) ? 2 : 1;
-    static constexpr int SF_SLOTS_FIT = (512 - ACC_BUFS * BN) / SF_COLS;
-    static constexpr int SF_SLOTS = SF_SLOTS_FIT < STAGES ? SF_SLOTS_FIT : STAGES;
-    static constexpr int TM_SF = ACC_BUFS * BN;            // slot j at TM_SF + j * SF_COLS
-    static constexpr int TM_USED = ACC_BUFS * BN + SF_SLOTS * SF_COLS;
+    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
+    static constexpr int ACC_BUFS = (512 - 2 * BN) / SF_COLS >= 4 ? 2 : 1;
+    static constexpr int SLOTS_FIT = (512 - ACC_BUFS * BN) / SF_COLS;
+    static constexpr int STAGES_MIN2 = STAGES_FIT < SLOTS_FIT ? STAGES_FIT : SLOTS_FIT;
+    static constexpr int STAGES = STAGES_MIN2 > 6 ? 6 : STAGES_MIN2;
+    static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
+    static constexpr int TM_SF = ACC_BUFS * BN;            // slot s at TM_SF + s * SF_COLS
+    static constexpr int TM_USED = ACC_BUFS * BN + STAGES * SF_COLS;
     static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
     // copy jobs per stage: the A scales, then each 128-row block of B scales;
     // one warp per job (a tcgen05.cp takes ~100 cycles to issue, so the jobs
@@ -187,8 +190,7 @@ struct GemmCfg {
         ((uint32_t)(BM >> 4) << 24);
     static_assert(BN == 128 || BN == 192 || BN == 256, "tile width");
     static_assert(TM_USED <= 512, "tensor memory overflow");
-    static_assert(SF_SLOTS >= 2, "tensor memory too small for two scale slots");
-    static_assert(STAGES >= 2, "shared memory too small for two stages");
+    static_assert(STAGES >= 3, "too few pipeline stages");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory overflow");
 };
 
@@ -236,27 +238,30 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
-    const uint32_t full0 = smem_u32(bars);                 // [STAGES]  TMA -> copy warps, MMA
-    const uint32_t empty0 = full0 + 8 * C::STAGES;         // [STAGES]  MMA -> TMA
-    const uint32_t sffull0 = empty0 + 8 * C::STAGES;       // [SF_SLOTS] copy warps -> MMA
-    const uint32_t sfempty0 = sffull0 + 8 * C::SF_SLOTS;   // [SF_SLOTS] MMA -> copy warps
-    const uint32_t tfull0 = sfempty0 + 8 * C::SF_SLOTS;    // [2]  MMA -> epilogue
+    // The MMA lane waits once per stage (the tensor pipe holds little more
+    // than one MMA in flight, so its barrier checks are idle pipe time):
+    //   full[s]   A and B tiles landed (tx) + the copy warps' commits of the
+    //             stage's scales into tensor-memory slot s
+    //   sfdata[s] the stage's scale tiles landed (tx): the copy warps' wait
+    //   empty[s]  the stage's MMAs completed: frees shared-memory stage s
+    //             and scale slot s
+    const uint32_t full0 = smem_u32(bars);                 // [STAGES]
+    const uint32_t empty0 = full0 + 8 * C::STAGES;         // [STAGES]
+    const uint32_t sfdata0 = empty0 + 8 * C::STAGES;       // [STAGES]
+    const uint32_t tfull0 = sfdata0 + 8 * C::STAGES;       // [2]  MMA -> epilogue
     const uint32_t tempty0 = tfull0 + 8 * 2;               // [2]  epilogue -> MMA
     const uint32_t drain = tempty0 + 8 * 2;                // MMA warp's own completion
     const uint32_t sfdrain = drain + 8;                    // copy warps' own completion
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 2 * C::SF_SLOTS + 6);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* never = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(full0 + 8 * s, 1);
+            mbar_init(full0 + 8 * s, 1 + C::SF_WARPS);
             mbar_init(empty0 + 8 * s, 1);
-        }
-        for (int j = 0; j < C::SF_SLOTS; ++j) {
-            mbar_init(sffull0 + 8 * j, C::SF_WARPS);
-            mbar_init(sfempty0 + 8 * j, 1);
+            mbar_init(sfdata0 + 8 * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
@@ -303,22 +308,25 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                         break;
                     }
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
-                    const uint32_t fb = full0 + 8 * s;
-                    mbar_arrive_expect_tx(fb, C::TX_BYTES);
-                    tma_load_2d(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), (int32_t)(mb * C::BM));
-                    tma_load_2d(st + C::OFF_B, &tmap_b, fb, (int32_t)(kt * C::KBYTES), (int32_t)(nb * BN));
-                    // plain bulk copies have no out-of-range fill: a B tile that
-                    // runs past N (its rows are not stored) reads the last scale tile
+                    const uint32_t fb = full0 + 8 * s, sb = sfdata0 + 8 * s;
+                    mbar_arrive_expect_tx(sb, C::SF_BYTES);
+                    mbar_arrive_expect_tx(fb, C::AB_BYTES);
+                    // scale tiles first: the copy warps need them before the MMAs
+                    // can run.  Plain bulk copies have no out-of-range fill: a B
+                    // tile that runs past N (its rows are not stored) reads the
+                    // last scale tile.
                     bulk_load(st + C::OFF_SFA,
                               p.sfa + ((size_t)mb * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
-                              C::SFA_BYTES, fb);
+                              C::SFA_BYTES, sb);
 #pragma unroll
                     for (int h = 0; h < C::SFB_H; ++h) {
                         const uint32_t bt = min(a0 + h, p.sfb_rtiles - 1);
                         bulk_load(st + C::OFF_SFB + h * C::SF_ATOMS * 512,
                                   p.sfb + ((size_t)bt * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
-                                  C::SF_ATOMS * 512, fb);
+                                  C::SF_ATOMS * 512, sb);
                     }
+                    tma_load_2d(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), (int32_t)(mb * C::BM));
+                    tma_load_2d(st + C::OFF_B, &tmap_b, fb, (int32_t)(kt * C::KBYTES), (int32_t)(nb * BN));
                     ++it;
                 }
             }
@@ -327,8 +335,10 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 atomicOr(p.status, 1u);
             }
             // every load this thread issued must land before the CTA exits
-            for (uint32_t j = it > (uint32_t)C::STAGES ? it - C::STAGES : 0; j < it; ++j)
+            for (uint32_t j = it > (uint32_t)C::STAGES ? it - C::STAGES : 0; j < it; ++j) {
+                mbar_wait_bounded(sfdata0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
                 mbar_wait_bounded(full0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
+            }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
@@ -348,15 +358,13 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 const uint32_t d_tmem = tmem + buf * BN;
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt, ++it) {
                     const uint32_t s = it % C::STAGES, su = it / C::STAGES;
-                    const uint32_t slot = it % C::SF_SLOTS, sv = it / C::SF_SLOTS;
-                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs) ||
-                        !mbar_wait_bounded(sffull0 + 8 * slot, sv & 1, abort_flag, kWaitLimitNs)) {
+                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
-                    const uint32_t sfa_t = tmem + C::TM_SF + slot * C::SF_COLS;
+                    const uint32_t sfa_t = tmem + C::TM_SF + s * C::SF_COLS;
                     const uint32_t sfb_t = sfa_t + C::SFA_COLS;
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k) {
@@ -372,8 +380,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                                         (sfb_t + sfb_shift) | ((uint32_t)k << 30), acc);
                         }
                     }
-                    tc_commit(empty0 + 8 * s);        // shared-memory stage free
-                    tc_commit(sfempty0 + 8 * slot);   // scale slot free
+                    tc_commit(empty0 + 8 * s);        // shared-memory stage and scale slot free
                 }
                 if (!ok) break;
                 tc_commit(tfull0 + 8 * buf);
@@ -392,15 +399,15 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             bool ok = true;
             for (uint32_t it = 0; it < total_iters; ++it) {
                 const uint32_t s = it % C::STAGES, su = it / C::STAGES;
-                const uint32_t slot = it % C::SF_SLOTS, sv = it / C::SF_SLOTS;
-                if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs) ||
-                    (sv > 0 && !mbar_wait_bounded(sfempty0 + 8 * slot, (sv - 1) & 1, abort_flag, kWaitLimitNs))) {
+                // slot s is free once the MMAs of its previous use completed
+                if ((su > 0 && !mbar_wait_bounded(empty0 + 8 * s, (su - 1) & 1, abort_flag, kWaitLimitNs)) ||
+                    !mbar_wait_bounded(sfdata0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                sf_copy_job<C, false>(job, smem_u32(smem + s * C::STAGE_BYTES), tmem + C::TM_SF + slot * C::SF_COLS);
-                tc_commit(sffull0 + 8 * slot);
+                sf_copy_job<C, false>(job, smem_u32(smem + s * C::STAGE_BYTES), tmem + C::TM_SF + s * C::SF_COLS);
+                tc_commit(full0 + 8 * s);             // the copies' share of the MMA's wait
             }
             if (!ok) {
                 *abort_flag = 1;

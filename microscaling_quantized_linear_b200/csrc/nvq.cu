@@ -424,7 +424,12 @@ int launch_for_format(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_sc
                                           M, N, K, s);
     }
     // One CTA per tile: width 256 when N allows it (fewest scale-factor copies
-    // per MMA), else 192 (two tensor-memory accumulators), else 128 (two).
+    // per MMA), else 192, else 128 (two accumulators).  When 256-wide tiles
+    // would leave SMs idle (a short M: the weight stream is then the cost),
+    // 128-wide tiles spread it over twice as many SMs.
+    if ((M + 127) / 128 * ((N + 255) / 256) < d->num_sms)
+        return launch_gemm<FMT, 128>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M,
+                                     N, K, s);
     if (N % 256 == 0)
         return launch_gemm<FMT, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M,
                                      N, K, s);
