@@ -177,6 +177,25 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     DeviceInfo* d = nullptr;
     if ((rc = device_info(&d))) return rc;
     const uint32_t nblk = (uint32_t)(K / 16);
+    if (!calib_amax && (uint64_t)M * nblk <= kClusterMaxBlocks) {
+        // small tensor: one launch of one cluster, the maximum exchanged in
+        // distributed shared memory (the workspace is not touched)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kClusterCtas);
+        cfg.blockDim = dim3(kClusterThreads);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, nvfp4_quantize_cluster_kernel, static_cast<const uint16_t*>(x), (uint32_t)M, nblk,
+                               (uint32_t)ldx, codes, scales, global_scale, d->status) != cudaSuccess) {
+            cudaGetLastError();
+            return NVQ_ERR_CUDA;
+        }
+        return NVQ_OK;
+    }
     if (!calib_amax && g_quant_one_pass) {
         // One pass when every CTA's rows fit in shared memory (one CTA per SM).
         const int64_t rows_per_cta = (M + d->num_sms - 1) / d->num_sms;

@@ -270,6 +270,92 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
     zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kQuantThreads + threadIdx.x, stride);
 }
 
+// ------------------------------------------------------------------ NVFP4, small tensors
+// One cluster of kClusterCtas CTAs quantizes a tensor of at most
+// kClusterMaxBlocks 16-blocks in one launch: each thread holds up to
+// kClusterBlocksPerThread blocks in registers, each CTA reduces its maximum,
+// the CTAs exchange their maxima through distributed shared memory (all into
+// CTA 0's array, one cluster barrier), and every thread quantizes the blocks
+// it holds.  No workspace, no second read of the tensor, no grid barrier.
+constexpr int kClusterCtas = 8;
+constexpr int kClusterThreads = 1024;
+constexpr int kClusterBlocksPerThread = 4;
+constexpr uint32_t kClusterMaxBlocks = (uint32_t)kClusterCtas * kClusterThreads * kClusterBlocksPerThread;
+
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterThreads, 1)
+nvfp4_quantize_cluster_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nblk, uint32_t ldx,
+                              uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                              float* __restrict__ g_dec_out, unsigned int* __restrict__ status) {
+    __shared__ uint32_t red[kClusterThreads / 32];
+    __shared__ uint32_t cta_max[kClusterCtas];             // used in CTA 0: one slot per CTA
+    __shared__ float d6[128], rtab[128];
+    const uint32_t rank = cluster_ctarank();
+    const uint32_t nthr = kClusterCtas * kClusterThreads;
+    const uint32_t tid = rank * kClusterThreads + threadIdx.x;
+    const uint32_t total = rows * nblk;
+    griddep_wait();                                        // x may come from the previous grid
+    griddep_launch();
+    uint4 v[2 * kClusterBlocksPerThread];
+    const uint4 zero4 = make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int i = 0; i < kClusterBlocksPerThread; ++i) {
+        const uint32_t b = tid + (uint32_t)i * nthr;
+        if (b < total) {
+            const uint32_t r = b / nblk, c = b - r * nblk;
+            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
+            v[2 * i] = __ldg(src);
+            v[2 * i + 1] = __ldg(src + 1);
+        } else {
+            v[2 * i] = v[2 * i + 1] = zero4;
+        }
+    }
+    init_d6(d6);
+    uint32_t mb[kClusterBlocksPerThread], m = 0;
+#pragma unroll
+    for (int i = 0; i < kClusterBlocksPerThread; ++i) {
+        const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
+                               v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
+        mb[i] = block16_max(w);
+        m = max(m, mb[i]);
+    }
+    m = block_max_u32<kClusterThreads>(m, red);
+    if (threadIdx.x == 0) st_shared_cluster_u32(mapa_shared(smem_u32(&cta_max[rank]), 0), m);
+    cluster_sync();                                        // CTA 0's array complete (release / acquire)
+    uint32_t all = threadIdx.x < kClusterCtas ? ld_shared_cluster_u32(mapa_shared(smem_u32(&cta_max[threadIdx.x]), 0))
+                                              : 0u;
+    all = __reduce_max_sync(0xFFFFFFFFu, all);            // warp 0 holds the tensor's max
+    if (threadIdx.x == 0) red[0] = all;
+    cluster_sync();                                        // every CTA has read CTA 0's array
+    const uint32_t amax_bits = red[0];
+    if (amax_bits >= 0x7F80u && tid == 0) atomicOr(status, 2u);
+    const float amax = __uint_as_float(amax_bits << 16);
+    const float g_enc = encode_scale(amax);
+    if (tid == 0) *g_dec_out = decode_scale(amax);
+    init_rtab(rtab, g_enc);
+    __syncthreads();
+    const uint32_t ctiles = nblk >> 2;
+#pragma unroll
+    for (int i = 0; i < kClusterBlocksPerThread; ++i) {
+        const uint32_t b = tid + (uint32_t)i * nthr;
+        if (b - threadIdx.x % 32 >= total) break;          // whole warps past the end stop together
+        const bool active = b < total;
+        const uint32_t r = b / nblk, c = b - r * nblk;
+        const uint32_t w[8] = {v[2 * i].x, v[2 * i].y, v[2 * i].z, v[2 * i].w,
+                               v[2 * i + 1].x, v[2 * i + 1].y, v[2 * i + 1].z, v[2 * i + 1].w};
+        uint32_t lo, hi;
+        const uint32_t sc = nvfp4_block(mb[i], w, g_enc, d6, rtab, lo, hi);
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
+        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
+        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
+        if (active) {
+            *reinterpret_cast<uint2*>(codes + (size_t)b * 8) = make_uint2(lo, hi);
+            if ((c & 3u) == 0)
+                *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r, c, ctiles)) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        }
+    }
+    zero_pad_scale_rows(sf, rows, ctiles, tid, nthr);
+}
+
 // ------------------------------------------------------------------ NVFP4, one pass
 // For tensors whose rows fit in the shared memory of one CTA per SM: every
 // CTA copies its rows into shared memory once (bulk copies, 4 chunks with
