@@ -302,6 +302,8 @@ def run_ours(args, rank, world, device):
     }
     if args.mxfp8:
         res["mxfp8_ffdown"] = run_mxfp8_component(nvq, args, device, stream, peaks)
+    if args.small_m:
+        res["small_m"] = run_small_m_component(nvq, device, stream, peaks)
     return res
 
 
@@ -345,41 +347,115 @@ def run_e2e(nvq, args, device, stream, x_host_src, wq, M, N, K, flops, world):
             "ms_per_step": round(ms, 4), "steps": steps}
 
 
-def run_mxfp8_component(nvq, args, device, stream, peaks):
-    """MXFP8 FF-down linear (A [4608,12288] GELU(N(0,1)), W [3072,12288]):
-    per-kernel times of the MXFP8 quantizer and the MXFP8 GEMM."""
-    w = workloads.WORKLOADS["ffdown"]
-    M, N, K = w.M, w.N, w.K
-    xs = [workloads.activation("ffdown", seed=i).to(device) for i in range(2)]
-    wc, wsf, _ = nvq.quantize_weight("mxfp8", workloads.weight("ffdown").to(device))
+def _time_mxfp8(nvq, xs, wq, fmt, elem, rule, M, N, K, device, stream, iters=50):
+    wc, wsf = wq
     codes = torch.empty((M, K), dtype=torch.uint8, device=device)
-    scales = torch.empty(nvq.scale_bytes("mxfp8", M, K), dtype=torch.uint8, device=device)
+    scales = torch.empty(nvq.scale_bytes(fmt, M, K), dtype=torch.uint8, device=device)
     out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-    iters = 50
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
     for i in range(5 + iters):
         timed = i >= 5
         e = evs[i - 5] if timed else None
         if timed:
             e[0].record(stream)
-        nvq.mxfp8_quantize(xs[i % 2], codes, scales, stream=stream)
+        nvq.mxfp8_quantize(xs[i % 2], codes, scales, stream=stream, elem=elem, rule=rule)
         if timed:
             e[1].record(stream)
-        nvq.block_scaled_linear("mxfp8", codes, scales, None, wc, wsf, None, M, N, K, out=out, stream=stream)
+        nvq.block_scaled_linear(fmt, codes, scales, None, wc, wsf, None, M, N, K, out=out, stream=stream)
         if timed:
             e[2].record(stream)
     torch.cuda.synchronize(device)
     q_us = statistics.mean(e[0].elapsed_time(e[1]) * 1e3 for e in evs)
     g_us = statistics.mean(e[1].elapsed_time(e[2]) * 1e3 for e in evs)
+    return q_us, g_us
+
+
+def run_mxfp8_component(nvq, args, device, stream, peaks):
+    """MXFP8 FF-down linear (A [4608,12288] GELU(N(0,1)), W [3072,12288]):
+    per-kernel times of the MXFP8 quantizer and the MXFP8 GEMM, for E4M3
+    elements with the OCP floor exponent and for E5M2 elements with the
+    ceil exponent (quantizer) and the E5M2 x E5M2 GEMM."""
+    w = workloads.WORKLOADS["ffdown"]
+    M, N, K = w.M, w.N, w.K
+    xs = [workloads.activation("ffdown", seed=i).to(device) for i in range(2)]
+    wd = workloads.weight("ffdown").to(device)
     flops = 2.0 * M * N * K
     fp8_peak = peaks["bf16_tflops"] * 2.0
     qbytes = M * K * (2 + 1 + 1 / 32)
-    return {"workload": "MXFP8 FF-down 4608x3072x12288", "quant_us": round(q_us, 3),
-            "quant_gbs": round(qbytes / (q_us * 1e-6) / 1e9, 1),
-            "quant_frac_hbm": round(qbytes / (q_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
-            "gemm_us": round(g_us, 3), "gemm_tflops": round(flops / (g_us * 1e-6) / 1e12, 1),
-            "gemm_frac_fp8": round(flops / (g_us * 1e-6) / 1e12 / fp8_peak, 4),
-            "fp8_peak": round(fp8_peak, 1), "l2": "2 activation batches (226 MB) alternate"}
+    res = {"workload": "MXFP8 FF-down 4608x3072x12288", "l2": "2 activation batches (226 MB) alternate",
+           "fp8_peak": round(fp8_peak, 1)}
+    for fmt, elem, rule, key in (("mxfp8", "e4m3", "floor", ""), ("mxfp8_e5m2", "e5m2", "ceil", "e5m2_ceil_")):
+        wc, wsf, _ = nvq.quantize_weight(fmt, wd)
+        q_us, g_us = _time_mxfp8(nvq, xs, (wc, wsf), fmt, elem, rule, M, N, K, device, stream)
+        res.update({key + "quant_us": round(q_us, 3),
+                    key + "quant_gbs": round(qbytes / (q_us * 1e-6) / 1e9, 1),
+                    key + "quant_frac_hbm": round(qbytes / (q_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                    key + "gemm_us": round(g_us, 3), key + "gemm_tflops": round(flops / (g_us * 1e-6) / 1e12, 1),
+                    key + "gemm_frac_fp8": round(flops / (g_us * 1e-6) / 1e12 / fp8_peak, 4)})
+    return res
+
+
+def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200):
+    """Short batches of the FF-up linear (N 12288, K 3072, NVFP4): latency of
+    one quantize + GEMM step issued eagerly and replayed from a CUDA graph,
+    and the GEMM's weight stream (the bytes a short M cannot avoid)."""
+    w = workloads.WORKLOADS["ffup"]
+    N, K = w.N, w.K
+    wc, wsf, wg = nvq.quantize_weight("nvfp4", workloads.weight("ffup").to(device))
+    wbytes = N * K * 0.5625
+    res = {"workload": "NVFP4 FF-up N 12288 K 3072 at short M", "weight_bytes": int(wbytes)}
+    for M in Ms:
+        x = workloads.normal(M, K, seed=5).to(device)
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+        sf = torch.empty(nvq.scale_bytes("nvfp4", M, K), dtype=torch.uint8, device=device)
+        g = torch.empty(1, dtype=torch.float32, device=device)
+        ws = nvq.new_workspace(device)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+
+        def step(s):
+            nvq.nvfp4_quantize(x, codes, sf, g, workspace=ws, stream=s)
+            nvq.block_scaled_linear("nvfp4", codes, sf, g, wc, wsf, wg, M, N, K, out=out, stream=s)
+
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(10):
+            step(stream)
+        torch.cuda.synchronize(device)
+        a.record(stream)
+        for _ in range(iters):
+            step(stream)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        eager = a.elapsed_time(b) / iters * 1e3
+        a.record(stream)
+        for _ in range(iters):
+            nvq.block_scaled_linear("nvfp4", codes, sf, g, wc, wsf, wg, M, N, K, out=out, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        gemm = a.elapsed_time(b) / iters * 1e3
+        cs = torch.cuda.Stream(device)
+        cs.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cs):
+            step(cs)
+            torch.cuda.synchronize(device)
+            with torch.cuda.graph(graph, stream=cs):
+                step(cs)
+        torch.cuda.synchronize(device)
+        for _ in range(10):
+            graph.replay()
+        torch.cuda.synchronize(device)
+        a.record()
+        for _ in range(iters):
+            graph.replay()
+        b.record()
+        torch.cuda.synchronize(device)
+        graphed = a.elapsed_time(b) / iters * 1e3
+        del graph
+        res["M%d" % M] = {"step_us_eager": round(eager, 2), "step_us_graph": round(graphed, 2),
+                          "gemm_us": round(gemm, 2),
+                          "gemm_weight_gbs": round(wbytes / (gemm * 1e-6) / 1e9, 1),
+                          "gemm_weight_frac_hbm": round(wbytes / (gemm * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
+    return res
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -468,6 +544,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mxfp8", dest="mxfp8", action="store_false")
+    ap.add_argument("--no-small-m", dest="small_m", action="store_false")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
