@@ -60,6 +60,10 @@ def lib():
         L.oracle_mxfp8_quantize_ex.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int, _u8p, _u8p]
         L.oracle_mxfp8_dequantize_ex.restype = None
         L.oracle_mxfp8_dequantize_ex.argtypes = [_u8p, _u8p, _i64, _i64, ctypes.c_int, _f64p]
+        L.oracle_double_to_bf16.restype = ctypes.c_uint16
+        L.oracle_double_to_bf16.argtypes = [ctypes.c_double]
+        L.oracle_gelu_bf16.restype = ctypes.c_uint16
+        L.oracle_gelu_bf16.argtypes = [ctypes.c_uint16]
         L.oracle_e5m2_value.restype = ctypes.c_double
         L.oracle_e5m2_value.argtypes = [ctypes.c_int]
         L.oracle_e5m2_encode.restype = ctypes.c_int
@@ -158,6 +162,18 @@ def nvfp4_dequantize(codes, sf, g_dec, rows, K):
     out = np.empty((rows, K), dtype=np.float64)
     lib().oracle_nvfp4_dequantize(_ptr(codes, _u8p), _ptr(sf, _u8p), float(g_dec), rows, K, _ptr(out, _f64p))
     return out
+
+
+def double_to_bf16(v):
+    """binary64 -> BF16 bit pattern, one round-to-nearest-even."""
+    return int(lib().oracle_double_to_bf16(float(v)))
+
+
+def gelu_bf16(bits_arr):
+    """GELU (exact erf, binary64) of BF16 bit patterns, rounded once to BF16."""
+    a = np.ascontiguousarray(bits_arr, dtype=np.uint16)
+    f = lib().oracle_gelu_bf16
+    return np.vectorize(lambda b: f(int(b)), otypes=[np.uint16])(a)
 
 
 ELEMS = {"e4m3": 0, "e5m2": 1}

@@ -45,6 +45,9 @@
  *     S.11111.00 = infinity, S.11111.xx = NaN; encoding saturates at 57344.
  *   - Ragged row counts: codes are dense over the M rows; the scale tiles
  *     are padded to a multiple of 128 rows with zero bytes.
+ *   - The activation between the two linears of a feed-forward block is GELU
+ *     with the exact error function, 0.5 x (1 + erf(x / sqrt 2)), evaluated in
+ *     binary64 on the BF16 output of the first linear and rounded once to BF16.
  *   - Scale bytes are stored in the 128x4 tensor-core tile order (see
  *     oracle_sf_offset).
  *   - Codes are K-contiguous; two E2M1 codes per byte, even element in the
@@ -175,6 +178,42 @@ static float bf16_to_float(uint16_t h) {
     float f;
     memcpy(&f, &u, 4);
     return f;
+}
+
+/* binary64 -> BF16 bits, round to nearest even (one rounding; overflow to
+ * infinity, NaN kept quiet).  Written from the binary64 fields. */
+ORACLE_EXPORT uint16_t oracle_double_to_bf16(double v) {
+    uint64_t u;
+    memcpy(&u, &v, 8);
+    const uint16_t sign = (uint16_t)((u >> 48) & 0x8000u);
+    if (isnan(v)) return (uint16_t)(sign | 0x7FC0u);
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    /* a = m * 2^e with m in [1, 2) */
+    int e;
+    (void)frexp(a, &e);                  /* a = f * 2^e, f in [0.5, 1) */
+    e -= 1;                              /* a = (2f) * 2^e */
+    if (e > 127) return (uint16_t)(sign | 0x7F80u);
+    /* quantum of the BF16 grid at this exponent: 2^(e-7) for normals,
+     * 2^-133 for subnormals (e < -126) */
+    int qexp = (e < -126) ? -133 : e - 7;
+    double units = ldexp(a, -qexp);      /* exact: a / quantum */
+    double fl = floor(units), rem = units - fl;
+    double r = fl;
+    if (rem > 0.5 || (rem == 0.5 && fmod(fl, 2.0) != 0.0)) r = fl + 1.0;
+    double rounded = ldexp(r, qexp);     /* exact */
+    if (rounded >= 0x1p128) return (uint16_t)(sign | 0x7F80u);
+    float rf = (float)rounded;           /* exact: rounded is on the BF16 grid */
+    uint32_t b;
+    memcpy(&b, &rf, 4);
+    return (uint16_t)(sign | (uint16_t)((b >> 16) & 0x7FFFu));
+}
+
+/* GELU of a BF16 value, exact-erf form in binary64, rounded once to BF16. */
+ORACLE_EXPORT uint16_t oracle_gelu_bf16(uint16_t in) {
+    double x = (double)bf16_to_float(in);
+    double g = 0.5 * x * (1.0 + erf(x * 0.70710678118654752440));
+    return oracle_double_to_bf16(g);
 }
 
 /* ------------------------------------------------------------------ */

@@ -581,3 +581,71 @@ def test_ragged_rows_equal_the_zero_padded_tensor(M):
         assert np.array_equal(s8, s8p)
     nblk = K // 16
     assert all(s[oracle.sf_offset(r, j, nblk)] == 0 for r in range(M, Mp) for j in range(nblk))
+
+
+# --------------------------------------------------------------------------
+# Epilogue activation: binary64 -> BF16 rounding and GELU
+# --------------------------------------------------------------------------
+
+def _bf16_round_exact(v):
+    """Independent reference: round a binary64 value to BF16 with exact
+    rational arithmetic (nearest, ties to the even significand)."""
+    from fractions import Fraction
+    import math
+    if v == 0:
+        return 0x8000 if math.copysign(1.0, v) < 0 else 0
+    sign = 0x8000 if v < 0 else 0
+    a = Fraction(abs(v))
+    e = math.floor(math.log2(abs(v)))
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    q = Fraction(2) ** (max(e, -126) - 7)          # spacing of BF16 values here
+    n = a / q
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    r = fl + (1 if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2) else 0)
+    val = r * q
+    if val >= Fraction(2) ** 128:
+        return sign | 0x7F80
+    f32 = np.float32(float(val))
+    return sign | (int(np.array([f32]).view(np.uint32)[0]) >> 16) & 0x7FFF
+
+
+def test_double_to_bf16_matches_exact_rounding_and_torch():
+    # ties, values just off ties (where rounding through binary32 first would
+    # give the wrong answer), subnormals, overflow
+    cases = [1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -8 + 2 ** -40, 1.0 + 2 ** -8 - 2 ** -40,
+             -(1.0 + 2 ** -8 + 2 ** -40), 2.0 ** -133, 1.5 * 2.0 ** -133, 2.0 ** -134, 0.75 * 2.0 ** -133,
+             2.0 ** -126 * 1.00390625, 3.3895313892515355e38, 3.4e38, 1e300, -0.0]
+    for v in cases:
+        assert oracle.double_to_bf16(v) == _bf16_round_exact(v), v
+    # 1 + 2^-8 + 2^-40 is above the tie: rounds up, although binary32 rounding
+    # first would land on the tie and then round to even (down)
+    assert oracle.double_to_bf16(1.0 + 2 ** -8 + 2 ** -40) == 0x3F81
+    rng = np.random.default_rng(43)
+    vals = rng.standard_normal(5000) * np.exp2(rng.integers(-140, 120, 5000))
+    for v in vals[:400]:
+        assert oracle.double_to_bf16(float(v)) == _bf16_round_exact(float(v)), v
+    # values exactly representable in binary32: one rounding, as torch's cast
+    f32 = vals.astype(np.float32)
+    want = torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.double_to_bf16(float(v)) for v in f32], dtype=np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_gelu_bf16_matches_scipy_erf_and_limits():
+    from scipy.special import erf
+    x = torch.cat([workloads.normal(64, 64, seed=47, std=3.0).flatten(),
+                   torch.tensor([0.0, -0.0, 1.0, -1.0, 10.0, -10.0, 3e38, -3e38, 1e-30, -1e-30])]).to(torch.bfloat16)
+    b = x.view(torch.int16).numpy().view(np.uint16)
+    got = oracle.gelu_bf16(b)
+    xd = x.double().numpy()
+    ref = 0.5 * xd * (1.0 + erf(xd * 0.70710678118654752440))
+    want = np.array([_bf16_round_exact(float(v)) for v in ref], dtype=np.uint16)
+    assert np.array_equal(got, want)
+    # closed forms: GELU(0) = 0, GELU(x) = x for large x, GELU(-large) = -0,
+    # GELU(1) = Phi(1) = 0.8413447... -> BF16 0.83984375 (0x3F57)
+    tail = got[-10:].tolist()          # inputs 0, -0, 1, -1, 10, -10, 3e38, -3e38, 1e-30, -1e-30
+    assert tail[0] == 0 and tail[1] == 0x8000 and tail[2] == 0x3F57 and tail[4] == 0x4120 and tail[5] == 0x8000
