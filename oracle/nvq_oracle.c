@@ -180,9 +180,11 @@ static float bf16_to_float(uint16_t h) {
     return f;
 }
 
-/* binary64 -> BF16 bits, round to nearest even (one rounding; overflow to
- * infinity, NaN kept quiet).  Written from the binary64 fields. */
-ORACLE_EXPORT uint16_t oracle_double_to_bf16(double v) {
+/* binary64 -> BF16 bits, round to nearest (one rounding; overflow to
+ * infinity, NaN kept quiet).  A value exactly half-way between two BF16
+ * values goes to the even one (tie = 0), or toward +infinity (tie > 0) or
+ * -infinity (tie < 0).  Written from the binary64 fields. */
+static uint16_t bf16_round_tie(double v, int tie) {
     uint64_t u;
     memcpy(&u, &v, 8);
     const uint16_t sign = (uint16_t)((u >> 48) & 0x8000u);
@@ -200,7 +202,11 @@ ORACLE_EXPORT uint16_t oracle_double_to_bf16(double v) {
     double units = ldexp(a, -qexp);      /* exact: a / quantum */
     double fl = floor(units), rem = units - fl;
     double r = fl;
-    if (rem > 0.5 || (rem == 0.5 && fmod(fl, 2.0) != 0.0)) r = fl + 1.0;
+    int up;                              /* round the magnitude up */
+    if (rem != 0.5) up = rem > 0.5;
+    else if (tie == 0) up = fmod(fl, 2.0) != 0.0;
+    else up = (tie > 0) == (sign == 0); /* toward +inf grows a positive magnitude */
+    if (up) r = fl + 1.0;
     double rounded = ldexp(r, qexp);     /* exact */
     if (rounded >= 0x1p128) return (uint16_t)(sign | 0x7F80u);
     float rf = (float)rounded;           /* exact: rounded is on the BF16 grid */
@@ -209,11 +215,34 @@ ORACLE_EXPORT uint16_t oracle_double_to_bf16(double v) {
     return (uint16_t)(sign | (uint16_t)((b >> 16) & 0x7FFFu));
 }
 
-/* GELU of a BF16 value, exact-erf form in binary64, rounded once to BF16. */
+ORACLE_EXPORT uint16_t oracle_double_to_bf16(double v) { return bf16_round_tie(v, 0); }
+
+/* GELU of a BF16 value, x * Phi(x) with Phi the standard normal CDF (the
+ * exact-erf form), rounded once to BF16.
+ *   |x| >= 1:  x * erfc(-x / sqrt 2) / 2 in binary64; the same function as
+ *              x (1 + erf(x / sqrt 2)) / 2 without its cancellation for
+ *              negative x (GELU(-10) is -7.6e-23, not 0).
+ *   |x| < 1:   x/2 + (x/2) erf(x / sqrt 2), the exact sum of the two binary64
+ *              terms (TwoSum: s + err).  For a subnormal x, x/2 can fall
+ *              exactly half-way between two BF16 values; the second term,
+ *              about x^2 / sqrt(2 pi) > 0, then decides, although it is far
+ *              below binary64 resolution at x/2.
+ * GELU(+-0) = +-0; GELU(+inf) = +inf; GELU(-inf) is its limit, -0. */
 ORACLE_EXPORT uint16_t oracle_gelu_bf16(uint16_t in) {
-    double x = (double)bf16_to_float(in);
-    double g = 0.5 * x * (1.0 + erf(x * 0.70710678118654752440));
-    return oracle_double_to_bf16(g);
+    const double x = (double)bf16_to_float(in);
+    const double c = 0.70710678118654752440;
+    if (isnan(x)) return oracle_double_to_bf16(x);
+    if (isinf(x)) return x > 0 ? 0x7F80u : 0x8000u;
+    if (x == 0.0) return in;
+    if (fabs(x) >= 1.0) return oracle_double_to_bf16(0.5 * x * erfc(-x * c));
+    const double h = 0.5 * x;            /* exact */
+    const double t = h * erf(x * c);
+    const double s = h + t;
+    const double bb = s - h;
+    const double err = (h - (s - bb)) + (t - bb);
+    /* s + err = h + t exactly; s is the binary64 nearest to it, so only
+     * when s is itself a BF16 tie can err change the rounding */
+    return bf16_round_tie(s, err > 0 ? 1 : (err < 0 ? -1 : 0));
 }
 
 /* ------------------------------------------------------------------ */

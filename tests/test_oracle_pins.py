@@ -635,17 +635,70 @@ def test_double_to_bf16_matches_exact_rounding_and_torch():
     assert np.array_equal(got, want)
 
 
-def test_gelu_bf16_matches_scipy_erf_and_limits():
-    from scipy.special import erf
-    x = torch.cat([workloads.normal(64, 64, seed=47, std=3.0).flatten(),
-                   torch.tensor([0.0, -0.0, 1.0, -1.0, 10.0, -10.0, 3e38, -3e38, 1e-30, -1e-30])]).to(torch.bfloat16)
-    b = x.view(torch.int16).numpy().view(np.uint16)
-    got = oracle.gelu_bf16(b)
-    xd = x.double().numpy()
-    ref = 0.5 * xd * (1.0 + erf(xd * 0.70710678118654752440))
-    want = np.array([_bf16_round_exact(float(v)) for v in ref], dtype=np.uint16)
-    assert np.array_equal(got, want)
-    # closed forms: GELU(0) = 0, GELU(x) = x for large x, GELU(-large) = -0,
-    # GELU(1) = Phi(1) = 0.8413447... -> BF16 0.83984375 (0x3F57)
-    tail = got[-10:].tolist()          # inputs 0, -0, 1, -1, 10, -10, 3e38, -3e38, 1e-30, -1e-30
-    assert tail[0] == 0 and tail[1] == 0x8000 and tail[2] == 0x3F57 and tail[4] == 0x4120 and tail[5] == 0x8000
+def _bf16_round_fraction(a, negative):
+    """Nearest BF16 (ties to even) to the exact non-negative rational a."""
+    from fractions import Fraction
+    import math
+    sign = 0x8000 if negative else 0
+    if a == 0:
+        return sign
+    e = math.floor(math.log2(a.numerator) - math.log2(a.denominator))
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    q = Fraction(2) ** (max(e, -126) - 7)
+    n = a / q
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    # the reference values are transcendental and carry about 300 bits: the
+    # nearest one to a tie (a subnormal x, GELU(x) = x/2 + ~x^2 / sqrt(2 pi))
+    # is about 2^-133 of a quantum away from it, far above their error
+    assert abs(rem - Fraction(1, 2)) > Fraction(1, 2 ** 200)
+    r = fl + (1 if rem > Fraction(1, 2) else 0)
+    val = r * q
+    if val >= Fraction(2) ** 128:
+        return sign | 0x7F80
+    f32 = np.float32(float(val))
+    return sign | (int(np.array([f32]).view(np.uint32)[0]) >> 16) & 0x7FFF
+
+
+def test_gelu_bf16_exhaustive_against_mpmath():
+    """Every BF16 input: the oracle's GELU equals x * Phi(x) evaluated with
+    90 significant digits (mpmath, independent of the C library's erfc) and
+    rounded once to BF16 in exact rational arithmetic."""
+    import mpmath
+    from fractions import Fraction
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.gelu_bf16(bits)
+    xs = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    mpmath.mp.dps = 90
+    half_sqrt2 = mpmath.sqrt(2) / 2
+    tiny = mpmath.mpf(2) ** -135
+    for i in range(65536):
+        x = float(xs[i])
+        if np.isnan(x):
+            assert (int(got[i]) & 0x7FFF) > 0x7F80, hex(i)      # NaN in, NaN out
+            continue
+        if np.isinf(x):
+            assert int(got[i]) == (0x7F80 if x > 0 else 0x8000), hex(i)   # GELU(+inf) = inf, GELU(-inf) -> -0
+            continue
+        if x == 0.0:
+            assert int(got[i]) == i & 0x8000, hex(i)
+            continue
+        g = mpmath.mpf(x) / 2 * mpmath.erfc(-mpmath.mpf(x) * half_sqrt2)
+        if abs(g) < tiny:
+            # below half the smallest BF16 subnormal (2^-133): rounds to -0
+            # (x < -13.5; the value's exponent can reach -10^77)
+            assert int(got[i]) == 0x8000, (hex(i), x)
+            continue
+        sign, man, exp, _ = g._mpf_
+        a = Fraction(man) * (Fraction(2) ** exp if exp >= 0 else Fraction(1, 2 ** -exp))
+        assert int(got[i]) == _bf16_round_fraction(a, bool(sign)), (hex(i), x)
+    # closed forms: GELU(1) = Phi(1) = 0.8413447... -> BF16 0.83984375 (0x3F57);
+    # GELU(10) = 10 (Phi(10) = 1 - 7.6e-24); GELU(-10) = -7.62e-23, which the
+    # form 0.5 x (1 + erf(x / sqrt 2)) loses to cancellation in binary64
+    assert int(got[0x3F80]) == 0x3F57
+    assert int(got[0x4120]) == 0x4120
+    g_m10 = float(torch.tensor([int(got[0xC120])], dtype=torch.int32).to(torch.int16).view(torch.bfloat16).float())
+    assert -7.7e-23 < g_m10 < -7.5e-23
