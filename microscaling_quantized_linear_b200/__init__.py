@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libnvq.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         "libnvq.so is not built (expected at %s); run "
-        "`python -m microscaling_quantized_linear_b200.build` or __graft_entry__.build()" % LIB_PATH)
+        "`python microscaling_quantized_linear_b200/build.py` or __graft_entry__.build()" % LIB_PATH)
 
 _lib = ctypes.CDLL(LIB_PATH)
 
