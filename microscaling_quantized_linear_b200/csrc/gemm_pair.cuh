@@ -152,8 +152,11 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     // everything above overlaps the previous grid; no global data is
-    // touched before it has completed
+    // touched before it has completed.  The next grid in the stream may then
+    // launch: its CTAs wait at their own griddepcontrol.wait until this grid
+    // has completed, so only its launch latency overlaps this grid.
     griddep_wait();
+    griddep_launch();
     const uint32_t num_tiles = p.num_m_blocks * p.num_n_blocks;   // 256 x BN tiles
     const uint32_t total_iters = ((num_tiles > pair) ? (num_tiles - pair + npairs - 1) / npairs : 0) * p.num_k_tiles;
 

@@ -111,6 +111,29 @@ int check_quant_shape(int format, int64_t rows, int64_t K, int64_t ld) {
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? NVQ_OK : NVQ_ERR_CUDA; }
 
+// Launch with programmatic stream serialization: the grid may launch while
+// the previous grid in the stream is still running.  Every kernel launched
+// this way executes griddepcontrol.wait before it reads anything the
+// previous grid may write, so only launch latency overlaps.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) {
+        cudaGetLastError();
+        return NVQ_ERR_CUDA;
+    }
+    return NVQ_OK;
+}
+
 int launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, uint32_t* partial, int num_sms,
                 cudaStream_t stream, uint32_t* npartial_out) {
     const uint32_t vecs_per_row = (uint32_t)(K / 8), pitch_vecs = (uint32_t)(ld / 8);
@@ -119,10 +142,9 @@ int launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, uint32_t* pa
     uint32_t grid = (uint32_t)(want < 1 ? 1 : want);
     const uint32_t cap = (uint32_t)num_sms * 8 < (uint32_t)kMaxAmaxPartials ? (uint32_t)num_sms * 8 : kMaxAmaxPartials;
     if (grid > cap) grid = cap;
-    amax_partials_kernel<<<grid, kAmaxThreads, 0, stream>>>(static_cast<const uint4*>(x), (uint32_t)rows,
-                                                            vecs_per_row, pitch_vecs, partial);
     *npartial_out = grid;
-    return launch_status();
+    return launch_pdl(amax_partials_kernel, dim3(grid), dim3(kAmaxThreads), 0, stream, static_cast<const uint4*>(x),
+                      (uint32_t)rows, vecs_per_row, pitch_vecs, partial);
 }
 
 uint32_t quant_grid(uint64_t units, int num_sms) {
@@ -233,23 +255,9 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
         if ((rc = launch_amax(x, M, K, ldx, partial, d->num_sms, stream, &npartial))) return rc;
     }
     const uint64_t units = (uint64_t)M * nblk;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(quant_grid(units, d->num_sms));
-    cfg.blockDim = dim3(kQuantThreads);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = calib_amax ? 0 : 1;   // overlap only with our own amax pass
-    const uint16_t* xp = static_cast<const uint16_t*>(x);
-    const uint32_t* pp = partial;
-    if (cudaLaunchKernelEx(&cfg, nvfp4_quantize_kernel, xp, (uint32_t)M, nblk, (uint32_t)ldx, codes, scales,
-                           global_scale, pp, npartial, calib_amax, d->status) != cudaSuccess) {
-        cudaGetLastError();
-        return NVQ_ERR_CUDA;
-    }
-    return NVQ_OK;
+    return launch_pdl(nvfp4_quantize_kernel, dim3(quant_grid(units, d->num_sms)), dim3(kQuantThreads), 0, stream,
+                      static_cast<const uint16_t*>(x), (uint32_t)M, nblk, (uint32_t)ldx, codes, scales, global_scale,
+                      partial, npartial, calib_amax, d->status);
 }
 
 int mxfp8_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
@@ -268,8 +276,8 @@ int mxfp8_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     const bool e5 = elem == NVQ_MXFP8_E5M2, ceil_rule = rule == NVQ_SCALE_CEIL;
     auto kern = e5 ? (ceil_rule ? mxfp8_quantize_kernel<1, 1> : mxfp8_quantize_kernel<1, 0>)
                    : (ceil_rule ? mxfp8_quantize_kernel<0, 1> : mxfp8_quantize_kernel<0, 0>);
-    kern<<<grid, kQuantThreads, 0, stream>>>(xp, (uint32_t)M, nblk, (uint32_t)ldx, codes, scales);
-    return launch_status();
+    return launch_pdl(kern, dim3(grid), dim3(kQuantThreads), 0, stream, xp, (uint32_t)M, nblk, (uint32_t)ldx, codes,
+                      scales);
 }
 
 int encode_codes_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t kbytes, uint32_t box_rows) {
@@ -615,24 +623,10 @@ int nvfp4_quantize_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx, uin
     uint32_t npartial = 0;
     if ((rc = launch_amax(x, M, K, ldx, partials, d->num_sms, s, &npartial))) return rc;
     const uint32_t nblk = (uint32_t)(K / 16);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(quant_grid((uint64_t)M * nblk, d->num_sms));
-    cfg.blockDim = dim3(kQuantThreads);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const uint16_t* xp = static_cast<const uint16_t*>(x);
-    const uint32_t* pp = partials;
     const float* no_calib = nullptr;
-    if (cudaLaunchKernelEx(&cfg, nvfp4_quantize_kernel, xp, (uint32_t)M, nblk, (uint32_t)ldx, codes, scales,
-                           global_scale, pp, npartial, no_calib, d->status) != cudaSuccess) {
-        cudaGetLastError();
-        return NVQ_ERR_CUDA;
-    }
-    return NVQ_OK;
+    return launch_pdl(nvfp4_quantize_kernel, dim3(quant_grid((uint64_t)M * nblk, d->num_sms)), dim3(kQuantThreads), 0,
+                      s, static_cast<const uint16_t*>(x), (uint32_t)M, nblk, (uint32_t)ldx, codes, scales,
+                      global_scale, partials, npartial, no_calib, d->status);
 }
 
 }  // extern "C"

@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(kAmaxThreads)
 amax_partials_kernel(const uint4* __restrict__ x, uint32_t rows, uint32_t vecs_per_row,
                      uint32_t pitch_vecs, uint32_t* __restrict__ partial) {
     __shared__ uint32_t red[kAmaxThreads / 32];
+    griddep_wait();                       // x may come from the previous grid
     griddep_launch();                     // the quantize pass may start its prologue
     uint32_t m2 = 0;
     const uint32_t total = rows * vecs_per_row;
@@ -192,7 +193,11 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
         c1 -= nblk;
         ++r1;
     }
-    // the first iteration's loads do not depend on the amax: issue them first
+    // Calibrated: x may come from the previous grid, so nothing is read
+    // before it has completed.  Dynamic: the previous grid is this call's amax
+    // pass, which only reads x and lets this grid start once it has itself
+    // waited for x's producer, so the first iteration's loads go first.
+    if (calib_amax != nullptr) griddep_wait();
     uint4 v[4];
     const uint4 zero4 = make_uint4(0, 0, 0, 0);
     {
@@ -551,6 +556,8 @@ __global__ void __launch_bounds__(kQuantThreads)
 mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nblk, uint32_t ldx,
                       uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
     constexpr int EMAX = ELEM == 0 ? 8 : 15;
+    griddep_wait();                              // x may come from the previous grid
+    griddep_launch();
     const uint32_t total = rows * nblk;
     const uint32_t ctiles = nblk >> 2;
     const uint32_t stride = gridDim.x * kQuantThreads;
