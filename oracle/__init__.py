@@ -64,6 +64,10 @@ def lib():
         L.oracle_double_to_bf16.argtypes = [ctypes.c_double]
         L.oracle_gelu_bf16.restype = ctypes.c_uint16
         L.oracle_gelu_bf16.argtypes = [ctypes.c_uint16]
+        L.oracle_double_to_bf16_array.restype = None
+        L.oracle_double_to_bf16_array.argtypes = [_f64p, _i64, _u16p]
+        L.oracle_gelu_bf16_array.restype = None
+        L.oracle_gelu_bf16_array.argtypes = [_u16p, _i64, _u16p]
         L.oracle_e5m2_value.restype = ctypes.c_double
         L.oracle_e5m2_value.argtypes = [ctypes.c_int]
         L.oracle_e5m2_encode.restype = ctypes.c_int
@@ -176,6 +180,22 @@ def gelu_bf16(bits_arr):
     return np.vectorize(lambda b: f(int(b)), otypes=[np.uint16])(a)
 
 
+def double_to_bf16_array(v):
+    """Elementwise double_to_bf16 of a binary64 array (same shape, uint16 bits)."""
+    a = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(a.shape, dtype=np.uint16)
+    lib().oracle_double_to_bf16_array(_ptr(a, _f64p), a.size, _ptr(out, _u16p))
+    return out
+
+
+def gelu_bf16_array(bits_arr):
+    """Elementwise gelu_bf16 of BF16 bit patterns (same shape, uint16 bits)."""
+    a = np.ascontiguousarray(bits_arr, dtype=np.uint16)
+    out = np.empty(a.shape, dtype=np.uint16)
+    lib().oracle_gelu_bf16_array(_ptr(a, _u16p), a.size, _ptr(out, _u16p))
+    return out
+
+
 ELEMS = {"e4m3": 0, "e5m2": 1}
 RULES = {"floor": 0, "ceil": 1}
 
@@ -220,6 +240,22 @@ def gemm_rows(A_hat, B_hat, rows=None, bias_bits=None):
         bp = _ptr(bias, _u16p)
     lib().oracle_gemm_rows(_ptr(A, _f64p), _ptr(B, _f64p), N, K, _ptr(rows, _i64p), rows.size, bp, _ptr(out, _f64p))
     return out
+
+
+def linear_gelu_mxfp8(A_hat, B_hat, rows=None, bias_bits=None):
+    """The first linear of a feed-forward block followed by the next layer's
+    activation quantization, in the order the definitions give:
+      Y = A_hat[rows] . B_hat^T (+ bias), binary64        (gemm_rows)
+      D = Y rounded once to BF16                            (double_to_bf16)
+      G = GELU(D) = D * Phi(D), rounded once to BF16        (gelu_bf16)
+      codes, sf = MXFP8 of G (E4M3 elements, floor rule)    (mxfp8_quantize)
+    Returns (codes u8 [R, N], sf u8 (tile order over R rows), D bits, G bits, Y)
+    with R = len(rows)."""
+    Y = gemm_rows(A_hat, B_hat, rows=rows, bias_bits=bias_bits)
+    D = double_to_bf16_array(Y)
+    G = gelu_bf16_array(D)
+    codes, sf = mxfp8_quantize(G)
+    return codes, sf, D, G, Y
 
 
 def num_threads():

@@ -245,6 +245,17 @@ ORACLE_EXPORT uint16_t oracle_gelu_bf16(uint16_t in) {
     return bf16_round_tie(s, err > 0 ? 1 : (err < 0 ? -1 : 0));
 }
 
+/* Elementwise forms of the two functions above, over n values. */
+ORACLE_EXPORT void oracle_double_to_bf16_array(const double* v, int64_t n, uint16_t* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_double_to_bf16(v[i]);
+}
+
+ORACLE_EXPORT void oracle_gelu_bf16_array(const uint16_t* in, int64_t n, uint16_t* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_gelu_bf16(in[i]);
+}
+
 /* ------------------------------------------------------------------ */
 /* NVFP4 quantization ([P1] NVFP4; [P2] 3.1 three outputs)            */
 /* ------------------------------------------------------------------ */

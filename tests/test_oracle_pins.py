@@ -702,3 +702,53 @@ def test_gelu_bf16_exhaustive_against_mpmath():
     assert int(got[0x4120]) == 0x4120
     g_m10 = float(torch.tensor([int(got[0xC120])], dtype=torch.int32).to(torch.int16).view(torch.bfloat16).float())
     assert -7.7e-23 < g_m10 < -7.5e-23
+
+
+def test_array_forms_equal_the_pinned_scalars():
+    rng = np.random.default_rng(44)
+    vals = np.concatenate([rng.standard_normal(3000) * np.exp2(rng.integers(-140, 120, 3000)),
+                           [0.0, -0.0, np.inf, -np.inf, 1.0 + 2 ** -8, 1.0 + 2 ** -8 + 2 ** -40, 2.0 ** -134]])
+    want = np.array([oracle.double_to_bf16(float(v)) for v in vals], dtype=np.uint16)
+    assert np.array_equal(oracle.double_to_bf16_array(vals), want)
+    assert np.array_equal(oracle.double_to_bf16_array(vals[:3003].reshape(-1, 7)), want[:3003].reshape(-1, 7))
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    assert np.array_equal(oracle.gelu_bf16_array(bits), oracle.gelu_bf16(bits))
+
+
+def _bits_of(values):
+    return torch.tensor(values, dtype=torch.float64).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_linear_gelu_mxfp8_closed_forms():
+    """K = 32 with B the identity, so Y = A row by row (exact), then:
+    row 0, values >= 4:     GELU is the identity on them, so the codes are
+                            those of MXFP8(Y): block max 35 -> X = 5 - 8,
+                            scale byte 124, code of v is E4M3(8 v);
+    row 1, values <= -16:   GELU gives -0 everywhere: codes 0x80, scale 0
+                            (a zero block takes X = -127);
+    row 2, +-1 and 0:       GELU(1) = 0.8413 -> BF16 0x3F57 (0.83984375),
+                            GELU(-1) = -0.1587 -> BF16 0xBE22 (-0.158203125);
+                            block max 0.83984375 -> X = -1 - 8, codes of
+                            0.83984375 * 512 = 430 -> 416 (spacing 32 in
+                            [256, 512): 0x7D) and of -0.158203125 * 512 = -81
+                            -> -80 (spacing 8 in [64, 128): 0xEA), 0 -> 0."""
+    K = 32
+    B = np.eye(K)
+    row0 = np.arange(4, 36, dtype=np.float64)
+    row1 = -np.arange(16, 48, dtype=np.float64)
+    row2 = np.array([1.0, -1.0, 0.0, 1.0] * 8)
+    A = np.stack([row0, row1, row2])
+    codes, sf, D, G, Y = oracle.linear_gelu_mxfp8(A, B)
+    assert np.array_equal(Y, A)
+    assert np.array_equal(D, _bits_of(A))
+    assert np.array_equal(G[0], D[0])
+    assert np.all(G[1] == 0x8000)
+    assert list(G[2][:4]) == [0x3F57, 0xBE22, 0x0000, 0x3F57]
+    sfm = np.array([[sf[oracle.sf_offset(r, 0, 1)]] for r in range(3)])
+    assert list(sfm[:, 0]) == [124, 0, 118]
+    assert all(int(codes[0][i]) == oracle.e4m3_encode(8.0 * row0[i]) for i in range(K))
+    assert int(codes[0][0]) == 0x60                          # 4 * 8 = 32 = 2^5
+    assert np.all(codes[1] == 0x80)
+    assert list(codes[2][:4]) == [0x7D, 0xEA, 0x00, 0x7D]
+    # rows past the third, up to 128, are zero padding in the scale tile
+    assert np.all(np.array([sf[oracle.sf_offset(r, 0, 1)] for r in range(3, 128)]) == 0)

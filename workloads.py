@@ -103,6 +103,31 @@ def bias(N, seed=2):
     return (torch.randn(N, generator=_gen(seed)) * 0.1).to(torch.bfloat16)
 
 
+def exact_operand(rows, K, seed, significands=(1.0, 1.5, 1.75), top_row=None, min_exp=-3, block=16):
+    """BF16 [rows, K] whose values are c_r * e with e drawn from {0, +-0.5,
+    +-1, +-1.5, +-2, +-3, +-4, +-6} and every `block` consecutive values of a
+    row holding one +-6 * c_r; the row constants c_r = s * 2^i take s from
+    `significands` and i from [min_exp, 0].  If top_row is given, that row's
+    constant is 1.75 (the tensor's largest).  Returns (x, c) with c the
+    binary64 row constants.  Products and sums of such values stay on a
+    coarse binary grid, which makes a GEMM over them exact in binary32 for
+    moderate K (CPU)."""
+    g = _gen(seed)
+    mags = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    e = mags[torch.randint(0, 8, (rows, K), generator=g)]
+    e = torch.where(torch.rand(rows, K, generator=g) < 0.5, -e, e)
+    pos = torch.randint(0, block, (rows, K // block), generator=g) + torch.arange(0, K, block)
+    sign6 = torch.where(torch.rand(rows, K // block, generator=g) < 0.5, -6.0, 6.0)
+    e.scatter_(1, pos, sign6)
+    sig = torch.tensor(significands, dtype=torch.float64)
+    c = sig[torch.randint(0, len(significands), (rows,), generator=g)] * \
+        torch.pow(2.0, torch.randint(min_exp, 1, (rows,), generator=g).double())
+    if top_row is not None:
+        c[top_row] = 1.75
+    x = (e.double() * c[:, None]).to(torch.bfloat16)
+    return x, c.numpy()
+
+
 def normal(M, K, seed, std=1.0):
     """Plain BF16 N(0, std^2) tensor, for shape-sweep tests."""
     return (torch.randn(M, K, generator=_gen(seed)) * std).to(torch.bfloat16)
