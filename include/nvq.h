@@ -214,6 +214,44 @@ NVQ_API int block_scaled_linear(int format,
                         int64_t M, int64_t N, int64_t K, nvq_stream_t stream);
 
 /*
+ * block_scaled_linear_gelu_mxfp8 -- the first linear of a feed-forward block
+ * with the next layer's activation quantization fused into its epilogue:
+ *
+ *   D[m, n]  = bf16( alpha * sum_k a(m,k) sa(m,k/bs) b(n,k) sb(n,k/bs) + bias[n] )
+ *              exactly as block_scaled_linear computes it (D is not written)
+ *   G[m, n]  = GELU(D[m, n]) = D * Phi(D), Phi the standard normal CDF (the
+ *              exact-erf form), rounded once to BF16
+ *   y_codes, y_scales = mxfp8_quantize(G): per 32 consecutive columns of a
+ *              row, X = floor(log2(max |G|)) - 8, scale byte X + 127, codes
+ *              E4M3(G * 2^-X) (round to nearest even, saturate at 448)
+ *
+ * The output is the quantized activation of the following linear (format
+ * NVQ_MXFP8, K of that layer = N of this one), so the BF16 activation between
+ * the two layers never reaches memory (page "NVIDIA Blackwell平台FP4量化技术解析
+ * 与图像生成优化", section 2.1: the transformer's fully connected layers run in
+ * FP4; the activation between them is not named on the pages, and the exact-erf
+ * GELU is the reading taken).
+ *
+ *   format            NVQ_NVFP4 or NVQ_MXFP8 (A and B operands, as block_scaled_linear)
+ *   a_*, b_*, bias    as block_scaled_linear
+ *   y_codes           out, [M, N] E4M3 bytes, dense (nvq_codes_bytes(NVQ_MXFP8, M, N))
+ *   y_scales          out, nvq_scale_bytes(NVQ_MXFP8, M, N) bytes (E8M0, tile
+ *                     order; rows M .. ceil(M/128)*128 - 1 written as zero)
+ *   M, N, K           M any, N a multiple of 128 (whole scale tiles of the next
+ *                     layer), K a multiple of 256 (NVFP4) or 128 (MXFP8)
+ *
+ * For every BF16 value of D the GELU is the correctly rounded one, so y_codes
+ * and y_scales are a function of D alone; D itself carries the GEMM's
+ * tolerance (see block_scaled_linear).  Errors: as block_scaled_linear, and
+ * NVQ_ERR_FORMAT for NVQ_MXFP8_E5M2 operands.
+ */
+NVQ_API int block_scaled_linear_gelu_mxfp8(int format,
+                        const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                        const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global,
+                        const void* bias, uint8_t* y_codes, uint8_t* y_scales,
+                        int64_t M, int64_t N, int64_t K, nvq_stream_t stream);
+
+/*
  * nvq_device_status -- synchronizes `stream`, then returns the current
  * device's status word (NVQ_STATUS_* bits, 0 = clean) and clears it.
  * Returns NVQ_ERR_CUDA (< 0) if the synchronization or the read fails.
@@ -269,6 +307,16 @@ NVQ_API int nvfp4_quantize_noalloc(const void* x, int64_t M, int64_t K, int64_t 
  */
 NVQ_API int nvq_probe_convert(const float* in, int64_t n, uint8_t* e2m1_out, uint8_t* e4m3_out,
                       nvq_stream_t stream);
+
+/*
+ * nvq_probe_gelu -- GELU self-test (no counterpart on the pages).  Runs the
+ * BF16 GELU of block_scaled_linear_gelu_mxfp8's epilogue (same table, same
+ * lookup) on n BF16 bit patterns, so tests can compare all 65536 inputs with
+ * the CPU oracle.
+ *   in    n BF16 values (device)
+ *   out   n BF16 values (device)
+ */
+NVQ_API int nvq_probe_gelu(const uint16_t* in, int64_t n, uint16_t* out, nvq_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -67,10 +67,16 @@ _lib.nvq_probe_convert.restype = ctypes.c_int
 _lib.nvq_probe_convert.argtypes = [_vp, _i64, _vp, _vp, _vp]
 _lib.nvfp4_quantize_noalloc.restype = ctypes.c_int
 _lib.nvfp4_quantize_noalloc.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]
+_lib.block_scaled_linear_gelu_mxfp8.restype = ctypes.c_int
+_lib.block_scaled_linear_gelu_mxfp8.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                                _i64, _i64, _i64, _vp]
+_lib.nvq_probe_gelu.restype = ctypes.c_int
+_lib.nvq_probe_gelu.argtypes = [_vp, _i64, _vp, _vp]
 
 EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_quantize",
             "mxfp8_quantize", "mxfp8_quantize_ex", "quantize_weight", "block_scaled_linear",
-            "nvq_device_status", "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc")
+            "nvq_device_status", "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc",
+            "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu")
 
 NOALLOC_MAX_PARTIALS = 1024
 
@@ -205,6 +211,24 @@ def block_scaled_linear(fmt, a_codes, a_scales, a_global, b_codes, b_scales, b_g
     return out
 
 
+def block_scaled_linear_gelu_mxfp8(fmt, a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K,
+                                   bias=None, y_codes=None, y_scales=None, stream=None):
+    """The linear D = bf16(alpha * A . B^T + bias) with GELU and MXFP8 (E4M3)
+    quantization of the result fused into the epilogue; D is never written.
+    Returns (y_codes u8 [M, N], y_scales u8 (E8M0, tile order)): the next
+    linear's MXFP8 activation operand."""
+    f = _fmt(fmt)
+    dev = a_codes.device
+    y_codes = y_codes if y_codes is not None else torch.empty((M, N), dtype=torch.uint8, device=dev)
+    y_scales = y_scales if y_scales is not None else torch.empty(scale_bytes(MXFP8, M, N), dtype=torch.uint8,
+                                                                 device=dev)
+    _check(_lib.block_scaled_linear_gelu_mxfp8(f, _ptr(a_codes), _ptr(a_scales), _ptr(a_global), _ptr(b_codes),
+                                               _ptr(b_scales), _ptr(b_global), _ptr(bias), _ptr(y_codes),
+                                               _ptr(y_scales), M, N, K, _stream(stream, dev)),
+           "block_scaled_linear_gelu_mxfp8")
+    return y_codes, y_scales
+
+
 class QuantizedLinear:
     """A linear layer whose weight is quantized once (offline) and whose
     activations are quantized on every call, then multiplied on the
@@ -251,6 +275,14 @@ def device_status(stream=None, device=None):
     if rc < 0:
         raise NvqError(rc, "nvq_device_status")
     return rc
+
+
+def probe_gelu(bits, stream=None):
+    """Device BF16 GELU (the fused epilogue's) of BF16 bit patterns (int16/uint16 tensor)."""
+    n = bits.numel()
+    out = torch.empty(n, dtype=torch.int16, device=bits.device)
+    _check(_lib.nvq_probe_gelu(_ptr(bits), n, _ptr(out), _stream(stream, bits.device)), "nvq_probe_gelu")
+    return out
 
 
 def probe_convert(values, stream=None):

@@ -32,7 +32,9 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include "gelu.cuh"
 #include "ptx.cuh"
+#include "quantize.cuh"
 
 namespace nvq {
 
@@ -73,11 +75,23 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], float al
 // MMAs of the next tile wait for the loads and one conversion only.  The
 // BF16 sub-tiles are then written via the warp's 64-byte-swizzled staging
 // buffer and TMA stores.
-template <int BN>
+// Output of the epilogue that quantizes for the next layer (EPI 1):
+// GELU of the BF16 result, then MXFP8 (E4M3 elements, OCP floor exponent)
+// per 32 consecutive columns, the codes dense [m, n] and the E8M0 scales in
+// the 128x4 tile order of an [m, n/32] scale matrix (rows m .. m_pad - 1 of
+// the last row tile zero).
+struct EpiQuant {
+    uint8_t* codes;
+    uint8_t* sf;
+    uint32_t n, m, m_pad;
+};
+
+template <int BN, int EPI>
 __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half, int lane, float alpha,
                                                   const __nv_bfloat16* bias_tile, uint8_t* staging,
                                                   const CUtensorMap* tmap_d, int32_t row0, uint32_t n0,
-                                                  int nlim, uint32_t release_bar, bool release_remote) {
+                                                  int nlim, uint32_t release_bar, bool release_remote,
+                                                  const EpiQuant& eq, const uint16_t* gelu_tab) {
     constexpr int NC = BN / 64;                          // 32-column chunks per warp
     constexpr int JL = (NC - 1) & ~1;                    // first chunk of the last pair
     const int c0 = half * (BN / 2);
@@ -110,6 +124,34 @@ __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half,
         }
         epilogue_chunk(r0, alpha, bias_tile, c0 + 32 * JL, nlim, packed[JL]);
         if (JL + 1 < NC) epilogue_chunk(r1, alpha, bias_tile, c0 + 32 * (JL + 1), nlim, packed[JL + 1 < NC ? JL + 1 : JL]);
+    }
+    if constexpr (EPI == 1) {
+        // One thread = one row; each 32-column chunk is one MXFP8 block.  The
+        // NC scale bytes of the row's share are consecutive in the tile order
+        // (the share starts at a multiple of 4 blocks for BN 256, of 2 for
+        // BN 128), so they go out in one store.
+        static_assert(NC == 2 || NC == 4, "MXFP8 epilogue: 128- or 256-wide tiles");
+        const uint32_t row = (uint32_t)row0 + (uint32_t)lane;
+        const uint32_t cfirst = n0 + (uint32_t)c0;
+        if (cfirst >= eq.n || row >= eq.m_pad) return;
+        uint32_t scw = 0;
+        if (row < eq.m) {
+            uint8_t* dst = eq.codes + (size_t)row * eq.n + cfirst;
+#pragma unroll
+            for (int j = 0; j < NC; ++j) {
+                uint32_t g[16], q[8];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) g[e] = gelu_bf16x2(packed[j][e], gelu_tab);
+                scw |= mx_block<0, 0>(g, q) << (8 * j);
+                uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * j);
+                d4[0] = make_uint4(q[0], q[1], q[2], q[3]);
+                d4[1] = make_uint4(q[4], q[5], q[6], q[7]);
+            }
+        }
+        uint8_t* sfp = eq.sf + sf_tile_offset(row, cfirst / 32, eq.n / 128);
+        if (NC == 4) *reinterpret_cast<uint32_t*>(sfp) = scw;
+        else *reinterpret_cast<uint16_t*>(sfp) = (uint16_t)scw;
+        return;
     }
     const uint32_t swz = (uint32_t)((lane >> 1) & 3);     // 64-byte swizzle of this thread's row
 #pragma unroll
@@ -205,6 +247,11 @@ struct GemmParams {
     uint32_t sf_ctiles;          // (K / SF_BLOCK) / 4: scale tiles per 128 rows
     uint32_t n_total;            // N: output columns past it are neither stored nor biased
     uint32_t sfa_rtiles, sfb_rtiles;   // 128-row scale tiles in the A and B scale buffers
+    // quantizing epilogue (EPI 1) only: MXFP8 codes [m_total, n_total] and
+    // scales of GELU(D), m_pad = m_total rounded up to 128
+    uint8_t* q_codes;
+    uint8_t* q_sf;
+    uint32_t m_total, m_pad;
 };
 
 // Scale-factor copy warp `job` (0: A scales, 1..SFB_H: B scale row block
@@ -230,11 +277,15 @@ __device__ __forceinline__ void sf_copy_job(int job, uint32_t st, uint32_t sf_sl
     }
 }
 
-template <int FMT, int BN>
+// EPI 0: D = bf16(alpha A.B^T + bias) through tmap_d.  EPI 1: D is not
+// written; GELU(D) leaves as MXFP8 codes and scales (EpiQuant), and the
+// epilogue warps' staging area holds the GELU table instead.
+template <int FMT, int BN, int EPI>
 __global__ void __launch_bounds__(GemmCfg<FMT, BN>::THREADS, 1)
 bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
               const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
     using C = GemmCfg<FMT, BN>;
+    static_assert(EPI == 0 || kGeluTabBytes <= C::EPI_BYTES, "GELU table must fit the staging area");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
@@ -276,7 +327,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmap_a);
         prefetch_tensormap(&tmap_b);
-        prefetch_tensormap(&tmap_d);
+        if (EPI == 0) prefetch_tensormap(&tmap_d);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), C::TM_COLS);
@@ -425,6 +476,14 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         const int half = (warp - 2) >> 2;             // which half of the tile's columns
         const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
         uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * C::EPI_BUF_BYTES;
+        const uint16_t* gelu_tab = reinterpret_cast<const uint16_t*>(smem + C::OFF_EPI);
+        const EpiQuant eq = {p.q_codes, p.q_sf, p.n_total, p.m_total, p.m_pad};
+        if (EPI == 1) {
+            // built while the first tile's MMAs run (the epilogue warps are
+            // idle until then); the other roles never touch it
+            gelu_table_fill(reinterpret_cast<uint16_t*>(smem + C::OFF_EPI), threadIdx.x - 64, 32 * kEpiWarps);
+            named_barrier_sync(1, 32 * kEpiWarps);
+        }
         uint32_t t_local = 0;
         for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t_local) {
             const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
@@ -437,9 +496,10 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             }
             tc_fence_after();
             const uint32_t n0 = nb * BN;
-            drain_accumulator<BN>(tmem + ((uint32_t)(32 * q) << 16) + buf * BN, half, lane, alpha,
-                                  p.bias ? p.bias + n0 : nullptr, staging, &tmap_d,
-                                  (int32_t)(mb * C::BM + 32 * q), n0, (int)(p.n_total - n0), tempty0 + 8 * buf, false);
+            drain_accumulator<BN, EPI>(tmem + ((uint32_t)(32 * q) << 16) + buf * BN, half, lane, alpha,
+                                       p.bias ? p.bias + n0 : nullptr, staging, &tmap_d,
+                                       (int32_t)(mb * C::BM + 32 * q), n0, (int)(p.n_total - n0), tempty0 + 8 * buf,
+                                       false, eq, gelu_tab);
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();

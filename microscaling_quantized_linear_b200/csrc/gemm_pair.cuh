@@ -91,12 +91,14 @@ struct PairCfg {
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory overflow");
 };
 
-template <int FMT, int BN>
+// EPI as in bsgemm_kernel: 0 writes D, 1 writes MXFP8 codes and scales of GELU(D).
+template <int FMT, int BN, int EPI>
 __global__ void __launch_bounds__(PairCfg<FMT, BN>::THREADS, 1)
 bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                    const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
     using C = PairCfg<FMT, BN>;
+    static_assert(EPI == 0 || (BN == 256 && kGeluTabBytes <= C::EPI_BYTES), "GELU table must fit the staging area");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
@@ -141,7 +143,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
         prefetch_tensormap(&tmap_b);
         prefetch_tensormap(&tmap_sfa);
         prefetch_tensormap(&tmap_sfb);
-        prefetch_tensormap(&tmap_d);
+        if (EPI == 0) prefetch_tensormap(&tmap_d);
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_holder), C::TM_COLS);
@@ -290,6 +292,13 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
         const int half = (warp - 2) >> 2;
         const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
         uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * C::EPI_BUF_BYTES;
+        const uint16_t* gelu_tab = reinterpret_cast<const uint16_t*>(smem + C::OFF_EPI);
+        const EpiQuant eq = {p.q_codes, p.q_sf, p.n_total, p.m_total, p.m_pad};
+        if (EPI == 1) {
+            // built while the first tile's MMAs run; the other roles never touch it
+            gelu_table_fill(reinterpret_cast<uint16_t*>(smem + C::OFF_EPI), threadIdx.x - 64, 32 * kEpiWarps);
+            named_barrier_sync(1, 32 * kEpiWarps);
+        }
         uint32_t t_local = 0;
         for (uint32_t tile = pair; tile < num_tiles; tile += npairs, ++t_local) {
             const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
@@ -302,10 +311,10 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             }
             tc_fence_after();
             const uint32_t n0 = nb * BN;
-            drain_accumulator<BN>(tmem + ((uint32_t)(32 * q) << 16) + buf * BN, half, lane, alpha,
-                                  p.bias ? p.bias + n0 : nullptr, staging, &tmap_d,
-                                  (int32_t)(mb * 256 + 128 * rank + 32 * q), n0, (int)(p.n_total - n0),
-                                  mapa_shared(tempty0 + 8 * buf, 0), true);
+            drain_accumulator<BN, EPI>(tmem + ((uint32_t)(32 * q) << 16) + buf * BN, half, lane, alpha,
+                                       p.bias ? p.bias + n0 : nullptr, staging, &tmap_d,
+                                       (int32_t)(mb * 256 + 128 * rank + 32 * q), n0, (int)(p.n_total - n0),
+                                       mapa_shared(tempty0 + 8 * buf, 0), true, eq, gelu_tab);
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();

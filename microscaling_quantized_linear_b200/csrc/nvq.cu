@@ -43,8 +43,8 @@ struct DeviceInfo {
     bool arch_ok = false;
     int num_sms = 0;
     unsigned int* status = nullptr;
-    bool gemm_attr[3][3] = {};
-    bool pair_attr[3][2] = {};
+    bool gemm_attr[3][3][2] = {};    // [format][BN 128/192/256][epilogue]
+    bool pair_attr[3][2][2] = {};    // [format][BN 192/256][epilogue]
     bool fused_attr = false;
 };
 
@@ -315,32 +315,45 @@ int encode_scale_map(CUtensorMap* map, const void* scales, size_t bytes, uint32_
     return r == CUDA_SUCCESS ? NVQ_OK : NVQ_ERR_CUDA;
 }
 
-// 256 x BN tiles on CTA pairs (M % 256 == 0, N % BN == 0).
-template <int FMT, int BN>
+// Fields of GemmParams for the quantizing epilogue (EPI 1): MXFP8 codes and
+// scales of GELU(D) for an [M, N] output; unused (null) for EPI 0.
+void set_epi_quant(GemmParams& p, uint8_t* q_codes, uint8_t* q_sf, int64_t M) {
+    p.q_codes = q_codes;
+    p.q_sf = q_sf;
+    p.m_total = (uint32_t)M;
+    p.m_pad = (uint32_t)((M + 127) / 128 * 128);
+}
+
+// 256 x BN tiles on CTA pairs (M % 256 == 0, N % BN == 0).  EPI 0 writes D
+// (out, ldo); EPI 1 writes MXFP8 codes and scales of GELU(D) (q_codes, q_sf).
+template <int FMT, int BN, int EPI>
 int launch_gemm_pair(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                      const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
-                     void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+                     void* out, int64_t ldo, uint8_t* q_codes, uint8_t* q_sf, int64_t M, int64_t N, int64_t K,
+                     cudaStream_t stream) {
     using C = PairCfg<FMT, BN>;
     const int64_t kbytes = FMT == 0 ? K / 2 : K;
     const int fmt = FMT == 0 ? NVQ_NVFP4 : NVQ_MXFP8;   // scale geometry only
     CUtensorMap ma, mb, msa, msb, md;
+    memset(&md, 0, sizeof(md));
     int rc;
     if ((rc = encode_codes_map(&ma, a_codes, M, kbytes, 128))) return rc;
     if ((rc = encode_codes_map(&mb, b_codes, N, kbytes, C::BN_HALF))) return rc;
     if ((rc = encode_scale_map(&msa, a_scales, nvq_scale_bytes(fmt, M, K), C::SF_CHUNK / 256))) return rc;
     if ((rc = encode_scale_map(&msb, b_scales, nvq_scale_bytes(fmt, N, K), C::SF_CHUNK / 256))) return rc;
-    if ((rc = encode_out_map(&md, out, M, N, ldo))) return rc;
-    auto kern = bsgemm_pair_kernel<FMT, BN>;
+    if (EPI == 0 && (rc = encode_out_map(&md, out, M, N, ldo))) return rc;
+    auto kern = bsgemm_pair_kernel<FMT, BN, EPI>;
     {
         std::lock_guard<std::mutex> lock(g_mu);
-        if (!d->pair_attr[FMT][BN == 256]) {
+        if (!d->pair_attr[FMT][BN == 256][EPI]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
                 cudaSuccess)
                 return NVQ_ERR_CUDA;
-            d->pair_attr[FMT][BN == 256] = true;
+            d->pair_attr[FMT][BN == 256][EPI] = true;
         }
     }
     GemmParams p;
+    set_epi_quant(p, q_codes, q_sf, M);
     p.sfa = a_scales;
     p.sfb = b_scales;
     p.a_global = a_global;
@@ -378,29 +391,32 @@ int launch_gemm_pair(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_sca
     return NVQ_OK;
 }
 
-template <int FMT, int BN>
+template <int FMT, int BN, int EPI>
 int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                 const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
-                void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+                void* out, int64_t ldo, uint8_t* q_codes, uint8_t* q_sf, int64_t M, int64_t N, int64_t K,
+                cudaStream_t stream) {
     using C = GemmCfg<FMT, BN>;
     const int64_t kbytes = FMT == 0 ? K / 2 : K;
     CUtensorMap ma, mb, md;
+    memset(&md, 0, sizeof(md));
     int rc;
     if ((rc = encode_codes_map(&ma, a_codes, M, kbytes, C::BM))) return rc;
     if ((rc = encode_codes_map(&mb, b_codes, N, kbytes, BN))) return rc;
-    if ((rc = encode_out_map(&md, out, M, N, ldo))) return rc;
-    auto kern = bsgemm_kernel<FMT, BN>;
+    if (EPI == 0 && (rc = encode_out_map(&md, out, M, N, ldo))) return rc;
+    auto kern = bsgemm_kernel<FMT, BN, EPI>;
     const int wi = BN / 64 - 2;                      // 128 -> 0, 192 -> 1, 256 -> 2
     {
         std::lock_guard<std::mutex> lock(g_mu);
-        if (!d->gemm_attr[FMT][wi]) {
+        if (!d->gemm_attr[FMT][wi][EPI]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
                 cudaSuccess)
                 return NVQ_ERR_CUDA;
-            d->gemm_attr[FMT][wi] = true;
+            d->gemm_attr[FMT][wi][EPI] = true;
         }
     }
     GemmParams p;
+    set_epi_quant(p, q_codes, q_sf, M);
     p.sfa = a_scales;
     p.sfb = b_scales;
     p.a_global = a_global;
@@ -445,26 +461,43 @@ int launch_for_format(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_sc
     // accumulator is faster than 256 x 192 with two.  A ragged N takes 256.
     if (g_use_pairs && M > 128) {
         if (N % 384 == 0 && N % 256 != 0)
-            return launch_gemm_pair<FMT, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out,
-                                              ldo, M, N, K, s);
-        return launch_gemm_pair<FMT, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
-                                          M, N, K, s);
+            return launch_gemm_pair<FMT, 192, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
+                                                 out, ldo, nullptr, nullptr, M, N, K, s);
+        return launch_gemm_pair<FMT, 256, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
+                                             out, ldo, nullptr, nullptr, M, N, K, s);
     }
     // One CTA per tile: width 256 when N allows it (fewest scale-factor copies
     // per MMA), else 192, else 128 (two accumulators).  When 256-wide tiles
     // would leave SMs idle (a short M: the weight stream is then the cost),
     // 128-wide tiles spread it over twice as many SMs.
     if ((M + 127) / 128 * ((N + 255) / 256) < d->num_sms)
-        return launch_gemm<FMT, 128>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M,
-                                     N, K, s);
+        return launch_gemm<FMT, 128, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
+                                        nullptr, nullptr, M, N, K, s);
     if (N % 256 == 0)
-        return launch_gemm<FMT, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M,
-                                     N, K, s);
+        return launch_gemm<FMT, 256, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
+                                        nullptr, nullptr, M, N, K, s);
     if (N % 384 == 0)
-        return launch_gemm<FMT, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M,
-                                     N, K, s);
-    return launch_gemm<FMT, 128>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo, M, N,
-                                 K, s);
+        return launch_gemm<FMT, 192, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
+                                        nullptr, nullptr, M, N, K, s);
+    return launch_gemm<FMT, 128, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
+                                        nullptr, nullptr, M, N, K, s);
+}
+
+// The quantizing epilogue (GELU, then MXFP8 codes and scales) on 256-wide
+// tiles: CTA pairs as above, else one CTA per 128 x 256 tile, or 128 x 128
+// when 256-wide tiles would leave SMs idle.
+template <int FMT>
+int launch_gelu_mxfp8(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                      const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
+                      uint8_t* y_codes, uint8_t* y_scales, int64_t M, int64_t N, int64_t K, cudaStream_t s) {
+    if (g_use_pairs && M > 128)
+        return launch_gemm_pair<FMT, 256, 1>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
+                                             nullptr, 0, y_codes, y_scales, M, N, K, s);
+    if ((M + 127) / 128 * ((N + 255) / 256) < d->num_sms)
+        return launch_gemm<FMT, 128, 1>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, nullptr,
+                                        0, y_codes, y_scales, M, N, K, s);
+    return launch_gemm<FMT, 256, 1>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, nullptr, 0,
+                                    y_codes, y_scales, M, N, K, s);
 }
 
 }  // namespace nvq
@@ -547,6 +580,48 @@ int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_sca
                                     K, s);
     return launch_for_format<2>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M, N, K,
                                 s);
+}
+
+int block_scaled_linear_gelu_mxfp8(int format, const uint8_t* a_codes, const uint8_t* a_scales,
+                                   const float* a_global, const uint8_t* b_codes, const uint8_t* b_scales,
+                                   const float* b_global, const void* bias, uint8_t* y_codes, uint8_t* y_scales,
+                                   int64_t M, int64_t N, int64_t K, nvq_stream_t stream) {
+    if (format != NVQ_NVFP4 && format != NVQ_MXFP8) return NVQ_ERR_FORMAT;
+    const int64_t k_stage = format == NVQ_NVFP4 ? 256 : 128;
+    // N is the K of the next layer's MXFP8 operand: whole 4-block scale columns
+    if (M < 0 || N <= 0 || N % 128 || K <= 0 || K % k_stage) return NVQ_ERR_SHAPE;
+    if (K >= (int64_t(1) << 24) || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) ||
+        M * N >= (int64_t(1) << 40))
+        return NVQ_ERR_SHAPE;
+    if (M == 0) return NVQ_OK;
+    if (!a_codes || !a_scales || !b_codes || !b_scales || !y_codes || !y_scales) return NVQ_ERR_NULL;
+    if (format == NVQ_NVFP4 && (!a_global || !b_global)) return NVQ_ERR_NULL;
+    if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) ||
+        !aligned16(y_codes) || !aligned16(y_scales) || (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+        return NVQ_ERR_ALIGN;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc) return rc;
+    if ((rc = get_encoder())) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (format == NVQ_NVFP4)
+        return launch_gelu_mxfp8<0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, y_codes,
+                                    y_scales, M, N, K, s);
+    return launch_gelu_mxfp8<1>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, y_codes, y_scales,
+                                M, N, K, s);
+}
+
+int nvq_probe_gelu(const uint16_t* in, int64_t n, uint16_t* out, nvq_stream_t stream) {
+    if (!in || !out) return NVQ_ERR_NULL;
+    if (n < 0 || n >= (int64_t(1) << 31)) return NVQ_ERR_SHAPE;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc) return rc;
+    if (n == 0) return NVQ_OK;
+    uint64_t grid = ((uint64_t)n + 255) / 256;
+    if (grid > (uint64_t)d->num_sms) grid = (uint64_t)d->num_sms;
+    probe_gelu_kernel<<<(uint32_t)grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(in, (uint32_t)n, out);
+    return launch_status();
 }
 
 int nvq_device_status(nvq_stream_t stream) {

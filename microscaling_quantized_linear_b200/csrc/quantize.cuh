@@ -544,18 +544,49 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
 }
 
 // ------------------------------------------------------------------ MXFP8
-// One thread = one 32-element block.  Block b is (row b / nblk, column
-// b % nblk), nblk = K / 32; its codes are bytes [32b, 32b + 32).
-// ELEM 0: E4M3 elements (largest 448 = 1.75 * 2^8); ELEM 1: E5M2 (largest
-// 57344 = 1.75 * 2^15).  RULE 0: X = floor(log2 b) - emax (OCP); RULE 1:
-// the smallest X with b <= largest * 2^X, i.e. one more than the floor
-// value when b's significand exceeds 1.75 (both largest values are
-// 1.75 * 2^emax), so no element saturates.
+// One 32-element block, its 32 BF16 values in w[0..15] (element 2i in the
+// low half of w[i]).  ELEM 0: E4M3 elements (largest 448 = 1.75 * 2^8);
+// ELEM 1: E5M2 (largest 57344 = 1.75 * 2^15).  RULE 0: X = floor(log2 b) -
+// emax (OCP); RULE 1: the smallest X with b <= largest * 2^X, i.e. one more
+// than the floor value when b's significand exceeds 1.75 (both largest
+// values are 1.75 * 2^emax), so no element saturates.  Returns the E8M0
+// scale byte X + 127; q receives the 32 element codes, 4 per word.
+template <int ELEM, int RULE>
+__device__ __forceinline__ uint32_t mx_block(const uint32_t (&w)[16], uint32_t (&q)[8]) {
+    constexpr int EMAX = ELEM == 0 ? 8 : 15;
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m2 = absmax2(m2, w[i]);
+    const uint32_t mb = fold2(m2);                   // BF16 magnitude bits of the block max
+    int X;
+    if (mb == 0) {
+        X = -127;
+    } else {
+        const int E = (int)(mb >> 7);
+        const uint32_t mant = mb & 0x7Fu;
+        const int p = 31 - __clz((int)mant);          // subnormal: leading one of the mantissa
+        const int e = E ? E - 127 : p - 133;
+        int up = 0;
+        if (RULE == 1) up = E ? (mant > 96u) : (4u * mant > (7u << p));   // significand > 1.75
+        X = min(max(e - EMAX + up, -127), 127);
+    }
+    const float mult = __uint_as_float((uint32_t)(127 - X) << 23);   // 2^-X, -127 <= X <= 121
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 p0 = bf16x2_mul(w[2 * i], mult);
+        const float2 p1 = bf16x2_mul(w[2 * i + 1], mult);
+        q[i] = ELEM == 0 ? cvt_e4m3x4(p0.x, p0.y, p1.x, p1.y) : cvt_e5m2x4(p0.x, p0.y, p1.x, p1.y);
+    }
+    return (uint32_t)(X + 127);
+}
+
+// One thread = one 32-element block (mx_block above).  Block b is
+// (row b / nblk, column b % nblk), nblk = K / 32; its codes are bytes
+// [32b, 32b + 32).
 template <int ELEM, int RULE>
 __global__ void __launch_bounds__(kQuantThreads)
 mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nblk, uint32_t ldx,
                       uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
-    constexpr int EMAX = ELEM == 0 ? 8 : 15;
     griddep_wait();                              // x may come from the previous grid
     griddep_launch();
     const uint32_t total = rows * nblk;
@@ -577,31 +608,8 @@ mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
                 w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
             }
         }
-        uint32_t m2 = 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) m2 = absmax2(m2, w[i]);
-        const uint32_t mb = fold2(m2);               // BF16 magnitude bits of the block max
-        int X;
-        if (mb == 0) {
-            X = -127;
-        } else {
-            const int E = (int)(mb >> 7);
-            const uint32_t mant = mb & 0x7Fu;
-            const int p = 31 - __clz((int)mant);      // subnormal: leading one of the mantissa
-            const int e = E ? E - 127 : p - 133;
-            int up = 0;
-            if (RULE == 1) up = E ? (mant > 96u) : (4u * mant > (7u << p));   // significand > 1.75
-            X = min(max(e - EMAX + up, -127), 127);
-        }
-        const uint32_t sc = (uint32_t)(X + 127);
-        const float mult = __uint_as_float((uint32_t)(127 - X) << 23);   // 2^-X, -127 <= X <= 121
         uint32_t q[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float2 p0 = bf16x2_mul(w[2 * i], mult);
-            const float2 p1 = bf16x2_mul(w[2 * i + 1], mult);
-            q[i] = ELEM == 0 ? cvt_e4m3x4(p0.x, p0.y, p1.x, p1.y) : cvt_e5m2x4(p0.x, p0.y, p1.x, p1.y);
-        }
+        const uint32_t sc = mx_block<ELEM, RULE>(w, q);
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
         const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);

@@ -120,6 +120,29 @@ def test_block_scaled_linear_rejects_bad_arguments():
     assert gemm(out=P_ODD) == -3
 
 
+def gemm_gelu(fmt=0, a=P16, sa=P16, ga=P16, b=P16, sb=P16, gb=P16, bias=NULL, yc=P16, ys=P16, M=128, N=128,
+              K=256):
+    return L.block_scaled_linear_gelu_mxfp8(fmt, a, sa, ga, b, sb, gb, bias, yc, ys, M, N, K, NULL)
+
+
+def test_block_scaled_linear_gelu_mxfp8_rejects_bad_arguments():
+    assert gemm_gelu(fmt=2) == -7             # E5M2 operands are not offered here
+    assert gemm_gelu(fmt=5) == -7
+    assert gemm_gelu(M=-1) == -2
+    assert gemm_gelu(N=64) == -2               # N (the next layer's K) must be a multiple of 128
+    assert gemm_gelu(N=136) == -2
+    assert gemm_gelu(K=128) == -2              # NVFP4 K must be a multiple of 256
+    assert gemm_gelu(fmt=1, ga=NULL, gb=NULL, K=64) == -2
+    assert gemm_gelu(yc=NULL) == -1
+    assert gemm_gelu(ys=NULL) == -1
+    assert gemm_gelu(gb=NULL) == -1
+    assert gemm_gelu(yc=P_ODD) == -3
+    assert gemm_gelu(ys=P_ODD) == -3
+    assert gemm_gelu(M=0) == 0                 # empty batch: nothing to do
+    assert L.nvq_probe_gelu(NULL, 4, P16, NULL) == -1
+    assert L.nvq_probe_gelu(P16, -1, P16, NULL) == -2
+
+
 def test_valid_arguments_without_gpu_report_cuda_error():
     # Arguments pass the host checks; with no device the library reports a
     # CUDA error instead of launching.
@@ -133,3 +156,6 @@ def test_valid_arguments_without_gpu_report_cuda_error():
     assert gemm(M=96, N=64, ldo=64) == -5
     assert gemm(fmt=2, ga=NULL, gb=NULL, K=128) == -5
     assert L.mxfp8_quantize_ex(P16, 100, 128, 128, P16, P16, 2, 1, NULL) == -5
+    assert gemm_gelu() == -5
+    assert gemm_gelu(fmt=1, ga=NULL, gb=NULL, M=100, N=384, K=128) == -5
+    assert L.nvq_probe_gelu(P16, 16, P16, NULL) == -5

@@ -128,6 +128,13 @@ def exact_operand(rows, K, seed, significands=(1.0, 1.5, 1.75), top_row=None, mi
     return x, c.numpy()
 
 
+def grid_bias(N, seed=3):
+    """BF16 bias [N] of k / 16 with k uniform in [-16, 16] (on the same coarse
+    grid as exact_operand's products for its exponents >= -3) (CPU)."""
+    k = torch.randint(-16, 17, (N,), generator=_gen(seed))
+    return (k.double() / 16.0).to(torch.bfloat16)
+
+
 def normal(M, K, seed, std=1.0):
     """Plain BF16 N(0, std^2) tensor, for shape-sweep tests."""
     return (torch.randn(M, K, generator=_gen(seed)) * std).to(torch.bfloat16)
