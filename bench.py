@@ -307,6 +307,8 @@ def run_ours(args, rank, world, device):
         res["mxfp8_ffdown"] = run_mxfp8_component(nvq, args, device, stream, peaks)
     if args.small_m:
         res["small_m"] = run_small_m_component(nvq, device, stream, peaks)
+    if args.ff_block:
+        res["ff_block"] = run_ff_block_component(nvq, device, stream, peaks)
     return res
 
 
@@ -442,6 +444,67 @@ def run_mxfp8_component(nvq, args, device, stream, peaks):
                     key + "quant_frac_hbm": round(qbytes / (q_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
                     key + "gemm_us": round(g_us, 3), key + "gemm_tflops": round(flops / (g_us * 1e-6) / 1e12, 1),
                     key + "gemm_frac_fp8": round(flops / (g_us * 1e-6) / 1e12 / fp8_peak, 4)})
+    return res
+
+
+def run_ff_block_component(nvq, device, stream, peaks, iters=100):
+    """The FLUX-like feed-forward block, A [4608, 3072] -> FF-up (NVFP4,
+    N 12288) -> GELU -> FF-down (MXFP8, N 3072), with the GELU and the MXFP8
+    activation quantization fused into the FF-up GEMM's epilogue
+    (block_scaled_linear_gelu_mxfp8), against the same block with a plain
+    FF-up GEMM writing BF16 and a separate MXFP8 quantize pass (the unfused
+    chain has no GELU pass, which would cost it one more pass over the
+    113 MB activation)."""
+    up, down = workloads.WORKLOADS["ffup"], workloads.WORKLOADS["ffdown"]
+    M, H, F = up.M, up.K, up.N
+    xs = [workloads.activation("ffup", seed=20 + i).to(device) for i in range(2)]
+    w1c, w1s, w1g = nvq.quantize_weight("nvfp4", workloads.weight("ffup").to(device))
+    w2c, w2s, _ = nvq.quantize_weight("mxfp8", workloads.weight("ffdown").to(device))
+    ac = torch.empty((M, H // 2), dtype=torch.uint8, device=device)
+    as_ = torch.empty(nvq.scale_bytes("nvfp4", M, H), dtype=torch.uint8, device=device)
+    ag = torch.empty(1, dtype=torch.float32, device=device)
+    ws = nvq.new_workspace(device)
+    yc = torch.empty((M, F), dtype=torch.uint8, device=device)
+    ys = torch.empty(nvq.scale_bytes("mxfp8", M, F), dtype=torch.uint8, device=device)
+    d_up = torch.empty((M, F), dtype=torch.bfloat16, device=device)
+    out = torch.empty((M, H), dtype=torch.bfloat16, device=device)
+
+    def quant(i):
+        nvq.nvfp4_quantize(xs[i % 2], ac, as_, ag, workspace=ws, stream=stream)
+
+    def fused_up(i):
+        nvq.block_scaled_linear_gelu_mxfp8("nvfp4", ac, as_, ag, w1c, w1s, w1g, M, F, H, y_codes=yc, y_scales=ys,
+                                           stream=stream)
+
+    def plain_up(i):
+        nvq.block_scaled_linear("nvfp4", ac, as_, ag, w1c, w1s, w1g, M, F, H, out=d_up, stream=stream)
+
+    def requant(i):
+        nvq.mxfp8_quantize(d_up, yc, ys, stream=stream)
+
+    def ff_down(i):
+        nvq.block_scaled_linear("mxfp8", yc, ys, None, w2c, w2s, None, M, H, F, out=out, stream=stream)
+
+    def chain(*fns):
+        def run(i):
+            for f in fns:
+                f(i)
+        return run
+
+    t = {k: _back_to_back_us(f, iters, device, stream) for k, f in (
+        ("fused_ffup_us", fused_up), ("plain_ffup_us", plain_up), ("mxfp8_requant_us", requant),
+        ("block_fused_us", chain(quant, fused_up, ff_down)),
+        ("block_unfused_us", chain(quant, plain_up, requant, ff_down)))}
+    flops_up = 2.0 * M * F * H
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    res = {"workload": "FF block: A [4608,3072] -> NVFP4 FF-up [12288] -> GELU -> MXFP8 FF-down [3072]",
+           "metric": "TFLOP/s of the two GEMMs per block", "unit": "TFLOP/s",
+           "value_fused": round(2 * flops_up / (t["block_fused_us"] * 1e-6) / 1e12, 1),
+           "value_unfused": round(2 * flops_up / (t["block_unfused_us"] * 1e-6) / 1e12, 1),
+           "fused_ffup_tflops": round(flops_up / (t["fused_ffup_us"] * 1e-6) / 1e12, 1),
+           "fused_ffup_frac_fp4": round(flops_up / (t["fused_ffup_us"] * 1e-6) / 1e12 / fp4_peak, 4),
+           "note": "unfused chain: FF-up GEMM writes BF16, then mxfp8_quantize; it has no GELU pass"}
+    res.update({k: round(v, 3) for k, v in t.items()})
     return res
 
 
@@ -591,6 +654,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mxfp8", dest="mxfp8", action="store_false")
     ap.add_argument("--no-small-m", dest="small_m", action="store_false")
+    ap.add_argument("--no-ff-block", dest="ff_block", action="store_false")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -139,10 +139,9 @@ __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half,
             uint8_t* dst = eq.codes + (size_t)row * eq.n + cfirst;
 #pragma unroll
             for (int j = 0; j < NC; ++j) {
-                uint32_t g[16], q[8];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) g[e] = gelu_bf16x2(packed[j][e], gelu_tab);
-                scw |= mx_block<0, 0>(g, q) << (8 * j);
+                uint32_t q[8];
+                gelu_bf16x32(packed[j], gelu_tab);
+                scw |= mx_block<0, 0>(packed[j], q) << (8 * j);
                 uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * j);
                 d4[0] = make_uint4(q[0], q[1], q[2], q[3]);
                 d4[1] = make_uint4(q[4], q[5], q[6], q[7]);

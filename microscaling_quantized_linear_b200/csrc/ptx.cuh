@@ -340,7 +340,7 @@ __device__ __forceinline__ void tc_mma_mxf8_pair(uint32_t d_tmem, uint64_t a_des
 // nibble), round to nearest even, saturating to +-6.
 __device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
     uint32_t out;
-    asm volatile(
+    asm(
         "{\n\t.reg .b8 t;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
         "cvt.u32.u8 %0, t;\n\t}"
@@ -353,7 +353,7 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
 __device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, float a3,
                                                float a4, float a5, float a6, float a7) {
     uint32_t out;
-    asm volatile(
+    asm(
         "{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
@@ -368,7 +368,7 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, flo
 // Four FP32 -> four E4M3 codes in one word, a0 in bits 7:0.
 __device__ __forceinline__ uint32_t cvt_e4m3x4(float a0, float a1, float a2, float a3) {
     uint32_t out;
-    asm volatile(
+    asm(
         "{\n\t.reg .b16 h0, h1;\n\t"
         "cvt.rn.satfinite.e4m3x2.f32 h0, %2, %1;\n\t"
         "cvt.rn.satfinite.e4m3x2.f32 h1, %4, %3;\n\t"
@@ -381,7 +381,7 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4(float a0, float a1, float a2, flo
 // round-to-nearest-even; one packed f32x2 multiply).
 __device__ __forceinline__ float2 bf16x2_mul(uint32_t w, float m) {
     float2 c;
-    asm volatile(
+    asm(
         "{\n\t.reg .b32 lo, hi;\n\t.reg .b64 x, y, z;\n\t"
         "shl.b32 lo, %2, 16;\n\t"
         "and.b32 hi, %2, 0xFFFF0000;\n\t"
@@ -397,7 +397,7 @@ __device__ __forceinline__ float2 bf16x2_mul(uint32_t w, float m) {
 // even, saturating to +-57344.
 __device__ __forceinline__ uint32_t cvt_e5m2x4(float a0, float a1, float a2, float a3) {
     uint32_t out;
-    asm volatile(
+    asm(
         "{\n\t.reg .b16 h0, h1;\n\t"
         "cvt.rn.satfinite.e5m2x2.f32 h0, %2, %1;\n\t"
         "cvt.rn.satfinite.e5m2x2.f32 h1, %4, %3;\n\t"
@@ -422,7 +422,7 @@ __device__ __forceinline__ float2 f32x2_mul(float a, float b, float m) {
 // round to nearest even, saturating to +-448.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
     uint16_t out;
-    asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
     return out;
 }
 
