@@ -491,6 +491,9 @@ def run_ff_block_component(nvq, device, stream, peaks, iters=100):
                 f(i)
         return run
 
+    quant(0)                 # the standalone legs below read a real quantized activation
+    plain_up(0)
+    torch.cuda.synchronize(device)
     t = {k: _back_to_back_us(f, iters, device, stream) for k, f in (
         ("fused_ffup_us", fused_up), ("plain_ffup_us", plain_up), ("mxfp8_requant_us", requant),
         ("block_fused_us", chain(quant, fused_up, ff_down)),
