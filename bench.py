@@ -267,7 +267,7 @@ def run_ours(args, rank, world, device):
                   "all larger than the 126 MB L2" % (ROTATE, ROTATE * (M * K * 2 + N * K * 0.5625) / 1e6,
                                                      M * N * 2 / 1e6),
         },
-        "act_quant": run_act_quant_component(nvq, device, stream, peaks),
+        "act_quant": run_act_quant_component(nvq, device, stream, peaks) if args.act_quant else None,
         "act_quant_in_step": {
             "value": round(act_gbs, 1), "unit": "GB/s", "us_per_call": round(quant_mean, 3),
             "bytes_per_call": int(act_bytes), "launches_per_call": 2,
@@ -658,6 +658,7 @@ def main():
     ap.add_argument("--no-mxfp8", dest="mxfp8", action="store_false")
     ap.add_argument("--no-small-m", dest="small_m", action="store_false")
     ap.add_argument("--no-ff-block", dest="ff_block", action="store_false")
+    ap.add_argument("--no-act-quant", dest="act_quant", action="store_false")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
