@@ -45,8 +45,8 @@ ACT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # BF16 read, E2M1 codes + E4M3 scale
 # Taken on the FF-up workload; the summary is in
 # profiles/bsgemm_pair_kernel_nvfp4_ffup.md.
 GEMM_TRAFFIC = {"kernel": "bsgemm_pair_kernel<0, 256>",
-                "bytes_per_launch": 29252096 + 62992896,
-                "sources_sha256": "781e3491fa97916197ed8a6b4c0abfd8661351333a4ad40ac8b614c01329ed6c"}
+                "bytes_per_launch": 29267456 + 62559488,
+                "sources_sha256": "2e8387cfad5a9773ef4664cfe56fbd5b842c1d3ee18a34de1ea2a357b0bff2de"}
 KERNEL_SOURCES = ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh")
 
 
