@@ -78,6 +78,31 @@ def gemm_traffic(kernel):
     return GEMM_TRAFFIC["bytes_per_launch"]
 
 
+# --------------------------------------------------------------------------- ranks
+# One process per GPU (torch.distributed.run), every rank an independent
+# replica on its own seeded batch: the only collectives are the timing
+# barrier and the max-over-ranks of the elapsed time.
+
+def rank_seeds(rank, count, base=0):
+    """Seeds of the rank's input tensors: disjoint across ranks."""
+    return [1000 * rank + base + i for i in range(count)]
+
+
+def max_over_ranks(value, world, device=None):
+    """Largest value over all ranks (the job's time is the slowest rank's)."""
+    if world <= 1:
+        return value
+    dev = device if device is not None and device.type == "cuda" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.item()
+
+
+def job_throughput(world, flops_per_step, steps, elapsed_ms):
+    """Whole-job TFLOP/s: the work of every rank over the slowest rank's time."""
+    return world * flops_per_step * steps / (elapsed_ms * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -161,10 +186,10 @@ def run_ours(args, rank, world, device):
 
     # Inputs: ROTATE activation batches and ROTATE quantized weights (seeded per
     # rank), resident in HBM before the timed region.
-    xs = [workloads.activation(WORKLOAD, seed=1000 * rank + i).to(device) for i in range(ROTATE)]
+    xs = [workloads.activation(WORKLOAD, seed=sd).to(device) for sd in rank_seeds(rank, ROTATE)]
     wq = []
-    for i in range(ROTATE):
-        wd = workloads.weight(WORKLOAD, seed=1000 * rank + 100 + i).to(device)
+    for sd in rank_seeds(rank, ROTATE, base=100):
+        wd = workloads.weight(WORKLOAD, seed=sd).to(device)
         wq.append(nvq.quantize_weight("nvfp4", wd))
         del wd
     codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
@@ -209,12 +234,7 @@ def run_ours(args, rank, world, device):
         torch.cuda.synchronize(device)
         if world > 1:
             torch.distributed.barrier()
-        ms = t0.elapsed_time(t1)
-        if world > 1:
-            t = torch.tensor([ms], dtype=torch.float64, device=device)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = t.item()
-        return ms
+        return max_over_ranks(t0.elapsed_time(t1), world, device)
 
     # The headline region runs the steps exactly as a user issues them.  An
     # event recorded between the quantizer and the GEMM ends their launch
@@ -230,7 +250,7 @@ def run_ours(args, rank, world, device):
     quant_us = [ev[i][0].elapsed_time(ev[i][1]) * 1e3 for i in range(n_ev)]
     gemm_us = [ev[i][1].elapsed_time(ev[i][2]) * 1e3 for i in range(n_ev)]
     ms_per_step = elapsed_ms / args.steps
-    value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = job_throughput(world, flops, args.steps, elapsed_ms)
 
     peaks = load_peaks()
     sustained = elapsed_ms > 1000.0
@@ -368,12 +388,8 @@ def run_e2e(nvq, args, device, stream, x_host_src, wq, M, N, K, flops, world):
     s_out.wait_stream(stream)
     b.record(s_out)
     torch.cuda.synchronize(device)
-    ms = a.elapsed_time(b) / steps
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = t.item()
-    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, device)
+    return {"value": round(job_throughput(world, flops, 1, ms), 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(out_host[0].numel() * 2),
             "ms_per_step": round(ms, 4), "steps": steps,
             "pipelining": "input copy, compute and output copy on three streams, two device buffer sets"}
