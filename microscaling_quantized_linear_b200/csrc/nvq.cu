@@ -222,7 +222,8 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
         // One pass when every CTA's rows fit in shared memory (one CTA per SM).
         const int64_t rows_per_cta = (M + d->num_sms - 1) / d->num_sms;
         const size_t smem = fused_smem_bytes((size_t)rows_per_cta, (size_t)K);
-        if (smem <= kFusedSmemMax && (M + rows_per_cta - 1) / rows_per_cta <= kMaxFusedCtas) {
+        if (smem <= kFusedSmemMax && (M + rows_per_cta - 1) / rows_per_cta <= kMaxFusedCtas &&
+            rows_per_cta * (K / 16) <= (int64_t)kFusedMaxBlocks * kFusedThreads) {
             {
                 std::lock_guard<std::mutex> lock(g_mu);
                 if (!d->fused_attr) {
@@ -240,10 +241,28 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
             uint32_t epoch = next_epoch();
             unsigned int* status = d->status;
             void* args[] = {&xp, &rows32, &k32, &ld32, &rpc, &codes, &scales, &global_scale, &slots, &epoch, &status};
-            if (cudaLaunchCooperativeKernel((const void*)nvfp4_quantize_fused_kernel, dim3(grid),
-                                            dim3(kFusedThreads), args, smem, stream) != cudaSuccess) {
+            // co-resident CTAs (the kernel waits on every CTA's maximum),
+            // launched with programmatic stream serialization; a runtime that
+            // refuses the two together gets a plain cooperative launch
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(grid);
+            cfg.blockDim = dim3(kFusedThreads);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[2];
+            attr[0].id = cudaLaunchAttributeCooperative;
+            attr[0].val.cooperative = 1;
+            attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[1].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 2;
+            if (cudaLaunchKernelExC(&cfg, (const void*)nvfp4_quantize_fused_kernel, args) != cudaSuccess) {
                 cudaGetLastError();
-                return NVQ_ERR_CUDA;
+                if (cudaLaunchCooperativeKernel((const void*)nvfp4_quantize_fused_kernel, dim3(grid),
+                                                dim3(kFusedThreads), args, smem, stream) != cudaSuccess) {
+                    cudaGetLastError();
+                    return NVQ_ERR_CUDA;
+                }
             }
             return NVQ_OK;
         }

@@ -108,12 +108,12 @@ __device__ __forceinline__ float div6(uint32_t mb, const float* d6) {
     return __fdiv_rn(__uint_as_float(mb << 16), 6.0f);
 }
 
-// One 16-element block: block max bits mb, the 16 BF16 values in w[0..7].
-// Returns the E4M3 scale code; lo/hi receive the 16 E2M1 codes.  g_enc == 0
-// (a zero tensor) gives scale 0 and zero codes.
-__device__ __forceinline__ uint32_t nvfp4_block(uint32_t mb, const uint32_t (&w)[8], float g_enc,
-                                                const float* d6, const float* rtab, uint32_t& lo, uint32_t& hi) {
-    const float s = __fmul_rn(div6(mb, d6), g_enc);
+// One 16-element block given d = fl(b / 6) for its block max b, the 16 BF16
+// values in w[0..7].  Returns the E4M3 scale code; lo/hi receive the 16 E2M1
+// codes.  g_enc == 0 (a zero tensor) gives scale 0 and zero codes.
+__device__ __forceinline__ uint32_t nvfp4_block_d(float d, const uint32_t (&w)[8], float g_enc, const float* rtab,
+                                                  uint32_t& lo, uint32_t& hi) {
+    const float s = __fmul_rn(d, g_enc);
     const uint32_t sc = cvt_e4m3x2(0.0f, s) & 0xFFu;
     const float r = rtab[sc];
     float2 p[8];
@@ -123,6 +123,12 @@ __device__ __forceinline__ uint32_t nvfp4_block(uint32_t mb, const uint32_t (&w)
     hi = cvt_e2m1x8(p[4].x, p[4].y, p[5].x, p[5].y, p[6].x, p[6].y, p[7].x, p[7].y);
     if (sc == 0) lo = hi = 0;                         // scale rounded to zero: zero codes (no -0)
     return sc;
+}
+
+// The same block given its block max bits mb.
+__device__ __forceinline__ uint32_t nvfp4_block(uint32_t mb, const uint32_t (&w)[8], float g_enc,
+                                                const float* d6, const float* rtab, uint32_t& lo, uint32_t& hi) {
+    return nvfp4_block_d(div6(mb, d6), w, g_enc, rtab, lo, hi);
 }
 
 __device__ __forceinline__ float encode_scale(float amax) {
@@ -363,15 +369,15 @@ nvfp4_quantize_cluster_kernel(const uint16_t* __restrict__ x, uint32_t rows, uin
 
 // ------------------------------------------------------------------ NVFP4, one pass
 // For tensors whose rows fit in the shared memory of one CTA per SM: every
-// CTA copies its rows into shared memory once (bulk copies, 4 chunks with
-// their own mbarriers so the block maxima are taken while later chunks are
-// still landing, and kept in shared memory), publishes its partial amax in an
-// epoch-tagged 64-bit slot of the workspace, waits (bounded) until every
-// CTA's slot carries this call's epoch, and quantizes from shared memory.
-// HBM sees exactly one read of the activation.  Must be launched
-// cooperatively (all CTAs co-resident).
+// CTA copies its rows into shared memory once (each thread copies its own
+// blocks with 16-byte asynchronous copies, all issued at once, one commit
+// group per block, and takes each block's maximum and fl(b/6) as its group
+// lands), publishes its partial amax in an epoch-tagged 64-bit slot of the
+// workspace, waits (bounded) until every CTA's slot carries this call's
+// epoch, and quantizes from shared memory.  HBM sees exactly one read of the
+// activation.  Must be launched cooperatively (all CTAs co-resident).
 constexpr int kFusedThreads = 1024;
-constexpr int kFusedChunks = 4;
+constexpr int kFusedMaxBlocks = 8;                 // 16-blocks per thread: rows_per_cta * K / 16 <= 8192
 constexpr uint64_t kFusedWaitNs = 2000000000ull;   // 2 s
 
 // The slot word carries its epoch and its value together, so relaxed
@@ -398,9 +404,10 @@ __device__ __forceinline__ void lds_block32(const uint8_t* base, uint32_t b, uin
     v1 = sw ? first : second;
 }
 
-// Shared memory the one-pass kernel needs for rows_per_cta rows of K.
+// Shared memory the one-pass kernel needs for rows_per_cta rows of K: the
+// BF16 tile and fl(b / 6) of every block's max b.
 __host__ __device__ constexpr size_t fused_smem_bytes(size_t rows_per_cta, size_t K) {
-    return 128 /*align*/ + rows_per_cta * K * 2 /*tile*/ + rows_per_cta * (K / 16) * 2 /*block maxima*/;
+    return 128 /*align*/ + rows_per_cta * K * 2 /*tile*/ + rows_per_cta * (K / 16) * 4 /*fl(b/6)*/;
 }
 
 __global__ void __launch_bounds__(kFusedThreads, 1)
@@ -411,49 +418,59 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const uint32_t nblk = K >> 4;
-    uint16_t* bmax = reinterpret_cast<uint16_t*>(tile + (size_t)rows_per_cta * K * 2);
-    __shared__ __align__(8) uint64_t bars[kFusedChunks];
+    float* bdiv6 = reinterpret_cast<float*>(tile + (size_t)rows_per_cta * K * 2);
     __shared__ uint32_t red[kFusedThreads / 32];
+    __shared__ uint32_t s_pmax[kMaxFusedCtas / 32];
     __shared__ float d6[128], rtab[128];
     __shared__ int s_timeout;
 
+    // x may come from the previous grid, and that grid may still read the
+    // outputs: nothing global is touched before it has completed
+    griddep_wait();
+    griddep_launch();
     const uint32_t r0 = blockIdx.x * rows_per_cta;
     const uint32_t nr = min(rows_per_cta, rows - r0);
-    const uint32_t row_bytes = K * 2;
-    const uint32_t rows_per_chunk = (nr + kFusedChunks - 1) / kFusedChunks;
-    if (threadIdx.x == 0) {
-        s_timeout = 0;
-        for (int c = 0; c < kFusedChunks; ++c) mbar_init(smem_u32(&bars[c]), 1);
-        fence_mbarrier_init();
-        for (int c = 0; c < kFusedChunks; ++c) {
-            const uint32_t ra = min(nr, c * rows_per_chunk), rb = min(nr, (c + 1) * rows_per_chunk);
-            const uint32_t bar = smem_u32(&bars[c]);
-            mbar_arrive_expect_tx(bar, (rb - ra) * row_bytes);
-            if (ldx == K) {
-                if (rb > ra)
-                    bulk_load(smem_u32(tile + (size_t)ra * row_bytes), x + (size_t)(r0 + ra) * K,
-                              (rb - ra) * row_bytes, bar);
-            } else {
-                for (uint32_t r = ra; r < rb; ++r)
-                    bulk_load(smem_u32(tile + (size_t)r * row_bytes), x + (size_t)(r0 + r) * ldx, row_bytes, bar);
-            }
+    const uint32_t total = nr * nblk;
+    // Thread t copies blocks t, t + 1024, ... (the ones it quantizes later),
+    // one commit group per block slot so that each can be used as it lands;
+    // slots past the thread's blocks commit empty groups.
+#pragma unroll
+    for (int i = 0; i < kFusedMaxBlocks; ++i) {
+        const uint32_t b = threadIdx.x + (uint32_t)i * kFusedThreads;
+        if (b < total) {
+            const uint32_t rl = b / nblk, c = b - rl * nblk;
+            const uint16_t* src = x + (size_t)(r0 + rl) * ldx + (size_t)c * 16;
+            const uint32_t dst = smem_u32(tile + (size_t)b * 32);
+            cp_async16(dst, src);
+            cp_async16(dst + 16, src + 8);
         }
+        cp_async_commit();
     }
+    if (threadIdx.x == 0) s_timeout = 0;
     init_d6(d6);
     __syncthreads();
 
-    // block maxima, chunk by chunk as the copies land
+    // block maxima and fl(b/6), block by block as the copies land
     uint32_t m = 0;
-    for (int c = 0; c < kFusedChunks; ++c) {
-        const uint32_t ra = min(nr, c * rows_per_chunk), rb = min(nr, (c + 1) * rows_per_chunk);
-        if (!mbar_wait_bounded(smem_u32(&bars[c]), 0, &s_timeout, kFusedWaitNs)) s_timeout = 1;
-        if (s_timeout) break;
-        for (uint32_t b = ra * nblk + threadIdx.x; b < rb * nblk; b += kFusedThreads) {
+#pragma unroll
+    for (int i = 0; i < kFusedMaxBlocks; ++i) {
+        switch (i) {            // at most kFusedMaxBlocks - 1 - i groups may still be pending
+            case 0: cp_async_wait<kFusedMaxBlocks - 1>(); break;
+            case 1: cp_async_wait<kFusedMaxBlocks - 2>(); break;
+            case 2: cp_async_wait<kFusedMaxBlocks - 3>(); break;
+            case 3: cp_async_wait<kFusedMaxBlocks - 4>(); break;
+            case 4: cp_async_wait<kFusedMaxBlocks - 5>(); break;
+            case 5: cp_async_wait<kFusedMaxBlocks - 6>(); break;
+            case 6: cp_async_wait<kFusedMaxBlocks - 7>(); break;
+            default: cp_async_wait<0>(); break;
+        }
+        const uint32_t b = threadIdx.x + (uint32_t)i * kFusedThreads;
+        if (b < total) {
             uint4 v0, v1;
             lds_block32(tile, b, v0, v1);
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
             const uint32_t mb = block16_max(w);
-            bmax[b] = (uint16_t)mb;
+            bdiv6[b] = div6(mb, d6);           // the scale's first step, done while copies land
             m = max(m, mb);
         }
     }
@@ -461,45 +478,43 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
     if (threadIdx.x == 0)
         st_relaxed_u64(slots + (size_t)blockIdx.x * kFusedSlotStride, ((unsigned long long)epoch << 32) | cta_max);
 
-    // Every CTA's partial, tagged with this call's epoch.  One warp polls
-    // (lane l watches slots l, l + 32, ...); the other warps wait at the
-    // barrier below, so the poll traffic is one load per slot per CTA.
-    __shared__ uint32_t s_amax;
-    if (threadIdx.x < 32) {
-        uint32_t mine = 0, pending = 0;
-        for (uint32_t j = threadIdx.x, bit = 0; j < gridDim.x; j += 32, ++bit) pending |= 1u << bit;
+    // Every CTA's partial, tagged with this call's epoch.  Warp w polls slots
+    // 32w .. 32w + 31, one per lane, so a polling round costs one L2 round
+    // trip; the other warps wait at the barrier below.
+    const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t npoll = (gridDim.x + 31) >> 5;
+    if (warp < npoll) {
+        volatile int* timeout = &s_timeout;
+        const uint32_t j = warp * 32 + lane;
+        bool done = j >= gridDim.x;
+        uint32_t mine = 0;
         const uint64_t t0 = globaltimer_ns();
         while (true) {
-            for (uint32_t j = threadIdx.x, bit = 0; j < gridDim.x; j += 32, ++bit) {
-                if (!(pending & (1u << bit))) continue;
+            if (!done) {
                 const unsigned long long v = ld_relaxed_u64(slots + (size_t)j * kFusedSlotStride);
                 if ((uint32_t)(v >> 32) == epoch) {
-                    mine = max(mine, (uint32_t)(v & 0xFFFFFFFFull));
-                    pending &= ~(1u << bit);
+                    mine = (uint32_t)(v & 0xFFFFFFFFull);
+                    done = true;
                 }
             }
-            if (!__any_sync(0xFFFFFFFFu, pending != 0)) break;
+            if (__all_sync(0xFFFFFFFFu, done)) break;
             int give_up = 0;                          // decided by lane 0 so the warp leaves together
-            if (threadIdx.x == 0) give_up = s_timeout || globaltimer_ns() - t0 > kFusedWaitNs;
+            if (lane == 0) give_up = *timeout || globaltimer_ns() - t0 > kFusedWaitNs;
             if (__shfl_sync(0xFFFFFFFFu, give_up, 0)) {
-                if (threadIdx.x == 0) s_timeout = 1;
+                if (lane == 0) *timeout = 1;
                 break;
             }
         }
         mine = __reduce_max_sync(0xFFFFFFFFu, mine);
-        if (threadIdx.x == 0) s_amax = mine;
+        if (lane == 0) s_pmax[warp] = mine;
     }
     __syncthreads();
-    const uint32_t amax_bits = s_amax;
-    if (s_timeout) {                                  // a copy or a peer never arrived: write nothing
-        if (threadIdx.x == 0) {
-            atomicOr(status, 1u);
-            int never = 0;                            // let every issued copy land before the CTA exits
-            for (int c = 0; c < kFusedChunks; ++c) mbar_wait_bounded(smem_u32(&bars[c]), 0, &never, kFusedWaitNs);
-        }
-        __syncthreads();
-        return;
+    if (s_timeout) {                                  // a peer never arrived: write nothing
+        if (threadIdx.x == 0) atomicOr(status, 1u);
+        return;                                       // every copy of this thread has landed
     }
+    uint32_t amax_bits = 0;
+    for (uint32_t i = 0; i < npoll; ++i) amax_bits = max(amax_bits, s_pmax[i]);
     if (amax_bits >= 0x7F80u && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, 2u);
     const float amax = __uint_as_float(amax_bits << 16);
     const float g_enc = encode_scale(amax);
@@ -507,34 +522,55 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
     init_rtab(rtab, g_enc);
     __syncthreads();
 
-    const uint32_t total = nr * nblk;
+    // Two blocks per thread per iteration (b and b + kFusedThreads), both
+    // read before either is computed.
     const uint32_t ctiles = nblk >> 2;
     const uint32_t qs = kFusedThreads / nblk, rs = kFusedThreads - qs * nblk;
     uint32_t rl = threadIdx.x / nblk, c = threadIdx.x - rl * nblk;
     const size_t code_base = (size_t)r0 * nblk * 8;
-    for (uint32_t base = 0; base < total; base += kFusedThreads) {
-        const uint32_t b = base + threadIdx.x;
-        const bool active = b < total;
-        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-        uint32_t mb = 0;
-        if (active) {
-            lds_block32(tile, b, v0, v1);
-            mb = bmax[b];
+    for (uint32_t base = 0; base < total; base += 2 * kFusedThreads) {
+        uint32_t rlu[2], cu[2];
+        rlu[0] = rl;
+        cu[0] = c;
+        rlu[1] = rl + qs;
+        cu[1] = c + rs;
+        if (cu[1] >= nblk) {
+            cu[1] -= nblk;
+            ++rlu[1];
         }
-        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        uint32_t lo, hi;
-        const uint32_t sc = nvfp4_block(mb, w, g_enc, d6, rtab, lo, hi);
-        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
-        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
-        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
-        if (active) {
-            *reinterpret_cast<uint2*>(codes + code_base + (size_t)b * 8) = make_uint2(lo, hi);
-            if ((c & 3u) == 0)
-                *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r0 + rl, c, ctiles)) =
-                    sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        uint4 v[4];
+        float d[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const uint32_t b = base + u * kFusedThreads + threadIdx.x;
+            v[2 * u] = v[2 * u + 1] = make_uint4(0, 0, 0, 0);
+            d[u] = 0.0f;
+            if (b < total) {
+                lds_block32(tile, b, v[2 * u], v[2 * u + 1]);
+                d[u] = bdiv6[b];
+            }
         }
-        rl += qs;
-        c += rs;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const uint32_t b = base + u * kFusedThreads + threadIdx.x;
+            const bool active = b < total;           // whole warps stay for the shuffles
+            const uint32_t w[8] = {v[2 * u].x, v[2 * u].y, v[2 * u].z, v[2 * u].w,
+                                   v[2 * u + 1].x, v[2 * u + 1].y, v[2 * u + 1].z, v[2 * u + 1].w};
+            uint32_t lo, hi;
+            const uint32_t sc = nvfp4_block_d(d[u], w, g_enc, rtab, lo, hi);
+            const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
+            const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
+            const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
+            if (active) {
+                *reinterpret_cast<uint2*>(codes + code_base + (size_t)b * 8) = make_uint2(lo, hi);
+                if ((cu[u] & 3u) == 0)
+                    *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r0 + rlu[u], cu[u], ctiles)) =
+                        sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            }
+        }
+        // advance by two strides
+        rl = rlu[1] + qs;
+        c = cu[1] + rs;
         if (c >= nblk) {
             c -= nblk;
             ++rl;
