@@ -318,6 +318,18 @@ NVQ_API int nvq_probe_convert(const float* in, int64_t n, uint8_t* e2m1_out, uin
  */
 NVQ_API int nvq_probe_gelu(const uint16_t* in, int64_t n, uint16_t* out, nvq_stream_t stream);
 
+/*
+ * nvq_probe_wait -- bounded-wait self-test (no counterpart on the pages).
+ * Launches one thread that waits, with the same bounded wait every GEMM
+ * pipeline stage uses, on an mbarrier that nothing arrives on.  After
+ * limit_ns of wall time the wait gives up, sets NVQ_STATUS_TIMEOUT in the
+ * device status word (read it with nvq_device_status) and the kernel returns
+ * normally, so the context stays usable.  Nothing faults, traps or hangs.
+ *   limit_ns    the wait's limit, at most 1e9 (else NVQ_ERR_SHAPE)
+ *   waited_ns   device pointer to one 64-bit word: the nanoseconds waited
+ */
+NVQ_API int nvq_probe_wait(uint64_t limit_ns, unsigned long long* waited_ns, nvq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

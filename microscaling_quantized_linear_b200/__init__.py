@@ -72,11 +72,13 @@ _lib.block_scaled_linear_gelu_mxfp8.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp
                                                 _i64, _i64, _i64, _vp]
 _lib.nvq_probe_gelu.restype = ctypes.c_int
 _lib.nvq_probe_gelu.argtypes = [_vp, _i64, _vp, _vp]
+_lib.nvq_probe_wait.restype = ctypes.c_int
+_lib.nvq_probe_wait.argtypes = [ctypes.c_uint64, _vp, _vp]
 
 EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_quantize",
             "mxfp8_quantize", "mxfp8_quantize_ex", "quantize_weight", "block_scaled_linear",
             "nvq_device_status", "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc",
-            "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu")
+            "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu", "nvq_probe_wait")
 
 NOALLOC_MAX_PARTIALS = 1024
 
@@ -283,6 +285,15 @@ def probe_gelu(bits, stream=None):
     out = torch.empty(n, dtype=torch.int16, device=bits.device)
     _check(_lib.nvq_probe_gelu(_ptr(bits), n, _ptr(out), _stream(stream, bits.device)), "nvq_probe_gelu")
     return out
+
+
+def probe_wait(limit_ns, device=None, stream=None):
+    """Run the bounded-wait self-test; returns the nanoseconds the device waited
+    (the status word then holds NVQ_STATUS_TIMEOUT; read it with device_status)."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    waited = torch.zeros(1, dtype=torch.int64, device=dev)
+    _check(_lib.nvq_probe_wait(int(limit_ns), _ptr(waited), _stream(stream, dev)), "nvq_probe_wait")
+    return int(waited.item())
 
 
 def probe_convert(values, stream=None):

@@ -643,6 +643,16 @@ int nvq_probe_gelu(const uint16_t* in, int64_t n, uint16_t* out, nvq_stream_t st
     return launch_status();
 }
 
+int nvq_probe_wait(uint64_t limit_ns, unsigned long long* waited_ns, nvq_stream_t stream) {
+    if (!waited_ns) return NVQ_ERR_NULL;
+    if (limit_ns > 1000000000ull) return NVQ_ERR_SHAPE;    // at most 1 s
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc) return rc;
+    probe_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, d->status, waited_ns);
+    return launch_status();
+}
+
 int nvq_device_status(nvq_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NVQ_ERR_CUDA;
     DeviceInfo* d = nullptr;

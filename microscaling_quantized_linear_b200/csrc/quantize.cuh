@@ -677,4 +677,22 @@ __global__ void probe_convert_kernel(const float* __restrict__ in, uint32_t n,
     }
 }
 
+// Test hook for the bounded waits: one thread waits, through the same
+// mbar_wait_bounded the GEMM pipelines use, on a shared-memory mbarrier that
+// nothing arrives on.  When the wait gives up after limit_ns it sets
+// NVQ_STATUS_TIMEOUT (bit 0) in the status word, as a GEMM role would, and the
+// kernel returns normally.  *waited receives the nanoseconds spent.
+__global__ void probe_wait_kernel(uint64_t limit_ns, unsigned int* __restrict__ status,
+                                  unsigned long long* __restrict__ waited) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int never;
+    if (threadIdx.x != 0) return;
+    never = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbarrier_init();
+    const uint64_t t0 = globaltimer_ns();
+    if (!mbar_wait_bounded(smem_u32(&bar), 0, &never, limit_ns)) atomicOr(status, 1u);
+    *waited = globaltimer_ns() - t0;
+}
+
 }  // namespace nvq

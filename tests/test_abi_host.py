@@ -140,6 +140,8 @@ def test_block_scaled_linear_gelu_mxfp8_rejects_bad_arguments():
     assert gemm_gelu(ys=P_ODD) == -3
     assert gemm_gelu(M=0) == 0                 # empty batch: nothing to do
     assert L.nvq_probe_gelu(NULL, 4, P16, NULL) == -1
+    assert L.nvq_probe_wait(1000, NULL, NULL) == -1
+    assert L.nvq_probe_wait(2 * 10**9, P16, NULL) == -2
     assert L.nvq_probe_gelu(P16, -1, P16, NULL) == -2
 
 
@@ -159,3 +161,4 @@ def test_valid_arguments_without_gpu_report_cuda_error():
     assert gemm_gelu() == -5
     assert gemm_gelu(fmt=1, ga=NULL, gb=NULL, M=100, N=384, K=128) == -5
     assert L.nvq_probe_gelu(P16, 16, P16, NULL) == -5
+    assert L.nvq_probe_wait(1000, P16, NULL) == -5
