@@ -204,3 +204,75 @@ def test_feed_forward_block_end_to_end():
     o2c, o2s = oracle.mxfp8_quantize(bits(w2))
     Y2 = oracle.gemm_rows(oracle.mxfp8_dequantize(oc, osf, M, F), oracle.mxfp8_dequantize(o2c, o2s, H, F))
     check_gemm(out.float().cpu().numpy(), Y2)
+
+
+def _check_sampled_rows(yc, ys, oc, osf, rows, M, N):
+    nb = N // 32
+    gs = sf_matrix(ys, M, nb)[rows]
+    os_ = sf_matrix(osf, rows.size, nb)
+    sdiff = gs.astype(np.int64) - os_.astype(np.int64)
+    assert np.abs(sdiff).max() <= 1
+    assert np.count_nonzero(sdiff) <= max(2, 1e-3 * sdiff.size), np.count_nonzero(sdiff)
+    same_scale = np.repeat(sdiff == 0, 32, axis=1)
+    steps = e4m3_steps_apart(yc[rows], oc)[same_scale]
+    assert steps.max() <= 1, steps.max()
+    assert np.count_nonzero(steps) <= 1e-3 * steps.size, np.count_nonzero(steps)
+
+
+def test_ffup_workload_mxfp8_operands_sampled_rows():
+    """The same FF-up linear with MXFP8 (E4M3) activation and weight operands."""
+    x, w = act("ffup"), wgt("ffup")
+    M, K = x.shape
+    N = w.shape[0]
+    ops, A, B = quantize_both("mxfp8", x, w)
+    yc, ys = gpu_fused("mxfp8", ops, M, N, K)
+    rows = sample_rows(M, per_tile_every=3, extra=8)
+    oc, osf, _, _, _ = oracle.linear_gelu_mxfp8(A, B, rows=rows)
+    _check_sampled_rows(yc, ys, oc, osf, rows, M, N)
+
+
+SINGLE_CTA_FUSED_SCRIPT = r"""
+import sys, numpy as np
+sys.path.insert(0, ROOT_DIR)
+sys.path.insert(0, TEST_DIR)
+import test_gpu_fused as t
+import workloads, oracle
+from gpu_common import bits, sample_rows
+# exact-grid operands: bit-exact codes and scales through the one-CTA kernel
+for fmt, M, N, K in [("nvfp4", 512, 768, 512), ("nvfp4", 1280, 512, 256), ("mxfp8", 384, 512, 256)]:
+    if fmt == "nvfp4":
+        x, _ = workloads.exact_operand(M, K, seed=M + 3, top_row=1)
+        w, _ = workloads.exact_operand(N, K, seed=N + 5, top_row=2)
+    else:
+        x, _ = workloads.exact_operand(M, K, seed=M + 3, significands=(1.0, 1.5))
+        w, _ = workloads.exact_operand(N, K, seed=N + 5, significands=(1.0, 1.5))
+    ops, A, B = t.quantize_both(fmt, x, w)
+    yc, ys = t.gpu_fused(fmt, ops, M, N, K)
+    oc, osf, _, _, _ = oracle.linear_gelu_mxfp8(A, B)
+    assert np.array_equal(ys, osf) and np.array_equal(yc, oc), (fmt, M, N, K)
+    print(fmt, M, N, K, "bit-exact")
+# the FF-up workload: within one step of the oracle on sampled rows
+x, w = t.act("ffup"), t.wgt("ffup")
+M, K = x.shape
+N = w.shape[0]
+ops, A, B = t.quantize_both("nvfp4", x, w)
+yc, ys = t.gpu_fused("nvfp4", ops, M, N, K)
+rows = sample_rows(M, per_tile_every=6, extra=8)
+oc, osf, _, _, _ = oracle.linear_gelu_mxfp8(A, B, rows=rows)
+t._check_sampled_rows(yc, ys, oc, osf, rows, M, N)
+print("OK")
+"""
+
+
+def test_single_cta_kernel_fused_epilogue():
+    # NVQ_GEMM_PAIRS=0 (read when the library loads, hence a fresh process)
+    # sends every shape through the one-CTA kernel with the fused epilogue
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    env = dict(os.environ, NVQ_GEMM_PAIRS="0")
+    script = SINGLE_CTA_FUSED_SCRIPT.replace("ROOT_DIR", repr(root)).replace("TEST_DIR", repr(here))
+    out = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True, timeout=900)
+    assert out.returncode == 0 and out.stdout.strip().endswith("OK"), out.stdout + out.stderr
