@@ -554,15 +554,17 @@ def run_ff_block_component(nvq, device, stream, peaks, iters=100):
     return res
 
 
-def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200):
+def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200, graph_steps=20):
     """Short batches of the FF-up linear (N 12288, K 3072, NVFP4): latency of
-    one quantize + GEMM step issued eagerly and replayed from a CUDA graph,
-    and the GEMM's weight stream (the bytes a short M cannot avoid)."""
+    one quantize + GEMM step issued eagerly (back to back, GPU held behind the
+    host) and replayed from a CUDA graph holding `graph_steps` steps, and the
+    GEMM's weight stream (the bytes a short M cannot avoid)."""
     w = workloads.WORKLOADS["ffup"]
     N, K = w.N, w.K
     wc, wsf, wg = nvq.quantize_weight("nvfp4", workloads.weight("ffup").to(device))
     wbytes = N * K * 0.5625
-    res = {"workload": "NVFP4 FF-up N 12288 K 3072 at short M", "weight_bytes": int(wbytes)}
+    res = {"workload": "NVFP4 FF-up N 12288 K 3072 at short M", "weight_bytes": int(wbytes),
+           "graph": "%d steps per captured graph, replays back to back" % graph_steps}
     for M in Ms:
         x = workloads.normal(M, K, seed=5).to(device)
         codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
@@ -575,16 +577,7 @@ def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200
             nvq.nvfp4_quantize(x, codes, sf, g, workspace=ws, stream=s)
             nvq.block_scaled_linear("nvfp4", codes, sf, g, wc, wsf, wg, M, N, K, out=out, stream=s)
 
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        for _ in range(10):
-            step(stream)
-        torch.cuda.synchronize(device)
-        a.record(stream)
-        for _ in range(iters):
-            step(stream)
-        b.record(stream)
-        torch.cuda.synchronize(device)
-        eager = a.elapsed_time(b) / iters * 1e3
+        eager = _back_to_back_us(lambda i: step(stream), iters, device, stream)
         gemm = _back_to_back_us(lambda i: nvq.block_scaled_linear("nvfp4", codes, sf, g, wc, wsf, wg, M, N, K,
                                                                   out=out, stream=stream), iters, device, stream)
         cs = torch.cuda.Stream(device)
@@ -594,17 +587,12 @@ def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200
             step(cs)
             torch.cuda.synchronize(device)
             with torch.cuda.graph(graph, stream=cs):
-                step(cs)
+                for _ in range(graph_steps):
+                    step(cs)
         torch.cuda.synchronize(device)
-        for _ in range(10):
-            graph.replay()
-        torch.cuda.synchronize(device)
-        a.record()
-        for _ in range(iters):
-            graph.replay()
-        b.record()
-        torch.cuda.synchronize(device)
-        graphed = a.elapsed_time(b) / iters * 1e3
+        replays = max(1, iters // graph_steps)
+        graphed = _back_to_back_us(lambda i: graph.replay(), replays, device, torch.cuda.current_stream(device))
+        graphed /= graph_steps
         del graph
         res["M%d" % M] = {"step_us_eager": round(eager, 2), "step_us_graph": round(graphed, 2),
                           "gemm_us": round(gemm, 2),
