@@ -171,12 +171,13 @@ uint32_t next_epoch() {
 
 constexpr size_t kFusedSmemMax = 220 * 1024;
 
-// Dynamic NVFP4 quantization: two passes (amax, then quantize with
-// programmatic dependent launch) unless NVQ_QUANT_ONE_PASS=1 selects the
-// cooperative one-pass kernel for tensors that fit on chip.
+// Dynamic NVFP4 quantization: one pass (every CTA's rows held in shared
+// memory, one read of x) for tensors that fit on chip, else two passes
+// (amax, then quantize with programmatic dependent launch).
+// NVQ_QUANT_ONE_PASS=0 selects the two passes for every tensor.
 const bool g_quant_one_pass = [] {
     const char* e = getenv("NVQ_QUANT_ONE_PASS");
-    return e && e[0] == '1';
+    return !(e && e[0] == '0');
 }();
 
 // NVQ_GEMM_PAIRS=0 in the environment selects the one-CTA GEMM for every
@@ -219,7 +220,8 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
         return NVQ_OK;
     }
     if (!calib_amax && g_quant_one_pass) {
-        // One pass when every CTA's rows fit in shared memory (one CTA per SM).
+        // One pass when every CTA's rows fit in shared memory (one CTA per SM,
+        // at most as many CTAs as SMs).
         const int64_t rows_per_cta = (M + d->num_sms - 1) / d->num_sms;
         const size_t smem = fused_smem_bytes((size_t)rows_per_cta, (size_t)K);
         if (smem <= kFusedSmemMax && (M + rows_per_cta - 1) / rows_per_cta <= kMaxFusedCtas &&
@@ -241,28 +243,27 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
             uint32_t epoch = next_epoch();
             unsigned int* status = d->status;
             void* args[] = {&xp, &rows32, &k32, &ld32, &rpc, &codes, &scales, &global_scale, &slots, &epoch, &status};
-            // co-resident CTAs (the kernel waits on every CTA's maximum),
-            // launched with programmatic stream serialization; a runtime that
-            // refuses the two together gets a plain cooperative launch
+            // The kernel waits on every CTA's maximum, so every CTA must be
+            // resident at once: the grid is at most one CTA per SM (the
+            // registers of 1024 threads leave room for one), so all of them
+            // are resident once the previous grid in the stream has left the
+            // SMs.  A cooperative launch would guarantee it too but costs
+            // about 2.6 us more per call on B200; work on other streams that
+            // held SMs for seconds would end in NVQ_STATUS_TIMEOUT (bounded
+            // wait), not in a hang.
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(grid);
             cfg.blockDim = dim3(kFusedThreads);
             cfg.dynamicSmemBytes = smem;
             cfg.stream = stream;
-            cudaLaunchAttribute attr[2];
-            attr[0].id = cudaLaunchAttributeCooperative;
-            attr[0].val.cooperative = 1;
-            attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr[1].val.programmaticStreamSerializationAllowed = 1;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
             cfg.attrs = attr;
-            cfg.numAttrs = 2;
+            cfg.numAttrs = 1;
             if (cudaLaunchKernelExC(&cfg, (const void*)nvfp4_quantize_fused_kernel, args) != cudaSuccess) {
                 cudaGetLastError();
-                if (cudaLaunchCooperativeKernel((const void*)nvfp4_quantize_fused_kernel, dim3(grid),
-                                                dim3(kFusedThreads), args, smem, stream) != cudaSuccess) {
-                    cudaGetLastError();
-                    return NVQ_ERR_CUDA;
-                }
+                return NVQ_ERR_CUDA;
             }
             return NVQ_OK;
         }

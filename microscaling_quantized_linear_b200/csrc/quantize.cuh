@@ -5,7 +5,7 @@
 // 16-element block along K, in FP32 round-to-nearest-even:
 //   s = (b / 6) * g_enc, sc = E4M3(s), r = g_enc / E4M3(sc), q_i = E2M1(x_i * r)
 // with b the block's max |x| and g_enc = 2688 / amax of the tensor.
-//   one pass   nvfp4_quantize_fused_kernel (cooperative; rows fit on chip)
+//   one pass   nvfp4_quantize_fused_kernel (rows fit on chip; the default there)
 //   two pass   amax_partials_kernel, then nvfp4_quantize_kernel
 //   calibrated nvfp4_quantize_kernel alone, amax given by the caller
 // MXFP8 (page "NVIDIA量化推理：5步极速优化显存+成功率翻倍", section MXFP8量化格式):
@@ -375,7 +375,7 @@ nvfp4_quantize_cluster_kernel(const uint16_t* __restrict__ x, uint32_t rows, uin
 // lands), publishes its partial amax in an epoch-tagged 64-bit slot of the
 // workspace, waits (bounded) until every CTA's slot carries this call's
 // epoch, and quantizes from shared memory.  HBM sees exactly one read of the
-// activation.  Must be launched cooperatively (all CTAs co-resident).
+// activation.  Every CTA must be resident at once: at most one CTA per SM.
 constexpr int kFusedThreads = 1024;
 constexpr int kFusedMaxBlocks = 8;                 // 16-blocks per thread: rows_per_cta * K / 16 <= 8192
 constexpr uint64_t kFusedWaitNs = 2000000000ull;   // 2 s

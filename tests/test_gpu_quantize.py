@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import workloads
-from gpu_common import act, bits, sf_matrix, wgt
+from gpu_common import act, bits, oracle_nvfp4, sf_matrix, wgt
 
 pytestmark = pytest.mark.gpu
 
@@ -213,20 +213,35 @@ print("OK")
 """
 
 
-def test_nvfp4_one_pass_path():
-    # NVQ_QUANT_ONE_PASS=1 (read when the library loads, hence a fresh
-    # process) routes the dynamic NVFP4 quantizer through the cooperative
-    # one-pass kernel wherever the rows fit in shared memory; its results must
-    # be the oracle's, call after call on one workspace.
+def test_nvfp4_two_pass_path():
+    # The default dynamic NVFP4 quantizer takes one pass (rows held in shared
+    # memory) wherever the tensor fits on chip; NVQ_QUANT_ONE_PASS=0 (read
+    # when the library loads, hence a fresh process) sends every tensor
+    # through the two-pass kernels instead.  Both must give the oracle's
+    # results, call after call on one workspace.
     import os
     import subprocess
     import sys
     here = os.path.dirname(os.path.abspath(__file__))
     root = os.path.dirname(here)
-    env = dict(os.environ, NVQ_QUANT_ONE_PASS="1")
+    env = dict(os.environ, NVQ_QUANT_ONE_PASS="0")
     script = ONE_PASS_SCRIPT.replace("ROOT_DIR", repr(root)).replace("TEST_DIR", repr(here))
     out = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True, timeout=600)
     assert out.returncode == 0 and out.stdout.strip().endswith("OK"), out.stdout + out.stderr
+
+
+def test_nvfp4_one_pass_repeated_calls_and_epochs():
+    # the default (one-pass) path, many calls in a row on one workspace:
+    # every call's barrier must match only its own epoch
+    x = act("ffup")
+    ws = nvq.new_workspace()
+    want = oracle_nvfp4("ffup", lambda: act("ffup"))
+    xd = x.cuda()
+    for _ in range(20):
+        codes, sf, g = nvq.nvfp4_quantize(xd, workspace=ws)
+    torch.cuda.synchronize()
+    assert_nvfp4_equal((codes.cpu().numpy(), sf.cpu().numpy(), np.float32(g.item())), want, *x.shape)
+    assert nvq.device_status() == 0
 
 
 # ------------------------------------------------------------------ ragged rows
