@@ -45,8 +45,8 @@ ACT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # BF16 read, E2M1 codes + E4M3 scale
 # Taken on the FF-up workload; the summary is in
 # profiles/bsgemm_pair_kernel_nvfp4_ffup.md.
 GEMM_TRAFFIC = {"kernel": "bsgemm_pair_kernel<0, 256>",
-                "bytes_per_launch": 29267456 + 62559488,
-                "sources_sha256": "2e8387cfad5a9773ef4664cfe56fbd5b842c1d3ee18a34de1ea2a357b0bff2de"}
+                "bytes_per_launch": 29256192 + 63661056,
+                "sources_sha256": "a03d9422fc2055db74c9ba121cd85bb4039101306b07bbf6f651a34b3a33462b"}
 KERNEL_SOURCES = ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh")
 
 
@@ -573,17 +573,23 @@ def run_ff_block_component(nvq, device, stream, peaks, iters=100):
     return res
 
 
-def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200, graph_steps=20):
+def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200, graph_steps=20, rotate=10):
     """Short batches of the FF-up linear (N 12288, K 3072, NVFP4): latency of
     one quantize + GEMM step issued eagerly (back to back, GPU held behind the
     host) and replayed from a CUDA graph holding `graph_steps` steps, and the
-    GEMM's weight stream (the bytes a short M cannot avoid)."""
+    GEMM's weight stream (the bytes a short M cannot avoid).  Consecutive
+    calls cycle through `rotate` copies of the quantized weight (212 MB, more
+    than the 126 MB L2), so every call streams its weight from HBM, as the
+    layers of a model would."""
     w = workloads.WORKLOADS["ffup"]
     N, K = w.N, w.K
-    wc, wsf, wg = nvq.quantize_weight("nvfp4", workloads.weight("ffup").to(device))
+    wc0, wsf0, wg0 = nvq.quantize_weight("nvfp4", workloads.weight("ffup").to(device))
+    wsets = [(wc0.clone(), wsf0.clone(), wg0.clone()) for _ in range(rotate)]
+    del wc0, wsf0, wg0
     wbytes = N * K * 0.5625
     res = {"workload": "NVFP4 FF-up N 12288 K 3072 at short M", "weight_bytes": int(wbytes),
-           "graph": "%d steps per captured graph, replays back to back" % graph_steps}
+           "graph": "%d steps per captured graph, replays back to back" % graph_steps,
+           "l2": "%d weight copies (%.0f MB) cycled" % (rotate, rotate * wbytes / 1e6)}
     for M in Ms:
         x = workloads.normal(M, K, seed=5).to(device)
         codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
@@ -592,22 +598,25 @@ def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200
         ws = nvq.new_workspace(device)
         out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
 
-        def step(s):
-            nvq.nvfp4_quantize(x, codes, sf, g, workspace=ws, stream=s)
+        def gemm_call(i, s):
+            wc, wsf, wg = wsets[i % rotate]
             nvq.block_scaled_linear("nvfp4", codes, sf, g, wc, wsf, wg, M, N, K, out=out, stream=s)
 
-        eager = _back_to_back_us(lambda i: step(stream), iters, device, stream)
-        gemm = _back_to_back_us(lambda i: nvq.block_scaled_linear("nvfp4", codes, sf, g, wc, wsf, wg, M, N, K,
-                                                                  out=out, stream=stream), iters, device, stream)
+        def step(i, s):
+            nvq.nvfp4_quantize(x, codes, sf, g, workspace=ws, stream=s)
+            gemm_call(i, s)
+
+        eager = _back_to_back_us(lambda i: step(i, stream), iters, device, stream)
+        gemm = _back_to_back_us(lambda i: gemm_call(i, stream), iters, device, stream)
         cs = torch.cuda.Stream(device)
         cs.wait_stream(stream)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.stream(cs):
-            step(cs)
+            step(0, cs)
             torch.cuda.synchronize(device)
             with torch.cuda.graph(graph, stream=cs):
-                for _ in range(graph_steps):
-                    step(cs)
+                for j in range(graph_steps):
+                    step(j, cs)
         torch.cuda.synchronize(device)
         replays = max(1, iters // graph_steps)
         graphed = _back_to_back_us(lambda i: graph.replay(), replays, device, torch.cuda.current_stream(device))
