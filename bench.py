@@ -59,15 +59,17 @@ def kernel_sources_sha256():
     return h.hexdigest()
 
 
-def gemm_kernel_name(fmt, M, N):
-    """The GEMM kernel block_scaled_linear launches for this shape (the
-    library's tile choice: CTA pairs on 256-row tiles when M allows them)."""
+def gemm_kernel_name(nvq, fmt, M, N, K):
+    """The GEMM kernel block_scaled_linear launches for this shape, as the
+    library reports its choice (CTA pairs on 256-row tiles when M allows
+    them; a cluster splitting K at a short M)."""
     f = 0 if fmt == "nvfp4" else 1
-    pairs = os.environ.get("NVQ_GEMM_PAIRS", "1") != "0"
-    if pairs and M % 256 == 0 and (N % 256 == 0 or N % 384 == 0):
-        return "bsgemm_pair_kernel<%d, %d>" % (f, 256 if N % 256 == 0 else 192)
-    bn = 256 if N % 256 == 0 else 192 if N % 384 == 0 else 128
-    return "bsgemm_kernel<%d, %d>" % (f, bn)
+    tm, tn, ks = nvq.gemm_plan(fmt, M, N, K)
+    if tm == 256:
+        return "bsgemm_pair_kernel<%d, %d>" % (f, tn)
+    if ks > 1:
+        return "bsgemm_kernel<%d, %d, split-K %d>" % (f, tn, ks)
+    return "bsgemm_kernel<%d, %d>" % (f, tn)
 
 
 def gemm_traffic(kernel):
@@ -281,7 +283,7 @@ def run_ours(args, rank, world, device):
     act_gbs = act_bytes / (quant_mean * 1e-6) / 1e9
 
     e2e = run_e2e(nvq, args, device, stream, xs[0].cpu(), wq[0], M, N, K, flops, world)
-    kernel = gemm_kernel_name("nvfp4", M, N)
+    kernel = gemm_kernel_name(nvq, "nvfp4", M, N, K)
 
     res = {
         "metric": METRIC,
@@ -623,7 +625,7 @@ def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200
         graphed /= graph_steps
         del graph
         res["M%d" % M] = {"step_us_eager": round(eager, 2), "step_us_graph": round(graphed, 2),
-                          "gemm_us": round(gemm, 2),
+                          "gemm_us": round(gemm, 2), "gemm_kernel": gemm_kernel_name(nvq, "nvfp4", M, N, K),
                           "gemm_weight_gbs": round(wbytes / (gemm * 1e-6) / 1e9, 1),
                           "gemm_weight_frac_hbm": round(wbytes / (gemm * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
     return res

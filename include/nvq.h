@@ -202,8 +202,11 @@ NVQ_API int quantize_weight(int format, const void* w, int64_t N, int64_t K, int
  *                       K a multiple of 256 (NVFP4) or 128 (MXFP8)
  *
  * Accumulation is FP32 in tensor memory; the order of the K sum is the
- * hardware's.  Results match the FP64 sum over the dequantized operands to
- * a relative error (normalised by the output row's L2 norm) of 2e-3.
+ * hardware's.  At a short M (at most 128 rows) the K range may be split over
+ * a cluster of CTAs whose FP32 partial sums are then added in a fixed order
+ * (nvq_gemm_plan reports the choice).  Results match the FP64 sum over the
+ * dequantized operands to a relative error (normalised by the output row's
+ * L2 norm) of 2e-3.
  * Pipeline waits inside the kernel are bounded; if one gives up, the kernel
  * sets NVQ_STATUS_TIMEOUT, writes nothing further and exits.
  */
@@ -212,6 +215,22 @@ NVQ_API int block_scaled_linear(int format,
                         const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global,
                         const void* bias, void* out, int64_t ldo,
                         int64_t M, int64_t N, int64_t K, nvq_stream_t stream);
+
+/*
+ * nvq_gemm_plan -- the kernel block_scaled_linear launches for a shape on
+ * the current device: output tile tile_m x tile_n (tile_m 256 = CTA pairs,
+ * 128 = one CTA per tile) and k_split CTAs per tile summing disjoint K
+ * ranges (1 = no split).  Host-only: launches nothing, allocates nothing.
+ *
+ *   format               as block_scaled_linear
+ *   M, N, K              as block_scaled_linear (M >= 1)
+ *   tile_m, tile_n, k_split  out, host pointers
+ *
+ * Returns NVQ_OK, NVQ_ERR_FORMAT, NVQ_ERR_NULL, NVQ_ERR_SHAPE (the shape
+ * block_scaled_linear would reject), NVQ_ERR_ARCH or NVQ_ERR_CUDA (no
+ * device); outputs are written only on NVQ_OK.
+ */
+NVQ_API int nvq_gemm_plan(int format, int64_t M, int64_t N, int64_t K, int* tile_m, int* tile_n, int* k_split);
 
 /*
  * block_scaled_linear_gelu_mxfp8 -- the first linear of a feed-forward block

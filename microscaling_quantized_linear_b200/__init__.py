@@ -74,11 +74,13 @@ _lib.nvq_probe_gelu.restype = ctypes.c_int
 _lib.nvq_probe_gelu.argtypes = [_vp, _i64, _vp, _vp]
 _lib.nvq_probe_wait.restype = ctypes.c_int
 _lib.nvq_probe_wait.argtypes = [ctypes.c_uint64, _vp, _vp]
+_lib.nvq_gemm_plan.restype = ctypes.c_int
+_lib.nvq_gemm_plan.argtypes = [ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp]
 
 EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_quantize",
             "mxfp8_quantize", "mxfp8_quantize_ex", "quantize_weight", "block_scaled_linear",
             "nvq_device_status", "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc",
-            "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu", "nvq_probe_wait")
+            "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu", "nvq_probe_wait", "nvq_gemm_plan")
 
 NOALLOC_MAX_PARTIALS = 1024
 
@@ -211,6 +213,16 @@ def block_scaled_linear(fmt, a_codes, a_scales, a_global, b_codes, b_scales, b_g
                                     _ptr(b_scales), _ptr(b_global), _ptr(bias), _ptr(out), _pitch(out),
                                     M, N, K, _stream(stream, dev)), "block_scaled_linear")
     return out
+
+
+def gemm_plan(fmt, M, N, K):
+    """The kernel block_scaled_linear launches for this shape on the current
+    device: (tile_m, tile_n, k_split); tile_m 256 is a CTA pair, k_split > 1
+    a cluster of CTAs splitting K.  Host-only."""
+    tm, tn, ks = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(_lib.nvq_gemm_plan(_fmt(fmt), M, N, K, ctypes.byref(tm), ctypes.byref(tn), ctypes.byref(ks)),
+           "nvq_gemm_plan")
+    return tm.value, tn.value, ks.value
 
 
 def block_scaled_linear_gelu_mxfp8(fmt, a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K,

@@ -251,7 +251,80 @@ struct GemmParams {
     uint8_t* q_codes;
     uint8_t* q_sf;
     uint32_t m_total, m_pad;
+    // split-K kernels only: CTAs per cluster, each summing one contiguous
+    // share of the K tiles of the cluster's output tile; D is stored with
+    // plain stores (out, ldo elements per row)
+    uint32_t k_split = 1;
+    __nv_bfloat16* out = nullptr;
+    uint32_t ldo = 0;
 };
+
+// Split-K reduction for one output tile of at most 128 rows: every CTA of
+// the cluster holds its FP32 partial tile in its own shared memory, rows of
+// BN floats with the 16-byte groups of each 128-byte segment rotated by the
+// row (group f of row r at (f & ~7) | ((f ^ r) & 7)), so that the writes from
+// tensor memory (one row per thread) spread over all banks.  CTA `rank`
+// finishes the rank-th share of the tile's row-major 4-column groups: the
+// partials summed in rank order, times alpha, plus bias, rounded to BF16 and
+// stored.  Groups at columns >= n_total are not stored.  A thread takes
+// kReduceBatch groups at a time and reads them from one CTA after another,
+// so that many distributed-shared-memory loads are in flight at once.
+constexpr uint32_t kReduceBatch = 8;
+
+template <int BN>
+__device__ __forceinline__ void splitk_reduce(uint32_t part, uint32_t rank, uint32_t split, uint32_t rows,
+                                              uint32_t n0, uint32_t n_total, float alpha,
+                                              const __nv_bfloat16* bias, __nv_bfloat16* out, uint32_t ldo,
+                                              uint32_t tid, uint32_t nthreads) {
+    constexpr uint32_t F = BN / 4;
+    const uint32_t total = rows * F;
+    const uint32_t per = (total + split - 1) / split;
+    const uint32_t begin = rank * per;
+    const uint32_t end = min(total, begin + per);
+    for (uint32_t base = begin + tid; base < end; base += kReduceBatch * nthreads) {
+        uint32_t off[kReduceBatch];
+        float4 acc[kReduceBatch];
+#pragma unroll
+        for (uint32_t u = 0; u < kReduceBatch; ++u) {
+            const uint32_t idx = min(base + u * nthreads, end - 1);   // past the end: a repeat, not stored
+            const uint32_t row = idx / F, f = idx % F;
+            off[u] = part + (row * F + ((f & ~7u) | ((f ^ row) & 7u))) * 16;
+            acc[u] = ld_shared_cluster_f4(mapa_shared(off[u], 0));
+        }
+        for (uint32_t r = 1; r < split; ++r) {
+            float4 v[kReduceBatch];
+#pragma unroll
+            for (uint32_t u = 0; u < kReduceBatch; ++u) v[u] = ld_shared_cluster_f4(mapa_shared(off[u], r));
+#pragma unroll
+            for (uint32_t u = 0; u < kReduceBatch; ++u) {
+                acc[u].x = __fadd_rn(acc[u].x, v[u].x);
+                acc[u].y = __fadd_rn(acc[u].y, v[u].y);
+                acc[u].z = __fadd_rn(acc[u].z, v[u].z);
+                acc[u].w = __fadd_rn(acc[u].w, v[u].w);
+            }
+        }
+#pragma unroll
+        for (uint32_t u = 0; u < kReduceBatch; ++u) {
+            const uint32_t idx = base + u * nthreads;
+            const uint32_t row = idx / F, n = n0 + 4 * (idx % F);
+            if (idx >= end || n >= n_total) continue;
+            float o[4] = {__fmul_rn(acc[u].x, alpha), __fmul_rn(acc[u].y, alpha), __fmul_rn(acc[u].z, alpha),
+                          __fmul_rn(acc[u].w, alpha)};
+            if (bias) {
+                const __nv_bfloat162 b01 = *reinterpret_cast<const __nv_bfloat162*>(bias + n);
+                const __nv_bfloat162 b23 = *reinterpret_cast<const __nv_bfloat162*>(bias + n + 2);
+                o[0] = __fadd_rn(o[0], __bfloat162float(b01.x));
+                o[1] = __fadd_rn(o[1], __bfloat162float(b01.y));
+                o[2] = __fadd_rn(o[2], __bfloat162float(b23.x));
+                o[3] = __fadd_rn(o[3], __bfloat162float(b23.y));
+            }
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
+            *reinterpret_cast<uint2*>(out + (size_t)row * ldo + n) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+        }
+    }
+}
 
 // Scale-factor copy warp `job` (0: A scales, 1..SFB_H: B scale row block
 // job-1) for one pipeline stage: shared memory -> tensor-memory slot.
@@ -279,12 +352,21 @@ __device__ __forceinline__ void sf_copy_job(int job, uint32_t st, uint32_t sf_sl
 // EPI 0: D = bf16(alpha A.B^T + bias) through tmap_d.  EPI 1: D is not
 // written; GELU(D) leaves as MXFP8 codes and scales (EpiQuant), and the
 // epilogue warps' staging area holds the GELU table instead.
-template <int FMT, int BN, int EPI>
+// SPLITK (EPI 0, M <= 128): the grid is one cluster of p.k_split CTAs per
+// output tile.  CTA rank r of a cluster runs the mainloop over the r-th
+// contiguous share of the K tiles into its own accumulator, which the
+// epilogue warps copy to shared memory (the pipeline stages are idle by
+// then); splitk_reduce then sums the partials across the cluster.  Before it
+// waits for the previous grid, the producer asks L2 for the CTA's whole B
+// share, so at a short M the weight stream overlaps the producer of A.
+template <int FMT, int BN, int EPI, bool SPLITK = false>
 __global__ void __launch_bounds__(GemmCfg<FMT, BN>::THREADS, 1)
 bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
               const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
     using C = GemmCfg<FMT, BN>;
     static_assert(EPI == 0 || kGeluTabBytes <= C::EPI_BYTES, "GELU table must fit the staging area");
+    static_assert(!SPLITK || (EPI == 0 && 128 * BN * 4 <= C::STAGES * C::STAGE_BYTES),
+                  "split-K: plain epilogue, and the partial tile must fit the pipeline stages");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
@@ -323,10 +405,32 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         *never = 0;
         fence_mbarrier_init();
     }
+    // Tiles and K tiles of this CTA: persistent CTAs stride over the tiles
+    // with all K tiles each; a split-K cluster owns one tile and CTA rank
+    // ks of it the K tiles [kt_begin, kt_end).
+    const uint32_t num_tiles = p.num_m_blocks * p.num_n_blocks;
+    const uint32_t ks = SPLITK ? cluster_ctarank() : 0;
+    const uint32_t tile_first = SPLITK ? blockIdx.x / p.k_split : blockIdx.x;
+    const uint32_t tile_step = SPLITK ? num_tiles : gridDim.x;
+    const uint32_t kt_begin = SPLITK ? ks * p.num_k_tiles / p.k_split : 0;
+    const uint32_t kt_end = SPLITK ? (ks + 1) * p.num_k_tiles / p.k_split : p.num_k_tiles;
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmap_a);
         prefetch_tensormap(&tmap_b);
-        if (EPI == 0) prefetch_tensormap(&tmap_d);
+        if (EPI == 0 && !SPLITK) prefetch_tensormap(&tmap_d);
+        if (SPLITK && tile_first < num_tiles) {
+            const uint32_t nb = tile_first / p.num_m_blocks;
+            const uint32_t a0 = (nb * BN) / 128;
+            for (uint32_t kt = kt_begin; kt < kt_end; ++kt) {
+                prefetch_l2_tile_2d(&tmap_b, (int32_t)(kt * C::KBYTES), (int32_t)(nb * BN));
+#pragma unroll
+                for (int h = 0; h < C::SFB_H; ++h) {
+                    const uint32_t bt = min(a0 + h, p.sfb_rtiles - 1);
+                    prefetch_l2_bulk(p.sfb + ((size_t)bt * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
+                                     C::SF_ATOMS * 512);
+                }
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), C::TM_COLS);
@@ -342,19 +446,18 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     // has completed, so only its launch latency overlaps this grid.
     griddep_wait();
     griddep_launch();
-    const uint32_t num_tiles = p.num_m_blocks * p.num_n_blocks;
-    const uint32_t total_iters = ((num_tiles > blockIdx.x) ? (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0)
-                                 * p.num_k_tiles;
+    const uint32_t total_iters =
+        ((num_tiles > tile_first) ? (num_tiles - tile_first + tile_step - 1) / tile_step : 0) * (kt_end - kt_begin);
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (uint32_t tile = tile_first; tile < num_tiles && ok; tile += tile_step) {
                 const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
                 const uint32_t a0 = (nb * BN) / 128;             // first 128-row scale tile of B
-                for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt) {
+                for (uint32_t kt = kt_begin; kt < kt_end; ++kt) {
                     const uint32_t s = it % C::STAGES, use = it / C::STAGES;
                     if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
                         ok = false;
@@ -398,7 +501,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         if (lane == 0) {
             uint32_t it = 0, t_local = 0;
             bool ok = true;
-            for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t_local) {
+            for (uint32_t tile = tile_first; tile < num_tiles && ok; tile += tile_step, ++t_local) {
                 const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
                 const uint32_t use = C::ACC_BUFS == 2 ? (t_local >> 1) : t_local;
                 if (use > 0 && !mbar_wait_bounded(tempty0 + 8 * buf, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
@@ -409,7 +512,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 const uint32_t nb = tile / p.num_m_blocks;
                 const uint32_t sfb_shift = ((nb * BN) % 128) / 32;   // B tile starting mid scale tile (BN = 192)
                 const uint32_t d_tmem = tmem + buf * BN;
-                for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt, ++it) {
+                for (uint32_t kt = kt_begin; kt < kt_end; ++kt, ++it) {
                     const uint32_t s = it % C::STAGES, su = it / C::STAGES;
                     if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
                         ok = false;
@@ -423,7 +526,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     for (int k = 0; k < C::KSTEPS; ++k) {
                         const uint64_t adesc = smem_desc(st + k * C::MMA_K_BYTES, 16, 1024, 2);
                         const uint64_t bdesc = smem_desc(st + C::OFF_B + k * C::MMA_K_BYTES, 16, 1024, 2);
-                        const uint32_t acc = (kt | (uint32_t)k) != 0;
+                        const uint32_t acc = (kt != kt_begin) || k != 0;
                         if (FMT == 0) {
                             tc_mma_nvf4(d_tmem, adesc, bdesc, C::IDESC, sfa_t + 4 * k,
                                         sfb_t + C::SFB_COLS_PER_MMA * k + sfb_shift, acc);
@@ -483,8 +586,36 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             gelu_table_fill(reinterpret_cast<uint16_t*>(smem + C::OFF_EPI), threadIdx.x - 64, 32 * kEpiWarps);
             named_barrier_sync(1, 32 * kEpiWarps);
         }
+        if constexpr (SPLITK) {
+            // this CTA's partial tile -> its shared memory (rows < M only)
+            const uint32_t rows = min(p.m_total, (uint32_t)C::BM);
+            if (tile_first < num_tiles) {
+                if (!mbar_wait_bounded(tfull0, 0, abort_flag, kWaitLimitNs)) {
+                    *abort_flag = 1;
+                    atomicOr(p.status, 1u);
+                } else if ((uint32_t)(32 * q) < rows) {
+                    tc_fence_after();
+                    const uint32_t row = 32 * q + lane;
+                    float4* prow = reinterpret_cast<float4*>(smem) + row * (BN / 4);
+#pragma unroll 1
+                    for (int j = 0; j < BN / 64; ++j) {
+                        const int c = half * (BN / 2) + 32 * j;
+                        uint32_t r[32];
+                        tc_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + c, r);
+                        tc_wait_ld();
+                        if (row < rows) {
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                prow[c / 4 + (v ^ (int)(row & 7))] =
+                                    make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+                        }
+                    }
+                }
+            }
+        }
         uint32_t t_local = 0;
-        for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t_local) {
+        for (uint32_t tile = SPLITK ? num_tiles : tile_first; tile < num_tiles; tile += tile_step, ++t_local) {
             const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
             const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
             const uint32_t use = C::ACC_BUFS == 2 ? (t_local >> 1) : t_local;
@@ -502,6 +633,21 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();
+    }
+
+    if constexpr (SPLITK) {
+        // Every thread of the cluster passes both barriers, whatever its role
+        // did: the waits above are bounded, so none can hold a barrier.
+        __syncwarp();
+        cluster_sync();                       // every partial of the cluster is in shared memory
+        if (warp >= 2 && warp < kFirstSfWarp && tile_first < num_tiles) {
+            const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
+            const uint32_t nb = tile_first / p.num_m_blocks;
+            splitk_reduce<BN>(smem_u32(smem), ks, p.k_split, min(p.m_total, (uint32_t)C::BM), nb * BN, p.n_total,
+                              alpha, p.bias, p.out, p.ldo, threadIdx.x - 64, 32 * kEpiWarps);
+        }
+        __syncwarp();
+        cluster_sync();                       // no CTA leaves while another reads its partial
     }
 
     tc_fence_before();

@@ -45,6 +45,10 @@ struct DeviceInfo {
     unsigned int* status = nullptr;
     bool gemm_attr[3][3][2] = {};    // [format][BN 128/192/256][epilogue]
     bool pair_attr[3][2][2] = {};    // [format][BN 192/256][epilogue]
+    bool splitk_attr[3][3] = {};     // [format][BN 128/192/256]
+    // most clusters of k_split CTAs that fit on the device at once, + 1
+    // (0 = not yet asked): [format][BN 128/192/256][k_split]
+    int splitk_clusters[3][3][9] = {};
     bool fused_attr = false;
 };
 
@@ -184,6 +188,15 @@ const bool g_quant_one_pass = [] {
 // shape (the test suite runs both kernels on the same shapes).
 const bool g_use_pairs = [] {
     const char* e = getenv("NVQ_GEMM_PAIRS");
+    return !(e && e[0] == '0');
+}();
+
+// NVQ_GEMM_SPLITK=0 never splits K across a cluster for short M.  Split-K
+// sums FP32 partials in another order, so results may differ from the
+// unsplit kernel in the last bits (both within the GEMM tolerance; exact
+// sums agree bit for bit).
+const bool g_use_splitk = [] {
+    const char* e = getenv("NVQ_GEMM_SPLITK");
     return !(e && e[0] == '0');
 }();
 
@@ -469,38 +482,174 @@ int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, 
     return NVQ_OK;
 }
 
+// Split-K kernel for M <= 128: opt in to its shared memory, and the number
+// of clusters of `split` CTAs the device holds at once (cached).
+template <int FMT, int BN>
+int splitk_max_clusters(DeviceInfo* d, int split) {
+    using C = GemmCfg<FMT, BN>;
+    auto kern = bsgemm_kernel<FMT, BN, 0, true>;
+    const int wi = BN / 64 - 2;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!d->splitk_attr[FMT][wi]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        d->splitk_attr[FMT][wi] = true;
+    }
+    int& c = d->splitk_clusters[FMT][wi][split];
+    if (c == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(split);
+        cfg.blockDim = dim3(C::THREADS);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = split;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        c = n + 1;
+    }
+    return c - 1;
+}
+
+// One cluster of `split` CTAs per 128 x BN output tile (M <= 128); each CTA
+// sums a contiguous share of the K tiles and the cluster adds the partials.
+template <int FMT, int BN>
+int launch_gemm_splitk(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                       const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
+                       void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, int split, cudaStream_t stream) {
+    using C = GemmCfg<FMT, BN>;
+    const int64_t kbytes = FMT == 0 ? K / 2 : K;
+    if (splitk_max_clusters<FMT, BN>(d, split) <= 0) return NVQ_ERR_CUDA;
+    CUtensorMap ma, mb, md;
+    memset(&md, 0, sizeof(md));
+    int rc;
+    if ((rc = encode_codes_map(&ma, a_codes, M, kbytes, C::BM))) return rc;
+    if ((rc = encode_codes_map(&mb, b_codes, N, kbytes, BN))) return rc;
+    GemmParams p;
+    set_epi_quant(p, nullptr, nullptr, M);
+    p.sfa = a_scales;
+    p.sfb = b_scales;
+    p.a_global = a_global;
+    p.b_global = b_global;
+    p.bias = static_cast<const __nv_bfloat16*>(bias);
+    p.status = d->status;
+    p.num_m_blocks = 1;
+    p.num_n_blocks = (uint32_t)((N + BN - 1) / BN);
+    p.n_total = (uint32_t)N;
+    p.sfa_rtiles = 1;
+    p.sfb_rtiles = (uint32_t)((N + 127) / 128);
+    p.num_k_tiles = (uint32_t)(K / C::BK);
+    p.sf_ctiles = (uint32_t)(K / C::SF_BLOCK / 4);
+    p.k_split = (uint32_t)split;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.ldo = (uint32_t)ldo;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.num_n_blocks * (uint32_t)split);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = split;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, bsgemm_kernel<FMT, BN, 0, true>, ma, mb, md, p) != cudaSuccess) {
+        cudaGetLastError();
+        return NVQ_ERR_CUDA;
+    }
+    return NVQ_OK;
+}
+
+struct GemmPlan {
+    int tile_m, tile_n, k_split;
+};
+
+// The kernel block_scaled_linear runs for a shape.  CTA pairs (256-row
+// tiles) unless M fits one 128-row tile: 256 x 256 tiles, or 256 x 192 (two
+// accumulators for MXFP8) when N is a multiple of 384 but not of 256.
+// Measured on the FF-up shape, 256 x 256 with one accumulator is faster than
+// 256 x 192 with two.  A ragged N takes 256.  One CTA per tile otherwise:
+// width 256 when N allows it (fewest scale-factor copies per MMA), else 192,
+// else 128 (two accumulators); when 256-wide tiles would leave SMs idle (a
+// short M: the weight stream is then the cost), 128-wide tiles spread it over
+// twice as many SMs.  At M <= 128, K is split across a cluster when that
+// streams the weight through at least a quarter more SMs than the best
+// unsplit grid: the tile width (256, 192 or 128) and split that occupy the
+// most SMs in one wave of clusters (at least two K tiles per CTA, at most 8
+// CTAs per cluster, and no more clusters than the device holds at once: on
+// a B200 that is 74 clusters of 2 but only 45 of 3), the wider tile and then
+// the smaller split on a tie.
+template <int FMT>
+GemmPlan plan_gemm(DeviceInfo* d, int64_t M, int64_t N, int64_t K) {
+    if (g_use_pairs && M > 128) return {256, (N % 384 == 0 && N % 256 != 0) ? 192 : 256, 1};
+    int bn = 128;
+    if ((M + 127) / 128 * ((N + 255) / 256) >= d->num_sms) bn = N % 256 == 0 ? 256 : N % 384 == 0 ? 192 : 128;
+    GemmPlan plan = {128, bn, 1};
+    if (!g_use_splitk || M > 128) return plan;
+    const int64_t nkt = K / GemmCfg<FMT, 128>::BK;
+    const int64_t base = (N + bn - 1) / bn;
+    int64_t best = base;
+    GemmPlan split = plan;
+    for (int w : {256, 192, 128}) {
+        const int64_t tiles = (N + w - 1) / w;
+        for (int sp = 2; sp <= 8 && 2 * sp <= nkt && tiles * sp <= d->num_sms; ++sp) {
+            if (tiles * sp <= best) continue;
+            const int fit = w == 256   ? splitk_max_clusters<FMT, 256>(d, sp)
+                            : w == 192 ? splitk_max_clusters<FMT, 192>(d, sp)
+                                       : splitk_max_clusters<FMT, 128>(d, sp);
+            if (tiles > fit) continue;
+            best = tiles * sp;
+            split = {128, w, sp};
+        }
+    }
+    return best * 4 >= base * 5 ? split : plan;
+}
+
 }  // namespace
 // One launch per (format, tile shape); FMT 0 = NVFP4, 1 = MXFP8 (E4M3), 2 = MXFP8 (E5M2).
 template <int FMT>
 int launch_for_format(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                       const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
                       void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, cudaStream_t s) {
-    // CTA pairs (256-row tiles) unless M fits one 128-row tile: 256 x 256
-    // tiles, or 256 x 192 (two accumulators for MXFP8) when N is a multiple of
-    // 384 but not of 256.  Measured on the FF-up shape, 256 x 256 with one
-    // accumulator is faster than 256 x 192 with two.  A ragged N takes 256.
-    if (g_use_pairs && M > 128) {
-        if (N % 384 == 0 && N % 256 != 0)
+    const GemmPlan pl = plan_gemm<FMT>(d, M, N, K);
+    if (pl.tile_m == 256) {
+        if (pl.tile_n == 192)
             return launch_gemm_pair<FMT, 192, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
                                                  out, ldo, nullptr, nullptr, M, N, K, s);
         return launch_gemm_pair<FMT, 256, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
                                              out, ldo, nullptr, nullptr, M, N, K, s);
     }
-    // One CTA per tile: width 256 when N allows it (fewest scale-factor copies
-    // per MMA), else 192, else 128 (two accumulators).  When 256-wide tiles
-    // would leave SMs idle (a short M: the weight stream is then the cost),
-    // 128-wide tiles spread it over twice as many SMs.
-    if ((M + 127) / 128 * ((N + 255) / 256) < d->num_sms)
-        return launch_gemm<FMT, 128, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
-                                        nullptr, nullptr, M, N, K, s);
-    if (N % 256 == 0)
+    if (pl.k_split > 1) {
+        if (pl.tile_n == 256)
+            return launch_gemm_splitk<FMT, 256>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
+                                                out, ldo, M, N, K, pl.k_split, s);
+        if (pl.tile_n == 192)
+            return launch_gemm_splitk<FMT, 192>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
+                                                out, ldo, M, N, K, pl.k_split, s);
+        return launch_gemm_splitk<FMT, 128>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out,
+                                            ldo, M, N, K, pl.k_split, s);
+    }
+    if (pl.tile_n == 256)
         return launch_gemm<FMT, 256, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
                                         nullptr, nullptr, M, N, K, s);
-    if (N % 384 == 0)
+    if (pl.tile_n == 192)
         return launch_gemm<FMT, 192, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
                                         nullptr, nullptr, M, N, K, s);
     return launch_gemm<FMT, 128, 0>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out, ldo,
-                                        nullptr, nullptr, M, N, K, s);
+                                    nullptr, nullptr, M, N, K, s);
 }
 
 // The quantizing epilogue (GELU, then MXFP8 codes and scales) on 256-wide
@@ -600,6 +749,24 @@ int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_sca
                                     K, s);
     return launch_for_format<2>(d, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, bias, out, ldo, M, N, K,
                                 s);
+}
+
+int nvq_gemm_plan(int format, int64_t M, int64_t N, int64_t K, int* tile_m, int* tile_n, int* k_split) {
+    if (format != NVQ_NVFP4 && !is_mxfp8(format)) return NVQ_ERR_FORMAT;
+    if (!tile_m || !tile_n || !k_split) return NVQ_ERR_NULL;
+    const int64_t k_stage = format == NVQ_NVFP4 ? 256 : 128;
+    if (M <= 0 || N <= 0 || N % 8 || K <= 0 || K % k_stage) return NVQ_ERR_SHAPE;
+    if (K >= (int64_t(1) << 24) || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVQ_ERR_SHAPE;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc) return rc;
+    const GemmPlan pl = format == NVQ_NVFP4 ? plan_gemm<0>(d, M, N, K)
+                        : format == NVQ_MXFP8 ? plan_gemm<1>(d, M, N, K)
+                                              : plan_gemm<2>(d, M, N, K);
+    *tile_m = pl.tile_m;
+    *tile_n = pl.tile_n;
+    *k_split = pl.k_split;
+    return NVQ_OK;
 }
 
 int block_scaled_linear_gelu_mxfp8(int format, const uint8_t* a_codes, const uint8_t* a_scales,

@@ -145,6 +145,18 @@ def test_block_scaled_linear_gelu_mxfp8_rejects_bad_arguments():
     assert L.nvq_probe_gelu(P16, -1, P16, NULL) == -2
 
 
+def test_gemm_plan_rejects_bad_arguments():
+    def plan(fmt=0, M=1, N=12288, K=3072, tm=P16, tn=P16, ks=P16):
+        return L.nvq_gemm_plan(fmt, M, N, K, tm, tn, ks)
+    assert plan(fmt=3) == -7
+    assert plan(tm=NULL) == -1
+    assert plan(ks=NULL) == -1
+    assert plan(M=0) == -2                     # a plan needs at least one row
+    assert plan(N=12) == -2
+    assert plan(K=128) == -2                   # NVFP4 K must be a multiple of 256
+    assert plan(fmt=1, K=64) == -2
+
+
 def test_valid_arguments_without_gpu_report_cuda_error():
     # Arguments pass the host checks; with no device the library reports a
     # CUDA error instead of launching.
@@ -162,3 +174,6 @@ def test_valid_arguments_without_gpu_report_cuda_error():
     assert gemm_gelu(fmt=1, ga=NULL, gb=NULL, M=100, N=384, K=128) == -5
     assert L.nvq_probe_gelu(P16, 16, P16, NULL) == -5
     assert L.nvq_probe_wait(1000, P16, NULL) == -5
+    out = (ctypes.c_int * 3)()
+    assert L.nvq_gemm_plan(0, 1, 12288, 3072, ctypes.byref(out, 0), ctypes.byref(out, 4),
+                           ctypes.byref(out, 8)) == -5
