@@ -45,8 +45,8 @@ ACT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # BF16 read, E2M1 codes + E4M3 scale
 # Taken on the FF-up workload; the summary is in
 # profiles/bsgemm_pair_kernel_nvfp4_ffup.md.
 GEMM_TRAFFIC = {"kernel": "bsgemm_pair_kernel<0, 256>",
-                "bytes_per_launch": 29256192 + 63661056,
-                "sources_sha256": "a03d9422fc2055db74c9ba121cd85bb4039101306b07bbf6f651a34b3a33462b"}
+                "bytes_per_launch": 29286912 + 62546688,
+                "sources_sha256": "0bed530746fb5b5719a5339e133ac2aa066ef8dc7a55bc2dd4f58a0988a1aceb"}
 KERNEL_SOURCES = ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh")
 
 

@@ -202,7 +202,7 @@ NVQ_API int quantize_weight(int format, const void* w, int64_t N, int64_t K, int
  *                       K a multiple of 256 (NVFP4) or 128 (MXFP8)
  *
  * Accumulation is FP32 in tensor memory; the order of the K sum is the
- * hardware's.  At a short M (at most 128 rows) the K range may be split over
+ * hardware's.  At a short M (at most 32 rows) the K range may be split over
  * a cluster of CTAs whose FP32 partial sums are then added in a fixed order
  * (nvq_gemm_plan reports the choice).  Results match the FP64 sum over the
  * dequantized operands to a relative error (normalised by the output row's

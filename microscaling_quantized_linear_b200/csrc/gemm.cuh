@@ -267,8 +267,9 @@ struct GemmParams {
 // finishes the rank-th share of the tile's row-major 4-column groups: the
 // partials summed in rank order, times alpha, plus bias, rounded to BF16 and
 // stored.  Groups at columns >= n_total are not stored.  A thread takes
-// kReduceBatch groups at a time and reads them from one CTA after another,
-// so that many distributed-shared-memory loads are in flight at once.
+// kReduceBatch groups at a time and reads them from one CTA after another
+// (its own partial with plain shared-memory loads), so that many
+// distributed-shared-memory loads are in flight at once.
 constexpr uint32_t kReduceBatch = 8;
 
 template <int BN>
@@ -289,12 +290,13 @@ __device__ __forceinline__ void splitk_reduce(uint32_t part, uint32_t rank, uint
             const uint32_t idx = min(base + u * nthreads, end - 1);   // past the end: a repeat, not stored
             const uint32_t row = idx / F, f = idx % F;
             off[u] = part + (row * F + ((f & ~7u) | ((f ^ row) & 7u))) * 16;
-            acc[u] = ld_shared_cluster_f4(mapa_shared(off[u], 0));
+            acc[u] = rank == 0 ? ld_shared_f4(off[u]) : ld_shared_cluster_f4(mapa_shared(off[u], 0));
         }
         for (uint32_t r = 1; r < split; ++r) {
             float4 v[kReduceBatch];
 #pragma unroll
-            for (uint32_t u = 0; u < kReduceBatch; ++u) v[u] = ld_shared_cluster_f4(mapa_shared(off[u], r));
+            for (uint32_t u = 0; u < kReduceBatch; ++u)
+                v[u] = r == rank ? ld_shared_f4(off[u]) : ld_shared_cluster_f4(mapa_shared(off[u], r));
 #pragma unroll
             for (uint32_t u = 0; u < kReduceBatch; ++u) {
                 acc[u].x = __fadd_rn(acc[u].x, v[u].x);
@@ -357,8 +359,8 @@ __device__ __forceinline__ void sf_copy_job(int job, uint32_t st, uint32_t sf_sl
 // contiguous share of the K tiles into its own accumulator, which the
 // epilogue warps copy to shared memory (the pipeline stages are idle by
 // then); splitk_reduce then sums the partials across the cluster.  Before it
-// waits for the previous grid, the producer asks L2 for the CTA's whole B
-// share, so at a short M the weight stream overlaps the producer of A.
+// waits for the previous grid, one epilogue warp asks L2 for the CTA's whole
+// B share, so at a short M the weight stream overlaps the producer of A.
 template <int FMT, int BN, int EPI, bool SPLITK = false>
 __global__ void __launch_bounds__(GemmCfg<FMT, BN>::THREADS, 1)
 bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -418,19 +420,6 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         prefetch_tensormap(&tmap_a);
         prefetch_tensormap(&tmap_b);
         if (EPI == 0 && !SPLITK) prefetch_tensormap(&tmap_d);
-        if (SPLITK && tile_first < num_tiles) {
-            const uint32_t nb = tile_first / p.num_m_blocks;
-            const uint32_t a0 = (nb * BN) / 128;
-            for (uint32_t kt = kt_begin; kt < kt_end; ++kt) {
-                prefetch_l2_tile_2d(&tmap_b, (int32_t)(kt * C::KBYTES), (int32_t)(nb * BN));
-#pragma unroll
-                for (int h = 0; h < C::SFB_H; ++h) {
-                    const uint32_t bt = min(a0 + h, p.sfb_rtiles - 1);
-                    prefetch_l2_bulk(p.sfb + ((size_t)bt * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
-                                     C::SF_ATOMS * 512);
-                }
-            }
-        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), C::TM_COLS);
@@ -440,6 +429,22 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    if (SPLITK && warp == kFirstSfWarp - 1 && lane == 0 && tile_first < num_tiles) {
+        // the weight share into L2, from an epilogue warp (idle until the
+        // accumulator is ready), so the prologue of the other roles does not
+        // wait for the prefetch instructions to issue
+        const uint32_t nb = tile_first / p.num_m_blocks;
+        const uint32_t a0 = (nb * BN) / 128;
+        for (uint32_t kt = kt_begin; kt < kt_end; ++kt) {
+            prefetch_l2_tile_2d(&tmap_b, (int32_t)(kt * C::KBYTES), (int32_t)(nb * BN));
+#pragma unroll
+            for (int h = 0; h < C::SFB_H; ++h) {
+                const uint32_t bt = min(a0 + h, p.sfb_rtiles - 1);
+                prefetch_l2_bulk(p.sfb + ((size_t)bt * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
+                                 C::SF_ATOMS * 512);
+            }
+        }
+    }
     // everything above overlaps the previous grid; no global data is
     // touched before it has completed.  The next grid in the stream may then
     // launch: its CTAs wait at their own griddepcontrol.wait until this grid

@@ -585,20 +585,27 @@ struct GemmPlan {
 // width 256 when N allows it (fewest scale-factor copies per MMA), else 192,
 // else 128 (two accumulators); when 256-wide tiles would leave SMs idle (a
 // short M: the weight stream is then the cost), 128-wide tiles spread it over
-// twice as many SMs.  At M <= 128, K is split across a cluster when that
+// twice as many SMs.  At M <= kSplitKMaxRows, K is split across a cluster when that
 // streams the weight through at least a quarter more SMs than the best
 // unsplit grid: the tile width (256, 192 or 128) and split that occupy the
 // most SMs in one wave of clusters (at least two K tiles per CTA, at most 8
 // CTAs per cluster, and no more clusters than the device holds at once: on
 // a B200 that is 74 clusters of 2 but only 45 of 3), the wider tile and then
 // the smaller split on a tie.
+// Rows up to which a K split pays.  Each CTA's partial grows with M, and the
+// reduction (partials to shared memory, two cluster barriers, the exchange
+// through distributed shared memory) with it: on the FF-up weight the split
+// kernel measured 9.2 / 10.1 / 10.1 / 10.3 / 11.6 us at M = 1 / 16 / 32 / 64
+// / 128 against 10.8 / 10.9 / 10.7 / 9.8 / 9.4 us unsplit.
+constexpr int64_t kSplitKMaxRows = 32;
+
 template <int FMT>
 GemmPlan plan_gemm(DeviceInfo* d, int64_t M, int64_t N, int64_t K) {
     if (g_use_pairs && M > 128) return {256, (N % 384 == 0 && N % 256 != 0) ? 192 : 256, 1};
     int bn = 128;
     if ((M + 127) / 128 * ((N + 255) / 256) >= d->num_sms) bn = N % 256 == 0 ? 256 : N % 384 == 0 ? 192 : 128;
     GemmPlan plan = {128, bn, 1};
-    if (!g_use_splitk || M > 128) return plan;
+    if (!g_use_splitk || M > kSplitKMaxRows) return plan;
     const int64_t nkt = K / GemmCfg<FMT, 128>::BK;
     const int64_t base = (N + bn - 1) / bn;
     int64_t best = base;

@@ -1,4 +1,4 @@
-"""GPU parity of the short-M GEMM path: at M <= 128 block_scaled_linear may
+"""GPU parity of the short-M GEMM path: at M <= 32 block_scaled_linear may
 split the K range of each output tile over a cluster of CTAs, each summing
 its share into its own FP32 accumulator, the cluster then adding the partials
 in rank order through distributed shared memory.
@@ -32,13 +32,13 @@ nvq = pytest.importorskip("microscaling_quantized_linear_b200")
 
 
 SPLIT = [
-    # fmt, M, N, K, bias
+    # fmt, M, N, K, bias (the library splits K for M <= 32)
     ("nvfp4", 1, 12288, 3072, False),        # FF-up weight at batch 1
     ("nvfp4", 16, 12288, 3072, True),
-    ("nvfp4", 128, 9216, 3072, False),       # QKV width
-    ("nvfp4", 37, 1000, 2048, True),         # ragged N: the last tile mostly past N
-    ("mxfp8", 100, 3072, 12288, True),       # FF-down weight at a short M
-    ("mxfp8_e5m2", 64, 2048, 1024, False),
+    ("nvfp4", 32, 9216, 3072, False),        # QKV width
+    ("nvfp4", 7, 1000, 2048, True),          # ragged N: the last tile mostly past N
+    ("mxfp8", 24, 3072, 12288, True),        # FF-down weight at a short M
+    ("mxfp8_e5m2", 3, 2048, 1024, False),
 ]
 
 
@@ -49,6 +49,8 @@ def test_plan_splits_short_m_only():
         print(fmt, M, N, K, "->", tm, tn, ks)
         assert tm == 128 and 2 <= ks <= 8 and tn in (128, 192, 256)
         assert -(-N // tn) * ks <= sms
+    assert nvq.gemm_plan("nvfp4", 33, 12288, 3072)[2] == 1     # past the rows where a split pays
+    assert nvq.gemm_plan("nvfp4", 128, 12288, 3072) == (128, 128, 1)
     assert nvq.gemm_plan("nvfp4", 129, 12288, 3072) == (256, 256, 1)
     assert nvq.gemm_plan("nvfp4", 4608, 12288, 3072) == (256, 256, 1)
     assert nvq.gemm_plan("nvfp4", 1, 256, 256)[2] == 1        # one K tile: nothing to split
@@ -81,8 +83,8 @@ def test_split_k_flux_like_batch1_and_deterministic():
 EXACT = [
     # fmt, M, N, K, bias
     ("nvfp4", 1, 12288, 3072, True),
-    ("nvfp4", 100, 1000, 2048, False),
-    ("mxfp8", 64, 3072, 3072, True),
+    ("nvfp4", 20, 1000, 2048, False),
+    ("mxfp8", 32, 3072, 3072, True),
 ]
 
 
