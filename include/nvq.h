@@ -233,6 +233,25 @@ NVQ_API int block_scaled_linear(int format,
 NVQ_API int nvq_gemm_plan(int format, int64_t M, int64_t N, int64_t K, int* tile_m, int* tile_n, int* k_split);
 
 /*
+ * nvq_gemm_plan_host -- the same choice for stated device facts instead of
+ * the current device's, so that it can be reasoned about (and tested)
+ * without a GPU.  Host-only.
+ *
+ *   num_sms        SMs of the device (> 0)
+ *   max_clusters   host int[3][9]: [w][s] = the most clusters of s CTAs with
+ *                  w-wide tiles the device holds at once, w = 0 / 1 / 2 for
+ *                  128 / 192 / 256 (cudaOccupancyMaxActiveClusters at one CTA
+ *                  per SM); entries s < 2 are not read
+ *   use_pairs      0 forbids CTA pairs (as NVQ_GEMM_PAIRS=0 does)
+ *   use_splitk     0 forbids the K split (as NVQ_GEMM_SPLITK=0 does)
+ *
+ * Returns as nvq_gemm_plan, without NVQ_ERR_ARCH / NVQ_ERR_CUDA;
+ * NVQ_ERR_SHAPE also for num_sms <= 0.
+ */
+NVQ_API int nvq_gemm_plan_host(int format, int64_t M, int64_t N, int64_t K, int num_sms, const int* max_clusters,
+                               int use_pairs, int use_splitk, int* tile_m, int* tile_n, int* k_split);
+
+/*
  * block_scaled_linear_gelu_mxfp8 -- the first linear of a feed-forward block
  * with the next layer's activation quantization fused into its epilogue:
  *

@@ -76,11 +76,15 @@ _lib.nvq_probe_wait.restype = ctypes.c_int
 _lib.nvq_probe_wait.argtypes = [ctypes.c_uint64, _vp, _vp]
 _lib.nvq_gemm_plan.restype = ctypes.c_int
 _lib.nvq_gemm_plan.argtypes = [ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp]
+_lib.nvq_gemm_plan_host.restype = ctypes.c_int
+_lib.nvq_gemm_plan_host.argtypes = [ctypes.c_int, _i64, _i64, _i64, ctypes.c_int, _vp, ctypes.c_int, ctypes.c_int,
+                                    _vp, _vp, _vp]
 
 EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_quantize",
             "mxfp8_quantize", "mxfp8_quantize_ex", "quantize_weight", "block_scaled_linear",
             "nvq_device_status", "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc",
-            "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu", "nvq_probe_wait", "nvq_gemm_plan")
+            "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu", "nvq_probe_wait", "nvq_gemm_plan",
+            "nvq_gemm_plan_host")
 
 NOALLOC_MAX_PARTIALS = 1024
 
@@ -223,6 +227,20 @@ def gemm_plan(fmt, M, N, K):
     _check(_lib.nvq_gemm_plan(_fmt(fmt), M, N, K, ctypes.byref(tm), ctypes.byref(tn), ctypes.byref(ks)),
            "nvq_gemm_plan")
     return tm.value, tn.value, ks.value
+
+
+def gemm_plan_host(fmt, M, N, K, num_sms, max_clusters, use_pairs=True, use_splitk=True):
+    """gemm_plan for stated device facts: num_sms and max_clusters, a mapping
+    {(tile_n, k_split): clusters the device holds at once} (missing entries
+    count as 0).  Host-only; needs no GPU."""
+    table = (ctypes.c_int * 27)()
+    for (tn, ks), n in max_clusters.items():
+        table[(tn // 64 - 2) * 9 + ks] = int(n)
+    tm, tn_, ks_ = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(_lib.nvq_gemm_plan_host(_fmt(fmt), M, N, K, int(num_sms), table, int(bool(use_pairs)),
+                                   int(bool(use_splitk)), ctypes.byref(tm), ctypes.byref(tn_), ctypes.byref(ks_)),
+           "nvq_gemm_plan_host")
+    return tm.value, tn_.value, ks_.value
 
 
 def block_scaled_linear_gelu_mxfp8(fmt, a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K,

@@ -599,30 +599,41 @@ struct GemmPlan {
 // / 128 against 10.8 / 10.9 / 10.7 / 9.8 / 9.4 us unsplit.
 constexpr int64_t kSplitKMaxRows = 32;
 
-template <int FMT>
-GemmPlan plan_gemm(DeviceInfo* d, int64_t M, int64_t N, int64_t K) {
-    if (g_use_pairs && M > 128) return {256, (N % 384 == 0 && N % 256 != 0) ? 192 : 256, 1};
+// The plan as a function of the shape and of the device's facts: its SM
+// count and fit(w, sp), the most clusters of sp CTAs with w-wide tiles that
+// it holds at once.  bk = K elements per pipeline stage.
+template <typename Fit>
+GemmPlan plan_gemm_core(int64_t bk, int64_t M, int64_t N, int64_t K, int num_sms, bool pairs, bool splitk,
+                        Fit fit) {
+    if (pairs && M > 128) return {256, (N % 384 == 0 && N % 256 != 0) ? 192 : 256, 1};
     int bn = 128;
-    if ((M + 127) / 128 * ((N + 255) / 256) >= d->num_sms) bn = N % 256 == 0 ? 256 : N % 384 == 0 ? 192 : 128;
+    if ((M + 127) / 128 * ((N + 255) / 256) >= num_sms) bn = N % 256 == 0 ? 256 : N % 384 == 0 ? 192 : 128;
     GemmPlan plan = {128, bn, 1};
-    if (!g_use_splitk || M > kSplitKMaxRows) return plan;
-    const int64_t nkt = K / GemmCfg<FMT, 128>::BK;
+    if (!splitk || M > kSplitKMaxRows) return plan;
+    const int64_t nkt = K / bk;
     const int64_t base = (N + bn - 1) / bn;
     int64_t best = base;
     GemmPlan split = plan;
     for (int w : {256, 192, 128}) {
         const int64_t tiles = (N + w - 1) / w;
-        for (int sp = 2; sp <= 8 && 2 * sp <= nkt && tiles * sp <= d->num_sms; ++sp) {
+        for (int sp = 2; sp <= 8 && 2 * sp <= nkt && tiles * sp <= num_sms; ++sp) {
             if (tiles * sp <= best) continue;
-            const int fit = w == 256   ? splitk_max_clusters<FMT, 256>(d, sp)
-                            : w == 192 ? splitk_max_clusters<FMT, 192>(d, sp)
-                                       : splitk_max_clusters<FMT, 128>(d, sp);
-            if (tiles > fit) continue;
+            if (tiles > fit(w, sp)) continue;
             best = tiles * sp;
             split = {128, w, sp};
         }
     }
     return best * 4 >= base * 5 ? split : plan;
+}
+
+template <int FMT>
+GemmPlan plan_gemm(DeviceInfo* d, int64_t M, int64_t N, int64_t K) {
+    return plan_gemm_core(GemmCfg<FMT, 128>::BK, M, N, K, d->num_sms, g_use_pairs, g_use_splitk,
+                          [d](int w, int sp) {
+                              return w == 256   ? splitk_max_clusters<FMT, 256>(d, sp)
+                                     : w == 192 ? splitk_max_clusters<FMT, 192>(d, sp)
+                                                : splitk_max_clusters<FMT, 128>(d, sp);
+                          });
 }
 
 }  // namespace
@@ -758,14 +769,38 @@ int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_sca
                                 s);
 }
 
-int nvq_gemm_plan(int format, int64_t M, int64_t N, int64_t K, int* tile_m, int* tile_n, int* k_split) {
+namespace {
+int check_plan_args(int format, int64_t M, int64_t N, int64_t K, const int* tile_m, const int* tile_n,
+                    const int* k_split) {
     if (format != NVQ_NVFP4 && !is_mxfp8(format)) return NVQ_ERR_FORMAT;
     if (!tile_m || !tile_n || !k_split) return NVQ_ERR_NULL;
     const int64_t k_stage = format == NVQ_NVFP4 ? 256 : 128;
     if (M <= 0 || N <= 0 || N % 8 || K <= 0 || K % k_stage) return NVQ_ERR_SHAPE;
     if (K >= (int64_t(1) << 24) || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVQ_ERR_SHAPE;
+    return NVQ_OK;
+}
+}  // namespace
+
+int nvq_gemm_plan_host(int format, int64_t M, int64_t N, int64_t K, int num_sms, const int* max_clusters,
+                       int use_pairs, int use_splitk, int* tile_m, int* tile_n, int* k_split) {
+    int rc = check_plan_args(format, M, N, K, tile_m, tile_n, k_split);
+    if (rc) return rc;
+    if (!max_clusters) return NVQ_ERR_NULL;
+    if (num_sms <= 0) return NVQ_ERR_SHAPE;
+    const int64_t bk = format == NVQ_NVFP4 ? 256 : 128;
+    const GemmPlan pl = plan_gemm_core(bk, M, N, K, num_sms, use_pairs != 0, use_splitk != 0,
+                                       [max_clusters](int w, int sp) { return max_clusters[(w / 64 - 2) * 9 + sp]; });
+    *tile_m = pl.tile_m;
+    *tile_n = pl.tile_n;
+    *k_split = pl.k_split;
+    return NVQ_OK;
+}
+
+int nvq_gemm_plan(int format, int64_t M, int64_t N, int64_t K, int* tile_m, int* tile_n, int* k_split) {
+    int rc = check_plan_args(format, M, N, K, tile_m, tile_n, k_split);
+    if (rc) return rc;
     DeviceInfo* d = nullptr;
-    int rc = device_info(&d);
+    rc = device_info(&d);
     if (rc) return rc;
     const GemmPlan pl = format == NVQ_NVFP4 ? plan_gemm<0>(d, M, N, K)
                         : format == NVQ_MXFP8 ? plan_gemm<1>(d, M, N, K)
