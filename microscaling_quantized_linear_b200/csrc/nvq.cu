@@ -528,6 +528,8 @@ int launch_gemm_splitk(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_s
                        void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, int split, cudaStream_t stream) {
     using C = GemmCfg<FMT, BN>;
     const int64_t kbytes = FMT == 0 ? K / 2 : K;
+    // one 128-row block, and at least one K tile per CTA of the cluster
+    if (M > C::BM || split < 2 || split > 8 || K / C::BK < split) return NVQ_ERR_SHAPE;
     if (splitk_max_clusters<FMT, BN>(d, split) <= 0) return NVQ_ERR_CUDA;
     CUtensorMap ma, mb, md;
     memset(&md, 0, sizeof(md));
