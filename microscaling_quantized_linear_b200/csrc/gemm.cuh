@@ -27,6 +27,9 @@
 //           memory -> registers (tcgen05.ld), scale by alpha, add bias,
 //           round to BF16, release the accumulator, then stage 32 x 32
 //           sub-tiles in 64-byte-swizzled shared memory for TMA stores.
+// At a short M the same kernel (SPLITK) runs one cluster of CTAs per output
+// tile instead, each CTA over a share of K, the partial sums added through
+// distributed shared memory (see bsgemm_kernel).
 // Every mbarrier wait is bounded in wall time; a wait that gives up sets the
 // status word and an abort flag that releases the other roles.
 #pragma once
@@ -445,10 +448,11 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             }
         }
     }
-    // everything above overlaps the previous grid; no global data is
-    // touched before it has completed.  The next grid in the stream may then
-    // launch: its CTAs wait at their own griddepcontrol.wait until this grid
-    // has completed, so only its launch latency overlaps this grid.
+    // everything above overlaps the previous grid; no global data is read
+    // or written before it has completed (the split-K prefetch only warms
+    // L2, the device's point of coherence).  The next grid in the stream may
+    // then launch: its CTAs wait at their own griddepcontrol.wait until this
+    // grid has completed, so only its launch latency overlaps this grid.
     griddep_wait();
     griddep_launch();
     const uint32_t total_iters =

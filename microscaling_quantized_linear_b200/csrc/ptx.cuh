@@ -248,8 +248,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
-// ---------------------------------------------------------------- CTA pairs (cta_group::2)
-// A cluster of two CTAs on two SMs drives one 256-row MMA: each CTA stages
+// ---------------------------------------------------------------- clusters
+// Rank, barrier and distributed-shared-memory access within a thread-block
+// cluster: the CTA pairs, and the split-K clusters of gemm.cuh.
+//
+// CTA pairs (cta_group::2): a cluster of two CTAs on two SMs drives one
+// 256-row MMA: each CTA stages
 // half of A and half of B in its own shared memory and holds half of the
 // accumulator in its own tensor memory; the even CTA (the leader) issues the
 // tensor-core instructions for both.
@@ -260,7 +264,7 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
     return r;
 }
 
-// All threads of both CTAs of the cluster.
+// All threads of every CTA of the cluster.
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
