@@ -41,6 +41,8 @@ def lib():
         L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
         L.oracle_e4m3_encode.restype = ctypes.c_int
         L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_e4m3_encode_array.restype = None
+        L.oracle_e4m3_encode_array.argtypes = [_f32p, _i64, _u8p]
         L.oracle_take_nan_flag.restype = ctypes.c_int
         L.oracle_sf_bytes.restype = _i64
         L.oracle_sf_bytes.argtypes = [_i64, _i64]
@@ -120,6 +122,14 @@ def e2m1_encode(v):
 
 def e4m3_encode(v):
     return lib().oracle_e4m3_encode(float(np.float32(v)))
+
+
+def e4m3_encode_array(v):
+    """Elementwise e4m3_encode of an array of FP32 values (same shape, uint8 codes)."""
+    a = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(a.shape, dtype=np.uint8)
+    lib().oracle_e4m3_encode_array(_ptr(a, _f32p), a.size, _ptr(out, _u8p))
+    return out
 
 
 def take_nan_flag():

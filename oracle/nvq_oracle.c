@@ -144,6 +144,13 @@ ORACLE_EXPORT int oracle_e5m2_encode(float v) {
     return sign | round_to_table(fabs((double)v), 0x7B, oracle_e5m2_value);
 }
 
+/* Elementwise oracle_e4m3_encode of n FP32 values: the array form that a
+ * test uses to bound MXFP8 element codes (E4M3 elements, page "NVIDIA量化推理：
+ * 5步极速优化显存+成功率翻倍", section MXFP8量化格式). */
+ORACLE_EXPORT void oracle_e4m3_encode_array(const float* in, int64_t n, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = (uint8_t)oracle_e4m3_encode(in[i]);
+}
+
 /* Returns 1 if any NaN input reached an encoder since the last call. */
 ORACLE_EXPORT int oracle_take_nan_flag(void) { int f = g_nan_seen; g_nan_seen = 0; return f; }
 

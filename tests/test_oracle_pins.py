@@ -93,6 +93,23 @@ def test_e4m3_encode_random_matches_torch():
     assert np.array_equal(ours, _torch_e4m3_code(v))
 
 
+def test_e4m3_encode_array_matches_torch_and_saturates():
+    # The array form: every midpoint +- 1 ulp and random values against
+    # torch's RNE cast (below 464), then saturation, infinities and -0.
+    vals = [oracle.e4m3_value(c) for c in range(0x7F)]
+    probes = []
+    for lo, hi in zip(vals[:-1], vals[1:]):
+        mid = np.float32((lo + hi) / 2)
+        probes += [mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(1e9)), lo]
+    rng = np.random.default_rng(11)
+    probes += list(np.float32(2.0) ** rng.uniform(-20, 8.85, 20000).astype(np.float32))
+    p = np.array(probes, dtype=np.float32)
+    p = np.concatenate([p, -p])
+    assert np.array_equal(oracle.e4m3_encode_array(p).astype(np.int64), _torch_e4m3_code(p))
+    big = np.array([448.0, 464.0, 486.4, 1e6, np.inf, -np.inf, -0.0, -1e-9], dtype=np.float32)
+    assert oracle.e4m3_encode_array(big).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0x80, 0x80]
+
+
 def test_e4m3_saturation():
     assert oracle.e4m3_encode(448.0) == 0x7E
     assert oracle.e4m3_encode(464.0) == 0x7E       # tie with the missing 480 -> even 0x7E
