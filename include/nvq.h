@@ -15,8 +15,12 @@
  * ---------------------------------------
  *  - All data pointers are DEVICE pointers owned by the caller; the library
  *    never allocates, frees or keeps them.  It allocates no device memory of
- *    its own: the only library state on the device is one status word per
- *    GPU (a static device variable), read by nvq_device_status().
+ *    its own.  Its device state is static device variables, present on every
+ *    GPU that loads the library: one status word per GPU, read by
+ *    nvq_device_status(), and the 4 KB scratch array of
+ *    nvfp4_quantize_noalloc().  The library looks up their device addresses
+ *    once per GPU and keeps them; a device reset (cudaDeviceReset) invalidates
+ *    them, so no library call may follow one in the same process.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *    default stream).  The return value reports only host-side argument
  *    checks and launch errors.  Errors found by the host launch nothing.
@@ -87,8 +91,9 @@ enum {
 
 /* Bits of the device status word (nvq_device_status). */
 enum {
-    NVQ_STATUS_TIMEOUT = 1,     /* a GEMM pipeline wait gave up (bounded spin) */
-    NVQ_STATUS_NONFINITE = 2    /* nvfp4_quantize saw a NaN/Inf amax */
+    NVQ_STATUS_TIMEOUT = 1,     /* a bounded wait inside a kernel gave up (see the entry points) */
+    NVQ_STATUS_NONFINITE = 2,   /* nvfp4_quantize saw a NaN/Inf amax */
+    NVQ_STATUS_WORKSPACE = 4    /* nvfp4_quantize was given a workspace it did not leave (not zero-filled) */
 };
 
 /* Bytes of the code buffer for a [rows, K] tensor: rows*K/2 (NVFP4), rows*K (MXFP8, either element). */
@@ -99,9 +104,18 @@ NVQ_API size_t nvq_codes_bytes(int format, int64_t rows, int64_t K);
 NVQ_API size_t nvq_scale_bytes(int format, int64_t rows, int64_t K);
 
 /* Bytes of device scratch that nvfp4_quantize / quantize_weight(NVQ_NVFP4)
- * need (per-CTA partial maxima of the tensor; fully rewritten by every call,
- * so it needs no initialization).  Constant for the life of the library. */
+ * need: the per-CTA partial maxima of the tensor and the tagged slots and
+ * generation word of the one-pass kernel's grid barrier.  Constant for the
+ * life of the library.  A workspace must be zero-filled once before its
+ * first use (nvq_workspace_init, or any memset to zero); every call leaves
+ * it ready for the next, so it is never cleared again.  Calls that can run
+ * at the same time (different streams, no ordering) must not share one. */
 NVQ_API size_t nvq_workspace_bytes(void);
+
+/* nvq_workspace_init -- zero-fills a workspace of nvq_workspace_bytes() bytes
+ * (asynchronously on `stream`), as its first use requires.  No counterpart
+ * on the pages.  NVQ_ERR_NULL / NVQ_ERR_ALIGN / NVQ_ERR_CUDA. */
+NVQ_API int nvq_workspace_init(void* workspace, nvq_stream_t stream);
 
 /*
  * nvfp4_quantize -- dynamic BF16 -> NVFP4 activation quantization.
@@ -118,8 +132,10 @@ NVQ_API size_t nvq_workspace_bytes(void);
  *                device float holding a calibrated per-tensor amax (page
  *                "FP8量化技术提升SD3.5...", section 校准): the amax pass is
  *                skipped; elements beyond the calibrated range saturate.
- *   workspace    device scratch of nvq_workspace_bytes(); must not be shared
- *                by two calls that can run at the same time.
+ *   workspace    device scratch of nvq_workspace_bytes(), zero-filled before
+ *                its first use (see nvq_workspace_bytes); must not be shared
+ *                by two calls that can run at the same time.  Required on the
+ *                dynamic path; with calib_amax it is not read (may be NULL).
  *
  * Arithmetic, in FP32 round-to-nearest-even, bit-exact with the CPU oracle:
  *   g_enc = 2688 / amax, g_dec = amax / 2688; per 16-block along K,
@@ -127,6 +143,19 @@ NVQ_API size_t nvq_workspace_bytes(void);
  *   (round to nearest even, saturate, sign kept).  A block whose scale
  *   rounds to zero gets zero codes.  amax < 2^-100 (zero included) gives
  *   all-zero codes and scales and g_dec = 0.
+ *
+ * The dynamic path takes one of three kernels by size: one cluster of CTAs
+ * for small tensors; one pass (amax and quantization in one launch, x read
+ * once) when one CTA per SM can hold its rows in shared memory; else an amax
+ * pass and a quantize pass.  All give the same bits.  The one-pass kernel's
+ * CTAs exchange partial maxima through the workspace and so must all be
+ * resident at once; kernels on other streams that hold SMs can delay some of
+ * them.  A CTA that has waited past the limit (2 s) reads the amax from x
+ * itself: the results stay exact, the call is slower, and NVQ_STATUS_TIMEOUT
+ * is set.  A graph capture of this call replays correctly: the barrier's
+ * state lives in the workspace.  A workspace that was not zero-filled can
+ * make the one-pass kernel report NVQ_STATUS_WORKSPACE (results then still
+ * exact) or, undetectably, use a stale partial maximum.
  */
 NVQ_API int nvfp4_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
                    uint8_t* codes, uint8_t* scales, float* global_scale,
@@ -173,7 +202,8 @@ NVQ_API int mxfp8_quantize_ex(const void* x, int64_t M, int64_t K, int64_t ldx,
  *
  *   format        NVQ_NVFP4, NVQ_MXFP8 or NVQ_MXFP8_E5M2 (floor block exponent)
  *   global_scale  NVFP4: out, required.  MXFP8: ignored (may be NULL).
- *   workspace     NVFP4: required (nvq_workspace_bytes()).  MXFP8: ignored.
+ *   workspace     NVFP4: required (nvq_workspace_bytes(), zero-filled before
+ *                 its first use).  MXFP8: ignored.
  */
 NVQ_API int quantize_weight(int format, const void* w, int64_t N, int64_t K, int64_t ldw,
                     uint8_t* codes, uint8_t* scales, float* global_scale,
@@ -207,8 +237,10 @@ NVQ_API int quantize_weight(int format, const void* w, int64_t N, int64_t K, int
  * (nvq_gemm_plan reports the choice).  Results match the FP64 sum over the
  * dequantized operands to a relative error (normalised by the output row's
  * L2 norm) of 2e-3.
- * Pipeline waits inside the kernel are bounded; if one gives up, the kernel
- * sets NVQ_STATUS_TIMEOUT, writes nothing further and exits.
+ * Pipeline waits inside the kernel are bounded (4 s, or nvq_set_wait_limit);
+ * if one gives up, the kernel sets NVQ_STATUS_TIMEOUT, writes nothing further
+ * (the output is then unspecified) and exits after waiting, again bounded,
+ * for its own copies and tensor-core work in flight.
  */
 NVQ_API int block_scaled_linear(int format,
                         const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
@@ -300,6 +332,19 @@ NVQ_API int nvq_device_status(nvq_stream_t stream);
 NVQ_API const char* nvq_status_string(int code);
 
 /*
+ * nvq_set_wait_limit -- test hook (no counterpart on the pages).  Sets, for
+ * the whole process, the limit of the bounded waits between the roles of a
+ * kernel that later launches use: the GEMM pipeline waits (default 4 s) and
+ * the one-pass quantizer's grid barrier (default 2 s).  0 restores the
+ * defaults; at most 4e9 (else NVQ_ERR_SHAPE).  It lets a test make those
+ * waits run out on purpose and check that the kernel reports
+ * NVQ_STATUS_TIMEOUT and returns, with the context intact.  The waits with
+ * which a kernel drains its own copies and tensor-core work before it exits
+ * keep their 4 s limit.  Launches already issued are not affected.
+ */
+NVQ_API int nvq_set_wait_limit(uint64_t limit_ns);
+
+/*
  * nvfp4_quantize_noalloc -- nvfp4_quantize for callers that cannot allocate
  * device memory.  The paper has no counterpart to this entry point.
  *
@@ -324,10 +369,13 @@ NVQ_API const char* nvq_status_string(int code);
  *   stream are safe.  The scratch keeps the last call's contents; nothing in
  *   it needs to start at zero, because every call rewrites every partial it
  *   reads.
- *   Returns NVQ_ERR_SHAPE, launching nothing, if the amax pass would need
- *   more partial maxima than the scratch holds (it never launches more than
- *   NVQ_NOALLOC_MAX_PARTIALS CTAs, so this only guards the limit), plus the
- *   errors of nvfp4_quantize.
+ *   The amax pass sizes its grid to the scratch: one CTA per partial
+ *   maximum, never more than NVQ_NOALLOC_MAX_PARTIALS CTAs (each reads more
+ *   rows when the tensor is large), so every tensor that the shape contract
+ *   admits (rows * K < 2^31) fits; anything larger is NVQ_ERR_SHAPE and
+ *   launches nothing.  Errors otherwise as nvfp4_quantize (without a
+ *   workspace to check).  The scratch address is looked up once per device,
+ *   like the status word: a device reset invalidates it.
  */
 #define NVQ_NOALLOC_MAX_PARTIALS 1024
 NVQ_API int nvfp4_quantize_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx,

@@ -37,6 +37,7 @@ _RULES = {"floor": SCALE_FLOOR, "ceil": SCALE_CEIL}
 
 NVQ_STATUS_TIMEOUT = 1
 NVQ_STATUS_NONFINITE = 2
+NVQ_STATUS_WORKSPACE = 4
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -76,6 +77,10 @@ _lib.nvq_probe_wait.restype = ctypes.c_int
 _lib.nvq_probe_wait.argtypes = [ctypes.c_uint64, _vp, _vp]
 _lib.nvq_gemm_plan.restype = ctypes.c_int
 _lib.nvq_gemm_plan.argtypes = [ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp]
+_lib.nvq_set_wait_limit.restype = ctypes.c_int
+_lib.nvq_set_wait_limit.argtypes = [ctypes.c_uint64]
+_lib.nvq_workspace_init.restype = ctypes.c_int
+_lib.nvq_workspace_init.argtypes = [_vp, _vp]
 _lib.nvq_gemm_plan_host.restype = ctypes.c_int
 _lib.nvq_gemm_plan_host.argtypes = [ctypes.c_int, _i64, _i64, _i64, ctypes.c_int, _vp, ctypes.c_int, ctypes.c_int,
                                     _vp, _vp, _vp]
@@ -84,7 +89,7 @@ EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_
             "mxfp8_quantize", "mxfp8_quantize_ex", "quantize_weight", "block_scaled_linear",
             "nvq_device_status", "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc",
             "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu", "nvq_probe_wait", "nvq_gemm_plan",
-            "nvq_gemm_plan_host")
+            "nvq_gemm_plan_host", "nvq_set_wait_limit", "nvq_workspace_init")
 
 NOALLOC_MAX_PARTIALS = 1024
 
@@ -141,7 +146,14 @@ def workspace_bytes():
 
 
 def new_workspace(device="cuda"):
-    return torch.empty(workspace_bytes(), dtype=torch.uint8, device=device)
+    """A workspace for nvfp4_quantize / quantize_weight, zero-filled as its
+    first use requires (every call then leaves it ready for the next)."""
+    return torch.zeros(workspace_bytes(), dtype=torch.uint8, device=device)
+
+
+def workspace_init(workspace, stream=None):
+    """Zero-fill a workspace through the library (nvq_workspace_init)."""
+    _check(_lib.nvq_workspace_init(_ptr(workspace), _stream(stream, workspace.device)), "nvq_workspace_init")
 
 
 # --------------------------------------------------------------------------- quantizers
@@ -315,6 +327,12 @@ def probe_gelu(bits, stream=None):
     out = torch.empty(n, dtype=torch.int16, device=bits.device)
     _check(_lib.nvq_probe_gelu(_ptr(bits), n, _ptr(out), _stream(stream, bits.device)), "nvq_probe_gelu")
     return out
+
+
+def set_wait_limit(limit_ns):
+    """Test hook: limit (ns) of the kernels' pipeline waits for later launches
+    in this process; 0 restores the defaults (nvq_set_wait_limit)."""
+    _check(_lib.nvq_set_wait_limit(int(limit_ns)), "nvq_set_wait_limit")
 
 
 def probe_wait(limit_ns, device=None, stream=None):

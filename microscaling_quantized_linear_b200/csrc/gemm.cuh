@@ -41,6 +41,9 @@
 
 namespace nvq {
 
+// Limit of the waits with which a CTA drains its own in-flight copies and
+// tensor-core work before it exits.  The pipeline waits take theirs from
+// GemmParams::wait_ns (the same 4 s unless a test shortens it).
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s per wait
 // Warp roles: 0 TMA producer, 1 MMA issuer, 2..9 epilogue (two warps per
 // tensor-memory lane quarter, each owning half of the tile's columns),
@@ -260,7 +263,13 @@ struct GemmParams {
     uint32_t k_split = 1;
     __nv_bfloat16* out = nullptr;
     uint32_t ldo = 0;
+    // limit of every pipeline wait in ns (a role that gives up sets the
+    // status word and the abort flag); the drain waits keep kWaitLimitNs.
+    // 32 bits, in the struct's tail padding: the kernels' code is the same
+    // size as without it.
+    uint32_t wait_ns = (uint32_t)kWaitLimitNs;
 };
+static_assert(sizeof(GemmParams) == 128, "GemmParams keeps its 128 bytes");
 
 // Split-K reduction for one output tile of at most 128 rows: every CTA of
 // the cluster holds its FP32 partial tile in its own shared memory, rows of
@@ -468,7 +477,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 const uint32_t a0 = (nb * BN) / 128;             // first 128-row scale tile of B
                 for (uint32_t kt = kt_begin; kt < kt_end; ++kt) {
                     const uint32_t s = it % C::STAGES, use = it / C::STAGES;
-                    if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
+                    if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, abort_flag, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -513,7 +522,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             for (uint32_t tile = tile_first; tile < num_tiles && ok; tile += tile_step, ++t_local) {
                 const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
                 const uint32_t use = C::ACC_BUFS == 2 ? (t_local >> 1) : t_local;
-                if (use > 0 && !mbar_wait_bounded(tempty0 + 8 * buf, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
+                if (use > 0 && !mbar_wait_bounded(tempty0 + 8 * buf, (use - 1) & 1, abort_flag, p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -523,7 +532,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 const uint32_t d_tmem = tmem + buf * BN;
                 for (uint32_t kt = kt_begin; kt < kt_end; ++kt, ++it) {
                     const uint32_t s = it % C::STAGES, su = it / C::STAGES;
-                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
+                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -565,8 +574,8 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             for (uint32_t it = 0; it < total_iters; ++it) {
                 const uint32_t s = it % C::STAGES, su = it / C::STAGES;
                 // slot s is free once the MMAs of its previous use completed
-                if ((su > 0 && !mbar_wait_bounded(empty0 + 8 * s, (su - 1) & 1, abort_flag, kWaitLimitNs)) ||
-                    !mbar_wait_bounded(sfdata0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
+                if ((su > 0 && !mbar_wait_bounded(empty0 + 8 * s, (su - 1) & 1, abort_flag, p.wait_ns)) ||
+                    !mbar_wait_bounded(sfdata0 + 8 * s, su & 1, abort_flag, p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -599,7 +608,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             // this CTA's partial tile -> its shared memory (rows < M only)
             const uint32_t rows = min(p.m_total, (uint32_t)C::BM);
             if (tile_first < num_tiles) {
-                if (!mbar_wait_bounded(tfull0, 0, abort_flag, kWaitLimitNs)) {
+                if (!mbar_wait_bounded(tfull0, 0, abort_flag, p.wait_ns)) {
                     *abort_flag = 1;
                     atomicOr(p.status, 1u);
                 } else if ((uint32_t)(32 * q) < rows) {
@@ -628,7 +637,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
             const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
             const uint32_t use = C::ACC_BUFS == 2 ? (t_local >> 1) : t_local;
-            if (!mbar_wait_bounded(tfull0 + 8 * buf, use & 1, abort_flag, kWaitLimitNs)) {
+            if (!mbar_wait_bounded(tfull0 + 8 * buf, use & 1, abort_flag, p.wait_ns)) {
                 *abort_flag = 1;
                 atomicOr(p.status, 1u);
                 break;

@@ -175,7 +175,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 const uint32_t sfb_atom = (nb * BN) / 128;            // first scale tile of the B tile
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt) {
                     const uint32_t s = it % C::STAGES, use = it / C::STAGES;
-                    if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
+                    if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, abort_flag, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -203,11 +203,21 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 *abort_flag = 1;
                 atomicOr(p.status, 1u);
             }
-            if (rank == 0)      // the leader's barriers count both CTAs' bytes: wait for the last stages
+            // Neither CTA leaves while a load it issued may still be in flight.
+            if (rank == 0) {    // the leader's barriers count both CTAs' bytes: wait for the last stages
                 for (uint32_t j = it > (uint32_t)C::STAGES ? it - C::STAGES : 0; j < it; ++j) {
                     mbar_wait_bounded(sfdata0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
                     mbar_wait_bounded(full0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
                 }
+            } else {
+                // The peer's loads complete on the leader's barriers, which it
+                // cannot wait on; the MMAs that consume a stage complete only
+                // after its loads landed, and their commit reaches this CTA's
+                // empty[s].  (After an abort that commit may never come: the
+                // bounded wait then ends long after any load has landed.)
+                for (uint32_t j = it > (uint32_t)C::STAGES ? it - C::STAGES : 0; j < it; ++j)
+                    mbar_wait_bounded(empty0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
+            }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer (leader only)
@@ -217,7 +227,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             for (uint32_t tile = pair; tile < num_tiles && ok; tile += npairs, ++t_local) {
                 const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
                 const uint32_t use = C::ACC_BUFS == 2 ? (t_local >> 1) : t_local;
-                if (use > 0 && !mbar_wait_bounded(tempty0 + 8 * buf, (use - 1) & 1, abort_flag, kWaitLimitNs)) {
+                if (use > 0 && !mbar_wait_bounded(tempty0 + 8 * buf, (use - 1) & 1, abort_flag, p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -227,7 +237,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 const uint32_t sfb_shift = (((tile / p.num_m_blocks) * BN) % 128) / 32;
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt, ++it) {
                     const uint32_t s = it % C::STAGES, su = it / C::STAGES;
-                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
+                    if (!mbar_wait_bounded(full0 + 8 * s, su & 1, abort_flag, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -270,8 +280,8 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 const uint32_t s = it % C::STAGES, su = it / C::STAGES;
                 // slot s is free once the MMAs of its previous use completed
                 // (the same commit that freed the shared-memory stage)
-                if ((su > 0 && !mbar_wait_bounded(empty0 + 8 * s, (su - 1) & 1, abort_flag, kWaitLimitNs)) ||
-                    !mbar_wait_bounded(sfdata0 + 8 * s, su & 1, abort_flag, kWaitLimitNs)) {
+                if ((su > 0 && !mbar_wait_bounded(empty0 + 8 * s, (su - 1) & 1, abort_flag, p.wait_ns)) ||
+                    !mbar_wait_bounded(sfdata0 + 8 * s, su & 1, abort_flag, p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -304,7 +314,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
             const uint32_t buf = C::ACC_BUFS == 2 ? (t_local & 1) : 0;
             const uint32_t use = C::ACC_BUFS == 2 ? (t_local >> 1) : t_local;
-            if (!mbar_wait_bounded(tfull0 + 8 * buf, use & 1, abort_flag, kWaitLimitNs)) {
+            if (!mbar_wait_bounded(tfull0 + 8 * buf, use & 1, abort_flag, p.wait_ns)) {
                 *abort_flag = 1;
                 atomicOr(p.status, 1u);
                 break;

@@ -7,10 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <unistd.h>
-
 #include <atomic>
-#include <chrono>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -33,6 +30,12 @@ __device__ unsigned int g_status;
 // Shared by every call on a device; fully rewritten by each call's amax pass
 // before it is read.
 static __device__ __align__(256) uint32_t g_noalloc_partials[NVQ_NOALLOC_MAX_PARTIALS];
+// The amax pass never launches more CTAs than it has partial slots for, so
+// it fits the static array too.
+static_assert(kMaxAmaxPartials <= NVQ_NOALLOC_MAX_PARTIALS, "amax partials must fit the no-alloc scratch");
+static_assert(kStatusTimeout == NVQ_STATUS_TIMEOUT && kStatusNonfinite == NVQ_STATUS_NONFINITE &&
+                  kStatusWorkspace == NVQ_STATUS_WORKSPACE,
+              "status bits");
 
 namespace {
 
@@ -50,6 +53,7 @@ struct DeviceInfo {
     // (0 = not yet asked): [format][BN 128/192/256][k_split]
     int splitk_clusters[3][3][9] = {};
     bool fused_attr = false;
+    int fused_occupancy = -1;        // CTAs of the one-pass quantizer per SM at its largest tile (-1: not asked)
 };
 
 std::mutex g_mu;
@@ -138,13 +142,17 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
     return NVQ_OK;
 }
 
-int launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, uint32_t* partial, int num_sms,
-                cudaStream_t stream, uint32_t* npartial_out) {
+// The amax pass: one CTA per 8 x 256 16-byte vectors, at most 8 per SM and
+// at most `capacity` CTAs (one partial maximum each).
+int launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, uint32_t* partial, uint32_t capacity,
+                int num_sms, cudaStream_t stream, uint32_t* npartial_out) {
     const uint32_t vecs_per_row = (uint32_t)(K / 8), pitch_vecs = (uint32_t)(ld / 8);
     const uint64_t total = (uint64_t)rows * vecs_per_row;
     uint64_t want = (total + 8 * kAmaxThreads - 1) / (8 * kAmaxThreads);
     uint32_t grid = (uint32_t)(want < 1 ? 1 : want);
-    const uint32_t cap = (uint32_t)num_sms * 8 < (uint32_t)kMaxAmaxPartials ? (uint32_t)num_sms * 8 : kMaxAmaxPartials;
+    uint32_t cap = (uint32_t)num_sms * 8 < (uint32_t)kMaxAmaxPartials ? (uint32_t)num_sms * 8 : kMaxAmaxPartials;
+    if (cap > capacity) cap = capacity;
+    if (cap == 0) return NVQ_ERR_SHAPE;
     if (grid > cap) grid = cap;
     *npartial_out = grid;
     return launch_pdl(amax_partials_kernel, dim3(grid), dim3(kAmaxThreads), 0, stream, static_cast<const uint4*>(x),
@@ -158,22 +166,43 @@ uint32_t quant_grid(uint64_t units, int num_sms) {
     return (uint32_t)(blocks < 1 ? 1 : blocks);
 }
 
-// Epoch tags of the one-pass quantizer's workspace slots: process-wide,
-// monotonic, started at a per-process random value so that slots left in
-// reused memory by another process cannot match.
-std::atomic<uint32_t> g_epoch{0};
-std::once_flag g_epoch_once;
+// Limit of the kernels' pipeline waits set by nvq_set_wait_limit (0: the
+// defaults, 4 s in the GEMMs and 2 s in the one-pass quantizer's barrier).
+std::atomic<uint64_t> g_wait_limit_ns{0};
 
-uint32_t next_epoch() {
-    std::call_once(g_epoch_once, [] {
-        const uint64_t t = (uint64_t)std::chrono::steady_clock::now().time_since_epoch().count();
-        g_epoch.store((uint32_t)(t ^ (t >> 32) ^ ((uint64_t)getpid() << 16)));
-    });
-    uint32_t e = g_epoch.fetch_add(1) + 1;
-    return e;
+uint64_t pipeline_wait_ns(uint64_t dflt) {
+    const uint64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
+    return v ? v : dflt;
 }
 
 constexpr size_t kFusedSmemMax = 220 * 1024;
+
+// One-pass quantizer: opt in to its shared memory and ask how many of its
+// CTAs an SM holds with the largest tile it is given (cached per device).
+// Its grid barrier needs every CTA resident at once; the grid is at most one
+// CTA per SM, so it runs only where that answer is at least one.
+int fused_quantizer_fits(DeviceInfo* d, bool* fits) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!d->fused_attr) {
+        if (cudaFuncSetAttribute(nvfp4_quantize_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kFusedSmemMax + 128) != cudaSuccess) {
+            cudaGetLastError();
+            return NVQ_ERR_CUDA;
+        }
+        d->fused_attr = true;
+    }
+    if (d->fused_occupancy < 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4_quantize_fused_kernel, kFusedThreads,
+                                                          kFusedSmemMax) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        d->fused_occupancy = n;
+    }
+    *fits = d->fused_occupancy >= 1;
+    return NVQ_OK;
+}
 
 // Dynamic NVFP4 quantization: one pass (every CTA's rows held in shared
 // memory, one read of x) for tensors that fit on chip, else two passes
@@ -237,33 +266,29 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
         // at most as many CTAs as SMs).
         const int64_t rows_per_cta = (M + d->num_sms - 1) / d->num_sms;
         const size_t smem = fused_smem_bytes((size_t)rows_per_cta, (size_t)K);
+        bool fits = false;
         if (smem <= kFusedSmemMax && (M + rows_per_cta - 1) / rows_per_cta <= kMaxFusedCtas &&
-            rows_per_cta * (K / 16) <= (int64_t)kFusedMaxBlocks * kFusedThreads) {
-            {
-                std::lock_guard<std::mutex> lock(g_mu);
-                if (!d->fused_attr) {
-                    if (cudaFuncSetAttribute(nvfp4_quantize_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kFusedSmemMax + 128) != cudaSuccess)
-                        return NVQ_ERR_CUDA;
-                    d->fused_attr = true;
-                }
-            }
+            rows_per_cta * (K / 16) <= (int64_t)kFusedMaxBlocks * kFusedThreads &&
+            (rc = fused_quantizer_fits(d, &fits)) == NVQ_OK && fits) {
             const uint32_t grid = (uint32_t)((M + rows_per_cta - 1) / rows_per_cta);
             const uint16_t* xp = static_cast<const uint16_t*>(x);
             uint32_t rows32 = (uint32_t)M, k32 = (uint32_t)K, ld32 = (uint32_t)ldx, rpc = (uint32_t)rows_per_cta;
             unsigned long long* slots = reinterpret_cast<unsigned long long*>(
                 static_cast<uint8_t*>(workspace) + kWorkspaceSlotsOffset);
-            uint32_t epoch = next_epoch();
+            unsigned long long* gen = reinterpret_cast<unsigned long long*>(
+                static_cast<uint8_t*>(workspace) + kWorkspaceGenOffset);
+            uint64_t wait_ns = pipeline_wait_ns(kFusedWaitNs);
             unsigned int* status = d->status;
-            void* args[] = {&xp, &rows32, &k32, &ld32, &rpc, &codes, &scales, &global_scale, &slots, &epoch, &status};
+            void* args[] = {&xp,     &rows32, &k32, &ld32,    &rpc,   &codes, &scales,
+                            &global_scale, &slots, &gen, &wait_ns, &status};
             // The kernel waits on every CTA's maximum, so every CTA must be
-            // resident at once: the grid is at most one CTA per SM (the
-            // registers of 1024 threads leave room for one), so all of them
-            // are resident once the previous grid in the stream has left the
-            // SMs.  A cooperative launch would guarantee it too but costs
-            // about 2.6 us more per call on B200; work on other streams that
-            // held SMs for seconds would end in NVQ_STATUS_TIMEOUT (bounded
-            // wait), not in a hang.
+            // resident at once: the grid is at most one CTA per SM and an SM
+            // holds one (checked above), so all of them are resident once the
+            // previous grid in the stream has left the SMs.  A cooperative
+            // launch would guarantee it too but costs about 2.6 us more per
+            // call on B200.  Work on other streams that holds SMs past the
+            // wait's limit makes the waiting CTAs read the amax from x
+            // themselves: exact results, NVQ_STATUS_TIMEOUT set.
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(grid);
             cfg.blockDim = dim3(kFusedThreads);
@@ -280,12 +305,13 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
             }
             return NVQ_OK;
         }
+        if (rc) return rc;
     }
     uint32_t npartial = 0;
     uint32_t* partial = calib_amax ? nullptr
                                    : reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + kWorkspacePartialsOffset);
     if (!calib_amax) {
-        if ((rc = launch_amax(x, M, K, ldx, partial, d->num_sms, stream, &npartial))) return rc;
+        if ((rc = launch_amax(x, M, K, ldx, partial, kMaxAmaxPartials, d->num_sms, stream, &npartial))) return rc;
     }
     const uint64_t units = (uint64_t)M * nblk;
     return launch_pdl(nvfp4_quantize_kernel, dim3(quant_grid(units, d->num_sms)), dim3(kQuantThreads), 0, stream,
@@ -393,6 +419,7 @@ int launch_gemm_pair(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_sca
     p.b_global = b_global;
     p.bias = static_cast<const __nv_bfloat16*>(bias);
     p.status = d->status;
+    p.wait_ns = (uint32_t)pipeline_wait_ns(kWaitLimitNs);
     p.num_m_blocks = (uint32_t)((M + 255) / 256);
     p.num_n_blocks = (uint32_t)((N + BN - 1) / BN);
     p.n_total = (uint32_t)N;
@@ -456,6 +483,7 @@ int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, 
     p.b_global = b_global;
     p.bias = static_cast<const __nv_bfloat16*>(bias);
     p.status = d->status;
+    p.wait_ns = (uint32_t)pipeline_wait_ns(kWaitLimitNs);
     p.num_m_blocks = (uint32_t)((M + C::BM - 1) / C::BM);
     p.num_n_blocks = (uint32_t)((N + BN - 1) / BN);
     p.n_total = (uint32_t)N;
@@ -544,6 +572,7 @@ int launch_gemm_splitk(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_s
     p.b_global = b_global;
     p.bias = static_cast<const __nv_bfloat16*>(bias);
     p.status = d->status;
+    p.wait_ns = (uint32_t)pipeline_wait_ns(kWaitLimitNs);
     p.num_m_blocks = 1;
     p.num_n_blocks = (uint32_t)((N + BN - 1) / BN);
     p.n_total = (uint32_t)N;
@@ -865,6 +894,22 @@ int nvq_probe_wait(uint64_t limit_ns, unsigned long long* waited_ns, nvq_stream_
     return launch_status();
 }
 
+int nvq_set_wait_limit(uint64_t limit_ns) {
+    if (limit_ns > kWaitLimitNs) return NVQ_ERR_SHAPE;       // at most the 4 s default
+    g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+    return NVQ_OK;
+}
+
+int nvq_workspace_init(void* workspace, nvq_stream_t stream) {
+    if (!workspace) return NVQ_ERR_NULL;
+    if (!aligned16(workspace)) return NVQ_ERR_ALIGN;
+    if (cudaMemsetAsync(workspace, 0, kWorkspaceBytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return NVQ_ERR_CUDA;
+    }
+    return NVQ_OK;
+}
+
 int nvq_device_status(nvq_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NVQ_ERR_CUDA;
     DeviceInfo* d = nullptr;
@@ -928,16 +973,11 @@ int nvfp4_quantize_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx, uin
         }
         partials = scratch[dev];
     }
-    // the amax pass writes one partial per CTA: it must fit the static scratch
-    const uint64_t vectors = (uint64_t)M * (uint64_t)(K / 8);
-    uint64_t grid = (vectors + 8 * kAmaxThreads - 1) / (8 * kAmaxThreads);
-    const uint64_t cap = (uint64_t)d->num_sms * 8 < (uint64_t)kMaxAmaxPartials ? (uint64_t)d->num_sms * 8
-                                                                               : (uint64_t)kMaxAmaxPartials;
-    if (grid > cap) grid = cap;
-    if (grid > NVQ_NOALLOC_MAX_PARTIALS) return NVQ_ERR_SHAPE;
+    // the amax pass writes one partial per CTA and launches at most as many
+    // CTAs as the static scratch holds
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint32_t npartial = 0;
-    if ((rc = launch_amax(x, M, K, ldx, partials, d->num_sms, s, &npartial))) return rc;
+    if ((rc = launch_amax(x, M, K, ldx, partials, NVQ_NOALLOC_MAX_PARTIALS, d->num_sms, s, &npartial))) return rc;
     const uint32_t nblk = (uint32_t)(K / 16);
     const float* no_calib = nullptr;
     return launch_pdl(nvfp4_quantize_kernel, dim3(quant_grid((uint64_t)M * nblk, d->num_sms)), dim3(kQuantThreads), 0,

@@ -29,13 +29,22 @@ namespace nvq {
 
 constexpr int kAmaxThreads = 256;
 constexpr int kMaxAmaxPartials = 1024;        // u32 partial maxima of the two-pass path
-constexpr int kMaxFusedCtas = 256;            // epoch-tagged slots of the one-pass path
+constexpr int kMaxFusedCtas = 256;            // generation-tagged slots of the one-pass path
 constexpr int kFusedSlotStride = 16;          // u64 per slot: one 128-byte line each, so polls spread over L2
+// Workspace: the one-pass slots, the two-pass partial maxima, then the
+// one-pass generation word on a line of its own.  The caller zero-fills it
+// once before its first use; every call leaves it valid for the next.
 constexpr size_t kWorkspaceSlotsOffset = 0;
 constexpr size_t kWorkspacePartialsOffset = (size_t)kMaxFusedCtas * kFusedSlotStride * 8;
-constexpr size_t kWorkspaceBytes = kWorkspacePartialsOffset + kMaxAmaxPartials * 4;
+constexpr size_t kWorkspaceGenOffset = kWorkspacePartialsOffset + kMaxAmaxPartials * 4;
+constexpr size_t kWorkspaceBytes = kWorkspaceGenOffset + 128;
 constexpr int kQuantThreads = 256;
 constexpr float kAmaxFloor = 0x1p-100f;       // below this the tensor quantizes to zero
+
+// Bits of the device status word (the NVQ_STATUS_* values of nvq.h).
+constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusNonfinite = 2u;
+constexpr unsigned int kStatusWorkspace = 4u;
 
 // max over the two 16-bit magnitudes packed in u
 __device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t u) {
@@ -372,15 +381,30 @@ nvfp4_quantize_cluster_kernel(const uint16_t* __restrict__ x, uint32_t rows, uin
 // CTA copies its rows into shared memory once (each thread copies its own
 // blocks with 16-byte asynchronous copies, all issued at once, one commit
 // group per block, and takes each block's maximum and fl(b/6) as its group
-// lands), publishes its partial amax in an epoch-tagged 64-bit slot of the
-// workspace, waits (bounded) until every CTA's slot carries this call's
-// epoch, and quantizes from shared memory.  HBM sees exactly one read of the
+// lands), publishes its partial amax in a tagged 64-bit slot of the
+// workspace, waits (bounded) until every CTA's slot carries this call's tag,
+// and quantizes from shared memory.  HBM sees exactly one read of the
 // activation.  Every CTA must be resident at once: at most one CTA per SM.
+//
+// The tag comes from a generation word in the workspace, never from the
+// host, so a launch replayed from a CUDA graph is as correct as a fresh one.
+// A call reads the word g (zero in a fresh workspace) and tags its slots
+// with E = g + 1.  Every tag an earlier call wrote is <= g, so no stale slot
+// can pass for this call's.  Once CTA 0 has seen every slot tagged E it
+// raises the word to E; every CTA read g before publishing, so all CTAs of
+// the call agree on E.  A CTA whose wait gives up raises the word to its own
+// tag too, so the next call's tag is above every tag written in this one,
+// whichever CTAs gave up; it then takes the amax by reading the whole tensor
+// itself, so its outputs are exact all the same, and reports
+// NVQ_STATUS_TIMEOUT.  A word at or above 2^48 - 1 (2^48 calls away from a
+// zero-filled workspace) was not left by this library: every CTA takes the
+// direct amax and the call reports NVQ_STATUS_WORKSPACE.
 constexpr int kFusedThreads = 1024;
 constexpr int kFusedMaxBlocks = 8;                 // 16-blocks per thread: rows_per_cta * K / 16 <= 8192
 constexpr uint64_t kFusedWaitNs = 2000000000ull;   // 2 s
+constexpr unsigned long long kGenMax = (1ull << 48) - 1;   // a slot holds a 48-bit tag above a 16-bit maximum
 
-// The slot word carries its epoch and its value together, so relaxed
+// The slot word carries its tag and its value together, so relaxed
 // single-copy-atomic 64-bit accesses suffice: nothing else is published.
 __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
@@ -390,6 +414,31 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
     unsigned long long v;
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
+}
+
+// The generation word is raised with a relaxed maximum.  CTA 0 raises it to
+// E only after it has read every slot tagged E, and a CTA's tag is computed
+// from the word it read: for a CTA of the same call to read the raised word,
+// its own slot would have to hold a tag derived from that read, which CTA 0
+// could not have seen before raising it (the memory model's no-thin-air
+// rule), so no fence is needed, and no thread waits for one.
+__device__ __forceinline__ void red_relaxed_max_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
+}
+
+// BF16 magnitude bits of max |x| over the whole [rows, K] tensor (pitch ldx),
+// read by one CTA: the one-pass kernel's amax when its wait gives up.
+__device__ __forceinline__ uint32_t cta_tensor_absmax(const uint16_t* __restrict__ x, uint32_t rows, uint32_t K,
+                                                      uint32_t ldx, uint32_t* red) {
+    const uint32_t vpr = K >> 3;                        // 16-byte vectors per row
+    const uint32_t total = rows * vpr;
+    uint32_t m2 = 0;
+    for (uint32_t i = threadIdx.x; i < total; i += kFusedThreads) {
+        const uint32_t r = i / vpr, c = i - r * vpr;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)r * ldx) + c);
+        m2 = absmax2(absmax2(absmax2(absmax2(m2, v.x), v.y), v.z), v.w);
+    }
+    return block_max_u32<kFusedThreads>(fold2(m2), red);
 }
 
 // Two 16-byte halves of the 32-byte block at smem byte offset 32*b.  Threads
@@ -414,7 +463,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t K, uint32_t ldx,
                             uint32_t rows_per_cta, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                             float* __restrict__ g_dec_out, unsigned long long* __restrict__ slots,
-                            uint32_t epoch, unsigned int* __restrict__ status) {
+                            unsigned long long* __restrict__ gen, uint64_t wait_ns,
+                            unsigned int* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const uint32_t nblk = K >> 4;
@@ -423,6 +473,7 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
     __shared__ uint32_t s_pmax[kMaxFusedCtas / 32];
     __shared__ float d6[128], rtab[128];
     __shared__ int s_timeout;
+    __shared__ unsigned long long s_gen;
 
     // x may come from the previous grid, and that grid may still read the
     // outputs: nothing global is touched before it has completed
@@ -449,6 +500,14 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
     if (threadIdx.x == 0) s_timeout = 0;
     init_d6(d6);
     __syncthreads();
+    // The generation this call starts from; no CTA of the call can raise it
+    // before every CTA has read it.  Thread 0 reads it here, after its copies
+    // and the barrier, and needs the value only when it publishes, so the
+    // load's latency hides under the copies'.  A relaxed load suffices: the
+    // slot it publishes carries a tag computed from the value read, and that
+    // data dependency keeps the publication after the read.
+    unsigned long long g_seen = 0;
+    if (threadIdx.x == 0) g_seen = ld_relaxed_u64(gen);
 
     // block maxima and fl(b/6), block by block as the copies land
     uint32_t m = 0;
@@ -474,48 +533,60 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
             m = max(m, mb);
         }
     }
-    const uint32_t cta_max = block_max_u32<kFusedThreads>(m, red);
-    if (threadIdx.x == 0)
-        st_relaxed_u64(slots + (size_t)blockIdx.x * kFusedSlotStride, ((unsigned long long)epoch << 32) | cta_max);
-
-    // Every CTA's partial, tagged with this call's epoch.  Warp w polls slots
-    // 32w .. 32w + 31, one per lane, so a polling round costs one L2 round
-    // trip; the other warps wait at the barrier below.
+    if (threadIdx.x == 0) s_gen = g_seen;
+    const uint32_t cta_max = block_max_u32<kFusedThreads>(m, red);   // (its barriers publish s_gen)
+    const unsigned long long g0 = s_gen;
+    const bool trusted = g0 < kGenMax;
+    const unsigned long long tag = g0 + 1;
     const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t npoll = (gridDim.x + 31) >> 5;
-    if (warp < npoll) {
-        volatile int* timeout = &s_timeout;
-        const uint32_t j = warp * 32 + lane;
-        bool done = j >= gridDim.x;
-        uint32_t mine = 0;
-        const uint64_t t0 = globaltimer_ns();
-        while (true) {
-            if (!done) {
-                const unsigned long long v = ld_relaxed_u64(slots + (size_t)j * kFusedSlotStride);
-                if ((uint32_t)(v >> 32) == epoch) {
-                    mine = (uint32_t)(v & 0xFFFFFFFFull);
-                    done = true;
+    if (trusted) {
+        if (threadIdx.x == 0) st_relaxed_u64(slots + (size_t)blockIdx.x * kFusedSlotStride, (tag << 16) | cta_max);
+        // Every CTA's partial, tagged with this call's tag.  Warp w polls
+        // slots 32w .. 32w + 31, one per lane, so a polling round costs one
+        // L2 round trip; the other warps wait at the barrier below.
+        if (warp < npoll) {
+            volatile int* timeout = &s_timeout;
+            const uint32_t j = warp * 32 + lane;
+            bool done = j >= gridDim.x;
+            uint32_t mine = 0;
+            const uint64_t t0 = globaltimer_ns();
+            while (true) {
+                if (!done) {
+                    const unsigned long long v = ld_relaxed_u64(slots + (size_t)j * kFusedSlotStride);
+                    if ((v >> 16) == tag) {
+                        mine = (uint32_t)(v & 0xFFFFull);
+                        done = true;
+                    }
+                }
+                if (__all_sync(0xFFFFFFFFu, done)) break;
+                int give_up = 0;                      // decided by lane 0 so the warp leaves together
+                if (lane == 0) give_up = *timeout || globaltimer_ns() - t0 > wait_ns;
+                if (__shfl_sync(0xFFFFFFFFu, give_up, 0)) {
+                    if (lane == 0) *timeout = 1;
+                    break;
                 }
             }
-            if (__all_sync(0xFFFFFFFFu, done)) break;
-            int give_up = 0;                          // decided by lane 0 so the warp leaves together
-            if (lane == 0) give_up = *timeout || globaltimer_ns() - t0 > kFusedWaitNs;
-            if (__shfl_sync(0xFFFFFFFFu, give_up, 0)) {
-                if (lane == 0) *timeout = 1;
-                break;
-            }
+            mine = __reduce_max_sync(0xFFFFFFFFu, mine);
+            if (lane == 0) s_pmax[warp] = mine;
         }
-        mine = __reduce_max_sync(0xFFFFFFFFu, mine);
-        if (lane == 0) s_pmax[warp] = mine;
     }
     __syncthreads();
-    if (s_timeout) {                                  // a peer never arrived: write nothing
-        if (threadIdx.x == 0) atomicOr(status, 1u);
-        return;                                       // every copy of this thread has landed
-    }
     uint32_t amax_bits = 0;
-    for (uint32_t i = 0; i < npoll; ++i) amax_bits = max(amax_bits, s_pmax[i]);
-    if (amax_bits >= 0x7F80u && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, 2u);
+    if (!trusted || s_timeout) {
+        // The barrier is off (a peer never arrived within the limit, or the
+        // generation word is not one this library left): the amax straight
+        // from x, so the outputs are exact all the same.
+        if (threadIdx.x == 0) {
+            atomicOr(status, trusted ? kStatusTimeout : kStatusWorkspace);
+            if (trusted) red_relaxed_max_u64(gen, tag);
+        }
+        amax_bits = cta_tensor_absmax(x, rows, K, ldx, red);
+    } else {
+        for (uint32_t i = 0; i < npoll; ++i) amax_bits = max(amax_bits, s_pmax[i]);
+        if (blockIdx.x == 0 && threadIdx.x == 0) red_relaxed_max_u64(gen, tag);
+    }
+    if (amax_bits >= 0x7F80u && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, kStatusNonfinite);
     const float amax = __uint_as_float(amax_bits << 16);
     const float g_enc = encode_scale(amax);
     if (blockIdx.x == 0 && threadIdx.x == 0) *g_dec_out = decode_scale(amax);

@@ -177,3 +177,15 @@ def test_valid_arguments_without_gpu_report_cuda_error():
     out = (ctypes.c_int * 3)()
     assert L.nvq_gemm_plan(0, 1, 12288, 3072, ctypes.byref(out, 0), ctypes.byref(out, 4),
                            ctypes.byref(out, 8)) == -5
+
+
+def test_wait_limit_hook_and_workspace_init_check_arguments():
+    # the test hook only stores a process-wide limit: no device needed
+    assert L.nvq_set_wait_limit(4_000_000_001) == -2        # above the 4 s default
+    assert L.nvq_set_wait_limit(1000) == 0
+    assert L.nvq_set_wait_limit(0) == 0                     # back to the defaults
+    assert L.nvq_workspace_init(NULL, NULL) == -1
+    assert L.nvq_workspace_init(P_ODD, NULL) == -3
+    # the workspace holds the one-pass slots (one 128-byte line per CTA, up to
+    # 256), the two-pass partials and the generation word's line
+    assert nvq.workspace_bytes() == 256 * 128 + 1024 * 4 + 128
