@@ -11,10 +11,13 @@ unique only where the GEMM is exact, so:
     partial sum of the GEMM is a binary32 number, whatever order the tensor
     core adds in, so D equals the oracle's D and codes and scales must match
     bit for bit (the test first checks that the grid bound holds);
-  * on the FLUX-like FF-up workload D may differ from the oracle's BF16
-    rounding in the last place where the binary64 sum lies near a rounding
-    boundary: scale bytes and codes must agree except for a small fraction,
-    and where they differ it is by one step;
+  * on the FLUX-like FF-up workload D is known only to the GEMM tolerance,
+    so several results are correct.  From the oracle's Y and the tolerance
+    the test derives, for every element, the BF16 values D may take, the
+    smallest and largest GELU over them, hence for every 32-block the
+    admissible E8M0 exponents and for every element the admissible E4M3
+    codes under the exponent the kernel chose; no byte may fall outside
+    (check_admissible);
   * the whole feed-forward block (fused FF-up, then the MXFP8 FF-down GEMM
     on its output) meets the GEMM tolerance against the oracle's chain.
 """
@@ -24,6 +27,7 @@ import torch
 
 import oracle
 import workloads
+from admissible import check_admissible
 from gpu_common import act, bits, check_gemm, sample_rows, sf_matrix, wgt
 
 pytestmark = pytest.mark.gpu
@@ -148,40 +152,24 @@ def test_exact_grid_deterministic_and_reusable_outputs():
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
-def e4m3_steps_apart(a, b):
-    """Distance in E4M3 codes between two codes of the same sign (codes are
-    monotone in magnitude within a sign); large if the signs differ and
-    either value is non-zero."""
-    a = a.astype(np.int64)
-    b = b.astype(np.int64)
-    same_sign = (a & 0x80) == (b & 0x80)
-    zero = ((a & 0x7F) == 0) & ((b & 0x7F) == 0)
-    return np.where(same_sign | zero, np.abs((a & 0x7F) - (b & 0x7F)), 1000)
+def check_sampled_rows(yc, ys, A, B, rows, M, N):
+    """The kernel's outputs on the sampled rows, against the admissible sets."""
+    Y = oracle.gemm_rows(A, B, rows=rows)
+    check_admissible(yc[rows], sf_matrix(ys, M, N // 32)[rows], Y)
+    # every sampled row was written (no canary row left)
+    assert not np.all(yc[rows] == 0xA5, axis=1).any()
 
 
 def test_ffup_workload_sampled_rows():
     """FF-up of the FLUX-like block at full size (4608 x 12288 x 3072, NVFP4),
-    in the launch configuration the benchmark uses."""
+    in the launch configuration the benchmark uses: every byte of every other
+    128-row tile's first and last row (and random rows) admissible."""
     x, w = act("ffup"), wgt("ffup")
     M, K = x.shape
     N = w.shape[0]
     ops, A, B = quantize_both("nvfp4", x, w)
     yc, ys = gpu_fused("nvfp4", ops, M, N, K)
-    rows = sample_rows(M, per_tile_every=2, extra=16)
-    oc, osf, D, G, Y = oracle.linear_gelu_mxfp8(A, B, rows=rows)
-    nb = N // 32
-    gs = sf_matrix(ys, M, nb)[rows]
-    os_ = sf_matrix(osf, rows.size, nb)
-    sdiff = gs.astype(np.int64) - os_.astype(np.int64)
-    assert np.abs(sdiff).max() <= 1
-    assert np.count_nonzero(sdiff) <= max(2, 1e-3 * sdiff.size), np.count_nonzero(sdiff)
-    g_codes = yc[rows]
-    same_scale = np.repeat(sdiff == 0, 32, axis=1)
-    steps = e4m3_steps_apart(g_codes, oc)[same_scale]
-    assert steps.max() <= 1, steps.max()
-    assert np.count_nonzero(steps) <= 1e-3 * steps.size, np.count_nonzero(steps)
-    # every row of the output was written (no canary left in the sampled rows)
-    assert not np.all(g_codes == 0xA5, axis=1).any()
+    check_sampled_rows(yc, ys, A, B, sample_rows(M, per_tile_every=2, extra=16), M, N)
 
 
 def test_feed_forward_block_end_to_end():
@@ -206,19 +194,6 @@ def test_feed_forward_block_end_to_end():
     check_gemm(out.float().cpu().numpy(), Y2)
 
 
-def _check_sampled_rows(yc, ys, oc, osf, rows, M, N):
-    nb = N // 32
-    gs = sf_matrix(ys, M, nb)[rows]
-    os_ = sf_matrix(osf, rows.size, nb)
-    sdiff = gs.astype(np.int64) - os_.astype(np.int64)
-    assert np.abs(sdiff).max() <= 1
-    assert np.count_nonzero(sdiff) <= max(2, 1e-3 * sdiff.size), np.count_nonzero(sdiff)
-    same_scale = np.repeat(sdiff == 0, 32, axis=1)
-    steps = e4m3_steps_apart(yc[rows], oc)[same_scale]
-    assert steps.max() <= 1, steps.max()
-    assert np.count_nonzero(steps) <= 1e-3 * steps.size, np.count_nonzero(steps)
-
-
 def test_ffup_workload_mxfp8_operands_sampled_rows():
     """The same FF-up linear with MXFP8 (E4M3) activation and weight operands."""
     x, w = act("ffup"), wgt("ffup")
@@ -226,9 +201,7 @@ def test_ffup_workload_mxfp8_operands_sampled_rows():
     N = w.shape[0]
     ops, A, B = quantize_both("mxfp8", x, w)
     yc, ys = gpu_fused("mxfp8", ops, M, N, K)
-    rows = sample_rows(M, per_tile_every=3, extra=8)
-    oc, osf, _, _, _ = oracle.linear_gelu_mxfp8(A, B, rows=rows)
-    _check_sampled_rows(yc, ys, oc, osf, rows, M, N)
+    check_sampled_rows(yc, ys, A, B, sample_rows(M, per_tile_every=2, extra=8), M, N)
 
 
 SINGLE_CTA_FUSED_SCRIPT = r"""
@@ -251,15 +224,16 @@ for fmt, M, N, K in [("nvfp4", 512, 768, 512), ("nvfp4", 1280, 512, 256), ("mxfp
     oc, osf, _, _, _ = oracle.linear_gelu_mxfp8(A, B)
     assert np.array_equal(ys, osf) and np.array_equal(yc, oc), (fmt, M, N, K)
     print(fmt, M, N, K, "bit-exact")
-# the FF-up workload: within one step of the oracle on sampled rows
+# the FF-up workload, NVFP4 and MXFP8 operands: every byte admissible on the
+# sampled rows of every other 128-row tile
 x, w = t.act("ffup"), t.wgt("ffup")
 M, K = x.shape
 N = w.shape[0]
-ops, A, B = t.quantize_both("nvfp4", x, w)
-yc, ys = t.gpu_fused("nvfp4", ops, M, N, K)
-rows = sample_rows(M, per_tile_every=6, extra=8)
-oc, osf, _, _, _ = oracle.linear_gelu_mxfp8(A, B, rows=rows)
-t._check_sampled_rows(yc, ys, oc, osf, rows, M, N)
+for fmt in ("nvfp4", "mxfp8"):
+    ops, A, B = t.quantize_both(fmt, x, w)
+    yc, ys = t.gpu_fused(fmt, ops, M, N, K)
+    t.check_sampled_rows(yc, ys, A, B, sample_rows(M, per_tile_every=2, extra=8), M, N)
+    print(fmt, "FF-up admissible")
 print("OK")
 """
 
