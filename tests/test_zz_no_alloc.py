@@ -20,7 +20,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
+from gpu_common import bits
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +30,8 @@ nvq = pytest.importorskip("microscaling_quantized_linear_b200")
 
 
 def quantize_noalloc_cabi(x):
-    """Calls the C entry point directly with caller-allocated outputs."""
+    """Calls the C entry point directly with caller-allocated outputs (x may
+    be a row-pitched view)."""
     M, K = x.shape
     codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
     scales = torch.empty(nvq.scale_bytes("nvfp4", M, K), dtype=torch.uint8, device="cuda")
@@ -67,7 +70,56 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
         want = quantize_with_workspace(x)
         assert_same(first, want)
         assert_same(second, want)
+        assert_same(first, oracle_quantize(x.cpu()))
     assert nvq.device_status() == 0
+
+
+def oracle_quantize(x_cpu):
+    codes, sf, g = oracle.nvfp4_quantize(bits(x_cpu))
+    return codes, sf, np.array([g], dtype=np.float32)
+
+
+SHAPES = [
+    # ragged row counts (the scale rows up to the next multiple of 128 are
+    # written as zero), several CTAs' partial maxima, and a pitched view
+    (129, 512, None),
+    (1000, 1536, None),
+    (256, 448, 448 + 64),
+]
+
+
+@pytest.mark.parametrize("M,K,ldx", SHAPES)
+def test_noalloc_matches_oracle_on_ragged_and_pitched_inputs(M, K, ldx):
+    x = workloads.normal(M, K, seed=M + K, std=2.0)
+    if ldx is None:
+        xd = x.cuda()
+    else:
+        buf = torch.zeros((M, ldx), dtype=torch.bfloat16)
+        buf[:, :K] = x
+        xd = buf.cuda()[:, :K]
+    want = oracle_quantize(x)
+    assert_same(quantize_noalloc_cabi(xd), want)
+    assert_same(quantize_noalloc_cabi(xd), want)           # second call on the same scratch
+    assert_same(quantize_with_workspace(xd), want)
+    assert nvq.device_status() == 0
+
+
+def test_noalloc_python_wrapper_and_nonfinite_status():
+    # The package's wrapper passes caller-allocated outputs to the same entry
+    # point; an infinity in the input sets NVQ_STATUS_NONFINITE, and the next
+    # finite call is clean and exact again.
+    x = workloads.activation("ffup", seed=3)
+    M, K = x.shape
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty(nvq.scale_bytes("nvfp4", M, K), dtype=torch.uint8, device="cuda")
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    bad = x.clone()
+    bad[17, 5] = float("inf")
+    nvq.nvfp4_quantize_noalloc(bad.cuda(), codes, scales, g)
+    assert nvq.device_status() == nvq.NVQ_STATUS_NONFINITE
+    nvq.nvfp4_quantize_noalloc(x.cuda(), codes, scales, g)
+    assert nvq.device_status() == 0
+    assert_same((codes.cpu().numpy(), scales.cpu().numpy(), g.cpu().numpy()), oracle_quantize(x))
 
 
 def test_noalloc_rejects_bad_arguments_without_launching():
