@@ -42,8 +42,8 @@ ACT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # BF16 read, E2M1 codes + E4M3 scale
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum).  It holds for
 # the kernel sources it was taken on; once they change the figure is stale
 # and is reported as null.
-# Taken on the FF-up workload; the summary is in
-# profiles/bsgemm_pair_kernel_nvfp4_ffup.md.
+# Taken on the FF-up workload with one ncu capture of the GEMM launch; the
+# summary of that capture is kept with the other ncu summaries in profiles/.
 GEMM_TRAFFIC = {"kernel": "bsgemm_pair_kernel<0, 256>",
                 "bytes_per_launch": 29276160 + 62105856,
                 "sources_sha256": "15b9be929ff7e57d992921403dfceb3d29ef5eae359c92b5731dade815c17e65"}
@@ -144,7 +144,7 @@ class ClockSampler:
         0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index, period=0.02):
+    def __init__(self, device_index, period=0.002):
         self.samples = []
         self.reasons = 0
         self.ok = False
@@ -349,6 +349,8 @@ def run_ours(args, rank, world, device):
         res["small_m"] = run_small_m_component(nvq, device, stream, peaks)
     if args.ff_block:
         res["ff_block"] = run_ff_block_component(nvq, device, stream, peaks)
+    if args.qkv4:
+        res["qkv4"] = run_qkv4_component(nvq, device, stream, peaks)
     return res
 
 
@@ -575,6 +577,66 @@ def run_ff_block_component(nvq, device, stream, peaks, iters=100):
     return res
 
 
+def run_qkv4_component(nvq, device, stream, peaks, rotate=2, iters=40):
+    """NVFP4 QKV projection at batch 4: dynamic quantization of the BF16
+    activation [18432, 3072] ~ 0.5 * StudentT(3) (its rows do not fit on chip,
+    so the amax pass and the quantize pass), then the block-scaled GEMM
+    against the [9216, 3072] weight, writing BF16 [18432, 9216].  Two
+    activation batches and two weights alternate (226 MB + 36 MB, plus a
+    340 MB output per step, all beyond the 126 MB L2).  Per-kernel CUDA
+    events on the launching stream give the quantizer's GB/s and the GEMM's
+    TFLOP/s; the step without events gives the pair's throughput."""
+    w = workloads.WORKLOADS["qkv4"]
+    M, N, K = w.M, w.N, w.K
+    xs = [workloads.activation("qkv4", seed=40 + i).to(device) for i in range(rotate)]
+    wq = [nvq.quantize_weight("nvfp4", workloads.weight("qkv4", seed=50 + i).to(device)) for i in range(rotate)]
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+    sf = torch.empty(nvq.scale_bytes("nvfp4", M, K), dtype=torch.uint8, device=device)
+    g = torch.empty(1, dtype=torch.float32, device=device)
+    ws = nvq.new_workspace(device)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    flops = 2.0 * M * N * K
+    qbytes = M * K * ACT_BYTES_PER_ELEM + 4
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+
+    def quant(i):
+        nvq.nvfp4_quantize(xs[i % rotate], codes, sf, g, workspace=ws, stream=stream)
+
+    def gemm(i):
+        wc, wsf, wg = wq[i % rotate]
+        nvq.block_scaled_linear("nvfp4", codes, sf, g, wc, wsf, wg, M, N, K, out=out, stream=stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+    for i in range(5 + iters):
+        e = evs[i - 5] if i >= 5 else None
+        if e:
+            e[0].record(stream)
+        quant(i)
+        if e:
+            e[1].record(stream)
+        gemm(i)
+        if e:
+            e[2].record(stream)
+    torch.cuda.synchronize(device)
+    q_us = statistics.mean(e[0].elapsed_time(e[1]) * 1e3 for e in evs)
+    g_us = statistics.mean(e[1].elapsed_time(e[2]) * 1e3 for e in evs)
+    step_us = _back_to_back_us(lambda i: (quant(i), gemm(i)), iters, device, stream)
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    return {"workload": "NVFP4 QKV projection at batch 4: A BF16 [18432,3072] 0.5*StudentT(3), "
+                        "W BF16 [9216,3072] N(0,0.02), out BF16 [18432,9216]; dynamic per-tensor activation scale",
+            "M": M, "N": N, "K": K,
+            "l2": "%d activation batches (%.0f MB) and %d weights alternate; %.0f MB output per step"
+                  % (rotate, rotate * M * K * 2 / 1e6, rotate, M * N * 2 / 1e6),
+            "step_us": round(step_us, 3), "step_tflops": round(flops / (step_us * 1e-6) / 1e12, 1),
+            "gemm_kernel": gemm_kernel_name(nvq, "nvfp4", M, N, K),
+            "gemm_us": round(g_us, 3), "gemm_tflops": round(flops / (g_us * 1e-6) / 1e12, 1),
+            "gemm_frac_fp4": round(flops / (g_us * 1e-6) / 1e12 / fp4_peak, 4), "fp4_peak": round(fp4_peak, 1),
+            "quant_us": round(q_us, 3), "quant_gbs": round(qbytes / (q_us * 1e-6) / 1e9, 1),
+            "quant_frac_hbm": round(qbytes / (q_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+            "quant_launches": nvfp4_quant_launches(M, K, sms),
+            "per_kernel_timing": "CUDA events around each launch on the launching stream, %d steps" % iters}
+
+
 def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200, graph_steps=20, rotate=10):
     """Short batches of the FF-up linear (N 12288, K 3072, NVFP4): latency of
     one quantize + GEMM step issued eagerly (back to back, GPU held behind the
@@ -707,6 +769,51 @@ def run_reference(args):
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# --------------------------------------------------------------------------- ncu captures
+
+def run_profile(leg, iters, device):
+    """A fixed, short run of one leg's launches for an ncu capture: one
+    warm-up call, then `iters` calls, each synchronized.  Prints one line."""
+    import microscaling_quantized_linear_b200 as nvq
+
+    stream = torch.cuda.current_stream(device)
+    name = {"ffup": "ffup", "qkv4": "qkv4", "actq": "actq", "fused": "ffup", "m1": "ffup"}[leg]
+    w = workloads.WORKLOADS[name]
+    M, K = (1 if leg == "m1" else w.M), w.K
+    x = workloads.activation(name, seed=60, M=M).to(device)
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+    sf = torch.empty(nvq.scale_bytes("nvfp4", M, K), dtype=torch.uint8, device=device)
+    g = torch.empty(1, dtype=torch.float32, device=device)
+    ws = nvq.new_workspace(device)
+    if leg == "actq":
+        def call():
+            nvq.nvfp4_quantize(x, codes, sf, g, workspace=ws, stream=stream)
+    else:
+        N = w.N
+        wc, wsf, wg = nvq.quantize_weight("nvfp4", workloads.weight(name, seed=61).to(device))
+        if leg == "fused":
+            yc = torch.empty((M, N), dtype=torch.uint8, device=device)
+            ys = torch.empty(nvq.scale_bytes("mxfp8", M, N), dtype=torch.uint8, device=device)
+
+            def call():
+                nvq.nvfp4_quantize(x, codes, sf, g, workspace=ws, stream=stream)
+                nvq.block_scaled_linear_gelu_mxfp8("nvfp4", codes, sf, g, wc, wsf, wg, M, N, K, y_codes=yc,
+                                                   y_scales=ys, stream=stream)
+        else:
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+
+            def call():
+                nvq.nvfp4_quantize(x, codes, sf, g, workspace=ws, stream=stream)
+                nvq.block_scaled_linear("nvfp4", codes, sf, g, wc, wsf, wg, M, N, K, out=out, stream=stream)
+    for _ in range(1 + iters):
+        call()
+        torch.cuda.synchronize(device)
+    status = nvq.device_status()
+    print(json.dumps({"profile": leg, "iters": iters, "M": M, "K": K, "device_status": status}), flush=True)
+    if status != 0:
+        raise SystemExit("device status %d" % status)
+
+
 # --------------------------------------------------------------------------- main
 
 def main():
@@ -720,6 +827,10 @@ def main():
     ap.add_argument("--no-small-m", dest="small_m", action="store_false")
     ap.add_argument("--no-ff-block", dest="ff_block", action="store_false")
     ap.add_argument("--no-act-quant", dest="act_quant", action="store_false")
+    ap.add_argument("--no-qkv4", dest="qkv4", action="store_false")
+    ap.add_argument("--profile", choices=["ffup", "qkv4", "actq", "fused", "m1"], default=None,
+                    help="run only this leg's launches (one warm-up call + --iters calls) for an ncu capture")
+    ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -731,6 +842,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.profile:
+        torch.cuda.set_device(local)
+        run_profile(args.profile, args.iters, torch.device("cuda", local))
         return
 
     torch.cuda.set_device(local)
