@@ -13,13 +13,19 @@
 //   (from its MMA warp); the MMA commits arrive on the barriers of both CTAs
 //   (.multicast::cluster on the commit).
 //   Both CTAs' tile loads complete on the leader's barriers (.cta_group::2
-//   tensor loads; no load multicast anywhere): the scale tiles on sfdata[s],
-//   which only the copy warps wait for, and the A and B tiles on full[s],
-//   which also counts the copy warps' commits.  The MMA lane therefore waits
-//   once per stage: it issues the MMAs one after another (the tensor pipe
-//   holds little more than one in flight), so every barrier check in its
-//   loop is time the pipe stands idle.  Stage s owns scale slot s in tensor
-//   memory, and one commit per stage frees both.
+//   tensor loads; no load multicast anywhere).  The A and B tiles of a
+//   stage land on full[s], which also counts the copy warps' commits, so
+//   the MMA lane waits once per stage: it issues the MMAs one after another
+//   (the tensor pipe holds little more than one in flight), so every barrier
+//   check in its loop is time the pipe stands idle.  Stage s owns scale slot
+//   s in tensor memory, and one commit per stage frees both.
+//   The scale tiles travel apart from A and B: a producer warp of their own
+//   fills a ring of scale slots in shared memory (longer than the stages)
+//   as soon as the copies out of a slot have completed, so a stage's scales
+//   are in shared memory well before its tensor-memory slot frees, and the
+//   copy warps move them the moment it does.  The copy path (scale load,
+//   wake-up, twelve tcgen05.cp per stage, completion) otherwise sat on the
+//   critical path of every stage.
 //   Each CTA drains its own accumulator half; the peer's epilogue warps
 //   arrive remotely on the leader's accumulator-empty barrier.
 // Per SM this halves the B bytes staged from L2 and the tensor-core
@@ -53,33 +59,45 @@ struct PairCfg {
     static constexpr int SFB_BYTES = SFB_H * SF_CHUNK;
     static constexpr int AB_BYTES = A_BYTES + B_BYTES;                    // per CTA per stage
     static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;                  // per CTA per stage
-    static constexpr int STAGE_BYTES = (AB_BYTES + SF_BYTES + 1023) / 1024 * 1024;
+    // The A/B tiles of a stage and its scale tiles live apart: stages of
+    // A and B, and a longer ring of scale slots that runs ahead of them, so
+    // the copies of a stage's scales into tensor memory can start the moment
+    // its tensor-memory slot is free instead of after a load issued then.
+    static constexpr int STAGE_BYTES = (AB_BYTES + 1023) / 1024 * 1024;
     static constexpr int OFF_B = A_BYTES;
-    static constexpr int OFF_SFA = A_BYTES + B_BYTES;
-    static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
+    static constexpr int SF_SLOT_BYTES = (SF_BYTES + 127) / 128 * 128;
+    static constexpr int OFF_SFA = 0;                        // within a scale slot
+    static constexpr int OFF_SFB = SFA_BYTES;
     static constexpr int EPI_BUF_BYTES = 32 * 64;
     static constexpr int EPI_BYTES = kEpiWarps * EPI_BUF_BYTES;
+    static constexpr int BAR_BYTES = 1024;
     static constexpr int SMEM_LIMIT = 232448;
-    static constexpr int FIXED_BYTES = 1024 + 512 + EPI_BYTES;
+    static constexpr int FIXED_BYTES = 1024 /*align*/ + BAR_BYTES + EPI_BYTES;
     static constexpr int SFA_COLS = FMT == 0 ? 4 * KSTEPS : 4;
     static constexpr int SFB_COLS_PER_MMA = 4 * SFB_H;
     static constexpr int SFB_COLS = FMT == 0 ? SFB_COLS_PER_MMA * KSTEPS : SFB_COLS_PER_MMA;
     static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
-    // Each pipeline stage owns one tensor-memory scale slot, so the stage
-    // count is bounded by shared memory and by the columns left beside the
-    // accumulator(s).  Two accumulators only when at least 4 slots remain.
-    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
+    // Each stage owns one tensor-memory scale slot, so the stage count is
+    // bounded by the columns left beside the accumulator(s) and by shared
+    // memory with at least kMinRing scale slots; the ring takes what is
+    // left.  Two accumulators only when at least 4 slots remain.
+    static constexpr int kMinRing = 8;
+    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES - kMinRing * SF_SLOT_BYTES) / STAGE_BYTES;
     static constexpr int ACC_BUFS = (512 - 2 * BN) / SF_COLS >= 4 ? 2 : 1;
     static constexpr int SLOTS_FIT = (512 - ACC_BUFS * BN) / SF_COLS;
     static constexpr int STAGES_MIN2 = STAGES_FIT < SLOTS_FIT ? STAGES_FIT : SLOTS_FIT;
     static constexpr int STAGES = STAGES_MIN2 > 8 ? 8 : STAGES_MIN2;
-    static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
+    static constexpr int RING_FIT = (SMEM_LIMIT - FIXED_BYTES - STAGES * STAGE_BYTES) / SF_SLOT_BYTES;
+    static constexpr int SF_RING = RING_FIT > 16 ? 16 : RING_FIT;
+    static constexpr int OFF_SF = STAGES * STAGE_BYTES;
+    static constexpr int OFF_EPI = (OFF_SF + SF_RING * SF_SLOT_BYTES + 1023) / 1024 * 1024;
+    static constexpr int SMEM_BYTES = OFF_EPI + EPI_BYTES + BAR_BYTES + 1024 /*align*/;
     static constexpr int TM_SF = ACC_BUFS * BN;
     static constexpr int TM_USED = ACC_BUFS * BN + STAGES * SF_COLS;
     static constexpr int TM_COLS = TM_USED <= 256 ? 256 : 512;
     static constexpr int SF_WARPS = 1 + SFB_H;             // copy warps (used in the leader)
-    static constexpr int THREADS = 32 * (kFirstSfWarp + SF_WARPS);
+    static constexpr int SCALE_WARP = kFirstSfWarp + SF_WARPS;   // loads the scale tiles (both CTAs)
+    static constexpr int THREADS = 32 * (SCALE_WARP + 1);
     static constexpr uint32_t IDESC =
         (FMT != 1 ? (1u << 7) | (1u << 10) : 0u) |   // A, B type: E2M1 (NVFP4) / E5M2 (FMT 2); 0 = E4M3
         ((uint32_t)(BN >> 3) << 17) |
@@ -88,7 +106,9 @@ struct PairCfg {
     static_assert(BN == 256 || BN == 192, "pair tiles are 256 x 256 or 256 x 192");
     static_assert(TM_USED <= 512, "tensor memory overflow");
     static_assert(STAGES >= 4, "too few pipeline stages");
+    static_assert(SF_RING >= STAGES, "the scale ring must be at least as long as the stages");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory overflow");
+    static_assert((2 * STAGES + 2 * SF_RING + 6) * 8 + 12 <= BAR_BYTES, "barrier area");
 };
 
 // EPI as in bsgemm_kernel: 0 writes D, 1 writes MXFP8 codes and scales of GELU(D).
@@ -102,20 +122,23 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
-    // full[s]:   A and B tiles of both CTAs landed (tx) + the scale copies
-    //            into slot s committed (one arrival per copy warp): the MMA
-    //            warp's single wait per stage
-    // sfdata[s]: both CTAs' scale tiles landed (tx): the copy warps' wait
-    // empty[s]:  the stage's MMAs completed (commit multicast to both CTAs):
-    //            frees shared-memory stage s and tensor-memory scale slot s
+    // full[s]:     A and B tiles of both CTAs landed (tx) + the scale copies
+    //              into slot s committed (one arrival per copy warp): the MMA
+    //              warp's single wait per stage
+    // empty[s]:    the stage's MMAs completed (commit multicast to both CTAs):
+    //              frees shared-memory stage s and tensor-memory scale slot s
+    // sffull[r]:   both CTAs' scale tiles in ring slot r landed (tx)
+    // sfempty[r]:  the copies out of ring slot r completed (commits
+    //              multicast to both CTAs, one per copy warp): frees slot r
     const uint32_t full0 = smem_u32(bars);
     const uint32_t empty0 = full0 + 8 * C::STAGES;
-    const uint32_t sfdata0 = empty0 + 8 * C::STAGES;
-    const uint32_t tfull0 = sfdata0 + 8 * C::STAGES;
+    const uint32_t sffull0 = empty0 + 8 * C::STAGES;
+    const uint32_t sfempty0 = sffull0 + 8 * C::SF_RING;
+    const uint32_t tfull0 = sfempty0 + 8 * C::SF_RING;
     const uint32_t tempty0 = tfull0 + 8 * 2;
     const uint32_t drain = tempty0 + 8 * 2;
     const uint32_t sfdrain = drain + 8;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 6);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 2 * C::SF_RING + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* never = abort_flag + 1;
 
@@ -126,7 +149,10 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(full0 + 8 * s, 1 + C::SF_WARPS);
             mbar_init(empty0 + 8 * s, 1);
-            mbar_init(sfdata0 + 8 * s, 1);
+        }
+        for (int r = 0; r < C::SF_RING; ++r) {
+            mbar_init(sffull0 + 8 * r, 1);
+            mbar_init(sfempty0 + 8 * r, C::SF_WARPS);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
@@ -171,8 +197,6 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                 const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
                 const int32_t arow = (int32_t)(mb * 256 + 128 * rank);
                 const int32_t brow = (int32_t)(nb * BN + C::BN_HALF * rank);
-                const uint32_t sfa_atom = mb * 2 + rank;              // this CTA's 128 A rows
-                const uint32_t sfb_atom = (nb * BN) / 128;            // first scale tile of the B tile
                 for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt) {
                     const uint32_t s = it % C::STAGES, use = it / C::STAGES;
                     if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, abort_flag, p.wait_ns)) {
@@ -180,20 +204,8 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
                         break;
                     }
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
-                    const uint32_t fb = mapa_shared(full0 + 8 * s, 0);     // the leader's barriers
-                    const uint32_t sb = mapa_shared(sfdata0 + 8 * s, 0);
-                    if (rank == 0) {
-                        mbar_arrive_expect_tx(sfdata0 + 8 * s, 2 * C::SF_BYTES);
-                        mbar_arrive_expect_tx(full0 + 8 * s, 2 * C::AB_BYTES);
-                    }
-                    // scale tiles first (the copy warps need them before the
-                    // MMAs can run); the tensors are viewed as rows of 256 bytes
-                    tma_load_2d_pair(st + C::OFF_SFA, &tmap_sfa, sb, 0,
-                                     (int32_t)(((size_t)sfa_atom * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 2));
-#pragma unroll
-                    for (int h = 0; h < C::SFB_H; ++h)
-                        tma_load_2d_pair(st + C::OFF_SFB + h * C::SF_CHUNK, &tmap_sfb, sb, 0,
-                                         (int32_t)(((size_t)(sfb_atom + h) * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 2));
+                    const uint32_t fb = mapa_shared(full0 + 8 * s, 0);     // the leader's barrier
+                    if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * C::AB_BYTES);
                     tma_load_2d_pair(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), arow);
                     tma_load_2d_pair(st + C::OFF_B, &tmap_b, fb, (int32_t)(kt * C::KBYTES), brow);
                     ++it;
@@ -205,10 +217,8 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             }
             // Neither CTA leaves while a load it issued may still be in flight.
             if (rank == 0) {    // the leader's barriers count both CTAs' bytes: wait for the last stages
-                for (uint32_t j = it > (uint32_t)C::STAGES ? it - C::STAGES : 0; j < it; ++j) {
-                    mbar_wait_bounded(sfdata0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
+                for (uint32_t j = it > (uint32_t)C::STAGES ? it - C::STAGES : 0; j < it; ++j)
                     mbar_wait_bounded(full0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1, never, kWaitLimitNs);
-                }
             } else {
                 // The peer's loads complete on the leader's barriers, which it
                 // cannot wait on; the MMAs that consume a stage complete only
@@ -271,6 +281,52 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             tc_commit_pair(drain);
             mbar_wait_bounded(drain, 0, never, kWaitLimitNs);
         }
+    } else if (warp == C::SCALE_WARP) {
+        // ---------------------------------------------------------- scale-tile producer (both CTAs)
+        // Runs up to SF_RING stages ahead: a ring slot is reloaded as soon
+        // as the copies out of it have completed.
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (uint32_t tile = pair; tile < num_tiles && ok; tile += npairs) {
+                const uint32_t mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+                const uint32_t sfa_atom = mb * 2 + rank;              // this CTA's 128 A rows
+                const uint32_t sfb_atom = (nb * BN) / 128;            // first scale tile of the B tile
+                for (uint32_t kt = 0; kt < p.num_k_tiles; ++kt) {
+                    const uint32_t r = it % C::SF_RING, ru = it / C::SF_RING;
+                    if (ru > 0 && !mbar_wait_bounded(sfempty0 + 8 * r, (ru - 1) & 1, abort_flag, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t slot = smem_u32(smem + C::OFF_SF + r * C::SF_SLOT_BYTES);
+                    const uint32_t sb = mapa_shared(sffull0 + 8 * r, 0);   // the leader's barrier
+                    if (rank == 0) mbar_arrive_expect_tx(sffull0 + 8 * r, 2 * C::SF_BYTES);
+                    // the scale tensors are viewed as rows of 256 bytes
+                    tma_load_2d_pair(slot + C::OFF_SFA, &tmap_sfa, sb, 0,
+                                     (int32_t)(((size_t)sfa_atom * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 2));
+#pragma unroll
+                    for (int h = 0; h < C::SFB_H; ++h)
+                        tma_load_2d_pair(slot + C::OFF_SFB + h * C::SF_CHUNK, &tmap_sfb, sb, 0,
+                                         (int32_t)(((size_t)(sfb_atom + h) * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 2));
+                    ++it;
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+            }
+            // Its own loads must land before the CTA leaves: the leader's
+            // ring barriers count both CTAs' bytes; the copies out of a slot
+            // complete only after its loads landed, and their commits reach
+            // both CTAs' sfempty (after an abort they may never come: the
+            // bounded wait then ends long after any load has landed).
+            for (uint32_t j = it > (uint32_t)C::SF_RING ? it - C::SF_RING : 0; j < it; ++j) {
+                if (rank == 0)
+                    mbar_wait_bounded(sffull0 + 8 * (j % C::SF_RING), (j / C::SF_RING) & 1, never, kWaitLimitNs);
+                else
+                    mbar_wait_bounded(sfempty0 + 8 * (j % C::SF_RING), (j / C::SF_RING) & 1, never, kWaitLimitNs);
+            }
+        }
     } else if (warp >= kFirstSfWarp) {
         // ---------------------------------------------------------- scale-factor copy warps (leader)
         if (lane == 0 && rank == 0) {
@@ -278,16 +334,19 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
             bool ok = true;
             for (uint32_t it = 0; it < total_iters; ++it) {
                 const uint32_t s = it % C::STAGES, su = it / C::STAGES;
-                // slot s is free once the MMAs of its previous use completed
-                // (the same commit that freed the shared-memory stage)
+                const uint32_t r = it % C::SF_RING, ru = it / C::SF_RING;
+                // tensor-memory slot s is free once the MMAs of its previous
+                // use completed; ring slot r holds this stage's scale tiles
                 if ((su > 0 && !mbar_wait_bounded(empty0 + 8 * s, (su - 1) & 1, abort_flag, p.wait_ns)) ||
-                    !mbar_wait_bounded(sfdata0 + 8 * s, su & 1, abort_flag, p.wait_ns)) {
+                    !mbar_wait_bounded(sffull0 + 8 * r, ru & 1, abort_flag, p.wait_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                sf_copy_job<C, true>(job, smem_u32(smem + s * C::STAGE_BYTES), tmem + C::TM_SF + s * C::SF_COLS);
+                sf_copy_job<C, true>(job, smem_u32(smem + C::OFF_SF + r * C::SF_SLOT_BYTES),
+                                     tmem + C::TM_SF + s * C::SF_COLS);
                 tc_commit_pair(full0 + 8 * s);               // the copies' share of the MMA's wait
+                tc_commit_pair_mc(sfempty0 + 8 * r, 0x3);    // ring slot r free in both CTAs
             }
             if (!ok) {
                 *abort_flag = 1;
