@@ -621,6 +621,7 @@ def run_qkv4_component(nvq, device, stream, peaks, rotate=2, iters=40):
     q_us = statistics.mean(e[0].elapsed_time(e[1]) * 1e3 for e in evs)
     g_us = statistics.mean(e[1].elapsed_time(e[2]) * 1e3 for e in evs)
     step_us = _back_to_back_us(lambda i: (quant(i), gemm(i)), iters, device, stream)
+    alone_us = _back_to_back_us(quant, 4 * iters, device, stream)
     sms = torch.cuda.get_device_properties(device).multi_processor_count
     return {"workload": "NVFP4 QKV projection at batch 4: A BF16 [18432,3072] 0.5*StudentT(3), "
                         "W BF16 [9216,3072] N(0,0.02), out BF16 [18432,9216]; dynamic per-tensor activation scale",
@@ -634,6 +635,11 @@ def run_qkv4_component(nvq, device, stream, peaks, rotate=2, iters=40):
             "quant_us": round(q_us, 3), "quant_gbs": round(qbytes / (q_us * 1e-6) / 1e9, 1),
             "quant_frac_hbm": round(qbytes / (q_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
             "quant_launches": nvfp4_quant_launches(M, K, sms),
+            "quant_alone_us": round(alone_us, 3), "quant_alone_gbs": round(qbytes / (alone_us * 1e-6) / 1e9, 1),
+            "quant_alone_frac_hbm": round(qbytes / (alone_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+            "quant_note": "quant_us is the quantizer's event interval inside the quantize + GEMM step, which also "
+                          "holds the write-back of the previous GEMM's 340 MB output; quant_alone_us is calls back to "
+                          "back over the two activation batches",
             "per_kernel_timing": "CUDA events around each launch on the launching stream, %d steps" % iters}
 
 

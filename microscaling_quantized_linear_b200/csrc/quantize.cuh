@@ -186,10 +186,24 @@ amax_partials_kernel(const uint4* __restrict__ x, uint32_t rows, uint32_t vecs_p
 }
 
 // ------------------------------------------------------------------ NVFP4, streaming
-// One thread = two 16-element blocks per iteration (b and b + stride, both
+// One thread = two 16-element blocks per iteration (b and b - stride, both
 // loaded before either is computed).  Block b is (row b / nblk, column
 // b % nblk), nblk = K / 16; its codes are bytes [8b, 8b + 8).  The amax is the
 // reduction of the two-pass partials, or *calib_amax.
+// The grid walks the tensor from its end to its start: after the amax pass,
+// which reads x from start to end, the rows read last are the likeliest
+// still in L2, so they are quantized first.  Within a warp the blocks stay
+// in ascending order (the scale gather below needs four neighbours).
+__device__ __forceinline__ void block_step_down(uint32_t& r, uint32_t& c, uint32_t qs, uint32_t rs, uint32_t nblk) {
+    if (c < rs) {
+        c += nblk - rs;
+        r -= qs + 1;
+    } else {
+        c -= rs;
+        r -= qs;
+    }
+}
+
 __global__ void __launch_bounds__(kQuantThreads, 6)
 nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nblk, uint32_t ldx,
                       uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ g_dec_out,
@@ -200,14 +214,16 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
     const uint32_t total = rows * nblk;
     const uint32_t stride = gridDim.x * kQuantThreads;
     const uint32_t qs = stride / nblk, rs = stride - qs * nblk;
-    uint32_t b = blockIdx.x * kQuantThreads + threadIdx.x;
+    // This thread's blocks are b0 + k * stride; the CTA walks k from its
+    // last (nk - 1) down to 0, two per iteration: b = b0 + k * stride and
+    // b1 = b - stride.  Only at k = nk - 1 can b lie past the end.
+    const uint32_t base_cta = blockIdx.x * kQuantThreads;
+    const uint32_t nk = total > base_cta ? (total - base_cta + stride - 1) / stride : 0;
+    int32_t k = (int32_t)nk - 1;
+    uint32_t b = base_cta + threadIdx.x + (uint32_t)(k > 0 ? k : 0) * stride;
     uint32_t r = b / nblk, c = b - r * nblk;
-    // Each iteration handles blocks b and b + stride; (r1, c1) is the second.
-    uint32_t r1 = r + qs, c1 = c + rs;
-    if (c1 >= nblk) {
-        c1 -= nblk;
-        ++r1;
-    }
+    uint32_t r1 = r, c1 = c;
+    block_step_down(r1, c1, qs, rs, nblk);       // block b - stride (not used when k < 1)
     // Calibrated: x may come from the previous grid, so nothing is read
     // before it has completed.  Dynamic: the previous grid is this call's amax
     // pass, which only reads x and lets this grid start once it has itself
@@ -216,12 +232,13 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
     uint4 v[4];
     const uint4 zero4 = make_uint4(0, 0, 0, 0);
     {
+        const bool a0 = k >= 0 && b < total, a1 = k >= 1;
         const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
         const uint4* s1 = reinterpret_cast<const uint4*>(x + (size_t)r1 * ldx + (size_t)c1 * 16);
-        v[0] = b < total ? __ldg(s0) : zero4;
-        v[1] = b < total ? __ldg(s0 + 1) : zero4;
-        v[2] = b + stride < total ? __ldg(s1) : zero4;
-        v[3] = b + stride < total ? __ldg(s1 + 1) : zero4;
+        v[0] = a0 ? __ldg(s0) : zero4;
+        v[1] = a0 ? __ldg(s0 + 1) : zero4;
+        v[2] = a1 ? __ldg(s1) : zero4;
+        v[3] = a1 ? __ldg(s1 + 1) : zero4;
     }
     init_d6(d6);
     // x is final (the amax pass that may still be running only reads it);
@@ -235,7 +252,7 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
         uint32_t m = 0;
         for (uint32_t i = threadIdx.x; i < npartial; i += kQuantThreads) m = max(m, partial[i]);
         m = block_max_u32<kQuantThreads>(m, red);
-        if (m >= 0x7F80u && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, 2u);
+        if (m >= 0x7F80u && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, kStatusNonfinite);
         amax = __uint_as_float(m << 16);
     }
     const float g_enc = encode_scale(amax);
@@ -244,20 +261,20 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
     __syncthreads();
 
     const uint32_t ctiles = nblk >> 2;
-    const uint32_t stride2 = 2 * stride, qs2 = stride2 / nblk, rs2 = stride2 - qs2 * nblk;
-    for (bool first = true; b - threadIdx.x < total; first = false) {
+    for (bool first = true; k >= 0; k -= 2, first = false) {
+        const bool a0 = b < total, a1 = k >= 1;      // whole warps stay in the loop for the shuffles
         if (!first) {
             const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
             const uint4* s1 = reinterpret_cast<const uint4*>(x + (size_t)r1 * ldx + (size_t)c1 * 16);
-            v[0] = b < total ? __ldg(s0) : zero4;
-            v[1] = b < total ? __ldg(s0 + 1) : zero4;
-            v[2] = b + stride < total ? __ldg(s1) : zero4;
-            v[3] = b + stride < total ? __ldg(s1 + 1) : zero4;
+            v[0] = a0 ? __ldg(s0) : zero4;
+            v[1] = a0 ? __ldg(s0 + 1) : zero4;
+            v[2] = a1 ? __ldg(s1) : zero4;
+            v[3] = a1 ? __ldg(s1 + 1) : zero4;
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const uint32_t bu = b + u * stride, ru = u ? r1 : r, cu = u ? c1 : c;
-            const bool active = bu < total;   // whole warps stay in the loop for the shuffles
+            const uint32_t bu = u ? b - stride : b, ru = u ? r1 : r, cu = u ? c1 : c;
+            const bool active = u ? a1 : a0;
             const uint4 p0 = v[2 * u], p1 = v[2 * u + 1];
             const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
             uint32_t lo, hi;
@@ -273,18 +290,14 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
                         sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
             }
         }
-        b += stride2;
-        r += qs2;
-        c += rs2;
-        if (c >= nblk) {
-            c -= nblk;
-            ++r;
-        }
-        r1 += qs2;
-        c1 += rs2;
-        if (c1 >= nblk) {
-            c1 -= nblk;
-            ++r1;
+        if (k >= 2) {                                // the next pair: b - 2 stride, b - 3 stride
+            b -= 2 * stride;
+            r = r1;
+            c = c1;
+            block_step_down(r, c, qs, rs, nblk);
+            r1 = r;
+            c1 = c;
+            block_step_down(r1, c1, qs, rs, nblk);
         }
     }
     zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kQuantThreads + threadIdx.x, stride);
@@ -441,16 +454,15 @@ __device__ __forceinline__ uint32_t cta_tensor_absmax(const uint16_t* __restrict
     return block_max_u32<kFusedThreads>(fold2(m2), red);
 }
 
-// Two 16-byte halves of the 32-byte block at smem byte offset 32*b.  Threads
-// 4..7 of every 8 read the halves in the opposite order, which makes each
-// 8-thread shared-memory phase touch 8 distinct 4-bank groups.
-__device__ __forceinline__ void lds_block32(const uint8_t* base, uint32_t b, uint4& v0, uint4& v1) {
-    const uint4* p = reinterpret_cast<const uint4*>(base + (size_t)b * 32);
-    const uint32_t sw = (threadIdx.x >> 2) & 1u;
-    const uint4 first = p[sw];
-    const uint4 second = p[sw ^ 1u];
-    v0 = sw ? second : first;
-    v1 = sw ? first : second;
+// Shared-memory layout of the one-pass kernel's tile: the CTA's rows in
+// row-major order, cut into 64-byte groups of two 16-element blocks (blocks
+// 2g and 2g + 1), the four 16-byte chunks of group g stored in the order
+// chunk ^ ((g >> 1) & 3).  A warp whose consecutive lanes read the same chunk
+// of consecutive groups then touches eight different 16-byte bank groups in
+// every quarter-warp phase, and each thread reads its chunks in their logical
+// order.  Block b's two halves are its group's chunks 2(b & 1) and 2(b & 1) + 1.
+__device__ __forceinline__ uint32_t group_chunk(uint32_t g, uint32_t k) {
+    return 64u * g + 16u * (k ^ ((g >> 1) & 3u));
 }
 
 // Shared memory the one-pass kernel needs for rows_per_cta rows of K: the
@@ -491,9 +503,9 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
         if (b < total) {
             const uint32_t rl = b / nblk, c = b - rl * nblk;
             const uint16_t* src = x + (size_t)(r0 + rl) * ldx + (size_t)c * 16;
-            const uint32_t dst = smem_u32(tile + (size_t)b * 32);
-            cp_async16(dst, src);
-            cp_async16(dst + 16, src + 8);
+            const uint32_t t0 = smem_u32(tile);
+            cp_async16(t0 + group_chunk(b >> 1, 2 * (b & 1)), src);          // the block's two halves,
+            cp_async16(t0 + group_chunk(b >> 1, 2 * (b & 1) + 1), src + 8);  // one 32-byte source
         }
         cp_async_commit();
     }
@@ -525,8 +537,8 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
         }
         const uint32_t b = threadIdx.x + (uint32_t)i * kFusedThreads;
         if (b < total) {
-            uint4 v0, v1;
-            lds_block32(tile, b, v0, v1);
+            const uint4 v0 = *reinterpret_cast<const uint4*>(tile + group_chunk(b >> 1, 2 * (b & 1)));
+            const uint4 v1 = *reinterpret_cast<const uint4*>(tile + group_chunk(b >> 1, 2 * (b & 1) + 1));
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
             const uint32_t mb = block16_max(w);
             bdiv6[b] = div6(mb, d6);           // the scale's first step, done while copies land
@@ -593,13 +605,18 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
     init_rtab(rtab, g_enc);
     __syncthreads();
 
-    // Two blocks per thread per iteration (b and b + kFusedThreads), both
-    // read before either is computed.
+    // Encode: thread t takes the 2-block groups g = t, t + 1024, ..., two
+    // groups per iteration, both read before either is computed.  A group's
+    // 16 code bytes leave in one store; the 4 scale bytes of blocks 4j ..
+    // 4j + 3 (groups 2j, 2j + 1: lanes l, l + 1) in one 32-bit store by the
+    // even lane.  Groups never straddle rows (K / 16 is a multiple of 4).
     const uint32_t ctiles = nblk >> 2;
-    const uint32_t qs = kFusedThreads / nblk, rs = kFusedThreads - qs * nblk;
-    uint32_t rl = threadIdx.x / nblk, c = threadIdx.x - rl * nblk;
-    const size_t code_base = (size_t)r0 * nblk * 8;
-    for (uint32_t base = 0; base < total; base += 2 * kFusedThreads) {
+    const uint32_t ngroups = total >> 1;
+    const uint32_t qs = 2 * kFusedThreads / nblk, rs = 2 * kFusedThreads - qs * nblk;   // one group stride, in blocks
+    uint32_t rl = 2 * threadIdx.x / nblk, c = 2 * threadIdx.x - rl * nblk;            // first block of group t
+    const float2* bd2 = reinterpret_cast<const float2*>(bdiv6);
+    uint8_t* code_cta = codes + (size_t)r0 * nblk * 8;
+    for (uint32_t base = 0; base < ngroups; base += 2 * kFusedThreads) {
         uint32_t rlu[2], cu[2];
         rlu[0] = rl;
         cu[0] = c;
@@ -609,37 +626,40 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
             cu[1] -= nblk;
             ++rlu[1];
         }
-        uint4 v[4];
-        float d[2];
+        uint4 v[2][4];
+        float2 d[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const uint32_t b = base + u * kFusedThreads + threadIdx.x;
-            v[2 * u] = v[2 * u + 1] = make_uint4(0, 0, 0, 0);
-            d[u] = 0.0f;
-            if (b < total) {
-                lds_block32(tile, b, v[2 * u], v[2 * u + 1]);
-                d[u] = bdiv6[b];
+            const uint32_t g = base + u * kFusedThreads + threadIdx.x;
+            d[u] = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[u][k] = make_uint4(0, 0, 0, 0);
+            if (g < ngroups) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[u][k] = *reinterpret_cast<const uint4*>(tile + group_chunk(g, k));
+                d[u] = bd2[g];
             }
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const uint32_t b = base + u * kFusedThreads + threadIdx.x;
-            const bool active = b < total;           // whole warps stay for the shuffles
-            const uint32_t w[8] = {v[2 * u].x, v[2 * u].y, v[2 * u].z, v[2 * u].w,
-                                   v[2 * u + 1].x, v[2 * u + 1].y, v[2 * u + 1].z, v[2 * u + 1].w};
-            uint32_t lo, hi;
-            const uint32_t sc = nvfp4_block_d(d[u], w, g_enc, rtab, lo, hi);
-            const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
-            const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
-            const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
+            const uint32_t g = base + u * kFusedThreads + threadIdx.x;
+            const bool active = g < ngroups;         // whole warps stay for the shuffle
+            const uint32_t w0[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                                    v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+            const uint32_t w1[8] = {v[u][2].x, v[u][2].y, v[u][2].z, v[u][2].w,
+                                    v[u][3].x, v[u][3].y, v[u][3].z, v[u][3].w};
+            uint32_t lo0, hi0, lo1, hi1;
+            const uint32_t sc0 = nvfp4_block_d(d[u].x, w0, g_enc, rtab, lo0, hi0);
+            const uint32_t sc1 = nvfp4_block_d(d[u].y, w1, g_enc, rtab, lo1, hi1);
+            const uint32_t pair = sc0 | (sc1 << 8);
+            const uint32_t next = __shfl_down_sync(0xFFFFFFFFu, pair, 1);
             if (active) {
-                *reinterpret_cast<uint2*>(codes + code_base + (size_t)b * 8) = make_uint2(lo, hi);
-                if ((cu[u] & 3u) == 0)
-                    *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r0 + rlu[u], cu[u], ctiles)) =
-                        sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+                *reinterpret_cast<uint4*>(code_cta + (size_t)g * 16) = make_uint4(lo0, hi0, lo1, hi1);
+                if ((g & 1u) == 0)
+                    *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r0 + rlu[u], cu[u], ctiles)) = pair | (next << 16);
             }
         }
-        // advance by two strides
+        // advance by two group strides
         rl = rlu[1] + qs;
         c = cu[1] + rs;
         if (c >= nblk) {
