@@ -783,6 +783,23 @@ def run_profile(leg, iters, device):
     import microscaling_quantized_linear_b200 as nvq
 
     stream = torch.cuda.current_stream(device)
+    if leg == "ffdown":
+        w = workloads.WORKLOADS["ffdown"]
+        M, N, K = w.M, w.N, w.K
+        x = workloads.activation("ffdown", seed=60).to(device)
+        wc, wsf, _ = nvq.quantize_weight("mxfp8", workloads.weight("ffdown", seed=61).to(device))
+        codes = torch.empty((M, K), dtype=torch.uint8, device=device)
+        sf = torch.empty(nvq.scale_bytes("mxfp8", M, K), dtype=torch.uint8, device=device)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        for _ in range(1 + iters):
+            nvq.mxfp8_quantize(x, codes, sf, stream=stream)
+            nvq.block_scaled_linear("mxfp8", codes, sf, None, wc, wsf, None, M, N, K, out=out, stream=stream)
+            torch.cuda.synchronize(device)
+        status = nvq.device_status()
+        print(json.dumps({"profile": leg, "iters": iters, "M": M, "K": K, "device_status": status}), flush=True)
+        if status != 0:
+            raise SystemExit("device status %d" % status)
+        return
     name = {"ffup": "ffup", "qkv4": "qkv4", "actq": "actq", "fused": "ffup", "m1": "ffup"}[leg]
     w = workloads.WORKLOADS[name]
     M, K = (1 if leg == "m1" else w.M), w.K
@@ -834,7 +851,7 @@ def main():
     ap.add_argument("--no-ff-block", dest="ff_block", action="store_false")
     ap.add_argument("--no-act-quant", dest="act_quant", action="store_false")
     ap.add_argument("--no-qkv4", dest="qkv4", action="store_false")
-    ap.add_argument("--profile", choices=["ffup", "qkv4", "actq", "fused", "m1"], default=None,
+    ap.add_argument("--profile", choices=["ffup", "qkv4", "actq", "fused", "m1", "ffdown"], default=None,
                     help="run only this leg's launches (one warm-up call + --iters calls) for an ncu capture")
     ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args()
