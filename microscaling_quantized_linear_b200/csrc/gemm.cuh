@@ -176,7 +176,10 @@ __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half,
     }
 }
 
-template <int FMT, int BN_>
+// Rows of the output that the split-K kernel takes (one short row block).
+constexpr uint32_t kSplitKRows = 32;
+
+template <int FMT, int BN_, bool SPLITK = false>
 struct GemmCfg {
     static constexpr int BM = 128;
     static constexpr int BN = BN_;
@@ -201,8 +204,14 @@ struct GemmCfg {
     // epilogue staging: 8 warps x (32 rows x 64 bytes)
     static constexpr int EPI_BUF_BYTES = 32 * 64;
     static constexpr int EPI_BYTES = kEpiWarps * EPI_BUF_BYTES;
+    // split-K: the receive area for the partial sums that the cluster's CTAs
+    // push here (kSplitKRows rows of BN FP32 values, plus the padding of
+    // the per-rank slots) takes the place of the staging area, which that
+    // kernel does not use
+    static constexpr int RECV_BYTES = SPLITK ? (int)kSplitKRows * BN * 4 + 2048 : 0;
+    static constexpr int EPI_AREA = EPI_BYTES > RECV_BYTES ? EPI_BYTES : RECV_BYTES;
     static constexpr int SMEM_LIMIT = 232448;
-    static constexpr int FIXED_BYTES = 1024 /*align*/ + 512 /*barriers*/ + EPI_BYTES;
+    static constexpr int FIXED_BYTES = 1024 /*align*/ + 512 /*barriers*/ + EPI_AREA;
     // tensor-memory columns: accumulator(s), then scale factors of A and B
     static constexpr int SFA_COLS = FMT == 0 ? 4 * KSTEPS : 4;
     static constexpr int SFB_COLS_PER_MMA = 4 * SFB_H;
@@ -271,72 +280,70 @@ struct GemmParams {
 };
 static_assert(sizeof(GemmParams) == 128, "GemmParams keeps its 128 bytes");
 
-// Split-K reduction for one output tile of at most 128 rows: every CTA of
-// the cluster holds its FP32 partial tile in its own shared memory, rows of
-// BN floats with the 16-byte groups of each 128-byte segment rotated by the
-// row (group f of row r at (f & ~7) | ((f ^ r) & 7)), so that the writes from
-// tensor memory (one row per thread) spread over all banks.  CTA `rank`
-// finishes the rank-th share of the tile's row-major 4-column groups: the
-// partials summed in rank order, times alpha, plus bias, rounded to BF16 and
-// stored.  Groups at columns >= n_total are not stored.  A thread takes
-// kReduceBatch groups at a time and reads them from one CTA after another
-// (its own partial with plain shared-memory loads), so that many
-// distributed-shared-memory loads are in flight at once.
-constexpr uint32_t kReduceBatch = 8;
+// Split-K exchange for one output tile of at most kSplitKRows rows.  The
+// tile's 4-column groups are numbered row-major (group idx = row * BN/4 +
+// column/4) and cut into `split` contiguous shares of `per` groups; CTA rank
+// r of the cluster finishes share r.  Every CTA pushes its FP32 partial of
+// share r into slot (its own rank) of CTA r's receive area; a slot covers
+// the share's aligned groups of eight, with group idx stored at position
+// (idx & ~7) | ((idx ^ row) & 7) from the share's first aligned group, so
+// that the pushes of one row per lane hit all banks.
+struct SplitShares {
+    uint32_t total, per, slot;   // groups in the tile, per share, per slot (16 bytes each)
+};
 
 template <int BN>
-__device__ __forceinline__ void splitk_reduce(uint32_t part, uint32_t rank, uint32_t split, uint32_t rows,
+__device__ __forceinline__ SplitShares split_shares(uint32_t rows, uint32_t split) {
+    SplitShares sh;
+    sh.total = rows * (BN / 4);
+    sh.per = (sh.total + split - 1) / split;
+    sh.slot = ((sh.per + 7) & ~7u) + 8;
+    return sh;
+}
+
+// Position (in 16-byte groups) of group idx, of tile row `row`, within its
+// slot; b8 = the owner's first group rounded down to a multiple of eight.
+__device__ __forceinline__ uint32_t split_pos(uint32_t idx, uint32_t row, uint32_t b8) {
+    return ((idx & ~7u) | ((idx ^ row) & 7u)) - b8;
+}
+
+// CTA `rank` finishes its share from its receive area (every slot filled):
+// the partials summed in rank order, times alpha, plus bias, rounded to BF16
+// and stored.  Groups at columns >= n_total are not stored.
+template <int BN>
+__device__ __forceinline__ void splitk_finish(uint32_t recv, const SplitShares& sh, uint32_t rank, uint32_t split,
                                               uint32_t n0, uint32_t n_total, float alpha,
                                               const __nv_bfloat16* bias, __nv_bfloat16* out, uint32_t ldo,
                                               uint32_t tid, uint32_t nthreads) {
     constexpr uint32_t F = BN / 4;
-    const uint32_t total = rows * F;
-    const uint32_t per = (total + split - 1) / split;
-    const uint32_t begin = rank * per;
-    const uint32_t end = min(total, begin + per);
-    for (uint32_t base = begin + tid; base < end; base += kReduceBatch * nthreads) {
-        uint32_t off[kReduceBatch];
-        float4 acc[kReduceBatch];
-#pragma unroll
-        for (uint32_t u = 0; u < kReduceBatch; ++u) {
-            const uint32_t idx = min(base + u * nthreads, end - 1);   // past the end: a repeat, not stored
-            const uint32_t row = idx / F, f = idx % F;
-            off[u] = part + (row * F + ((f & ~7u) | ((f ^ row) & 7u))) * 16;
-            acc[u] = rank == 0 ? ld_shared_f4(off[u]) : ld_shared_cluster_f4(mapa_shared(off[u], 0));
-        }
+    const uint32_t begin = rank * sh.per;
+    const uint32_t end = min(sh.total, begin + sh.per);
+    for (uint32_t idx = begin + tid; idx < end; idx += nthreads) {
+        const uint32_t row = idx / F, n = n0 + 4 * (idx % F);
+        const uint32_t off = recv + split_pos(idx, row, begin & ~7u) * 16;
+        float4 acc = ld_shared_f4(off);
         for (uint32_t r = 1; r < split; ++r) {
-            float4 v[kReduceBatch];
-#pragma unroll
-            for (uint32_t u = 0; u < kReduceBatch; ++u)
-                v[u] = r == rank ? ld_shared_f4(off[u]) : ld_shared_cluster_f4(mapa_shared(off[u], r));
-#pragma unroll
-            for (uint32_t u = 0; u < kReduceBatch; ++u) {
-                acc[u].x = __fadd_rn(acc[u].x, v[u].x);
-                acc[u].y = __fadd_rn(acc[u].y, v[u].y);
-                acc[u].z = __fadd_rn(acc[u].z, v[u].z);
-                acc[u].w = __fadd_rn(acc[u].w, v[u].w);
-            }
+            const float4 v = ld_shared_f4(off + r * sh.slot * 16);
+            acc.x = __fadd_rn(acc.x, v.x);
+            acc.y = __fadd_rn(acc.y, v.y);
+            acc.z = __fadd_rn(acc.z, v.z);
+            acc.w = __fadd_rn(acc.w, v.w);
         }
-#pragma unroll
-        for (uint32_t u = 0; u < kReduceBatch; ++u) {
-            const uint32_t idx = base + u * nthreads;
-            const uint32_t row = idx / F, n = n0 + 4 * (idx % F);
-            if (idx >= end || n >= n_total) continue;
-            float o[4] = {__fmul_rn(acc[u].x, alpha), __fmul_rn(acc[u].y, alpha), __fmul_rn(acc[u].z, alpha),
-                          __fmul_rn(acc[u].w, alpha)};
-            if (bias) {
-                const __nv_bfloat162 b01 = *reinterpret_cast<const __nv_bfloat162*>(bias + n);
-                const __nv_bfloat162 b23 = *reinterpret_cast<const __nv_bfloat162*>(bias + n + 2);
-                o[0] = __fadd_rn(o[0], __bfloat162float(b01.x));
-                o[1] = __fadd_rn(o[1], __bfloat162float(b01.y));
-                o[2] = __fadd_rn(o[2], __bfloat162float(b23.x));
-                o[3] = __fadd_rn(o[3], __bfloat162float(b23.y));
-            }
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
-            *reinterpret_cast<uint2*>(out + (size_t)row * ldo + n) =
-                make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+        if (n >= n_total) continue;
+        float o[4] = {__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha), __fmul_rn(acc.z, alpha),
+                      __fmul_rn(acc.w, alpha)};
+        if (bias) {
+            const __nv_bfloat162 b01 = *reinterpret_cast<const __nv_bfloat162*>(bias + n);
+            const __nv_bfloat162 b23 = *reinterpret_cast<const __nv_bfloat162*>(bias + n + 2);
+            o[0] = __fadd_rn(o[0], __bfloat162float(b01.x));
+            o[1] = __fadd_rn(o[1], __bfloat162float(b01.y));
+            o[2] = __fadd_rn(o[2], __bfloat162float(b23.x));
+            o[3] = __fadd_rn(o[3], __bfloat162float(b23.y));
         }
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
+        *reinterpret_cast<uint2*>(out + (size_t)row * ldo + n) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
     }
 }
 
@@ -366,24 +373,28 @@ __device__ __forceinline__ void sf_copy_job(int job, uint32_t st, uint32_t sf_sl
 // EPI 0: D = bf16(alpha A.B^T + bias) through tmap_d.  EPI 1: D is not
 // written; GELU(D) leaves as MXFP8 codes and scales (EpiQuant), and the
 // epilogue warps' staging area holds the GELU table instead.
-// SPLITK (EPI 0, M <= 128): the grid is one cluster of p.k_split CTAs per
-// output tile.  CTA rank r of a cluster runs the mainloop over the r-th
-// contiguous share of the K tiles into its own accumulator, which the
-// epilogue warps copy to shared memory (the pipeline stages are idle by
-// then); splitk_reduce then sums the partials across the cluster.  Before it
-// waits for the previous grid, one epilogue warp asks L2 for the CTA's whole
-// B share, so at a short M the weight stream overlaps the producer of A.
+// SPLITK (EPI 0, M <= kSplitKRows): the grid is one cluster of p.k_split
+// CTAs per output tile.  CTA rank r of a cluster runs the mainloop over the
+// r-th contiguous share of the K tiles into its own accumulator.  Its
+// epilogue warps read the accumulator once and push each share of it with
+// st.async into the receive area of the CTA that finishes that share; every
+// CTA then waits on one mbarrier for the pushes of the whole cluster and
+// finishes its share (splitk_finish).  A cluster barrier split into arrive
+// and wait guards the exchange: its first phase makes the receive barriers'
+// initialisation visible before any push, its second keeps every CTA alive
+// until all pushes are issued.  Before it waits for the previous grid, one
+// epilogue warp asks L2 for the CTA's whole B share, so at a short M the
+// weight stream overlaps the producer of A.
 template <int FMT, int BN, int EPI, bool SPLITK = false>
 __global__ void __launch_bounds__(GemmCfg<FMT, BN>::THREADS, 1)
 bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
               const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
-    using C = GemmCfg<FMT, BN>;
+    using C = GemmCfg<FMT, BN, SPLITK>;
     static_assert(EPI == 0 || kGeluTabBytes <= C::EPI_BYTES, "GELU table must fit the staging area");
-    static_assert(!SPLITK || (EPI == 0 && 128 * BN * 4 <= C::STAGES * C::STAGE_BYTES),
-                  "split-K: plain epilogue, and the partial tile must fit the pipeline stages");
+    static_assert(!SPLITK || EPI == 0, "split-K: plain epilogue only");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_BYTES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_AREA);
     // The MMA lane waits once per stage (the tensor pipe holds little more
     // than one MMA in flight, so its barrier checks are idle pipe time):
     //   full[s]   A and B tiles landed (tx) + the copy warps' commits of the
@@ -398,7 +409,8 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     const uint32_t tempty0 = tfull0 + 8 * 2;               // [2]  epilogue -> MMA
     const uint32_t drain = tempty0 + 8 * 2;                // MMA warp's own completion
     const uint32_t sfdrain = drain + 8;                    // copy warps' own completion
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 6);
+    const uint32_t recvbar = sfdrain + 8;                  // split-K: the cluster's pushes landed (tx)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 7);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* never = abort_flag + 1;
 
@@ -415,6 +427,15 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         }
         mbar_init(drain, 1);
         mbar_init(sfdrain, C::SF_WARPS);
+        if (SPLITK) {
+            // expects the partials of this CTA's share from every CTA of the
+            // cluster, its own included
+            const SplitShares sh = split_shares<BN>(min(p.m_total, kSplitKRows), p.k_split);
+            const uint32_t begin = cluster_ctarank() * sh.per;
+            const uint32_t groups = begin < sh.total ? min(sh.total - begin, sh.per) : 0;
+            mbar_init(recvbar, 1);
+            mbar_arrive_expect_tx(recvbar, p.k_split * groups * 16);
+        }
         *abort_flag = 0;
         *never = 0;
         fence_mbarrier_init();
@@ -440,7 +461,9 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (SPLITK) cluster_arrive_relaxed();   // this CTA's receive barrier is initialised
     const uint32_t tmem = *tmem_holder;
+    bool split_got = true;                  // split-K: this thread's wait for the pushes ended in time
     if (SPLITK && warp == kFirstSfWarp - 1 && lane == 0 && tile_first < num_tiles) {
         // the weight share into L2, from an epilogue warp (idle until the
         // accumulator is ready), so the prologue of the other roles does not
@@ -605,31 +628,77 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             named_barrier_sync(1, 32 * kEpiWarps);
         }
         if constexpr (SPLITK) {
-            // this CTA's partial tile -> its shared memory (rows < M only)
-            const uint32_t rows = min(p.m_total, (uint32_t)C::BM);
-            if (tile_first < num_tiles) {
-                if (!mbar_wait_bounded(tfull0, 0, abort_flag, p.wait_ns)) {
-                    *abort_flag = 1;
-                    atomicOr(p.status, 1u);
-                } else if ((uint32_t)(32 * q) < rows) {
-                    tc_fence_after();
-                    const uint32_t row = 32 * q + lane;
-                    float4* prow = reinterpret_cast<float4*>(smem) + row * (BN / 4);
-#pragma unroll 1
-                    for (int j = 0; j < BN / 64; ++j) {
-                        const int c = half * (BN / 2) + 32 * j;
-                        uint32_t r[32];
-                        tc_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + c, r);
-                        tc_wait_ld();
-                        if (row < rows) {
+            // Rows < kSplitKRows: the first tensor-memory lane quarter holds
+            // them all, so the two warps with q == 0 read the accumulator
+            // (one row per lane, half of the columns each) and push every
+            // 4-column group to the slot of this CTA in its owner's receive
+            // area.
+            const uint32_t rows = min(p.m_total, kSplitKRows);
+            const SplitShares sh = split_shares<BN>(rows, p.k_split);
+            const uint32_t recv = smem_u32(smem + C::OFF_EPI);
+            // one decision per warp: the tensor-memory loads below are warp-wide
+            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(tfull0, 0, abort_flag, p.wait_ns));
+            cluster_wait();                   // every receive barrier of the cluster is initialised
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+            }
+            if (q == 0) {
+                // After a wait that gave up, the pushes' bytes are counted on
+                // their owners' barriers without data (the output is then
+                // unspecified), so every receive barrier still completes.
+                // A lane's BN/8 groups are consecutive, so the owner only
+                // steps on at a share boundary.
+                const uint32_t row = lane;
+                uint32_t idx = row * (BN / 4) + half * (BN / 8);
+                uint32_t owner = idx / sh.per;
+                uint32_t bound = (owner + 1) * sh.per;
+                uint32_t b8 = (owner * sh.per) & ~7u;
+                uint32_t rbase = mapa_shared(recv + ks * sh.slot * 16, owner);
+                uint32_t rbar = mapa_shared(recvbar, owner);
+                if (ok) tc_fence_after();
 #pragma unroll
-                            for (int v = 0; v < 8; ++v)
-                                prow[c / 4 + (v ^ (int)(row & 7))] =
-                                    make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+                for (int c0 = 0; c0 < BN / 2; c0 += 64) {   // 64 columns per load batch
+                    const int nc = BN / 2 - c0 < 64 ? BN / 2 - c0 : 64;
+                    uint32_t r[64];
+                    if (ok) {
+                        tc_ld_32x32b_x32(tmem + half * (BN / 2) + c0, *reinterpret_cast<uint32_t(*)[32]>(r));
+                        if (nc > 32)
+                            tc_ld_32x32b_x32(tmem + half * (BN / 2) + c0 + 32,
+                                             *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+                        tc_wait_ld();
+                    }
+                    if (row < rows) {
+#pragma unroll
+                        for (int v = 0; v < nc / 4; ++v, ++idx) {
+                            if (idx == bound) {
+                                ++owner;
+                                b8 = bound & ~7u;
+                                bound += sh.per;
+                                rbase = mapa_shared(recv + ks * sh.slot * 16, owner);
+                                rbar = mapa_shared(recvbar, owner);
+                            }
+                            if (ok)
+                                st_async_f4(rbase + split_pos(idx, row, b8) * 16,
+                                            make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                        __uint_as_float(r[4 * v + 2]),
+                                                        __uint_as_float(r[4 * v + 3])),
+                                            rbar);
+                            else
+                                mbar_complete_tx_cluster(rbar, 16);
                         }
                     }
                 }
+            }
+            __syncwarp();
+            cluster_arrive_relaxed();         // this thread's pushes are issued
+            split_got = mbar_wait_bounded_cluster(recvbar, 0, abort_flag, p.wait_ns);
+            if (!split_got) {
+                *abort_flag = 1;
+                atomicOr(p.status, 1u);
+            } else {
+                splitk_finish<BN>(recv, sh, ks, p.k_split, (tile_first / p.num_m_blocks) * BN, p.n_total, alpha,
+                                  p.bias, p.out, p.ldo, threadIdx.x - 64, 32 * kEpiWarps);
             }
         }
         uint32_t t_local = 0;
@@ -654,18 +723,20 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     }
 
     if constexpr (SPLITK) {
-        // Every thread of the cluster passes both barriers, whatever its role
-        // did: the waits above are bounded, so none can hold a barrier.
+        // The roles outside the exchange pass the first phase of the cluster
+        // barrier and arrive on the second here; the epilogue warps did both
+        // around their pushes.  Every wait above is bounded, so each thread of
+        // the cluster arrives.  After the second phase every push to this CTA
+        // (or its stand-in count) has been issued, so a thread whose wait for
+        // them gave up waits here until they have landed: no CTA exits while
+        // a push into its shared memory is in flight.
         __syncwarp();
-        cluster_sync();                       // every partial of the cluster is in shared memory
-        if (warp >= 2 && warp < kFirstSfWarp && tile_first < num_tiles) {
-            const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
-            const uint32_t nb = tile_first / p.num_m_blocks;
-            splitk_reduce<BN>(smem_u32(smem), ks, p.k_split, min(p.m_total, (uint32_t)C::BM), nb * BN, p.n_total,
-                              alpha, p.bias, p.out, p.ldo, threadIdx.x - 64, 32 * kEpiWarps);
+        if (warp < 2 || warp >= kFirstSfWarp) {
+            cluster_wait();
+            cluster_arrive_relaxed();
         }
-        __syncwarp();
-        cluster_sync();                       // no CTA leaves while another reads its partial
+        cluster_wait();
+        if (!split_got) mbar_wait_bounded_cluster(recvbar, 0, never, kWaitLimitNs);
     }
 
     tc_fence_before();

@@ -510,11 +510,11 @@ int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, 
     return NVQ_OK;
 }
 
-// Split-K kernel for M <= 128: opt in to its shared memory, and the number
+// Split-K kernel for M <= kSplitKRows: opt in to its shared memory, and the number
 // of clusters of `split` CTAs the device holds at once (cached).
 template <int FMT, int BN>
 int splitk_max_clusters(DeviceInfo* d, int split) {
-    using C = GemmCfg<FMT, BN>;
+    using C = GemmCfg<FMT, BN, true>;
     auto kern = bsgemm_kernel<FMT, BN, 0, true>;
     const int wi = BN / 64 - 2;
     std::lock_guard<std::mutex> lock(g_mu);
@@ -548,16 +548,17 @@ int splitk_max_clusters(DeviceInfo* d, int split) {
     return c - 1;
 }
 
-// One cluster of `split` CTAs per 128 x BN output tile (M <= 128); each CTA
-// sums a contiguous share of the K tiles and the cluster adds the partials.
+// One cluster of `split` CTAs per output tile of M <= kSplitKRows rows and
+// BN columns; each CTA sums a contiguous share of the K tiles and the
+// cluster adds the partials.
 template <int FMT, int BN>
 int launch_gemm_splitk(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                        const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
                        void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, int split, cudaStream_t stream) {
-    using C = GemmCfg<FMT, BN>;
+    using C = GemmCfg<FMT, BN, true>;
     const int64_t kbytes = FMT == 0 ? K / 2 : K;
-    // one 128-row block, and at least one K tile per CTA of the cluster
-    if (M > C::BM || split < 2 || split > 8 || K / C::BK < split) return NVQ_ERR_SHAPE;
+    // rows that the receive areas hold, and at least one K tile per CTA of the cluster
+    if (M > (int64_t)kSplitKRows || split < 2 || split > 8 || K / C::BK < split) return NVQ_ERR_SHAPE;
     if (splitk_max_clusters<FMT, BN>(d, split) <= 0) return NVQ_ERR_CUDA;
     CUtensorMap ma, mb, md;
     memset(&md, 0, sizeof(md));
@@ -623,12 +624,12 @@ struct GemmPlan {
 // CTAs per cluster, and no more clusters than the device holds at once: on
 // a B200 that is 74 clusters of 2 but only 45 of 3), the wider tile and then
 // the smaller split on a tie.
-// Rows up to which a K split pays.  Each CTA's partial grows with M, and the
-// reduction (partials to shared memory, two cluster barriers, the exchange
-// through distributed shared memory) with it: on the FF-up weight the split
-// kernel measured 9.2 / 10.1 / 10.1 / 10.3 / 11.6 us at M = 1 / 16 / 32 / 64
-// / 128 against 10.8 / 10.9 / 10.7 / 9.8 / 9.4 us unsplit.
-constexpr int64_t kSplitKMaxRows = 32;
+// Rows up to which a K split pays, which are also the rows the split
+// kernel's receive areas hold.  The exchange grows with M: with partials
+// read back through distributed shared memory, the split kernel measured
+// 9.2 / 10.1 / 10.1 / 10.3 / 11.6 us on the FF-up weight at M = 1 / 16 / 32
+// / 64 / 128 against 10.8 / 10.9 / 10.7 / 9.8 / 9.4 us unsplit.
+constexpr int64_t kSplitKMaxRows = kSplitKRows;
 
 // The plan as a function of the shape and of the device's facts: its SM
 // count and fit(w, sp), the most clusters of sp CTAs with w-wide tiles that

@@ -269,6 +269,17 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// The two halves of a cluster barrier, for a barrier whose wait comes long
+// after its arrive.  The relaxed arrive publishes no memory writes, except
+// mbarrier initialisations made visible by fence.mbarrier_init.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // Address of the same shared-memory location in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
     uint32_t r;
@@ -299,6 +310,41 @@ __device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t cluster_addr) {
     asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(cluster_addr) : "memory");
     return v;
+}
+
+// Asynchronous 16-byte store into the shared memory of (possibly) another
+// CTA of the cluster, counted as 16 bytes on the transaction count of the
+// mbarrier at `cluster_bar`, which lies in the same CTA as the destination.
+// The source is registers, so the issuing thread waits for nothing.
+__device__ __forceinline__ void st_async_f4(uint32_t cluster_addr, float4 v, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 :: "r"(cluster_addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cluster_bar) : "memory");
+}
+
+// Count `bytes` on the transaction count of the mbarrier at `cluster_bar`
+// (possibly in another CTA of the cluster) without writing data: stands in
+// for pushes that will not come, so that the barrier's phase still ends.
+__device__ __forceinline__ void mbar_complete_tx_cluster(uint32_t cluster_bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.relaxed.cluster.shared::cluster.b64 [%0], %1;"
+                 :: "r"(cluster_bar), "r"(bytes) : "memory");
+}
+
+// Bounded wait with acquire semantics at cluster scope, for a phase that
+// other CTAs' writes complete (st.async into this CTA's shared memory).
+__device__ __forceinline__ bool mbar_wait_bounded_cluster(uint32_t bar, uint32_t parity,
+                                                          const volatile int* abort, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+        if (ok) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
 }
 
 // Arrive on an mbarrier in (possibly) another CTA of the cluster.

@@ -5,13 +5,13 @@ gives up, the kernel sets NVQ_STATUS_TIMEOUT in the device status word and
 returns, so the context stays usable.  nvq_probe_wait runs that bounded wait
 on an mbarrier nothing arrives on (a flag that nothing sets).  The test hook
 nvq_set_wait_limit shortens the real kernels' waits so that they run out: the
-one-CTA GEMM's pipeline waits and the one-pass quantizer's grid barrier.  The
-tests read the status on the host and then check that the context still
-computes correct results.  Nothing faults, traps or hangs: every kernel still
-waits, with its usual 4 s limit, for its own copies and tensor-core work
-before it exits.  (The CTA-pair GEMM's abort path is not driven here: its
-peer CTA's loads complete on the leader's barriers, and this file keeps to
-shapes that run on one CTA.)
+one-CTA GEMM's pipeline waits and the one-pass quantizer's grid barrier and the split-K
+cluster's exchange.  The tests read the status on the host and then check
+that the context still computes correct results.  Nothing faults, traps or
+hangs: every kernel still waits, with its usual 4 s limit, for its own
+copies and tensor-core work before it exits, and a split-K CTA for every
+push into its shared memory.  (The CTA-pair GEMM's abort path is not driven
+here: its peer CTA's loads complete on the leader's barriers.)
 """
 import numpy as np
 import pytest
@@ -97,6 +97,38 @@ def test_gemm_pipeline_wait_runs_out_and_the_context_survives():
     nvq.set_wait_limit(1)
     try:
         nvq.block_scaled_linear("nvfp4", ac, as_, ag, wc, ws, wg, M, N, K)
+        status = nvq.device_status()
+    finally:
+        nvq.set_wait_limit(0)
+    assert status == nvq.NVQ_STATUS_TIMEOUT
+    D = nvq.block_scaled_linear("nvfp4", ac, as_, ag, wc, ws, wg, M, N, K)
+    assert nvq.device_status() == 0
+    oc, os_, og = oracle.nvfp4_quantize(bits(x))
+    Y = oracle.gemm_rows(oracle.nvfp4_dequantize(oc, os_, og, M, K),
+                         oracle.nvfp4_dequantize(*oracle.nvfp4_quantize(bits(w)), N, K))
+    check_gemm(D.float().cpu().numpy(), Y)
+
+
+def test_split_k_waits_run_out_and_the_context_survives():
+    # The FF-up weight at M = 1 runs as clusters of two CTAs, each over half
+    # of K.  With a 1 ns limit the pipeline waits give up; the epilogue warps
+    # then count the bytes of the pushes they will not make on their owners'
+    # receive barriers, so every CTA's wait for the cluster's pushes ends, and
+    # no CTA exits while a push into its shared memory is in flight.  The
+    # next call, at the default limit, must be clean and match the oracle.
+    w = workloads.weight("ffup")
+    N, K = w.shape
+    x = workloads.activation("ffup", seed=5, M=1)
+    M = 1
+    tm, tn, ks = nvq.gemm_plan("nvfp4", M, N, K)
+    assert ks > 1
+    ac, as_, ag = nvq.nvfp4_quantize(x.cuda())
+    wc, ws, wg = nvq.quantize_weight("nvfp4", w.cuda())
+    assert nvq.device_status() == 0
+    nvq.set_wait_limit(1)
+    try:
+        for _ in range(3):
+            nvq.block_scaled_linear("nvfp4", ac, as_, ag, wc, ws, wg, M, N, K)
         status = nvq.device_status()
     finally:
         nvq.set_wait_limit(0)

@@ -1,7 +1,8 @@
 """GPU parity of the short-M GEMM path: at M <= 32 block_scaled_linear may
 split the K range of each output tile over a cluster of CTAs, each summing
-its share into its own FP32 accumulator, the cluster then adding the partials
-in rank order through distributed shared memory.
+its share into its own FP32 accumulator.  Each CTA then pushes its partial of
+every share of the tile into the shared memory of the CTA that finishes that
+share, which adds the partials in rank order.
 
   * the library's plan (nvq_gemm_plan) splits the short-M shapes below and
     leaves the others alone;
@@ -39,6 +40,10 @@ SPLIT = [
     ("nvfp4", 7, 1000, 2048, True),          # ragged N: the last tile mostly past N
     ("mxfp8", 24, 3072, 12288, True),        # FF-down weight at a short M
     ("mxfp8_e5m2", 3, 2048, 1024, False),
+    # shares that do not fall on whole rows or on groups of eight columns
+    ("nvfp4", 29, 256, 4096, True),          # 192 wide, split 8, ragged N
+    ("nvfp4", 13, 4096, 3072, True),         # 192 wide, split 6
+    ("mxfp8", 32, 2048, 3072, False),        # 128 wide, split 6
 ]
 
 
