@@ -93,7 +93,8 @@ enum {
 enum {
     NVQ_STATUS_TIMEOUT = 1,     /* a bounded wait inside a kernel gave up (see the entry points) */
     NVQ_STATUS_NONFINITE = 2,   /* nvfp4_quantize saw a NaN/Inf amax */
-    NVQ_STATUS_WORKSPACE = 4    /* nvfp4_quantize was given a workspace it did not leave (not zero-filled) */
+    NVQ_STATUS_WORKSPACE = 4,   /* nvfp4_quantize was given a workspace it did not leave (not zero-filled) */
+    NVQ_STATUS_BOUNDS = 8       /* debug build only: a kernel's bounds check failed (nvq_debug_build) */
 };
 
 /* Bytes of the code buffer for a [rows, K] tensor: rows*K/2 (NVFP4), rows*K (MXFP8, either element). */
@@ -415,6 +416,30 @@ NVQ_API int nvq_probe_gelu(const uint16_t* in, int64_t n, uint16_t* out, nvq_str
  *   waited_ns   device pointer to one 64-bit word: the nanoseconds waited
  */
 NVQ_API int nvq_probe_wait(uint64_t limit_ns, unsigned long long* waited_ns, nvq_stream_t stream);
+
+/*
+ * nvq_debug_build -- 1 in the debug build of this library (libnvq_debug.so,
+ * compiled with NVQ_DEBUG), 0 in the normal one (no counterpart on the
+ * pages).  In the debug build every kernel checks, before each global
+ * access whose address it computes from its indices, that the accessed bytes
+ * lie inside the buffer the call passed (its extent follows from the call's
+ * sizes: rows, K, pitches, tile counts).  A failed check sets
+ * NVQ_STATUS_BOUNDS in the device status word and skips the access: a store
+ * writes nothing, a load reads zeros, and a skipped bulk copy into a
+ * pipeline stage is counted on the stage's barrier without data, so no wait
+ * runs out because of it.  Nothing traps.  Results are otherwise identical
+ * to the normal build's.  The normal build contains no checks.
+ */
+NVQ_API int nvq_debug_build(void);
+
+/*
+ * nvq_probe_bounds -- bounds-check self-test (no counterpart on the pages).
+ * Launches one kernel that evaluates one failing bounds check and makes no
+ * memory access.  In the debug build the device status word then holds
+ * NVQ_STATUS_BOUNDS (read it with nvq_device_status); in the normal build it
+ * stays clean.
+ */
+NVQ_API int nvq_probe_bounds(nvq_stream_t stream);
 
 #ifdef __cplusplus
 }

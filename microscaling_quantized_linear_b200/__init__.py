@@ -9,6 +9,10 @@ shared library is missing, importing this package fails.
 
 Names follow the C ABI: ``nvfp4_quantize``, ``mxfp8_quantize``,
 ``quantize_weight``, ``block_scaled_linear``, plus the size helpers.
+
+With NVQ_DEBUG=1 in the environment at import, the debug build
+``libnvq_debug.so`` (bounds-checked kernels, see ``build.py``) is loaded
+instead; ``DEBUG_BUILD`` says which one is in use.
 """
 import ctypes
 import os
@@ -16,12 +20,14 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libnvq.so")
+_WANT_DEBUG = os.environ.get("NVQ_DEBUG", "") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "libnvq_debug.so" if _WANT_DEBUG else "libnvq.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        "libnvq.so is not built (expected at %s); run "
-        "`python microscaling_quantized_linear_b200/build.py` or __graft_entry__.build()" % LIB_PATH)
+        "%s is not built (expected at %s); run "
+        "`python microscaling_quantized_linear_b200/build.py%s` or __graft_entry__.build()"
+        % (os.path.basename(LIB_PATH), LIB_PATH, " --debug" if _WANT_DEBUG else ""))
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -38,6 +44,7 @@ _RULES = {"floor": SCALE_FLOOR, "ceil": SCALE_CEIL}
 NVQ_STATUS_TIMEOUT = 1
 NVQ_STATUS_NONFINITE = 2
 NVQ_STATUS_WORKSPACE = 4
+NVQ_STATUS_BOUNDS = 8
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -77,6 +84,10 @@ _lib.nvq_probe_wait.restype = ctypes.c_int
 _lib.nvq_probe_wait.argtypes = [ctypes.c_uint64, _vp, _vp]
 _lib.nvq_gemm_plan.restype = ctypes.c_int
 _lib.nvq_gemm_plan.argtypes = [ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp]
+_lib.nvq_debug_build.restype = ctypes.c_int
+_lib.nvq_debug_build.argtypes = []
+_lib.nvq_probe_bounds.restype = ctypes.c_int
+_lib.nvq_probe_bounds.argtypes = [_vp]
 _lib.nvq_set_wait_limit.restype = ctypes.c_int
 _lib.nvq_set_wait_limit.argtypes = [ctypes.c_uint64]
 _lib.nvq_workspace_init.restype = ctypes.c_int
@@ -89,7 +100,10 @@ EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_
             "mxfp8_quantize", "mxfp8_quantize_ex", "quantize_weight", "block_scaled_linear",
             "nvq_device_status", "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc",
             "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu", "nvq_probe_wait", "nvq_gemm_plan",
-            "nvq_gemm_plan_host", "nvq_set_wait_limit", "nvq_workspace_init")
+            "nvq_gemm_plan_host", "nvq_set_wait_limit", "nvq_workspace_init", "nvq_debug_build",
+            "nvq_probe_bounds")
+
+DEBUG_BUILD = bool(_lib.nvq_debug_build())
 
 NOALLOC_MAX_PARTIALS = 1024
 
@@ -342,6 +356,13 @@ def probe_wait(limit_ns, device=None, stream=None):
     waited = torch.zeros(1, dtype=torch.int64, device=dev)
     _check(_lib.nvq_probe_wait(int(limit_ns), _ptr(waited), _stream(stream, dev)), "nvq_probe_wait")
     return int(waited.item())
+
+
+def probe_bounds(device=None, stream=None):
+    """Run the bounds-check self-test (one failing check, no memory access):
+    in the debug build the status word then holds NVQ_STATUS_BOUNDS."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    _check(_lib.nvq_probe_bounds(_stream(stream, dev)), "nvq_probe_bounds")
 
 
 def probe_convert(values, stream=None):

@@ -90,6 +90,7 @@ struct EpiQuant {
     uint8_t* codes;
     uint8_t* sf;
     uint32_t n, m, m_pad;
+    unsigned int* status;   // bounds checks of the debug build
 };
 
 template <int BN, int EPI>
@@ -148,12 +149,16 @@ __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half,
                 uint32_t q[8];
                 gelu_bf16x32(packed[j], gelu_tab);
                 scw |= mx_block<0, 0>(packed[j], q) << (8 * j);
-                uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * j);
-                d4[0] = make_uint4(q[0], q[1], q[2], q[3]);
-                d4[1] = make_uint4(q[4], q[5], q[6], q[7]);
+                if (in_bounds((uint64_t)row * eq.n + cfirst + 32 * j, 32, (uint64_t)eq.m * eq.n, eq.status)) {
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * j);
+                    d4[0] = make_uint4(q[0], q[1], q[2], q[3]);
+                    d4[1] = make_uint4(q[4], q[5], q[6], q[7]);
+                }
             }
         }
-        uint8_t* sfp = eq.sf + sf_tile_offset(row, cfirst / 32, eq.n / 128);
+        const uint32_t so = sf_tile_offset(row, cfirst / 32, eq.n / 128);
+        if (!in_bounds(so, NC, sf_extent(eq.m_pad, eq.n / 128), eq.status)) return;
+        uint8_t* sfp = eq.sf + so;
         if (NC == 4) *reinterpret_cast<uint32_t*>(sfp) = scw;
         else *reinterpret_cast<uint16_t*>(sfp) = (uint16_t)scw;
         return;
@@ -314,8 +319,9 @@ template <int BN>
 __device__ __forceinline__ void splitk_finish(uint32_t recv, const SplitShares& sh, uint32_t rank, uint32_t split,
                                               uint32_t n0, uint32_t n_total, float alpha,
                                               const __nv_bfloat16* bias, __nv_bfloat16* out, uint32_t ldo,
-                                              uint32_t tid, uint32_t nthreads) {
+                                              uint32_t tid, uint32_t nthreads, unsigned int* status) {
     constexpr uint32_t F = BN / 4;
+    const uint64_t out_elems = pitched_extent(sh.total / F, n_total, ldo);
     const uint32_t begin = rank * sh.per;
     const uint32_t end = min(sh.total, begin + sh.per);
     for (uint32_t idx = begin + tid; idx < end; idx += nthreads) {
@@ -342,8 +348,9 @@ __device__ __forceinline__ void splitk_finish(uint32_t recv, const SplitShares& 
         }
         const __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
         const __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
-        *reinterpret_cast<uint2*>(out + (size_t)row * ldo + n) =
-            make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+        if (in_bounds((uint64_t)row * ldo + n, 4, out_elems, status))
+            *reinterpret_cast<uint2*>(out + (size_t)row * ldo + n) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
     }
 }
 
@@ -475,8 +482,9 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
 #pragma unroll
             for (int h = 0; h < C::SFB_H; ++h) {
                 const uint32_t bt = min(a0 + h, p.sfb_rtiles - 1);
-                prefetch_l2_bulk(p.sfb + ((size_t)bt * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
-                                 C::SF_ATOMS * 512);
+                const uint64_t sfb_off = ((uint64_t)bt * p.sf_ctiles + (uint64_t)kt * C::SF_ATOMS) * 512;
+                if (in_bounds(sfb_off, C::SF_ATOMS * 512, (uint64_t)p.sfb_rtiles * p.sf_ctiles * 512, p.status))
+                    prefetch_l2_bulk(p.sfb + sfb_off, C::SF_ATOMS * 512);
             }
         }
     }
@@ -512,15 +520,21 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     // can run.  Plain bulk copies have no out-of-range fill: a B
                     // tile that runs past N (its rows are not stored) reads the
                     // last scale tile.
-                    bulk_load(st + C::OFF_SFA,
-                              p.sfa + ((size_t)mb * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
-                              C::SFA_BYTES, sb);
+                    const uint64_t sfa_off = ((uint64_t)mb * p.sf_ctiles + (uint64_t)kt * C::SF_ATOMS) * 512;
+                    if (in_bounds(sfa_off, C::SFA_BYTES, (uint64_t)p.sfa_rtiles * p.sf_ctiles * 512, p.status))
+                        bulk_load(st + C::OFF_SFA, p.sfa + sfa_off, C::SFA_BYTES, sb);
+                    else
+                        mbar_complete_tx(sb, C::SFA_BYTES);     // counted without data: no wait runs out
 #pragma unroll
                     for (int h = 0; h < C::SFB_H; ++h) {
                         const uint32_t bt = min(a0 + h, p.sfb_rtiles - 1);
-                        bulk_load(st + C::OFF_SFB + h * C::SF_ATOMS * 512,
-                                  p.sfb + ((size_t)bt * p.sf_ctiles + (size_t)kt * C::SF_ATOMS) * 512,
-                                  C::SF_ATOMS * 512, sb);
+                        const uint64_t sfb_off = ((uint64_t)bt * p.sf_ctiles + (uint64_t)kt * C::SF_ATOMS) * 512;
+                        if (in_bounds(sfb_off, C::SF_ATOMS * 512, (uint64_t)p.sfb_rtiles * p.sf_ctiles * 512,
+                                      p.status))
+                            bulk_load(st + C::OFF_SFB + h * C::SF_ATOMS * 512, p.sfb + sfb_off, C::SF_ATOMS * 512,
+                                      sb);
+                        else
+                            mbar_complete_tx(sb, C::SF_ATOMS * 512);
                     }
                     tma_load_2d(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), (int32_t)(mb * C::BM));
                     tma_load_2d(st + C::OFF_B, &tmap_b, fb, (int32_t)(kt * C::KBYTES), (int32_t)(nb * BN));
@@ -620,7 +634,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
         uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * C::EPI_BUF_BYTES;
         const uint16_t* gelu_tab = reinterpret_cast<const uint16_t*>(smem + C::OFF_EPI);
-        const EpiQuant eq = {p.q_codes, p.q_sf, p.n_total, p.m_total, p.m_pad};
+        const EpiQuant eq = {p.q_codes, p.q_sf, p.n_total, p.m_total, p.m_pad, p.status};
         if (EPI == 1) {
             // built while the first tile's MMAs run (the epilogue warps are
             // idle until then); the other roles never touch it
@@ -698,7 +712,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 atomicOr(p.status, 1u);
             } else {
                 splitk_finish<BN>(recv, sh, ks, p.k_split, (tile_first / p.num_m_blocks) * BN, p.n_total, alpha,
-                                  p.bias, p.out, p.ldo, threadIdx.x - 64, 32 * kEpiWarps);
+                                  p.bias, p.out, p.ldo, threadIdx.x - 64, 32 * kEpiWarps, p.status);
             }
         }
         uint32_t t_local = 0;

@@ -362,7 +362,7 @@ bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
         const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
         uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * C::EPI_BUF_BYTES;
         const uint16_t* gelu_tab = reinterpret_cast<const uint16_t*>(smem + C::OFF_EPI);
-        const EpiQuant eq = {p.q_codes, p.q_sf, p.n_total, p.m_total, p.m_pad};
+        const EpiQuant eq = {p.q_codes, p.q_sf, p.n_total, p.m_total, p.m_pad, p.status};
         if (EPI == 1) {
             // built while the first tile's MMAs run; the other roles never touch it
             gelu_table_fill(reinterpret_cast<uint16_t*>(smem + C::OFF_EPI), threadIdx.x - 64, 32 * kEpiWarps);

@@ -34,7 +34,7 @@ static __device__ __align__(256) uint32_t g_noalloc_partials[NVQ_NOALLOC_MAX_PAR
 // it fits the static array too.
 static_assert(kMaxAmaxPartials <= NVQ_NOALLOC_MAX_PARTIALS, "amax partials must fit the no-alloc scratch");
 static_assert(kStatusTimeout == NVQ_STATUS_TIMEOUT && kStatusNonfinite == NVQ_STATUS_NONFINITE &&
-                  kStatusWorkspace == NVQ_STATUS_WORKSPACE,
+                  kStatusWorkspace == NVQ_STATUS_WORKSPACE && kStatusBounds == NVQ_STATUS_BOUNDS,
               "status bits");
 
 namespace {
@@ -145,7 +145,7 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
 // The amax pass: one CTA per 8 x 256 16-byte vectors, at most 8 per SM and
 // at most `capacity` CTAs (one partial maximum each).
 int launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, uint32_t* partial, uint32_t capacity,
-                int num_sms, cudaStream_t stream, uint32_t* npartial_out) {
+                int num_sms, unsigned int* status, cudaStream_t stream, uint32_t* npartial_out) {
     const uint32_t vecs_per_row = (uint32_t)(K / 8), pitch_vecs = (uint32_t)(ld / 8);
     const uint64_t total = (uint64_t)rows * vecs_per_row;
     uint64_t want = (total + 8 * kAmaxThreads - 1) / (8 * kAmaxThreads);
@@ -156,7 +156,7 @@ int launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, uint32_t* pa
     if (grid > cap) grid = cap;
     *npartial_out = grid;
     return launch_pdl(amax_partials_kernel, dim3(grid), dim3(kAmaxThreads), 0, stream, static_cast<const uint4*>(x),
-                      (uint32_t)rows, vecs_per_row, pitch_vecs, partial);
+                      (uint32_t)rows, vecs_per_row, pitch_vecs, partial, capacity, status);
 }
 
 uint32_t quant_grid(uint64_t units, int num_sms) {
@@ -311,7 +311,7 @@ int nvfp4_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     uint32_t* partial = calib_amax ? nullptr
                                    : reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + kWorkspacePartialsOffset);
     if (!calib_amax) {
-        if ((rc = launch_amax(x, M, K, ldx, partial, kMaxAmaxPartials, d->num_sms, stream, &npartial))) return rc;
+        if ((rc = launch_amax(x, M, K, ldx, partial, kMaxAmaxPartials, d->num_sms, d->status, stream, &npartial))) return rc;
     }
     const uint64_t units = (uint64_t)M * nblk;
     return launch_pdl(nvfp4_quantize_kernel, dim3(quant_grid(units, d->num_sms)), dim3(kQuantThreads), 0, stream,
@@ -336,7 +336,7 @@ int mxfp8_quantize_impl(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     auto kern = e5 ? (ceil_rule ? mxfp8_quantize_kernel<1, 1> : mxfp8_quantize_kernel<1, 0>)
                    : (ceil_rule ? mxfp8_quantize_kernel<0, 1> : mxfp8_quantize_kernel<0, 0>);
     return launch_pdl(kern, dim3(grid), dim3(kQuantThreads), 0, stream, xp, (uint32_t)M, nblk, (uint32_t)ldx, codes,
-                      scales);
+                      scales, d->status);
 }
 
 int encode_codes_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t kbytes, uint32_t box_rows) {
@@ -895,6 +895,16 @@ int nvq_probe_wait(uint64_t limit_ns, unsigned long long* waited_ns, nvq_stream_
     return launch_status();
 }
 
+int nvq_debug_build(void) { return kDebugBuild ? 1 : 0; }
+
+int nvq_probe_bounds(nvq_stream_t stream) {
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc) return rc;
+    probe_bounds_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(d->status);
+    return launch_status();
+}
+
 int nvq_set_wait_limit(uint64_t limit_ns) {
     if (limit_ns > kWaitLimitNs) return NVQ_ERR_SHAPE;       // at most the 4 s default
     g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
@@ -978,7 +988,7 @@ int nvfp4_quantize_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx, uin
     // CTAs as the static scratch holds
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint32_t npartial = 0;
-    if ((rc = launch_amax(x, M, K, ldx, partials, NVQ_NOALLOC_MAX_PARTIALS, d->num_sms, s, &npartial))) return rc;
+    if ((rc = launch_amax(x, M, K, ldx, partials, NVQ_NOALLOC_MAX_PARTIALS, d->num_sms, d->status, s, &npartial))) return rc;
     const uint32_t nblk = (uint32_t)(K / 16);
     const float* no_calib = nullptr;
     return launch_pdl(nvfp4_quantize_kernel, dim3(quant_grid((uint64_t)M * nblk, d->num_sms)), dim3(kQuantThreads), 0,

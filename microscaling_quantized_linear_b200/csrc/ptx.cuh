@@ -329,6 +329,11 @@ __device__ __forceinline__ void mbar_complete_tx_cluster(uint32_t cluster_bar, u
                  :: "r"(cluster_bar), "r"(bytes) : "memory");
 }
 
+// The same for an mbarrier of this CTA.
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+
 // Bounded wait with acquire semantics at cluster scope, for a phase that
 // other CTAs' writes complete (st.async into this CTA's shared memory).
 __device__ __forceinline__ bool mbar_wait_bounded_cluster(uint32_t bar, uint32_t parity,

@@ -23,6 +23,7 @@
 // scalar ones); every result is bit-identical to the CPU oracle.
 #pragma once
 #include <cstdint>
+#include "debug.cuh"
 #include "ptx.cuh"
 
 namespace nvq {
@@ -85,11 +86,12 @@ __device__ __forceinline__ uint32_t sf_tile_offset(uint32_t r, uint32_t c, uint3
 // tensor-core tile holds 128 rows).  One 32-bit word = the 4 scale bytes of
 // one row in one column tile; thread `t` of `nthreads` writes its share.
 __device__ __forceinline__ void zero_pad_scale_rows(uint8_t* sf, uint32_t rows, uint32_t ctiles, uint32_t t,
-                                                    uint32_t nthreads) {
+                                                    uint32_t nthreads, unsigned int* status) {
     const uint32_t pad_rows = ((rows + 127u) & ~127u) - rows;
     for (uint32_t i = t; i < pad_rows * ctiles; i += nthreads) {
         const uint32_t r = rows + i / ctiles, ct = i - (i / ctiles) * ctiles;
-        *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r, 4 * ct, ctiles)) = 0u;
+        const uint32_t off = sf_tile_offset(r, 4 * ct, ctiles);
+        if (in_bounds(off, 4, sf_extent(rows, ctiles), status)) *reinterpret_cast<uint32_t*>(sf + off) = 0u;
     }
 }
 
@@ -153,13 +155,15 @@ __device__ __forceinline__ float decode_scale(float amax) {
 // `pitch_vecs` vectors; partial[blockIdx.x] = max |x| bits (BF16 magnitude).
 __global__ void __launch_bounds__(kAmaxThreads)
 amax_partials_kernel(const uint4* __restrict__ x, uint32_t rows, uint32_t vecs_per_row,
-                     uint32_t pitch_vecs, uint32_t* __restrict__ partial) {
+                     uint32_t pitch_vecs, uint32_t* __restrict__ partial, uint32_t capacity,
+                     unsigned int* __restrict__ status) {
     __shared__ uint32_t red[kAmaxThreads / 32];
     griddep_wait();                       // x may come from the previous grid
     griddep_launch();                     // the quantize pass may start its prologue
     uint32_t m2 = 0;
     const uint32_t total = rows * vecs_per_row;
     const uint32_t stride = gridDim.x * kAmaxThreads;
+    const uint64_t x_vecs = pitched_extent(rows, vecs_per_row, pitch_vecs);
     uint32_t i = blockIdx.x * kAmaxThreads + threadIdx.x;
     if (pitch_vecs == vecs_per_row) {
         // contiguous: batches of 8 independent 16-byte loads, all issued
@@ -169,7 +173,9 @@ amax_partials_kernel(const uint4* __restrict__ x, uint32_t rows, uint32_t vecs_p
             uint4 v[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                v[u] = (i + u * stride < total) ? __ldg(x + i + u * stride) : make_uint4(0, 0, 0, 0);
+                v[u] = (i + u * stride < total && in_bounds(i + u * stride, 1, x_vecs, status))
+                           ? __ldg(x + i + u * stride)
+                           : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 m2 = absmax2(absmax2(absmax2(absmax2(m2, v[u].x), v[u].y), v[u].z), v[u].w);
@@ -177,12 +183,13 @@ amax_partials_kernel(const uint4* __restrict__ x, uint32_t rows, uint32_t vecs_p
     } else {
         for (; i < total; i += stride) {
             const uint32_t r = i / vecs_per_row, c = i - r * vecs_per_row;
-            uint4 v = __ldg(x + (size_t)r * pitch_vecs + c);
+            const uint64_t off = (uint64_t)r * pitch_vecs + c;
+            const uint4 v = in_bounds(off, 1, x_vecs, status) ? __ldg(x + off) : make_uint4(0, 0, 0, 0);
             m2 = absmax2(absmax2(absmax2(absmax2(m2, v.x), v.y), v.z), v.w);
         }
     }
     const uint32_t m = block_max_u32<kAmaxThreads>(fold2(m2), red);
-    if (threadIdx.x == 0) partial[blockIdx.x] = m;
+    if (threadIdx.x == 0 && in_bounds(blockIdx.x, 1, capacity, status)) partial[blockIdx.x] = m;
 }
 
 // ------------------------------------------------------------------ NVFP4, streaming
@@ -214,6 +221,7 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
     const uint32_t total = rows * nblk;
     const uint32_t stride = gridDim.x * kQuantThreads;
     const uint32_t qs = stride / nblk, rs = stride - qs * nblk;
+    const uint64_t x_elems = pitched_extent(rows, nblk * 16, ldx);
     // This thread's blocks are b0 + k * stride; the CTA walks k from its
     // last (nk - 1) down to 0, two per iteration: b = b0 + k * stride and
     // b1 = b - stride.  Only at k = nk - 1 can b lie past the end.
@@ -235,10 +243,12 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
         const bool a0 = k >= 0 && b < total, a1 = k >= 1;
         const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
         const uint4* s1 = reinterpret_cast<const uint4*>(x + (size_t)r1 * ldx + (size_t)c1 * 16);
-        v[0] = a0 ? __ldg(s0) : zero4;
-        v[1] = a0 ? __ldg(s0 + 1) : zero4;
-        v[2] = a1 ? __ldg(s1) : zero4;
-        v[3] = a1 ? __ldg(s1 + 1) : zero4;
+        const bool l0 = a0 && in_bounds((uint64_t)r * ldx + c * 16, 16, x_elems, status);
+        const bool l1 = a1 && in_bounds((uint64_t)r1 * ldx + c1 * 16, 16, x_elems, status);
+        v[0] = l0 ? __ldg(s0) : zero4;
+        v[1] = l0 ? __ldg(s0 + 1) : zero4;
+        v[2] = l1 ? __ldg(s1) : zero4;
+        v[3] = l1 ? __ldg(s1 + 1) : zero4;
     }
     init_d6(d6);
     // x is final (the amax pass that may still be running only reads it);
@@ -266,10 +276,12 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
         if (!first) {
             const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
             const uint4* s1 = reinterpret_cast<const uint4*>(x + (size_t)r1 * ldx + (size_t)c1 * 16);
-            v[0] = a0 ? __ldg(s0) : zero4;
-            v[1] = a0 ? __ldg(s0 + 1) : zero4;
-            v[2] = a1 ? __ldg(s1) : zero4;
-            v[3] = a1 ? __ldg(s1 + 1) : zero4;
+            const bool l0 = a0 && in_bounds((uint64_t)r * ldx + c * 16, 16, x_elems, status);
+            const bool l1 = a1 && in_bounds((uint64_t)r1 * ldx + c1 * 16, 16, x_elems, status);
+            v[0] = l0 ? __ldg(s0) : zero4;
+            v[1] = l0 ? __ldg(s0 + 1) : zero4;
+            v[2] = l1 ? __ldg(s1) : zero4;
+            v[3] = l1 ? __ldg(s1 + 1) : zero4;
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
@@ -284,10 +296,11 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
             const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
             const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
             if (active) {
-                *reinterpret_cast<uint2*>(codes + (size_t)bu * 8) = make_uint2(lo, hi);
-                if ((cu & 3u) == 0)
-                    *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(ru, cu, ctiles)) =
-                        sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+                if (in_bounds((uint64_t)bu * 8, 8, (uint64_t)total * 8, status))
+                    *reinterpret_cast<uint2*>(codes + (size_t)bu * 8) = make_uint2(lo, hi);
+                const uint32_t so = sf_tile_offset(ru, cu, ctiles);
+                if ((cu & 3u) == 0 && in_bounds(so, 4, sf_extent(rows, ctiles), status))
+                    *reinterpret_cast<uint32_t*>(sf + so) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
             }
         }
         if (k >= 2) {                                // the next pair: b - 2 stride, b - 3 stride
@@ -300,7 +313,7 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
             block_step_down(r1, c1, qs, rs, nblk);
         }
     }
-    zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kQuantThreads + threadIdx.x, stride);
+    zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kQuantThreads + threadIdx.x, stride, status);
 }
 
 // ------------------------------------------------------------------ NVFP4, small tensors
@@ -333,7 +346,8 @@ nvfp4_quantize_cluster_kernel(const uint16_t* __restrict__ x, uint32_t rows, uin
 #pragma unroll
     for (int i = 0; i < kClusterBlocksPerThread; ++i) {
         const uint32_t b = tid + (uint32_t)i * nthr;
-        if (b < total) {
+        if (b < total && in_bounds((uint64_t)(b / nblk) * ldx + (b % nblk) * 16, 16,
+                                   pitched_extent(rows, nblk * 16, ldx), status)) {
             const uint32_t r = b / nblk, c = b - r * nblk;
             const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 16);
             v[2 * i] = __ldg(src);
@@ -381,12 +395,14 @@ nvfp4_quantize_cluster_kernel(const uint16_t* __restrict__ x, uint32_t rows, uin
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
         const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
         if (active) {
-            *reinterpret_cast<uint2*>(codes + (size_t)b * 8) = make_uint2(lo, hi);
-            if ((c & 3u) == 0)
-                *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r, c, ctiles)) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            if (in_bounds((uint64_t)b * 8, 8, (uint64_t)total * 8, status))
+                *reinterpret_cast<uint2*>(codes + (size_t)b * 8) = make_uint2(lo, hi);
+            const uint32_t so = sf_tile_offset(r, c, ctiles);
+            if ((c & 3u) == 0 && in_bounds(so, 4, sf_extent(rows, ctiles), status))
+                *reinterpret_cast<uint32_t*>(sf + so) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
         }
     }
-    zero_pad_scale_rows(sf, rows, ctiles, tid, nthr);
+    zero_pad_scale_rows(sf, rows, ctiles, tid, nthr, status);
 }
 
 // ------------------------------------------------------------------ NVFP4, one pass
@@ -442,12 +458,13 @@ __device__ __forceinline__ void red_relaxed_max_u64(unsigned long long* p, unsig
 // BF16 magnitude bits of max |x| over the whole [rows, K] tensor (pitch ldx),
 // read by one CTA: the one-pass kernel's amax when its wait gives up.
 __device__ __forceinline__ uint32_t cta_tensor_absmax(const uint16_t* __restrict__ x, uint32_t rows, uint32_t K,
-                                                      uint32_t ldx, uint32_t* red) {
+                                                      uint32_t ldx, uint32_t* red, unsigned int* status) {
     const uint32_t vpr = K >> 3;                        // 16-byte vectors per row
     const uint32_t total = rows * vpr;
     uint32_t m2 = 0;
     for (uint32_t i = threadIdx.x; i < total; i += kFusedThreads) {
         const uint32_t r = i / vpr, c = i - r * vpr;
+        if (!in_bounds((uint64_t)r * ldx + c * 8, 8, pitched_extent(rows, K, ldx), status)) continue;
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)r * ldx) + c);
         m2 = absmax2(absmax2(absmax2(absmax2(m2, v.x), v.y), v.z), v.w);
     }
@@ -500,8 +517,8 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
 #pragma unroll
     for (int i = 0; i < kFusedMaxBlocks; ++i) {
         const uint32_t b = threadIdx.x + (uint32_t)i * kFusedThreads;
-        if (b < total) {
-            const uint32_t rl = b / nblk, c = b - rl * nblk;
+        const uint32_t rl = b / nblk, c = b - rl * nblk;
+        if (b < total && in_bounds((uint64_t)(r0 + rl) * ldx + c * 16, 16, pitched_extent(rows, K, ldx), status)) {
             const uint16_t* src = x + (size_t)(r0 + rl) * ldx + (size_t)c * 16;
             const uint32_t t0 = smem_u32(tile);
             cp_async16(t0 + group_chunk(b >> 1, 2 * (b & 1)), src);          // the block's two halves,
@@ -553,7 +570,8 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
     const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t npoll = (gridDim.x + 31) >> 5;
     if (trusted) {
-        if (threadIdx.x == 0) st_relaxed_u64(slots + (size_t)blockIdx.x * kFusedSlotStride, (tag << 16) | cta_max);
+        if (threadIdx.x == 0 && in_bounds(blockIdx.x, 1, kMaxAmaxPartials, status))
+            st_relaxed_u64(slots + (size_t)blockIdx.x * kFusedSlotStride, (tag << 16) | cta_max);
         // Every CTA's partial, tagged with this call's tag.  Warp w polls
         // slots 32w .. 32w + 31, one per lane, so a polling round costs one
         // L2 round trip; the other warps wait at the barrier below.
@@ -593,7 +611,7 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
             atomicOr(status, trusted ? kStatusTimeout : kStatusWorkspace);
             if (trusted) red_relaxed_max_u64(gen, tag);
         }
-        amax_bits = cta_tensor_absmax(x, rows, K, ldx, red);
+        amax_bits = cta_tensor_absmax(x, rows, K, ldx, red, status);
     } else {
         for (uint32_t i = 0; i < npoll; ++i) amax_bits = max(amax_bits, s_pmax[i]);
         if (blockIdx.x == 0 && threadIdx.x == 0) red_relaxed_max_u64(gen, tag);
@@ -654,9 +672,11 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
             const uint32_t pair = sc0 | (sc1 << 8);
             const uint32_t next = __shfl_down_sync(0xFFFFFFFFu, pair, 1);
             if (active) {
-                *reinterpret_cast<uint4*>(code_cta + (size_t)g * 16) = make_uint4(lo0, hi0, lo1, hi1);
-                if ((g & 1u) == 0)
-                    *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r0 + rlu[u], cu[u], ctiles)) = pair | (next << 16);
+                if (in_bounds((uint64_t)r0 * nblk * 8 + (uint64_t)g * 16, 16, (uint64_t)rows * nblk * 8, status))
+                    *reinterpret_cast<uint4*>(code_cta + (size_t)g * 16) = make_uint4(lo0, hi0, lo1, hi1);
+                const uint32_t so = sf_tile_offset(r0 + rlu[u], cu[u], ctiles);
+                if ((g & 1u) == 0 && in_bounds(so, 4, sf_extent(rows, ctiles), status))
+                    *reinterpret_cast<uint32_t*>(sf + so) = pair | (next << 16);
             }
         }
         // advance by two group strides
@@ -667,7 +687,8 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
             ++rl;
         }
     }
-    zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kFusedThreads + threadIdx.x, gridDim.x * kFusedThreads);
+    zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kFusedThreads + threadIdx.x, gridDim.x * kFusedThreads,
+                        status);
 }
 
 // ------------------------------------------------------------------ MXFP8
@@ -713,7 +734,7 @@ __device__ __forceinline__ uint32_t mx_block(const uint32_t (&w)[16], uint32_t (
 template <int ELEM, int RULE>
 __global__ void __launch_bounds__(kQuantThreads)
 mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nblk, uint32_t ldx,
-                      uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+                      uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, unsigned int* __restrict__ status) {
     griddep_wait();                              // x may come from the previous grid
     griddep_launch();
     const uint32_t total = rows * nblk;
@@ -727,7 +748,7 @@ mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) w[i] = 0;
-        if (active) {
+        if (active && in_bounds((uint64_t)r * ldx + c * 32, 32, pitched_extent(rows, nblk * 32, ldx), status)) {
             const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)r * ldx + (size_t)c * 32);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -741,12 +762,14 @@ mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
         const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
         if (active) {
-            uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)b * 32);
-            dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
-            dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
-            if ((c & 3u) == 0)
-                *reinterpret_cast<uint32_t*>(sf + sf_tile_offset(r, c, ctiles)) =
-                    sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            if (in_bounds((uint64_t)b * 32, 32, (uint64_t)total * 32, status)) {
+                uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)b * 32);
+                dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+                dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+            }
+            const uint32_t so = sf_tile_offset(r, c, ctiles);
+            if ((c & 3u) == 0 && in_bounds(so, 4, sf_extent(rows, ctiles), status))
+                *reinterpret_cast<uint32_t*>(sf + so) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
         }
         r += qs;
         c += rs;
@@ -755,7 +778,7 @@ mxfp8_quantize_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t nb
             ++r;
         }
     }
-    zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kQuantThreads + threadIdx.x, stride);
+    zero_pad_scale_rows(sf, rows, ctiles, blockIdx.x * kQuantThreads + threadIdx.x, stride, status);
 }
 
 // ------------------------------------------------------------------ probe
@@ -773,6 +796,13 @@ __global__ void probe_convert_kernel(const float* __restrict__ in, uint32_t n,
 // nothing arrives on.  When the wait gives up after limit_ns it sets
 // NVQ_STATUS_TIMEOUT (bit 0) in the status word, as a GEMM role would, and the
 // kernel returns normally.  *waited receives the nanoseconds spent.
+// One failing bounds check and nothing else: the debug build's report path
+// (the status bit) without any memory access.  In the normal build the
+// check compiles away and the kernel does nothing.
+__global__ void probe_bounds_kernel(unsigned int* __restrict__ status) {
+    if (threadIdx.x == 0) (void)in_bounds(1, 1, 1, status);
+}
+
 __global__ void probe_wait_kernel(uint64_t limit_ns, unsigned int* __restrict__ status,
                                   unsigned long long* __restrict__ waited) {
     __shared__ __align__(8) uint64_t bar;
