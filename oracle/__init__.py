@@ -277,11 +277,44 @@ def num_threads():
 GEMM_TOL = 2e-3
 
 
-def gemm_row_errors(D, Y):
-    """Per-row max_n |D - Y| / ||Y[row, :]||_2 (all-zero reference rows: max |D|)."""
+def bf16_rounding_interval(D):
+    """[lo, hi]: the real values that round to nearest (ties to even, taken
+    inclusively) to the BF16 value D, elementwise.  D must hold BF16 values
+    (the output's own format).  Half the spacing to the next BF16 magnitude
+    lies above |D| and half the spacing to the previous one below it (the
+    two differ at a power of two); +-0 covers half the smallest subnormal on
+    each side.  Non-finite D gives an empty interval (lo = +inf, hi = -inf)."""
     D = np.asarray(D, dtype=np.float64)
+    f = D.astype(np.float32)
+    bits = f.view(np.uint32)
+    assert np.all((f.astype(np.float64) == D) | np.isnan(D)) and np.all((bits & 0xFFFF) == 0), \
+        "D must hold BF16 values"
+    m = (bits >> 16) & 0x7FFF
+    val = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    mag = val(m)
+    finite = m < 0x7F80
+    prev = val(np.where(m > 0, m - 1, 0))
+    nxt = val(np.where(m + 1 < 0x7F80, m + 1, 0))
+    up = np.where(m + 1 < 0x7F80, nxt - mag, mag - prev)     # spacing above |D| (the top binade's, at the largest)
+    down_half = np.where(m > 0, (mag - prev) / 2, 2.0 ** -134)
+    neg = (bits >> 31) == 1
+    with np.errstate(invalid="ignore"):
+        lo = np.where(neg, -(mag + up / 2), mag - down_half)
+        hi = np.where(neg, -(mag - down_half), mag + up / 2)
+    return np.where(finite, lo, np.inf), np.where(finite, hi, -np.inf)
+
+
+def gemm_row_errors(D, Y):
+    """The GEMM acceptance rule: the output is judged before its BF16
+    rounding, which the tests cannot observe, so a BF16 output D[row, n] is
+    correct when some value that rounds to it lies near Y[row, n].  Per row:
+    max_n dist(Y[row, n], rounding interval of D[row, n]) / ||Y[row, :]||_2,
+    with an all-zero reference row allowing only +-0 outputs (its error is 0
+    or inf).  D = BF16 rounding of Y gives 0 on every row."""
     Y = np.asarray(Y, dtype=np.float64)
-    err = np.abs(D - Y).max(axis=1)
+    lo, hi = bf16_rounding_interval(D)
+    err = np.maximum(np.maximum(lo - Y, Y - hi), 0.0)
+    err = np.where(np.isfinite(lo), err, np.inf).max(axis=1)
     nrm = np.linalg.norm(Y, axis=1)
     zero_row = np.where(err > 0, np.inf, 0.0)
     return np.where(nrm > 0, err / np.where(nrm > 0, nrm, 1.0), zero_row)

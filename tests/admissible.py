@@ -1,8 +1,9 @@
 """Admissible outputs of the fused GELU + MXFP8 epilogue (test infrastructure).
 
 The epilogue's codes and scales are a function of the linear's BF16 result D,
-and D is known only to the GEMM's tolerance: any BF16 value within
-tol * ||Y row||_2 of the oracle's binary64 sum Y is a correct D.  So several
+and D is known only to the GEMM's tolerance, which judges the result before
+its BF16 rounding: the BF16 rounding of any value within tol * ||Y row||_2 of
+the oracle's binary64 sum Y is a correct D (oracle.gemm_row_errors).  So several
 outputs are correct, and check_admissible() accepts exactly those bytes that
 some admissible D explains, element by element and block by block, with no
 allowance for a count of mismatches.  Every value it compares comes from the
@@ -12,31 +13,8 @@ import numpy as np
 import oracle
 
 
-# BF16 bit patterns <-> a key that orders them by value (-0 just below +0).
 def _bf16_val(bits):
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-
-
-def _key(bits):
-    b = np.asarray(bits, dtype=np.int64)
-    return np.where(b & 0x8000, 0x7FFF - (b & 0x7FFF), 0x8000 + b)
-
-
-def _unkey(k):
-    k = np.asarray(k, dtype=np.int64)
-    return np.where(k >= 0x8000, k - 0x8000, 0x8000 | (0x7FFF - k)).astype(np.uint16)
-
-
-def _bf16_ceil(v):
-    """Smallest BF16 value >= v (finite v), as bits."""
-    r = oracle.double_to_bf16_array(v)
-    return _unkey(np.where(_bf16_val(r) < v, _key(r) + 1, _key(r)))
-
-
-def _bf16_floor(v):
-    """Largest BF16 value <= v (finite v), as bits."""
-    r = oracle.double_to_bf16_array(v)
-    return _unkey(np.where(_bf16_val(r) > v, _key(r) - 1, _key(r)))
 
 
 # GELU falls, then rises, with its minimum at x* = -0.7518 (between the BF16
@@ -49,12 +27,15 @@ _E4M3_VALUES = np.array([np.nan if c & 0x7F == 0x7F else oracle.e4m3_value(c) fo
 
 def admissible_gelu(Y, tol=oracle.GEMM_TOL):
     """For every element: the smallest and largest BF16 GELU(D) over the BF16
-    values D within tol * ||Y row||_2 of the binary64 sum Y (the GEMM's
-    acceptance rule).  GELU decreases below x* and increases above it, and
-    rounding to BF16 keeps that order, so the largest value sits at an end of
-    the interval and the smallest at an end or at the BF16 neighbour of x*."""
+    values D that are the rounding of a value within tol * ||Y row||_2 of the
+    binary64 sum Y (the GEMM's acceptance rule).  Rounding to nearest is
+    monotone, so those D are the BF16 values from the rounding of Y - t to
+    the rounding of Y + t.  GELU decreases below x* and increases above it,
+    and rounding to BF16 keeps that order, so the largest value sits at an
+    end of that range and the smallest at an end or at the BF16 neighbour of
+    x*."""
     t = tol * np.linalg.norm(Y, axis=1, keepdims=True)
-    a, b = _bf16_ceil(Y - t), _bf16_floor(Y + t)
+    a, b = oracle.double_to_bf16_array(Y - t), oracle.double_to_bf16_array(Y + t)
     va, vb = _bf16_val(a), _bf16_val(b)
     ga, gb = _bf16_val(oracle.gelu_bf16_array(a)), _bf16_val(oracle.gelu_bf16_array(b))
     gmin, gmax = np.minimum(ga, gb), np.maximum(ga, gb)

@@ -449,12 +449,41 @@ def test_gemm_rows_brute_force_exact_on_integers():
 
 
 def test_acceptance_rule():
+    # The output is judged before its BF16 rounding: the error of a BF16
+    # output is the distance from Y to the values that round to it.
     Y = np.array([[3.0, 4.0], [0.0, 0.0]])
     assert oracle.gemm_row_errors(Y, Y).tolist() == [0.0, 0.0]
-    D = Y + np.array([[0.005, 0.0], [0.0, 0.0]])
-    assert abs(oracle.gemm_row_errors(D, Y)[0] - 0.001) < 1e-15
-    D = Y + np.array([[0.0, 0.0], [1e-30, 0.0]])
-    assert np.isinf(oracle.gemm_row_errors(D, Y)[1])
+    # 3 + 1/64 is the BF16 neighbour of 3 (spacing 1/64 in [2, 4)): the
+    # values that round to it start half a spacing below it, at 3 + 1/128
+    D = np.array([[3.015625, 4.0], [0.0, 0.0]])
+    assert oracle.gemm_row_errors(D, Y)[0] == 0.0078125 / 5.0
+    # at a power of two the spacing below (1/64) is half the spacing above
+    # (1/32): 4 covers [4 - 1/128, 4 + 1/64]; mirrored for -4
+    assert oracle.gemm_row_errors(np.array([[4.0, 0.0]]), np.array([[4.015, 0.0]]))[0] == 0.0
+    assert oracle.gemm_row_errors(np.array([[4.0, 0.0]]), np.array([[4.0165, 0.0]]))[0] > 0.0
+    assert oracle.gemm_row_errors(np.array([[-4.0, 0.0]]), np.array([[-4.015, 0.0]]))[0] == 0.0
+    err = oracle.gemm_row_errors(np.array([[4.0, 0.0]]), np.array([[3.99, 0.0]]))[0]
+    assert abs(err - (3.9921875 - 3.99) / 3.99) < 1e-15
+    # an all-zero reference row takes +-0 only; the smallest subnormal is wrong
+    D = np.array([[0.0, -0.0], [2.0 ** -133, 0.0]])
+    assert oracle.gemm_row_errors(D, np.zeros((2, 2))).tolist() == [0.0, np.inf]
+    assert np.isinf(oracle.gemm_row_errors(np.array([[np.inf, 4.0]]), np.array([[3.0, 4.0]]))[0])
+    with pytest.raises(AssertionError):
+        oracle.gemm_row_errors(np.array([[3.005, 4.0]]), Y[:1])      # not a BF16 value
+
+
+def test_acceptance_rule_accepts_every_correctly_rounded_output():
+    # D = the BF16 rounding of the exact sum is correct for any shape, short
+    # rows included: a row whose norm one element carries can lose up to
+    # 2^-8 of it to BF16 rounding alone, more than the 2e-3 budget.
+    rng = np.random.default_rng(8)
+    for n in (1, 2, 3, 24, 257):
+        Y = rng.standard_normal((64, n)) * np.exp2(rng.integers(-20, 20, (64, 1)))
+        Y[0, 0] = 1.0 + 2.0 ** -8 - 2.0 ** -40     # rounds down to 1 (relative error just under 2^-8)
+        D = (oracle.double_to_bf16_array(Y).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        assert np.all(oracle.gemm_row_errors(D, Y) == 0.0), n
+        if n == 1:      # |D - Y| itself is above the budget there
+            assert abs(D[0, 0] - Y[0, 0]) / abs(Y[0, 0]) > 2e-3
 
 
 # --------------------------------------------------------------------------
