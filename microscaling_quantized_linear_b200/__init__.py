@@ -291,7 +291,11 @@ class QuantizedLinear:
     """A linear layer whose weight is quantized once (offline) and whose
     activations are quantized on every call, then multiplied on the
     block-scaled tensor cores.  Holds device buffers only; each call is the
-    ABI sequence quantize -> block_scaled_linear on one stream."""
+    ABI sequence quantize -> block_scaled_linear on one stream.  The
+    activation buffers (one set per batch size) are reused by every call, so
+    calls on different streams must be ordered with respect to each other.
+    MXFP8 activations take the weight's element type (E4M3, or E5M2 for
+    "mxfp8_e5m2") and the floor exponent rule, as quantize_weight does."""
 
     def __init__(self, weight, fmt="nvfp4", bias=None):
         self.fmt = _fmt(fmt)
@@ -318,7 +322,7 @@ class QuantizedLinear:
         if self.fmt == NVFP4:
             nvfp4_quantize(x, codes, scales, g, workspace=self._ws, stream=stream)
         else:
-            mxfp8_quantize(x, codes, scales, stream=stream)
+            mxfp8_quantize(x, codes, scales, stream=stream, elem="e5m2" if self.fmt == MXFP8_E5M2 else "e4m3")
             g = None
         return block_scaled_linear(self.fmt, codes, scales, g, self.w_codes, self.w_scales, self.w_global,
                                    M, self.N, self.K, bias=self.bias, out=out, stream=stream)
