@@ -139,6 +139,37 @@ def _stream(stream, device):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _buf(t, dtype, nbytes, name):
+    """A device buffer that the call reads or writes as nbytes contiguous
+    bytes: checked before the library sees its pointer, since the C ABI
+    cannot check the size of what a pointer points to."""
+    if t.dtype != dtype:
+        raise ValueError("%s: expected %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s: expected a contiguous tensor" % name)
+    if t.numel() * t.element_size() < nbytes:
+        raise ValueError("%s: %d bytes, the call needs %d" % (name, t.numel() * t.element_size(), nbytes))
+    return t
+
+
+def _mat(t, dtype, rows, cols, name):
+    """A row-major [rows, cols] matrix with unit column stride (any row pitch)."""
+    if t.dtype != dtype:
+        raise ValueError("%s: expected %s, got %s" % (name, dtype, t.dtype))
+    if t.dim() != 2 or tuple(t.shape) != (rows, cols) or t.stride(1) != 1:
+        raise ValueError("%s: expected a [%d, %d] matrix with unit column stride, got shape %s strides %s"
+                         % (name, rows, cols, tuple(t.shape), tuple(t.stride())))
+    return t
+
+
+def _cuda(**tensors):
+    """Every tensor given (None skipped) lives on a CUDA device (checked after
+    the dtypes and sizes)."""
+    for name, t in tensors.items():
+        if t is not None and not t.is_cuda:
+            raise ValueError("%s: expected a CUDA tensor" % name)
+
+
 def _pitch(t):
     if t.dim() != 2 or t.stride(1) != 1:
         raise ValueError("expected a 2-D tensor with unit stride in the last dimension")
@@ -172,6 +203,14 @@ def workspace_init(workspace, stream=None):
 
 # --------------------------------------------------------------------------- quantizers
 
+def _nvfp4_args(x, codes, scales, global_scale):
+    M, K = x.shape
+    _mat(x, torch.bfloat16, M, K, "x")
+    _buf(codes, torch.uint8, codes_bytes(NVFP4, M, K), "codes")
+    _buf(scales, torch.uint8, scale_bytes(NVFP4, M, K), "scales")
+    _buf(global_scale, torch.float32, 4, "global_scale")
+
+
 def nvfp4_quantize(x, codes=None, scales=None, global_scale=None, calib_amax=None, workspace=None,
                    stream=None):
     """BF16 [M, K] -> (codes u8 [M, K/2], scales u8 (tile order), global_scale f32 [1])."""
@@ -182,6 +221,12 @@ def nvfp4_quantize(x, codes=None, scales=None, global_scale=None, calib_amax=Non
     global_scale = global_scale if global_scale is not None else torch.empty(1, dtype=torch.float32, device=dev)
     if workspace is None and calib_amax is None:
         workspace = new_workspace(dev)
+    _nvfp4_args(x, codes, scales, global_scale)
+    if calib_amax is not None:
+        _buf(calib_amax, torch.float32, 4, "calib_amax")
+    if workspace is not None:
+        _buf(workspace, torch.uint8, workspace_bytes(), "workspace")
+    _cuda(x=x, codes=codes, scales=scales, global_scale=global_scale, calib_amax=calib_amax, workspace=workspace)
     _check(_lib.nvfp4_quantize(_ptr(x), M, K, _pitch(x), _ptr(codes), _ptr(scales), _ptr(global_scale),
                                _ptr(calib_amax), _ptr(workspace), _stream(stream, dev)), "nvfp4_quantize")
     return codes, scales, global_scale
@@ -192,6 +237,8 @@ def nvfp4_quantize_noalloc(x, codes, scales, global_scale, stream=None):
     workspace and allocates nothing: its scratch is a static array inside the
     library.  The outputs must be given (this call allocates nothing)."""
     M, K = x.shape
+    _nvfp4_args(x, codes, scales, global_scale)
+    _cuda(x=x, codes=codes, scales=scales, global_scale=global_scale)
     _check(_lib.nvfp4_quantize_noalloc(_ptr(x), M, K, _pitch(x), _ptr(codes), _ptr(scales), _ptr(global_scale),
                                        _stream(stream, x.device)), "nvfp4_quantize_noalloc")
     return codes, scales, global_scale
@@ -204,6 +251,10 @@ def mxfp8_quantize(x, codes=None, scales=None, stream=None, elem="e4m3", rule="f
     dev = x.device
     codes = codes if codes is not None else torch.empty((M, K), dtype=torch.uint8, device=dev)
     scales = scales if scales is not None else torch.empty(scale_bytes(MXFP8, M, K), dtype=torch.uint8, device=dev)
+    _mat(x, torch.bfloat16, M, K, "x")
+    _buf(codes, torch.uint8, codes_bytes(MXFP8, M, K), "codes")
+    _buf(scales, torch.uint8, scale_bytes(MXFP8, M, K), "scales")
+    _cuda(x=x, codes=codes, scales=scales)
     if elem == "e4m3" and rule == "floor":
         rc = _lib.mxfp8_quantize(_ptr(x), M, K, _pitch(x), _ptr(codes), _ptr(scales), _stream(stream, dev))
     else:
@@ -226,6 +277,12 @@ def quantize_weight(fmt, w, codes=None, scales=None, global_scale=None, workspac
     if f == NVFP4:
         global_scale = global_scale if global_scale is not None else torch.empty(1, dtype=torch.float32, device=dev)
         workspace = workspace if workspace is not None else new_workspace(dev)
+        _buf(global_scale, torch.float32, 4, "global_scale")
+        _buf(workspace, torch.uint8, workspace_bytes(), "workspace")
+    _mat(w, torch.bfloat16, N, K, "w")
+    _buf(codes, torch.uint8, codes_bytes(f, N, K), "codes")
+    _buf(scales, torch.uint8, scale_bytes(f, N, K), "scales")
+    _cuda(w=w, codes=codes, scales=scales, global_scale=global_scale, workspace=workspace)
     _check(_lib.quantize_weight(f, _ptr(w), N, K, _pitch(w), _ptr(codes), _ptr(scales), _ptr(global_scale),
                                 _ptr(workspace), _stream(stream, dev)), "quantize_weight")
     return codes, scales, global_scale
@@ -233,12 +290,34 @@ def quantize_weight(fmt, w, codes=None, scales=None, global_scale=None, workspac
 
 # --------------------------------------------------------------------------- GEMM
 
+def _gemm_args(f, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, M, N, K):
+    _buf(a_codes, torch.uint8, codes_bytes(f, M, K), "a_codes")
+    _buf(a_scales, torch.uint8, scale_bytes(f, M, K), "a_scales")
+    _buf(b_codes, torch.uint8, codes_bytes(f, N, K), "b_codes")
+    _buf(b_scales, torch.uint8, scale_bytes(f, N, K), "b_scales")
+    if f == NVFP4:
+        if a_global is None or b_global is None:
+            raise ValueError("NVFP4 operands need their global scales")
+        _buf(a_global, torch.float32, 4, "a_global")
+        _buf(b_global, torch.float32, 4, "b_global")
+    if bias is not None:
+        _buf(bias, torch.bfloat16, 2 * N, "bias")
+
+
+def _gemm_cuda(a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, **outs):
+    _cuda(a_codes=a_codes, a_scales=a_scales, a_global=a_global, b_codes=b_codes, b_scales=b_scales,
+          b_global=b_global, bias=bias, **outs)
+
+
 def block_scaled_linear(fmt, a_codes, a_scales, a_global, b_codes, b_scales, b_global, M, N, K,
                         bias=None, out=None, stream=None):
     """D = bf16(alpha * A . B^T + bias) on the block-scaled tensor cores; returns out [M, N]."""
     f = _fmt(fmt)
     dev = a_codes.device
     out = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _gemm_args(f, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, M, N, K)
+    _mat(out, torch.bfloat16, M, N, "out")
+    _gemm_cuda(a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, out=out)
     _check(_lib.block_scaled_linear(f, _ptr(a_codes), _ptr(a_scales), _ptr(a_global), _ptr(b_codes),
                                     _ptr(b_scales), _ptr(b_global), _ptr(bias), _ptr(out), _pitch(out),
                                     M, N, K, _stream(stream, dev)), "block_scaled_linear")
@@ -280,6 +359,10 @@ def block_scaled_linear_gelu_mxfp8(fmt, a_codes, a_scales, a_global, b_codes, b_
     y_codes = y_codes if y_codes is not None else torch.empty((M, N), dtype=torch.uint8, device=dev)
     y_scales = y_scales if y_scales is not None else torch.empty(scale_bytes(MXFP8, M, N), dtype=torch.uint8,
                                                                  device=dev)
+    _gemm_args(f, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, M, N, K)
+    _buf(y_codes, torch.uint8, codes_bytes(MXFP8, M, N), "y_codes")
+    _buf(y_scales, torch.uint8, scale_bytes(MXFP8, M, N), "y_scales")
+    _gemm_cuda(a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias, y_codes=y_codes, y_scales=y_scales)
     _check(_lib.block_scaled_linear_gelu_mxfp8(f, _ptr(a_codes), _ptr(a_scales), _ptr(a_global), _ptr(b_codes),
                                                _ptr(b_scales), _ptr(b_global), _ptr(bias), _ptr(y_codes),
                                                _ptr(y_scales), M, N, K, _stream(stream, dev)),

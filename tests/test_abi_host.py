@@ -10,6 +10,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import microscaling_quantized_linear_b200 as nvq
 
@@ -189,3 +190,39 @@ def test_wait_limit_hook_and_workspace_init_check_arguments():
     # the workspace holds the one-pass slots (one 128-byte line per CTA, up to
     # 256), the two-pass partials and the generation word's line
     assert nvq.workspace_bytes() == 256 * 128 + 1024 * 4 + 128
+
+
+def test_binding_checks_buffers_before_the_library_sees_them():
+    # The C ABI takes raw pointers and cannot check what they point to; the
+    # binding checks dtype, contiguity and size (then the device) first.
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    u8 = lambda n: torch.zeros(n, dtype=torch.uint8)
+    f32 = lambda n: torch.zeros(n, dtype=torch.float32)
+    M, K = 128, 256
+    with pytest.raises(ValueError, match="x: expected torch.bfloat16"):
+        nvq.nvfp4_quantize(torch.zeros(M, K), u8(M * K // 2), u8(nvq.scale_bytes("nvfp4", M, K)), f32(1))
+    with pytest.raises(ValueError, match="codes: .* the call needs 16384"):
+        nvq.nvfp4_quantize(bf(M, K), u8(100), u8(nvq.scale_bytes("nvfp4", M, K)), f32(1))
+    with pytest.raises(ValueError, match="scales: .* the call needs"):
+        nvq.nvfp4_quantize_noalloc(bf(M, K), u8(M * K // 2), u8(8), f32(1))
+    with pytest.raises(ValueError, match="global_scale: expected torch.float32"):
+        nvq.nvfp4_quantize(bf(M, K), u8(M * K // 2), u8(nvq.scale_bytes("nvfp4", M, K)), u8(4))
+    with pytest.raises(ValueError, match="workspace: .* the call needs"):
+        nvq.nvfp4_quantize(bf(M, K), u8(M * K // 2), u8(nvq.scale_bytes("nvfp4", M, K)), f32(1), workspace=u8(16))
+    with pytest.raises(ValueError, match="codes: expected a contiguous tensor"):
+        nvq.mxfp8_quantize(bf(M, K), torch.zeros(M, 2 * K, dtype=torch.uint8)[:, ::2], u8(4096))
+    with pytest.raises(ValueError, match="w: expected a \\[256, 128\\] matrix with unit column stride"):
+        nvq.quantize_weight("mxfp8", bf(M, K).t(), u8(M * K), u8(nvq.scale_bytes("mxfp8", M, K)))
+    ops = dict(a_codes=u8(M * K // 2), a_scales=u8(nvq.scale_bytes("nvfp4", M, K)), a_global=f32(1),
+               b_codes=u8(M * K // 2), b_scales=u8(nvq.scale_bytes("nvfp4", M, K)), b_global=f32(1))
+    with pytest.raises(ValueError, match="out: expected a \\[128, 128\\] matrix"):
+        nvq.block_scaled_linear("nvfp4", M=M, N=M, K=K, out=bf(M, 64), **ops)
+    with pytest.raises(ValueError, match="bias: .* the call needs 256"):
+        nvq.block_scaled_linear("nvfp4", M=M, N=M, K=K, bias=bf(64), out=bf(M, M), **ops)
+    with pytest.raises(ValueError, match="NVFP4 operands need their global scales"):
+        nvq.block_scaled_linear("nvfp4", M=M, N=M, K=K, out=bf(M, M), **dict(ops, a_global=None))
+    with pytest.raises(ValueError, match="y_codes: .* the call needs"):
+        nvq.block_scaled_linear_gelu_mxfp8("nvfp4", M=M, N=M, K=K, y_codes=u8(10), y_scales=u8(1 << 14), **ops)
+    # right dtypes and sizes on the host: only the device is wrong
+    with pytest.raises(ValueError, match="expected a CUDA tensor"):
+        nvq.block_scaled_linear("nvfp4", M=M, N=M, K=K, out=bf(M, M), **ops)
