@@ -184,8 +184,11 @@ __device__ __forceinline__ void drain_accumulator(uint32_t tmem_acc_q, int half,
 // Rows of the output that the split-K kernel takes (one short row block).
 constexpr uint32_t kSplitKRows = 32;
 
-template <int FMT, int BN_, bool SPLITK = false>
+// SPLIT_ROWS: 0 for the persistent kernel; 16 or 32 for the split-K kernel
+// at M <= SPLIT_ROWS (the rows its receive area holds).
+template <int FMT, int BN_, int SPLIT_ROWS = 0>
 struct GemmCfg {
+    static constexpr bool SPLITK = SPLIT_ROWS > 0;
     static constexpr int BM = 128;
     static constexpr int BN = BN_;
     static constexpr int KBYTES = 128;                       // bytes of K per stage (one swizzle atom)
@@ -196,7 +199,11 @@ struct GemmCfg {
     static constexpr int SF_BLOCK = FMT == 0 ? 16 : 32;
     static constexpr int SF_ATOMS = BK / SF_BLOCK / 4;       // 128x4 scale tiles per 128 rows per stage
     static constexpr int SFB_H = BN == 128 ? 1 : 2;          // 128-row scale tiles spanned by a B tile
-    static constexpr int A_BYTES = BM * KBYTES;
+    // Split-K stages only the activation's first 32 rows (M <= 32; the box
+    // past M reads zeros).  The MMA still spans 128 rows: its rows 32..127
+    // read the stage's B tile, and those accumulator rows are never read.
+    static constexpr int A_ROWS = SPLITK ? 32 : BM;
+    static constexpr int A_BYTES = A_ROWS * KBYTES;
     static constexpr int B_BYTES = BN * KBYTES;
     static constexpr int SFA_BYTES = SF_ATOMS * 512;
     static constexpr int SFB_BYTES = SFB_H * SF_ATOMS * 512;
@@ -210,11 +217,11 @@ struct GemmCfg {
     static constexpr int EPI_BUF_BYTES = 32 * 64;
     static constexpr int EPI_BYTES = kEpiWarps * EPI_BUF_BYTES;
     // split-K: the receive area for the partial sums that the cluster's CTAs
-    // push here (kSplitKRows rows of BN FP32 values, plus the padding of
-    // the per-rank slots) takes the place of the staging area, which that
-    // kernel does not use
-    static constexpr int RECV_BYTES = SPLITK ? (int)kSplitKRows * BN * 4 + 2048 : 0;
-    static constexpr int EPI_AREA = EPI_BYTES > RECV_BYTES ? EPI_BYTES : RECV_BYTES;
+    // push here (SPLIT_ROWS rows of BN FP32 values, plus the padding of the
+    // per-rank slots) takes the place of the staging area, which that kernel
+    // does not use
+    static constexpr int RECV_BYTES = SPLITK ? SPLIT_ROWS * BN * 4 + 2048 : 0;
+    static constexpr int EPI_AREA = SPLITK ? RECV_BYTES : EPI_BYTES;
     static constexpr int SMEM_LIMIT = 232448;
     static constexpr int FIXED_BYTES = 1024 /*align*/ + 512 /*barriers*/ + EPI_AREA;
     // tensor-memory columns: accumulator(s), then scale factors of A and B
@@ -227,10 +234,13 @@ struct GemmCfg {
     // accumulator(s); two accumulators only when at least 4 slots remain.
     static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
-    static constexpr int ACC_BUFS = (512 - 2 * BN) / SF_COLS >= 4 ? 2 : 1;
+    // A split-K CTA owns one tile: one accumulator, and up to 8 stages (its
+    // share of K is short, so the more of it in flight at once the better).
+    static constexpr int ACC_BUFS = SPLITK ? 1 : ((512 - 2 * BN) / SF_COLS >= 4 ? 2 : 1);
     static constexpr int SLOTS_FIT = (512 - ACC_BUFS * BN) / SF_COLS;
     static constexpr int STAGES_MIN2 = STAGES_FIT < SLOTS_FIT ? STAGES_FIT : SLOTS_FIT;
-    static constexpr int STAGES = STAGES_MIN2 > 6 ? 6 : STAGES_MIN2;
+    static constexpr int STAGES_CAP = SPLITK ? 8 : 6;
+    static constexpr int STAGES = STAGES_MIN2 > STAGES_CAP ? STAGES_CAP : STAGES_MIN2;
     static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
     static constexpr int TM_SF = ACC_BUFS * BN;            // slot s at TM_SF + s * SF_COLS
@@ -380,7 +390,7 @@ __device__ __forceinline__ void sf_copy_job(int job, uint32_t st, uint32_t sf_sl
 // EPI 0: D = bf16(alpha A.B^T + bias) through tmap_d.  EPI 1: D is not
 // written; GELU(D) leaves as MXFP8 codes and scales (EpiQuant), and the
 // epilogue warps' staging area holds the GELU table instead.
-// SPLITK (EPI 0, M <= kSplitKRows): the grid is one cluster of p.k_split
+// SPLIT_ROWS > 0 (EPI 0, M <= SPLIT_ROWS): the grid is one cluster of p.k_split
 // CTAs per output tile.  CTA rank r of a cluster runs the mainloop over the
 // r-th contiguous share of the K tiles into its own accumulator.  Its
 // epilogue warps read the accumulator once and push each share of it with
@@ -392,11 +402,12 @@ __device__ __forceinline__ void sf_copy_job(int job, uint32_t st, uint32_t sf_sl
 // until all pushes are issued.  Before it waits for the previous grid, one
 // epilogue warp asks L2 for the CTA's whole B share, so at a short M the
 // weight stream overlaps the producer of A.
-template <int FMT, int BN, int EPI, bool SPLITK = false>
+template <int FMT, int BN, int EPI, int SPLIT_ROWS = 0>
 __global__ void __launch_bounds__(GemmCfg<FMT, BN>::THREADS, 1)
 bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
               const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
-    using C = GemmCfg<FMT, BN, SPLITK>;
+    using C = GemmCfg<FMT, BN, SPLIT_ROWS>;
+    constexpr bool SPLITK = SPLIT_ROWS > 0;
     static_assert(EPI == 0 || kGeluTabBytes <= C::EPI_BYTES, "GELU table must fit the staging area");
     static_assert(!SPLITK || EPI == 0, "split-K: plain epilogue only");
     extern __shared__ uint8_t smem_raw[];
@@ -437,7 +448,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         if (SPLITK) {
             // expects the partials of this CTA's share from every CTA of the
             // cluster, its own included
-            const SplitShares sh = split_shares<BN>(min(p.m_total, kSplitKRows), p.k_split);
+            const SplitShares sh = split_shares<BN>(min(p.m_total, (uint32_t)SPLIT_ROWS), p.k_split);
             const uint32_t begin = cluster_ctarank() * sh.per;
             const uint32_t groups = begin < sh.total ? min(sh.total - begin, sh.per) : 0;
             mbar_init(recvbar, 1);
@@ -642,12 +653,12 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             named_barrier_sync(1, 32 * kEpiWarps);
         }
         if constexpr (SPLITK) {
-            // Rows < kSplitKRows: the first tensor-memory lane quarter holds
+            // Rows < SPLIT_ROWS: the first tensor-memory lane quarter holds
             // them all, so the two warps with q == 0 read the accumulator
             // (one row per lane, half of the columns each) and push every
             // 4-column group to the slot of this CTA in its owner's receive
             // area.
-            const uint32_t rows = min(p.m_total, kSplitKRows);
+            const uint32_t rows = min(p.m_total, (uint32_t)SPLIT_ROWS);
             const SplitShares sh = split_shares<BN>(rows, p.k_split);
             const uint32_t recv = smem_u32(smem + C::OFF_EPI);
             // one decision per warp: the tensor-memory loads below are warp-wide

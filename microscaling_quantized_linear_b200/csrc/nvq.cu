@@ -48,7 +48,7 @@ struct DeviceInfo {
     unsigned int* status = nullptr;
     bool gemm_attr[3][3][2] = {};    // [format][BN 128/192/256][epilogue]
     bool pair_attr[3][2][2] = {};    // [format][BN 192/256][epilogue]
-    bool splitk_attr[3][3] = {};     // [format][BN 128/192/256]
+    bool splitk_attr[3][3][2] = {};  // [format][BN 128/192/256][receive rows 16/32]
     // most clusters of k_split CTAs that fit on the device at once, + 1
     // (0 = not yet asked): [format][BN 128/192/256][k_split]
     int splitk_clusters[3][3][9] = {};
@@ -510,21 +510,31 @@ int launch_gemm(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, 
     return NVQ_OK;
 }
 
-// Split-K kernel for M <= kSplitKRows: opt in to its shared memory, and the number
-// of clusters of `split` CTAs the device holds at once (cached).
+// Split-K kernel for M <= ROWS: opt in to its shared memory (once per device).
+// Call with g_mu held.
+template <int FMT, int BN, int ROWS>
+bool splitk_opt_in(DeviceInfo* d) {
+    bool& done = d->splitk_attr[FMT][BN / 64 - 2][ROWS == 32];
+    if (!done) {
+        if (cudaFuncSetAttribute(bsgemm_kernel<FMT, BN, 0, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<FMT, BN, ROWS>::SMEM_BYTES) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        done = true;
+    }
+    return true;
+}
+
+// The number of clusters of `split` split-K CTAs the device holds at once
+// (cached; asked of the 32-row kernel, the one with more shared memory).
 template <int FMT, int BN>
 int splitk_max_clusters(DeviceInfo* d, int split) {
-    using C = GemmCfg<FMT, BN, true>;
-    auto kern = bsgemm_kernel<FMT, BN, 0, true>;
+    using C = GemmCfg<FMT, BN, 32>;
+    auto kern = bsgemm_kernel<FMT, BN, 0, 32>;
     const int wi = BN / 64 - 2;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!d->splitk_attr[FMT][wi]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
-            cudaGetLastError();
-            return 0;
-        }
-        d->splitk_attr[FMT][wi] = true;
-    }
+    if (!splitk_opt_in<FMT, BN, 32>(d)) return 0;
     int& c = d->splitk_clusters[FMT][wi][split];
     if (c == 0) {
         cudaLaunchConfig_t cfg = {};
@@ -548,22 +558,28 @@ int splitk_max_clusters(DeviceInfo* d, int split) {
     return c - 1;
 }
 
-// One cluster of `split` CTAs per output tile of M <= kSplitKRows rows and
-// BN columns; each CTA sums a contiguous share of the K tiles and the
-// cluster adds the partials.
-template <int FMT, int BN>
-int launch_gemm_splitk(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
-                       const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
-                       void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, int split, cudaStream_t stream) {
-    using C = GemmCfg<FMT, BN, true>;
+// One cluster of `split` CTAs per output tile of M <= ROWS rows and BN
+// columns; each CTA sums a contiguous share of the K tiles and the cluster
+// adds the partials.  The receive area holds ROWS rows: 16 leaves shared
+// memory for more stages than 32.
+template <int FMT, int BN, int ROWS>
+int launch_gemm_splitk_rows(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                            const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global,
+                            const void* bias, void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, int split,
+                            cudaStream_t stream) {
+    using C = GemmCfg<FMT, BN, ROWS>;
     const int64_t kbytes = FMT == 0 ? K / 2 : K;
     // rows that the receive areas hold, and at least one K tile per CTA of the cluster
-    if (M > (int64_t)kSplitKRows || split < 2 || split > 8 || K / C::BK < split) return NVQ_ERR_SHAPE;
+    if (M > (int64_t)ROWS || split < 2 || split > 8 || K / C::BK < split) return NVQ_ERR_SHAPE;
     if (splitk_max_clusters<FMT, BN>(d, split) <= 0) return NVQ_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!splitk_opt_in<FMT, BN, ROWS>(d)) return NVQ_ERR_CUDA;
+    }
     CUtensorMap ma, mb, md;
     memset(&md, 0, sizeof(md));
     int rc;
-    if ((rc = encode_codes_map(&ma, a_codes, M, kbytes, C::BM))) return rc;
+    if ((rc = encode_codes_map(&ma, a_codes, M, kbytes, C::A_ROWS))) return rc;
     if ((rc = encode_codes_map(&mb, b_codes, N, kbytes, BN))) return rc;
     GemmParams p;
     set_epi_quant(p, nullptr, nullptr, M);
@@ -598,11 +614,22 @@ int launch_gemm_splitk(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_s
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, bsgemm_kernel<FMT, BN, 0, true>, ma, mb, md, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, bsgemm_kernel<FMT, BN, 0, ROWS>, ma, mb, md, p) != cudaSuccess) {
         cudaGetLastError();
         return NVQ_ERR_CUDA;
     }
     return NVQ_OK;
+}
+
+template <int FMT, int BN>
+int launch_gemm_splitk(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                       const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, const void* bias,
+                       void* out, int64_t ldo, int64_t M, int64_t N, int64_t K, int split, cudaStream_t stream) {
+    if (M <= 16)
+        return launch_gemm_splitk_rows<FMT, BN, 16>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global,
+                                                    bias, out, ldo, M, N, K, split, stream);
+    return launch_gemm_splitk_rows<FMT, BN, 32>(d, a_codes, a_scales, a_global, b_codes, b_scales, b_global, bias,
+                                                out, ldo, M, N, K, split, stream);
 }
 
 struct GemmPlan {
