@@ -393,13 +393,14 @@ __device__ __forceinline__ void sf_copy_job(int job, uint32_t st, uint32_t sf_sl
 // SPLIT_ROWS > 0 (EPI 0, M <= SPLIT_ROWS): the grid is one cluster of p.k_split
 // CTAs per output tile.  CTA rank r of a cluster runs the mainloop over the
 // r-th contiguous share of the K tiles into its own accumulator.  Its
-// epilogue warps read the accumulator once and push each share of it with
-// st.async into the receive area of the CTA that finishes that share; every
-// CTA then waits on one mbarrier for the pushes of the whole cluster and
-// finishes its share (splitk_finish).  A cluster barrier split into arrive
-// and wait guards the exchange: its first phase makes the receive barriers'
-// initialisation visible before any push, its second keeps every CTA alive
-// until all pushes are issued.  Before it waits for the previous grid, one
+// epilogue warps read the accumulator once and lay each share of it out in
+// the CTA's free pipeline stages, and one bulk copy per share sends it into
+// the receive area of the CTA that finishes that share; every CTA then waits
+// on one mbarrier for the copies of the whole cluster and finishes its share
+// (splitk_finish).  A cluster barrier split into arrive and wait guards the
+// exchange: its first phase makes the receive barriers' initialisation
+// visible before any copy, its second keeps every CTA alive until every
+// CTA's copies have landed.  Before it waits for the previous grid, one
 // epilogue warp asks L2 for the CTA's whole B share, so at a short M the
 // weight stream overlaps the producer of A.
 template <int FMT, int BN, int EPI, int SPLIT_ROWS = 0>
@@ -446,13 +447,10 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         mbar_init(drain, 1);
         mbar_init(sfdrain, C::SF_WARPS);
         if (SPLITK) {
-            // expects the partials of this CTA's share from every CTA of the
-            // cluster, its own included
+            // expects one whole slot from every CTA of the cluster, its own included
             const SplitShares sh = split_shares<BN>(min(p.m_total, (uint32_t)SPLIT_ROWS), p.k_split);
-            const uint32_t begin = cluster_ctarank() * sh.per;
-            const uint32_t groups = begin < sh.total ? min(sh.total - begin, sh.per) : 0;
             mbar_init(recvbar, 1);
-            mbar_arrive_expect_tx(recvbar, p.k_split * groups * 16);
+            mbar_arrive_expect_tx(recvbar, p.k_split * sh.slot * 16);
         }
         *abort_flag = 0;
         *never = 0;
@@ -655,23 +653,25 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         if constexpr (SPLITK) {
             // Rows < SPLIT_ROWS: the first tensor-memory lane quarter holds
             // them all, so the two warps with q == 0 read the accumulator
-            // (one row per lane, half of the columns each) and push every
-            // 4-column group to the slot of this CTA in its owner's receive
-            // area.
+            // (one row per lane, half of the columns each).  They lay each
+            // owner's share out in this CTA's own pipeline stages (free once
+            // the MMAs completed), in the slot layout of the owner's receive
+            // area, and one thread then sends each slot with one bulk copy
+            // that completes on the owner's receive barrier.
             const uint32_t rows = min(p.m_total, (uint32_t)SPLIT_ROWS);
             const SplitShares sh = split_shares<BN>(rows, p.k_split);
             const uint32_t recv = smem_u32(smem + C::OFF_EPI);
+            const uint32_t outbox = smem_u32(smem);           // slot for owner j at j * slot * 16
             // one decision per warp: the tensor-memory loads below are warp-wide
             const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(tfull0, 0, abort_flag, p.wait_ns));
             cluster_wait();                   // every receive barrier of the cluster is initialised
             if (!ok) {
+                // the slots still go out (their contents unspecified), so
+                // every receive barrier completes
                 *abort_flag = 1;
                 atomicOr(p.status, 1u);
             }
-            if (q == 0) {
-                // After a wait that gave up, the pushes' bytes are counted on
-                // their owners' barriers without data (the output is then
-                // unspecified), so every receive barrier still completes.
+            if (q == 0 && ok) {
                 // A lane's BN/8 groups are consecutive, so the owner only
                 // steps on at a share boundary.
                 const uint32_t row = lane;
@@ -679,20 +679,16 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 uint32_t owner = idx / sh.per;
                 uint32_t bound = (owner + 1) * sh.per;
                 uint32_t b8 = (owner * sh.per) & ~7u;
-                uint32_t rbase = mapa_shared(recv + ks * sh.slot * 16, owner);
-                uint32_t rbar = mapa_shared(recvbar, owner);
-                if (ok) tc_fence_after();
+                uint32_t obase = outbox + owner * sh.slot * 16;
+                tc_fence_after();
 #pragma unroll
                 for (int c0 = 0; c0 < BN / 2; c0 += 64) {   // 64 columns per load batch
                     const int nc = BN / 2 - c0 < 64 ? BN / 2 - c0 : 64;
                     uint32_t r[64];
-                    if (ok) {
-                        tc_ld_32x32b_x32(tmem + half * (BN / 2) + c0, *reinterpret_cast<uint32_t(*)[32]>(r));
-                        if (nc > 32)
-                            tc_ld_32x32b_x32(tmem + half * (BN / 2) + c0 + 32,
-                                             *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-                        tc_wait_ld();
-                    }
+                    tc_ld_32x32b_x32(tmem + half * (BN / 2) + c0, *reinterpret_cast<uint32_t(*)[32]>(r));
+                    if (nc > 32)
+                        tc_ld_32x32b_x32(tmem + half * (BN / 2) + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+                    tc_wait_ld();
                     if (row < rows) {
 #pragma unroll
                         for (int v = 0; v < nc / 4; ++v, ++idx) {
@@ -700,31 +696,34 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                                 ++owner;
                                 b8 = bound & ~7u;
                                 bound += sh.per;
-                                rbase = mapa_shared(recv + ks * sh.slot * 16, owner);
-                                rbar = mapa_shared(recvbar, owner);
+                                obase = outbox + owner * sh.slot * 16;
                             }
-                            if (ok)
-                                st_async_f4(rbase + split_pos(idx, row, b8) * 16,
-                                            make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                                        __uint_as_float(r[4 * v + 2]),
-                                                        __uint_as_float(r[4 * v + 3])),
-                                            rbar);
-                            else
-                                mbar_complete_tx_cluster(rbar, 16);
+                            st_shared_f4(obase + split_pos(idx, row, b8) * 16,
+                                         make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
                         }
                     }
                 }
+                fence_proxy_async_smem();     // the slots, to the bulk copies
             }
-            __syncwarp();
-            cluster_arrive_relaxed();         // this thread's pushes are issued
+            named_barrier_sync(2, 32 * kEpiWarps);
+            if (threadIdx.x == 64) {
+                for (uint32_t j = 0; j < p.k_split; ++j)
+                    bulk_copy_to_cluster(mapa_shared(recv + ks * sh.slot * 16, j), outbox + j * sh.slot * 16,
+                                         sh.slot * 16, mapa_shared(recvbar, j));
+            }
             split_got = mbar_wait_bounded_cluster(recvbar, 0, abort_flag, p.wait_ns);
             if (!split_got) {
                 *abort_flag = 1;
                 atomicOr(p.status, 1u);
+                // the copies into this CTA were all issued; let them land
+                mbar_wait_bounded_cluster(recvbar, 0, never, kWaitLimitNs);
             } else {
                 splitk_finish<BN>(recv, sh, ks, p.k_split, (tile_first / p.num_m_blocks) * BN, p.n_total, alpha,
                                   p.bias, p.out, p.ldo, threadIdx.x - 64, 32 * kEpiWarps, p.status);
             }
+            __syncwarp();
+            cluster_arrive_relaxed();         // this CTA's share has arrived: its copies out have been read
         }
         uint32_t t_local = 0;
         for (uint32_t tile = SPLITK ? num_tiles : tile_first; tile < num_tiles; tile += tile_step, ++t_local) {
@@ -750,18 +749,17 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     if constexpr (SPLITK) {
         // The roles outside the exchange pass the first phase of the cluster
         // barrier and arrive on the second here; the epilogue warps did both
-        // around their pushes.  Every wait above is bounded, so each thread of
-        // the cluster arrives.  After the second phase every push to this CTA
-        // (or its stand-in count) has been issued, so a thread whose wait for
-        // them gave up waits here until they have landed: no CTA exits while
-        // a push into its shared memory is in flight.
+        // around the exchange, arriving once their CTA's receive barrier
+        // completed (every copy into it landed, so every copy out of its
+        // sender's shared memory has been read).  Every wait above is
+        // bounded, so each thread of the cluster arrives, and no CTA exits
+        // while a copy into or out of its shared memory is in flight.
         __syncwarp();
         if (warp < 2 || warp >= kFirstSfWarp) {
             cluster_wait();
             cluster_arrive_relaxed();
         }
         cluster_wait();
-        if (!split_got) mbar_wait_bounded_cluster(recvbar, 0, never, kWaitLimitNs);
     }
 
     tc_fence_before();

@@ -298,6 +298,11 @@ __device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr)
     return v;
 }
 
+__device__ __forceinline__ void st_shared_f4(uint32_t addr, float4 v) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
     float4 v;
     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -312,30 +317,25 @@ __device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t cluster_addr) {
     return v;
 }
 
-// Asynchronous 16-byte store into the shared memory of (possibly) another
-// CTA of the cluster, counted as 16 bytes on the transaction count of the
-// mbarrier at `cluster_bar`, which lies in the same CTA as the destination.
-// The source is registers, so the issuing thread waits for nothing.
-__device__ __forceinline__ void st_async_f4(uint32_t cluster_addr, float4 v, uint32_t cluster_bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
-                 :: "r"(cluster_addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cluster_bar) : "memory");
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
+// from this CTA's shared memory into the shared memory of (possibly)
+// another CTA of the cluster, counted on the mbarrier at `cluster_bar` in
+// the destination CTA.  The source must stay unchanged until that barrier's
+// phase completes.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                                     uint32_t cluster_bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst_cluster), "r"(src), "r"(bytes), "r"(cluster_bar) : "memory");
 }
 
-// Count `bytes` on the transaction count of the mbarrier at `cluster_bar`
-// (possibly in another CTA of the cluster) without writing data: stands in
-// for pushes that will not come, so that the barrier's phase still ends.
-__device__ __forceinline__ void mbar_complete_tx_cluster(uint32_t cluster_bar, uint32_t bytes) {
-    asm volatile("mbarrier.complete_tx.relaxed.cluster.shared::cluster.b64 [%0], %1;"
-                 :: "r"(cluster_bar), "r"(bytes) : "memory");
-}
-
-// The same for an mbarrier of this CTA.
+// Count `bytes` on the transaction count of an mbarrier of this CTA without
+// writing data.
 __device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
 }
 
 // Bounded wait with acquire semantics at cluster scope, for a phase that
-// other CTAs' writes complete (st.async into this CTA's shared memory).
+// other CTAs' writes complete (bulk copies into this CTA's shared memory).
 __device__ __forceinline__ bool mbar_wait_bounded_cluster(uint32_t bar, uint32_t parity,
                                                           const volatile int* abort, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();

@@ -112,10 +112,10 @@ def test_gemm_pipeline_wait_runs_out_and_the_context_survives():
 def test_split_k_waits_run_out_and_the_context_survives():
     # The FF-up weight at M = 1 runs as clusters of two CTAs, each over half
     # of K.  With a 1 ns limit the pipeline waits give up; the epilogue warps
-    # then count the bytes of the pushes they will not make on their owners'
-    # receive barriers, so every CTA's wait for the cluster's pushes ends, and
-    # no CTA exits while a push into its shared memory is in flight.  The
-    # next call, at the default limit, must be clean and match the oracle.
+    # still send their (unspecified) slots, so every CTA's wait for the
+    # cluster's copies ends, and no CTA exits while a copy into or out of its
+    # shared memory is in flight.  The next call, at the default limit, must
+    # be clean and match the oracle.
     w = workloads.weight("ffup")
     N, K = w.shape
     x = workloads.activation("ffup", seed=5, M=1)
