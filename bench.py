@@ -676,26 +676,38 @@ def run_small_m_component(nvq, device, stream, peaks, Ms=(1, 16, 128), iters=200
             nvq.nvfp4_quantize(x, codes, sf, g, workspace=ws, stream=s)
             gemm_call(i, s)
 
+        def fused_step(i, s):
+            wc, wsf, wg = wsets[i % rotate]
+            nvq.nvfp4_linear_short_m(x, wc, wsf, wg, N, out=out, stream=s)
+
+        def graphed_us(fn):
+            cs = torch.cuda.Stream(device)
+            cs.wait_stream(stream)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(cs):
+                fn(0, cs)
+                torch.cuda.synchronize(device)
+                with torch.cuda.graph(graph, stream=cs):
+                    for j in range(graph_steps):
+                        fn(j, cs)
+            torch.cuda.synchronize(device)
+            replays = max(1, iters // graph_steps)
+            t = _back_to_back_us(lambda i: graph.replay(), replays, device, torch.cuda.current_stream(device))
+            del graph
+            return t / graph_steps
+
         eager = _back_to_back_us(lambda i: step(i, stream), iters, device, stream)
         gemm = _back_to_back_us(lambda i: gemm_call(i, stream), iters, device, stream)
-        cs = torch.cuda.Stream(device)
-        cs.wait_stream(stream)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(cs):
-            step(0, cs)
-            torch.cuda.synchronize(device)
-            with torch.cuda.graph(graph, stream=cs):
-                for j in range(graph_steps):
-                    step(j, cs)
-        torch.cuda.synchronize(device)
-        replays = max(1, iters // graph_steps)
-        graphed = _back_to_back_us(lambda i: graph.replay(), replays, device, torch.cuda.current_stream(device))
-        graphed /= graph_steps
-        del graph
+        graphed = graphed_us(step)
         res["M%d" % M] = {"step_us_eager": round(eager, 2), "step_us_graph": round(graphed, 2),
                           "gemm_us": round(gemm, 2), "gemm_kernel": gemm_kernel_name(nvq, "nvfp4", M, N, K),
                           "gemm_weight_gbs": round(wbytes / (gemm * 1e-6) / 1e9, 1),
                           "gemm_weight_frac_hbm": round(wbytes / (gemm * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
+        if M <= 16:
+            # the same step as one launch (nvfp4_linear_short_m: the GEMM quantizes the activation itself)
+            res["M%d" % M]["fused_step_us_eager"] = round(_back_to_back_us(lambda i: fused_step(i, stream), iters,
+                                                                            device, stream), 2)
+            res["M%d" % M]["fused_step_us_graph"] = round(graphed_us(fused_step), 2)
     return res
 
 

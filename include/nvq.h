@@ -323,6 +323,43 @@ NVQ_API int block_scaled_linear_gelu_mxfp8(int format,
                         int64_t M, int64_t N, int64_t K, nvq_stream_t stream);
 
 /*
+ * nvfp4_linear_short_m -- the NVFP4 linear of a short batch (M <= 16) in one
+ * launch: the dynamic activation quantization of nvfp4_quantize and the
+ * block-scaled GEMM of block_scaled_linear, fused, for latency at short
+ * batches (batch 1 of the pages' FLUX runs, page "Modelos de Difusão"; the
+ * small-batch latency discussion of page "NVIDIA量化推理：5步极速优化显存+成功率
+ * 翻倍").  Every CTA of the split-K GEMM takes the activation's
+ * amax itself and quantizes the rows of its own share of K into its pipeline
+ * stages, with the arithmetic of nvfp4_quantize, while the weight streams in.
+ *
+ *   out = block_scaled_linear(NVQ_NVFP4, nvfp4_quantize(x), w) bit for bit:
+ *   the same codes, scales and global scale, the same split-K order.
+ *
+ *   x          in, BF16 [M, K], row pitch ldx elements (ldx >= K, a multiple
+ *              of 8), 16-byte aligned
+ *   M, K, N    1 <= M <= 16 (0 is a no-op); K a multiple of 256; N a
+ *              multiple of 8
+ *   b_*        the weight as quantize_weight(NVQ_NVFP4) wrote it, [N, K]
+ *   bias       optional BF16 [N] (NULL for none)
+ *   out, ldo   out, BF16 [M, N] with row pitch ldo (>= N, a multiple of 8)
+ *   a_codes, a_scales, a_global
+ *              optional outs (each may be NULL): the activation's codes,
+ *              scales (tile order, padding rows zero) and global scale, as
+ *              nvfp4_quantize would write them
+ *
+ * The fused launch exists only where block_scaled_linear would split K
+ * across a cluster (nvq_gemm_plan returns k_split > 1) and every CTA's share
+ * of the K stages fits its pipeline at once; otherwise it returns
+ * NVQ_ERR_SHAPE and launches nothing, and the caller takes the two calls.
+ * A NaN/Inf amax sets NVQ_STATUS_NONFINITE.  Other errors as nvfp4_quantize
+ * and block_scaled_linear.
+ */
+NVQ_API int nvfp4_linear_short_m(const void* x, int64_t M, int64_t K, int64_t ldx, const uint8_t* b_codes,
+                                 const uint8_t* b_scales, const float* b_global, const void* bias, void* out,
+                                 int64_t ldo, int64_t N, uint8_t* a_codes, uint8_t* a_scales, float* a_global,
+                                 nvq_stream_t stream);
+
+/*
  * nvq_device_status -- synchronizes `stream`, then returns the current
  * device's status word (NVQ_STATUS_* bits, 0 = clean) and clears it.
  * Returns NVQ_ERR_CUDA (< 0) if the synchronization or the read fails.

@@ -78,6 +78,8 @@ _lib.nvfp4_quantize_noalloc.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _v
 _lib.block_scaled_linear_gelu_mxfp8.restype = ctypes.c_int
 _lib.block_scaled_linear_gelu_mxfp8.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                 _i64, _i64, _i64, _vp]
+_lib.nvfp4_linear_short_m.restype = ctypes.c_int
+_lib.nvfp4_linear_short_m.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]
 _lib.nvq_probe_gelu.restype = ctypes.c_int
 _lib.nvq_probe_gelu.argtypes = [_vp, _i64, _vp, _vp]
 _lib.nvq_probe_wait.restype = ctypes.c_int
@@ -101,7 +103,7 @@ EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_
             "nvq_device_status", "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc",
             "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu", "nvq_probe_wait", "nvq_gemm_plan",
             "nvq_gemm_plan_host", "nvq_set_wait_limit", "nvq_workspace_init", "nvq_debug_build",
-            "nvq_probe_bounds")
+            "nvq_probe_bounds", "nvfp4_linear_short_m")
 
 DEBUG_BUILD = bool(_lib.nvq_debug_build())
 
@@ -370,6 +372,42 @@ def block_scaled_linear_gelu_mxfp8(fmt, a_codes, a_scales, a_global, b_codes, b_
     return y_codes, y_scales
 
 
+NVQ_ERR_SHAPE = -2
+SHORT_M_FUSED_ROWS = 8      # QuantizedLinear's one-launch path: batches up to this many rows
+
+
+def nvfp4_linear_short_m(x, b_codes, b_scales, b_global, N, bias=None, out=None, a_codes=None, a_scales=None,
+                         a_global=None, stream=None):
+    """The NVFP4 linear of a short batch (M <= 16) in one launch: the dynamic
+    activation quantization and the block-scaled GEMM fused, bit for bit as
+    nvfp4_quantize + block_scaled_linear.  a_codes / a_scales / a_global, if
+    given, receive the activation's quantization.  Raises NvqError with code
+    NVQ_ERR_SHAPE where the fused launch does not apply (then take the two
+    calls)."""
+    M, K = x.shape
+    dev = x.device
+    out = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _mat(x, torch.bfloat16, M, K, "x")
+    _buf(b_codes, torch.uint8, codes_bytes(NVFP4, N, K), "b_codes")
+    _buf(b_scales, torch.uint8, scale_bytes(NVFP4, N, K), "b_scales")
+    _buf(b_global, torch.float32, 4, "b_global")
+    if bias is not None:
+        _buf(bias, torch.bfloat16, 2 * N, "bias")
+    _mat(out, torch.bfloat16, M, N, "out")
+    if a_codes is not None:
+        _buf(a_codes, torch.uint8, codes_bytes(NVFP4, M, K), "a_codes")
+    if a_scales is not None:
+        _buf(a_scales, torch.uint8, scale_bytes(NVFP4, M, K), "a_scales")
+    if a_global is not None:
+        _buf(a_global, torch.float32, 4, "a_global")
+    _cuda(x=x, b_codes=b_codes, b_scales=b_scales, b_global=b_global, bias=bias, out=out, a_codes=a_codes,
+          a_scales=a_scales, a_global=a_global)
+    _check(_lib.nvfp4_linear_short_m(_ptr(x), M, K, _pitch(x), _ptr(b_codes), _ptr(b_scales), _ptr(b_global),
+                                     _ptr(bias), _ptr(out), _pitch(out), N, _ptr(a_codes), _ptr(a_scales),
+                                     _ptr(a_global), _stream(stream, dev)), "nvfp4_linear_short_m")
+    return out
+
+
 class QuantizedLinear:
     """A linear layer whose weight is quantized once (offline) and whose
     activations are quantized on every call, then multiplied on the
@@ -378,7 +416,10 @@ class QuantizedLinear:
     activation buffers (one set per batch size) are reused by every call, so
     calls on different streams must be ordered with respect to each other.
     MXFP8 activations take the weight's element type (E4M3, or E5M2 for
-    "mxfp8_e5m2") and the floor exponent rule, as quantize_weight does."""
+    "mxfp8_e5m2") and the floor exponent rule, as quantize_weight does.
+    NVFP4 batches of at most 8 rows take the one-launch nvfp4_linear_short_m
+    where it applies (same result, bit for bit; measured faster than the two
+    calls up to 8 rows, slower at 16)."""
 
     def __init__(self, weight, fmt="nvfp4", bias=None):
         self.fmt = _fmt(fmt)
@@ -388,6 +429,7 @@ class QuantizedLinear:
         self.bias = bias
         self._ws = new_workspace(self.device) if self.fmt == NVFP4 else None
         self._bufs = {}
+        self._short = {}        # batch size -> whether the fused short-M launch applies
 
     def _act_bufs(self, M):
         b = self._bufs.get(M)
@@ -401,6 +443,15 @@ class QuantizedLinear:
 
     def __call__(self, x, out=None, stream=None):
         M = x.shape[0]
+        if self.fmt == NVFP4 and 0 < M <= SHORT_M_FUSED_ROWS and self._short.get(M, True):
+            # one launch for a short batch where the split GEMM allows it
+            try:
+                return nvfp4_linear_short_m(x, self.w_codes, self.w_scales, self.w_global, self.N, bias=self.bias,
+                                            out=out, stream=stream)
+            except NvqError as e:
+                if e.code != NVQ_ERR_SHAPE:
+                    raise
+                self._short[M] = False
         codes, scales, g = self._act_bufs(M)
         if self.fmt == NVFP4:
             nvfp4_quantize(x, codes, scales, g, workspace=self._ws, stream=stream)

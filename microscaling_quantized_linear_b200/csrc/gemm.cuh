@@ -186,9 +186,12 @@ constexpr uint32_t kSplitKRows = 32;
 
 // SPLIT_ROWS: 0 for the persistent kernel; 16 or 32 for the split-K kernel
 // at M <= SPLIT_ROWS (the rows its receive area holds).
-template <int FMT, int BN_, int SPLIT_ROWS = 0>
+template <int FMT, int BN_, int SPLIT_ROWS = 0, bool FUSEQ = false>
 struct GemmCfg {
     static constexpr bool SPLITK = SPLIT_ROWS > 0;
+    // fused short-M path: d6 and rtab tables (128 floats each) and a
+    // reduction slot per epilogue warp, after the barriers
+    static constexpr int SCRATCH_BYTES = FUSEQ ? 1280 : 0;
     static constexpr int BM = 128;
     static constexpr int BN = BN_;
     static constexpr int KBYTES = 128;                       // bytes of K per stage (one swizzle atom)
@@ -223,7 +226,7 @@ struct GemmCfg {
     static constexpr int RECV_BYTES = SPLITK ? SPLIT_ROWS * BN * 4 + 2048 : 0;
     static constexpr int EPI_AREA = SPLITK ? RECV_BYTES : EPI_BYTES;
     static constexpr int SMEM_LIMIT = 232448;
-    static constexpr int FIXED_BYTES = 1024 /*align*/ + 512 /*barriers*/ + EPI_AREA;
+    static constexpr int FIXED_BYTES = 1024 /*align*/ + 512 /*barriers*/ + EPI_AREA + SCRATCH_BYTES;
     // tensor-memory columns: accumulator(s), then scale factors of A and B
     static constexpr int SFA_COLS = FMT == 0 ? 4 * KSTEPS : 4;
     static constexpr int SFB_COLS_PER_MMA = 4 * SFB_H;
@@ -266,9 +269,15 @@ struct GemmCfg {
 };
 
 struct GemmParams {
-    const uint8_t* sfa;
+    union {
+        const uint8_t* sfa;
+        const uint16_t* x;       // fused short-M path: the BF16 activation [m_total, K], pitch ldx
+    };
     const uint8_t* sfb;
-    const float* a_global;
+    union {
+        const float* a_global;
+        float* a_global_out;     // fused short-M path: where the activation's global scale goes (or null)
+    };
     const float* b_global;
     const __nv_bfloat16* bias;
     unsigned int* status;
@@ -277,10 +286,15 @@ struct GemmParams {
     uint32_t n_total;            // N: output columns past it are neither stored nor biased
     uint32_t sfa_rtiles, sfb_rtiles;   // 128-row scale tiles in the A and B scale buffers
     // quantizing epilogue (EPI 1) only: MXFP8 codes [m_total, n_total] and
-    // scales of GELU(D), m_pad = m_total rounded up to 128
+    // scales of GELU(D), m_pad = m_total rounded up to 128.  Fused short-M
+    // path: the activation's NVFP4 codes and scales (either may be null)
     uint8_t* q_codes;
     uint8_t* q_sf;
-    uint32_t m_total, m_pad;
+    uint32_t m_total;
+    union {
+        uint32_t m_pad;
+        uint32_t ldx;            // fused short-M path: the activation's row pitch in elements
+    };
     // split-K kernels only: CTAs per cluster, each summing one contiguous
     // share of the K tiles of the cluster's output tile; D is stored with
     // plain stores (out, ldo elements per row)
@@ -364,6 +378,119 @@ __device__ __forceinline__ void splitk_finish(uint32_t recv, const SplitShares& 
     }
 }
 
+// Fused short-M path: the activation's dynamic NVFP4 quantization inside the
+// split-K GEMM, by the epilogue warps (idle until the accumulator is ready)
+// while the B tiles load.  Every CTA takes the amax of the whole activation
+// [M, K] (M <= 16: a few KB to 96 KB, read from L2), then quantizes the rows
+// of its own K tiles with the same arithmetic as the quantize kernels,
+// writing the E2M1 codes into its stages' A tiles (the 128-byte swizzle the
+// MMA reads: 16-byte chunk c of row r at chunk c ^ (r % 8)) and the E4M3
+// scales into their A scale tiles (128x4 order), then counts one arrival per
+// stage on full[] and sfdata[] once the tiles are written.  Rows M..31 of
+// the A tiles are left as they are: they only feed accumulator rows that
+// nothing reads.  With q_codes / q_sf / a_global_out set, the CTAs of the
+// first cluster also write the codes, scales (padding rows zero) and g_dec,
+// exactly as nvfp4_quantize would.  Returns g_dec.  Threads tid 0..255.
+template <typename C>
+__device__ __forceinline__ float fused_quantize_a(const GemmParams& p, uint8_t* smem, float* scratch,
+                                                  uint32_t kt_begin, uint32_t kt_end, bool first_cluster,
+                                                  uint32_t tid, uint32_t full0, uint32_t sfdata0) {
+    constexpr uint32_t NT = 32 * kEpiWarps;
+    float* d6 = scratch;
+    float* rtab = scratch + 128;
+    uint32_t* red = reinterpret_cast<uint32_t*>(scratch + 256);
+    const uint32_t rows = p.m_total;
+    const uint32_t K = p.num_k_tiles * 256u;
+    const uint32_t vpr = K / 8;                               // 16-byte vectors per row
+    const uint64_t x_elems = pitched_extent(rows, K, p.ldx);
+    // amax of the whole activation: batches of 8 independent 16-byte loads
+    // per thread, all issued before any is used
+    uint32_t m2 = 0;
+    for (uint32_t i0 = tid; i0 < rows * vpr; i0 += 8 * NT) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint32_t i = i0 + u * NT, r = i / vpr, c = i - r * vpr;
+            v[u] = (i < rows * vpr && in_bounds((uint64_t)r * p.ldx + c * 8, 8, x_elems, p.status))
+                       ? __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)r * p.ldx) + c)
+                       : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m2 = absmax2(absmax2(absmax2(absmax2(m2, v[u].x), v[u].y), v[u].z), v[u].w);
+    }
+    uint32_t m = __reduce_max_sync(0xFFFFFFFFu, fold2(m2));
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    if (tid < 128) d6[tid] = __fdiv_rn((float)(128 + tid), 6.0f);
+    named_barrier_sync(3, NT);
+    m = 0;
+#pragma unroll
+    for (int w = 0; w < kEpiWarps; ++w) m = max(m, red[w]);
+    if (m >= 0x7F80u && first_cluster && cluster_ctarank() == 0 && tid == 0) atomicOr(p.status, kStatusNonfinite);
+    const float amax = __uint_as_float(m << 16);
+    const float g_enc = encode_scale(amax);
+    const float g_dec = decode_scale(amax);
+    if (tid >= 128) {
+        const uint32_t c = tid - 128;
+        rtab[c] = c ? __fdiv_rn(g_enc, e4m3_decode_pos(c)) : 0.0f;
+    }
+    named_barrier_sync(3, NT);
+    // this CTA's K tiles: stage s holds K tile kt_begin + s
+    const uint32_t share = kt_end - kt_begin;
+    const uint32_t ctiles = K / 64;
+    // two blocks per thread per iteration, both loaded before either is used
+    const uint32_t nblocks = rows * share * 16;
+    for (uint32_t u0 = tid; u0 < nblocks; u0 += 2 * NT) {
+        uint4 v[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t u = u0 + h * NT;
+            const uint32_t r = u / (share * 16), rem = u - r * (share * 16);
+            const uint32_t col = (kt_begin + (rem >> 4)) * 256 + (rem & 15u) * 16;
+            const bool ld = u < nblocks && in_bounds((uint64_t)r * p.ldx + col, 16, x_elems, p.status);
+            const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)r * p.ldx + col);
+            v[2 * h] = ld ? __ldg(src) : make_uint4(0, 0, 0, 0);
+            v[2 * h + 1] = ld ? __ldg(src + 1) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+        const uint32_t u = u0 + h * NT;
+        if (u >= nblocks) break;
+        const uint32_t r = u / (share * 16), rem = u - r * (share * 16);
+        const uint32_t st = rem >> 4, b = rem & 15u, kt = kt_begin + st;
+        const uint32_t col = kt * 256 + b * 16;
+        const uint32_t w[8] = {v[2 * h].x, v[2 * h].y, v[2 * h].z, v[2 * h].w,
+                               v[2 * h + 1].x, v[2 * h + 1].y, v[2 * h + 1].z, v[2 * h + 1].w};
+        uint32_t lo, hi;
+        const uint32_t sc = nvfp4_block(block16_max(w), w, g_enc, d6, rtab, lo, hi);
+        const uint32_t stage = smem_u32(smem + st * C::STAGE_BYTES);
+        const uint32_t chunk = b >> 1;
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};"
+                     :: "r"(stage + r * 128 + ((chunk ^ (r & 7u)) << 4) + ((b & 1u) << 3)), "r"(lo), "r"(hi)
+                     : "memory");
+        asm volatile("st.shared.u8 [%0], %1;"
+                     :: "r"(stage + C::OFF_SFA + (b >> 2) * 512 + r * 16 + (b & 3u)), "r"(sc) : "memory");
+        if (first_cluster) {
+            if (p.q_codes && in_bounds((uint64_t)r * (K / 2) + col / 2, 8, (uint64_t)rows * (K / 2), p.status))
+                *reinterpret_cast<uint2*>(p.q_codes + (size_t)r * (K / 2) + col / 2) = make_uint2(lo, hi);
+            const uint32_t so = sf_tile_offset(r, col / 16, ctiles);
+            if (p.q_sf && in_bounds(so, 1, sf_extent(rows, ctiles), p.status)) p.q_sf[so] = (uint8_t)sc;
+        }
+        }
+    }
+    if (first_cluster && cluster_ctarank() == 0) {
+        if (p.q_sf) zero_pad_scale_rows(p.q_sf, rows, ctiles, tid, NT, p.status);
+        if (p.a_global_out && tid == 0) *p.a_global_out = g_dec;
+    }
+    fence_proxy_async_smem();                 // the tiles, to the tensor core and the scale copies
+    named_barrier_sync(3, NT);
+    if (tid == 0)
+        for (uint32_t st = 0; st < share; ++st) {
+            mbar_arrive(full0 + 8 * st);
+            mbar_arrive(sfdata0 + 8 * st);
+        }
+    return g_dec;
+}
+
 // Scale-factor copy warp `job` (0: A scales, 1..SFB_H: B scale row block
 // job-1) for one pipeline stage: shared memory -> tensor-memory slot.
 template <typename C, bool PAIR>
@@ -403,14 +530,17 @@ __device__ __forceinline__ void sf_copy_job(int job, uint32_t st, uint32_t sf_sl
 // CTA's copies have landed.  Before it waits for the previous grid, one
 // epilogue warp asks L2 for the CTA's whole B share, so at a short M the
 // weight stream overlaps the producer of A.
-template <int FMT, int BN, int EPI, int SPLIT_ROWS = 0>
+// FUSEQ (NVFP4 split-K only): the activation arrives as BF16 (p.x) and is
+// quantized inside the kernel (fused_quantize_a); tmap_a is not used.
+template <int FMT, int BN, int EPI, int SPLIT_ROWS = 0, bool FUSEQ = false>
 __global__ void __launch_bounds__(GemmCfg<FMT, BN>::THREADS, 1)
 bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
               const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
-    using C = GemmCfg<FMT, BN, SPLIT_ROWS>;
+    using C = GemmCfg<FMT, BN, SPLIT_ROWS, FUSEQ>;
     constexpr bool SPLITK = SPLIT_ROWS > 0;
     static_assert(EPI == 0 || kGeluTabBytes <= C::EPI_BYTES, "GELU table must fit the staging area");
     static_assert(!SPLITK || EPI == 0, "split-K: plain epilogue only");
+    static_assert(!FUSEQ || (SPLITK && FMT == 0), "fused activation quantization: NVFP4 split-K only");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + C::EPI_AREA);
@@ -436,9 +566,9 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(full0 + 8 * s, 1 + C::SF_WARPS);
+            mbar_init(full0 + 8 * s, 1 + C::SF_WARPS + (FUSEQ ? 1 : 0));
             mbar_init(empty0 + 8 * s, 1);
-            mbar_init(sfdata0 + 8 * s, 1);
+            mbar_init(sfdata0 + 8 * s, FUSEQ ? 2 : 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
@@ -466,7 +596,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     const uint32_t kt_begin = SPLITK ? ks * p.num_k_tiles / p.k_split : 0;
     const uint32_t kt_end = SPLITK ? (ks + 1) * p.num_k_tiles / p.k_split : p.num_k_tiles;
     if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmap_a);
+        if (!FUSEQ) prefetch_tensormap(&tmap_a);
         prefetch_tensormap(&tmap_b);
         if (EPI == 0 && !SPLITK) prefetch_tensormap(&tmap_d);
     }
@@ -523,17 +653,21 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     }
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
                     const uint32_t fb = full0 + 8 * s, sb = sfdata0 + 8 * s;
-                    mbar_arrive_expect_tx(sb, C::SF_BYTES);
-                    mbar_arrive_expect_tx(fb, C::AB_BYTES);
+                    // (fused activation quantization: the epilogue warps write
+                    // the A tile and its scales, and arrive on both barriers)
+                    mbar_arrive_expect_tx(sb, C::SF_BYTES - (FUSEQ ? C::SFA_BYTES : 0));
+                    mbar_arrive_expect_tx(fb, C::AB_BYTES - (FUSEQ ? C::A_BYTES : 0));
                     // scale tiles first: the copy warps need them before the MMAs
                     // can run.  Plain bulk copies have no out-of-range fill: a B
                     // tile that runs past N (its rows are not stored) reads the
                     // last scale tile.
                     const uint64_t sfa_off = ((uint64_t)mb * p.sf_ctiles + (uint64_t)kt * C::SF_ATOMS) * 512;
-                    if (in_bounds(sfa_off, C::SFA_BYTES, (uint64_t)p.sfa_rtiles * p.sf_ctiles * 512, p.status))
+                    if (FUSEQ) {
+                    } else if (in_bounds(sfa_off, C::SFA_BYTES, (uint64_t)p.sfa_rtiles * p.sf_ctiles * 512, p.status)) {
                         bulk_load(st + C::OFF_SFA, p.sfa + sfa_off, C::SFA_BYTES, sb);
-                    else
+                    } else {
                         mbar_complete_tx(sb, C::SFA_BYTES);     // counted without data: no wait runs out
+                    }
 #pragma unroll
                     for (int h = 0; h < C::SFB_H; ++h) {
                         const uint32_t bt = min(a0 + h, p.sfb_rtiles - 1);
@@ -545,7 +679,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                         else
                             mbar_complete_tx(sb, C::SF_ATOMS * 512);
                     }
-                    tma_load_2d(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), (int32_t)(mb * C::BM));
+                    if (!FUSEQ) tma_load_2d(st, &tmap_a, fb, (int32_t)(kt * C::KBYTES), (int32_t)(mb * C::BM));
                     tma_load_2d(st + C::OFF_B, &tmap_b, fb, (int32_t)(kt * C::KBYTES), (int32_t)(nb * BN));
                     ++it;
                 }
@@ -640,7 +774,13 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         // ---------------------------------------------------------- epilogue (warps 2-9)
         const int q = warp & 3;                       // tensor-memory lane quarter of this warp
         const int half = (warp - 2) >> 2;             // which half of the tile's columns
-        const float alpha = FMT == 0 ? __fmul_rn(*p.a_global, *p.b_global) : 1.0f;
+        float a_dec;
+        if constexpr (FUSEQ)
+            a_dec = fused_quantize_a<C>(p, smem, reinterpret_cast<float*>(bars + 64), kt_begin, kt_end,
+                                        tile_first == 0, threadIdx.x - 64, full0, sfdata0);
+        else
+            a_dec = FMT == 0 ? *p.a_global : 1.0f;
+        const float alpha = FMT == 0 ? __fmul_rn(a_dec, *p.b_global) : 1.0f;
         uint8_t* staging = smem + C::OFF_EPI + (warp - 2) * C::EPI_BUF_BYTES;
         const uint16_t* gelu_tab = reinterpret_cast<const uint16_t*>(smem + C::OFF_EPI);
         const EpiQuant eq = {p.q_codes, p.q_sf, p.n_total, p.m_total, p.m_pad, p.status};

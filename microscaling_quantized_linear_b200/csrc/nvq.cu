@@ -49,6 +49,7 @@ struct DeviceInfo {
     bool gemm_attr[3][3][2] = {};    // [format][BN 128/192/256][epilogue]
     bool pair_attr[3][2][2] = {};    // [format][BN 192/256][epilogue]
     bool splitk_attr[3][3][2] = {};  // [format][BN 128/192/256][receive rows 16/32]
+    bool short_attr[3] = {};         // fused short-M NVFP4 kernel: [BN 128/192/256]
     // most clusters of k_split CTAs that fit on the device at once, + 1
     // (0 = not yet asked): [format][BN 128/192/256][k_split]
     int splitk_clusters[3][3][9] = {};
@@ -632,6 +633,78 @@ int launch_gemm_splitk(DeviceInfo* d, const uint8_t* a_codes, const uint8_t* a_s
                                                 out, ldo, M, N, K, split, stream);
 }
 
+// Fused short-M NVFP4 linear: one cluster of `split` CTAs per 16 x BN output
+// tile, the activation quantized inside the kernel (fused_quantize_a).
+// Needs every CTA's share of the K tiles to fit its stages at once.
+template <int BN>
+int launch_linear_short(DeviceInfo* d, const void* x, int64_t ldx, const uint8_t* b_codes, const uint8_t* b_scales,
+                        const float* b_global, const void* bias, void* out, int64_t ldo, uint8_t* a_codes,
+                        uint8_t* a_scales, float* a_global, int64_t M, int64_t N, int64_t K, int split,
+                        cudaStream_t stream) {
+    using C = GemmCfg<0, BN, 16, true>;
+    auto kern = bsgemm_kernel<0, BN, 0, 16, true>;
+    const int64_t nkt = K / C::BK;
+    if (M > 16 || split < 2 || split > 8 || nkt < split || (nkt + split - 1) / split > C::STAGES)
+        return NVQ_ERR_SHAPE;
+    if (splitk_max_clusters<0, BN>(d, split) <= 0) return NVQ_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        bool& done = d->short_attr[BN / 64 - 2];
+        if (!done) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                return NVQ_ERR_CUDA;
+            }
+            done = true;
+        }
+    }
+    CUtensorMap mb, md;
+    memset(&md, 0, sizeof(md));
+    int rc;
+    if ((rc = encode_codes_map(&mb, b_codes, N, K / 2, BN))) return rc;
+    GemmParams p;
+    set_epi_quant(p, a_codes, a_scales, M);
+    p.ldx = (uint32_t)ldx;
+    p.x = static_cast<const uint16_t*>(x);
+    p.sfb = b_scales;
+    p.a_global_out = a_global;
+    p.b_global = b_global;
+    p.bias = static_cast<const __nv_bfloat16*>(bias);
+    p.status = d->status;
+    p.wait_ns = (uint32_t)pipeline_wait_ns(kWaitLimitNs);
+    p.num_m_blocks = 1;
+    p.num_n_blocks = (uint32_t)((N + BN - 1) / BN);
+    p.n_total = (uint32_t)N;
+    p.sfa_rtiles = 1;
+    p.sfb_rtiles = (uint32_t)((N + 127) / 128);
+    p.num_k_tiles = (uint32_t)nkt;
+    p.sf_ctiles = (uint32_t)(K / C::SF_BLOCK / 4);
+    p.k_split = (uint32_t)split;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.ldo = (uint32_t)ldo;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.num_n_blocks * (uint32_t)split);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = split;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    // tmap_a is not read on this path; the B map stands in for it
+    if (cudaLaunchKernelEx(&cfg, kern, mb, mb, md, p) != cudaSuccess) {
+        cudaGetLastError();
+        return NVQ_ERR_CUDA;
+    }
+    return NVQ_OK;
+}
+
 struct GemmPlan {
     int tile_m, tile_n, k_split;
 };
@@ -792,6 +865,35 @@ int quantize_weight(int format, const void* w, int64_t N, int64_t K, int64_t ldw
         return mxfp8_quantize_impl(w, N, K, ldw, codes, scales, format, NVQ_SCALE_FLOOR,
                                    reinterpret_cast<cudaStream_t>(stream));
     return NVQ_ERR_FORMAT;
+}
+
+int nvfp4_linear_short_m(const void* x, int64_t M, int64_t K, int64_t ldx, const uint8_t* b_codes,
+                         const uint8_t* b_scales, const float* b_global, const void* bias, void* out, int64_t ldo,
+                         int64_t N, uint8_t* a_codes, uint8_t* a_scales, float* a_global, nvq_stream_t stream) {
+    int rc = check_quant_shape(NVQ_NVFP4, M, K, ldx);
+    if (rc) return rc;
+    if (M > 16 || N <= 0 || N % 8 || K % 256) return NVQ_ERR_SHAPE;
+    if (ldo < N || ldo % 8 || ldo >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVQ_ERR_SHAPE;
+    if (M == 0) return NVQ_OK;
+    if (!x || !b_codes || !b_scales || !b_global || !out) return NVQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(b_codes) || !aligned16(b_scales) || !aligned16(out) ||
+        (a_codes && !aligned16(a_codes)) || (a_scales && !aligned16(a_scales)) ||
+        (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) || (a_global && (reinterpret_cast<uintptr_t>(a_global) & 3u)))
+        return NVQ_ERR_ALIGN;
+    DeviceInfo* d = nullptr;
+    if ((rc = device_info(&d))) return rc;
+    if ((rc = get_encoder())) return rc;
+    const GemmPlan pl = plan_gemm<0>(d, M, N, K);
+    if (pl.k_split < 2) return NVQ_ERR_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (pl.tile_n == 256)
+        return launch_linear_short<256>(d, x, ldx, b_codes, b_scales, b_global, bias, out, ldo, a_codes, a_scales,
+                                        a_global, M, N, K, pl.k_split, s);
+    if (pl.tile_n == 192)
+        return launch_linear_short<192>(d, x, ldx, b_codes, b_scales, b_global, bias, out, ldo, a_codes, a_scales,
+                                        a_global, M, N, K, pl.k_split, s);
+    return launch_linear_short<128>(d, x, ldx, b_codes, b_scales, b_global, bias, out, ldo, a_codes, a_scales,
+                                    a_global, M, N, K, pl.k_split, s);
 }
 
 int block_scaled_linear(int format, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,

@@ -226,3 +226,16 @@ def test_binding_checks_buffers_before_the_library_sees_them():
     # right dtypes and sizes on the host: only the device is wrong
     with pytest.raises(ValueError, match="expected a CUDA tensor"):
         nvq.block_scaled_linear("nvfp4", M=M, N=M, K=K, out=bf(M, M), **ops)
+
+
+def test_linear_short_m_rejects_bad_arguments():
+    def ls(x=P16, M=1, K=256, ldx=256, b=P16, sb=P16, gb=P16, bias=NULL, out=P16, ldo=128, N=128):
+        return L.nvfp4_linear_short_m(x, M, K, ldx, b, sb, gb, bias, out, ldo, N, NULL, NULL, NULL, NULL)
+    assert ls(M=17) == -2                     # short batches only
+    assert ls(K=192, ldx=192) == -2           # K a multiple of 256
+    assert ls(N=100, ldo=104) == -2           # N a multiple of 8
+    assert ls(ldo=120) == -2
+    assert ls(x=NULL) == -1
+    assert ls(gb=NULL) == -1
+    assert ls(out=P_ODD) == -3
+    assert ls(M=0) == 0                       # empty batch: nothing to do

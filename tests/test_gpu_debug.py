@@ -102,6 +102,18 @@ for fmt, M, N, K, use_bias in GEMMS:
     D = gpu_linear(fmt, x, w, bias=b)              # asserts a clean status word
     check_gemm(D.float().cpu().numpy(), oracle_linear(fmt, x, w, bias=b))
 
+for M, N, K in ((1, 12288, 3072), (7, 1000, 2048)):      # one-launch short-batch linear
+    x = workloads.normal(M, K, seed=M + 9)
+    w = workloads.normal(N, K, seed=N + 3, std=0.05)
+    wc, ws, wg = nvq.quantize_weight("nvfp4", w.cuda())
+    ac = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    asf = torch.empty(nvq.scale_bytes("nvfp4", M, K), dtype=torch.uint8, device="cuda")
+    D = nvq.nvfp4_linear_short_m(x.cuda(), wc, ws, wg, N, a_codes=ac, a_scales=asf)
+    clean("short-M linear %d x %d x %d" % (M, N, K))
+    oc, osf, _ = oracle.nvfp4_quantize(bits(x))
+    assert np.array_equal(ac.cpu().numpy(), oc) and np.array_equal(asf.cpu().numpy(), osf)
+    check_gemm(D.float().cpu().numpy(), oracle_linear("nvfp4", x, w))
+
 for fmt, M, N, K in (("nvfp4", 384, 768, 512), ("nvfp4", 100, 384, 256), ("mxfp8", 96, 256, 256)):
     if fmt == "nvfp4":
         x, _ = workloads.exact_operand(M, K, seed=M + K, top_row=M // 2)
