@@ -20,7 +20,6 @@ import json
 import os
 import statistics
 import sys
-import threading
 import time
 
 import numpy as np
@@ -135,8 +134,37 @@ def load_peaks():
 
 # --------------------------------------------------------------------------- clocks
 
+_SAMPLER = r"""
+import json, sys, threading, time
+import pynvml
+pynvml.nvmlInit()
+uuid, bus, period = sys.argv[1], sys.argv[2], float(sys.argv[3])
+try:
+    h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+except Exception:
+    h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+print(json.dumps({"max_mhz": pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)}), flush=True)
+stop = threading.Event()
+threading.Thread(target=lambda: (sys.stdin.read(), stop.set()), daemon=True).start()
+out = []
+while not stop.is_set():
+    t = time.perf_counter()
+    try:
+        out.append([t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                    pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)])
+    except Exception:
+        pass
+    time.sleep(period)
+print(json.dumps(out), flush=True)
+"""
+
+
 class ClockSampler:
-    """Samples SM clock and clock-event reasons of one GPU through NVML."""
+    """Samples SM clock and clock-event reasons of one GPU through NVML, in a
+    child process (a thread of this one would wait on the interpreter lock
+    while the host issues launches), every `period` seconds; summary() keeps
+    the samples taken between start() and stop() (perf_counter is the same
+    monotonic clock in both processes)."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
@@ -145,45 +173,41 @@ class ClockSampler:
     }
 
     def __init__(self, device_index, period=0.002):
+        import subprocess
         self.samples = []
         self.reasons = 0
         self.ok = False
-        self._stop = threading.Event()
+        self.t0 = self.t1 = None
         try:
-            import pynvml
-            pynvml.nvmlInit()
+            import pynvml  # noqa: F401  (the child imports it; fail here, not there)
             props = torch.cuda.get_device_properties(device_index)
-            try:
-                self._h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
-            except Exception:
-                bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
-                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-            self._nv = pynvml
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            self._p = subprocess.Popen([sys.executable, "-c", _SAMPLER, "GPU-" + str(props.uuid), bus, str(period)],
+                                       stdin=subprocess.PIPE, stdout=subprocess.PIPE, text=True)
+            self.max_mhz = json.loads(self._p.stdout.readline())["max_mhz"]
             self.ok = True
         except Exception as e:  # NVML missing: report no clock data rather than guess
             self.err = repr(e)
-        self._period = period
-        self._t = threading.Thread(target=self._run, daemon=True)
-
-    def _run(self):
-        nv = self._nv
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-            except Exception:
-                pass
-            time.sleep(self._period)
 
     def start(self):
-        if self.ok:
-            self._t.start()
+        self.t0 = time.perf_counter()
 
     def stop(self):
-        if self.ok:
-            self._stop.set()
-            self._t.join()
+        self.t1 = time.perf_counter()
+        if not self.ok:
+            return
+        try:
+            self._p.stdin.close()
+            rows = json.loads(self._p.stdout.readline())
+            self._p.wait(timeout=60)
+        except Exception as e:  # the sampler died: no clock data rather than a failed run
+            self.ok, self.err = False, repr(e)
+            self._p.kill()
+            return
+        for t, mhz, reasons in rows:
+            if self.t0 <= t <= self.t1:
+                self.samples.append(mhz)
+                self.reasons |= reasons
 
     def summary(self):
         if not self.ok:
