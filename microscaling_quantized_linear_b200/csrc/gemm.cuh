@@ -380,9 +380,13 @@ __device__ __forceinline__ void splitk_finish(uint32_t recv, const SplitShares& 
 
 // Fused short-M path: the activation's dynamic NVFP4 quantization inside the
 // split-K GEMM, by the epilogue warps (idle until the accumulator is ready)
-// while the B tiles load.  Every CTA takes the amax of the whole activation
-// [M, K] (M <= 16: a few KB to 96 KB, read from L2), then quantizes the rows
-// of its own K tiles with the same arithmetic as the quantize kernels,
+// while the B tiles load.  For more than kShortAmaxRows rows every CTA takes
+// the max |x| of its own K tiles' columns and sends it with st.async to every
+// CTA of its cluster (the cluster's shares cover K, so each CTA then holds
+// the tensor's amax; the receiving mbarrier expects one 4-byte value per
+// CTA); for fewer rows each CTA reads the whole activation, which is cheaper
+// than the exchange's latency.  Then every CTA quantizes the
+// rows of its own K tiles with the same arithmetic as the quantize kernels,
 // writing the E2M1 codes into its stages' A tiles (the 128-byte swizzle the
 // MMA reads: 16-byte chunk c of row r at chunk c ^ (r % 8)) and the E4M3
 // scales into their A scale tiles (128x4 order), then counts one arrival per
@@ -390,28 +394,40 @@ __device__ __forceinline__ void splitk_finish(uint32_t recv, const SplitShares& 
 // the A tiles are left as they are: they only feed accumulator rows that
 // nothing reads.  With q_codes / q_sf / a_global_out set, the CTAs of the
 // first cluster also write the codes, scales (padding rows zero) and g_dec,
-// exactly as nvfp4_quantize would.  Returns g_dec.  Threads tid 0..255.
+// exactly as nvfp4_quantize would.  With the exchange (more than
+// kShortAmaxRows rows) this waits on the cluster barrier's first phase before
+// the first st.async, and the caller does not wait on it again.  If the wait for the cluster's maxima gives up, the amax comes
+// from the whole activation read here (exact all the same) and the status
+// word records the timeout.  Returns g_dec.  Threads tid 0..255.
+constexpr uint32_t kShortAmaxRows = 4;
+
 template <typename C>
 __device__ __forceinline__ float fused_quantize_a(const GemmParams& p, uint8_t* smem, float* scratch,
                                                   uint32_t kt_begin, uint32_t kt_end, bool first_cluster,
-                                                  uint32_t tid, uint32_t full0, uint32_t sfdata0) {
+                                                  uint32_t tid, uint32_t full0, uint32_t sfdata0, uint32_t amaxbar,
+                                                  uint32_t rank, const volatile int* abort_flag,
+                                                  bool& amax_got) {
     constexpr uint32_t NT = 32 * kEpiWarps;
     float* d6 = scratch;
     float* rtab = scratch + 128;
     uint32_t* red = reinterpret_cast<uint32_t*>(scratch + 256);
+    uint32_t* slots = reinterpret_cast<uint32_t*>(scratch + 264);      // one per CTA of the cluster
+    volatile uint32_t* gave_up = reinterpret_cast<volatile uint32_t*>(scratch + 274);
     const uint32_t rows = p.m_total;
     const uint32_t K = p.num_k_tiles * 256u;
-    const uint32_t vpr = K / 8;                               // 16-byte vectors per row
     const uint64_t x_elems = pitched_extent(rows, K, p.ldx);
-    // amax of the whole activation: batches of 8 independent 16-byte loads
-    // per thread, all issued before any is used
+    // max |x| over this CTA's K tiles (or the whole tensor): batches of 8
+    // independent 16-byte loads per thread, all issued before any is used
+    const bool shared_amax = rows > kShortAmaxRows;
+    const uint32_t vps = shared_amax ? (kt_end - kt_begin) * 32 : K / 8;   // 16-byte vectors per row read
+    const uint32_t c0 = shared_amax ? kt_begin * 32 : 0;
     uint32_t m2 = 0;
-    for (uint32_t i0 = tid; i0 < rows * vpr; i0 += 8 * NT) {
+    for (uint32_t i0 = tid; i0 < rows * vps; i0 += 8 * NT) {
         uint4 v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const uint32_t i = i0 + u * NT, r = i / vpr, c = i - r * vpr;
-            v[u] = (i < rows * vpr && in_bounds((uint64_t)r * p.ldx + c * 8, 8, x_elems, p.status))
+            const uint32_t i = i0 + u * NT, r = i / vps, c = c0 + (i - r * vps);
+            v[u] = (i < rows * vps && in_bounds((uint64_t)r * p.ldx + c * 8, 8, x_elems, p.status))
                        ? __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)r * p.ldx) + c)
                        : make_uint4(0, 0, 0, 0);
         }
@@ -421,10 +437,47 @@ __device__ __forceinline__ float fused_quantize_a(const GemmParams& p, uint8_t* 
     uint32_t m = __reduce_max_sync(0xFFFFFFFFu, fold2(m2));
     if ((tid & 31) == 0) red[tid >> 5] = m;
     if (tid < 128) d6[tid] = __fdiv_rn((float)(128 + tid), 6.0f);
+    if (tid == 0) *gave_up = 0;
     named_barrier_sync(3, NT);
     m = 0;
+    if (!shared_amax) {
 #pragma unroll
-    for (int w = 0; w < kEpiWarps; ++w) m = max(m, red[w]);
+        for (int w = 0; w < kEpiWarps; ++w) m = max(m, red[w]);
+        amax_got = true;
+    } else {
+    cluster_wait();                           // every CTA's amax barrier is initialised
+    if (tid == 0) {
+#pragma unroll
+        for (int w = 0; w < kEpiWarps; ++w) m = max(m, red[w]);
+        for (uint32_t r = 0; r < p.k_split; ++r)
+            st_async_u32(mapa_shared(smem_u32(slots + rank), r), m, mapa_shared(amaxbar, r));
+    }
+    if (!mbar_wait_bounded_cluster(amaxbar, 0, abort_flag, p.wait_ns)) *gave_up = 1;
+    named_barrier_sync(3, NT);                // one decision for all: the branches below hold barriers
+    amax_got = *gave_up == 0;
+    m = 0;
+    if (amax_got) {
+        for (uint32_t r = 0; r < p.k_split; ++r) m = max(m, slots[r]);
+    } else {
+        // a CTA of the cluster did not send: the amax from the whole tensor
+        if (tid == 0) atomicOr(p.status, kStatusTimeout);
+        const uint32_t vpr = K / 8;
+        uint32_t a2 = 0;
+        for (uint32_t i = tid; i < rows * vpr; i += NT) {
+            const uint32_t r = i / vpr, c = i - r * vpr;
+            if (in_bounds((uint64_t)r * p.ldx + c * 8, 8, x_elems, p.status)) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)r * p.ldx) + c);
+                a2 = absmax2(absmax2(absmax2(absmax2(a2, v.x), v.y), v.z), v.w);
+            }
+        }
+        named_barrier_sync(3, NT);            // everyone has read red[] above
+        const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, fold2(a2));
+        if ((tid & 31) == 0) red[tid >> 5] = wm;
+        named_barrier_sync(3, NT);
+#pragma unroll
+        for (int w = 0; w < kEpiWarps; ++w) m = max(m, red[w]);
+    }
+    }
     if (m >= 0x7F80u && first_cluster && cluster_ctarank() == 0 && tid == 0) atomicOr(p.status, kStatusNonfinite);
     const float amax = __uint_as_float(m << 16);
     const float g_enc = encode_scale(amax);
@@ -559,6 +612,7 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     const uint32_t drain = tempty0 + 8 * 2;                // MMA warp's own completion
     const uint32_t sfdrain = drain + 8;                    // copy warps' own completion
     const uint32_t recvbar = sfdrain + 8;                  // split-K: the cluster's pushes landed (tx)
+    const uint32_t amaxbar = smem_u32(bars + 64) + 1088;   // fused short-M: the cluster's partial maxima (tx)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 7);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* never = abort_flag + 1;
@@ -576,6 +630,10 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         }
         mbar_init(drain, 1);
         mbar_init(sfdrain, C::SF_WARPS);
+        if (FUSEQ) {
+            mbar_init(amaxbar, 1);
+            if (p.m_total > kShortAmaxRows) mbar_arrive_expect_tx(amaxbar, p.k_split * 4);
+        }
         if (SPLITK) {
             // expects one whole slot from every CTA of the cluster, its own included
             const SplitShares sh = split_shares<BN>(min(p.m_total, (uint32_t)SPLIT_ROWS), p.k_split);
@@ -775,9 +833,11 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         const int q = warp & 3;                       // tensor-memory lane quarter of this warp
         const int half = (warp - 2) >> 2;             // which half of the tile's columns
         float a_dec;
+        bool amax_got = true;
         if constexpr (FUSEQ)
             a_dec = fused_quantize_a<C>(p, smem, reinterpret_cast<float*>(bars + 64), kt_begin, kt_end,
-                                        tile_first == 0, threadIdx.x - 64, full0, sfdata0);
+                                        tile_first == 0, threadIdx.x - 64, full0, sfdata0, amaxbar, ks,
+                                        abort_flag, amax_got);
         else
             a_dec = FMT == 0 ? *p.a_global : 1.0f;
         const float alpha = FMT == 0 ? __fmul_rn(a_dec, *p.b_global) : 1.0f;
@@ -804,7 +864,9 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             const uint32_t outbox = smem_u32(smem);           // slot for owner j at j * slot * 16
             // one decision per warp: the tensor-memory loads below are warp-wide
             const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(tfull0, 0, abort_flag, p.wait_ns));
-            cluster_wait();                   // every receive barrier of the cluster is initialised
+            // every receive barrier of the cluster is initialised (the fused
+            // path with the amax exchange has waited for this already)
+            if (!FUSEQ || p.m_total <= kShortAmaxRows) cluster_wait();
             if (!ok) {
                 // the slots still go out (their contents unspecified), so
                 // every receive barrier completes
@@ -862,6 +924,9 @@ bsgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 splitk_finish<BN>(recv, sh, ks, p.k_split, (tile_first / p.num_m_blocks) * BN, p.n_total, alpha,
                                   p.bias, p.out, p.ldo, threadIdx.x - 64, 32 * kEpiWarps, p.status);
             }
+            // (fused: a wait for the cluster's maxima that gave up lets the
+            // values already sent land first)
+            if (FUSEQ && !amax_got) mbar_wait_bounded_cluster(amaxbar, 0, never, kWaitLimitNs);
             __syncwarp();
             cluster_arrive_relaxed();         // this CTA's share has arrived: its copies out have been read
         }

@@ -328,6 +328,14 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint3
                  :: "r"(dst_cluster), "r"(src), "r"(bytes), "r"(cluster_bar) : "memory");
 }
 
+// Asynchronous 4-byte store into the shared memory of (possibly) another CTA
+// of the cluster, counted as 4 bytes on the mbarrier at `cluster_bar` in the
+// same CTA as the destination.
+__device__ __forceinline__ void st_async_u32(uint32_t cluster_addr, uint32_t v, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+                 :: "r"(cluster_addr), "r"(v), "r"(cluster_bar) : "memory");
+}
+
 // Count `bytes` on the transaction count of an mbarrier of this CTA without
 // writing data.
 __device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {

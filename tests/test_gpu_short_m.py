@@ -143,3 +143,27 @@ def test_quantized_linear_takes_the_fused_launch_at_short_batches():
         check_gemm(D.float().cpu().numpy(), oracle.gemm_rows(A, B))
     # batches up to SHORT_M_FUSED_ROWS rows took the fused launch, none was refused
     assert nvq.SHORT_M_FUSED_ROWS == 8 and layer._short == {}
+
+
+def test_waits_run_out_and_the_context_survives():
+    # With a 1 ns limit the cluster's exchange of partial maxima and the
+    # pipeline waits give up: the amax then comes from the whole activation
+    # (exact), the slots still go out, every wait stays bounded, and the host
+    # reads NVQ_STATUS_TIMEOUT.  The next call, at the default limit, is clean
+    # and equals the two-call path.
+    M, N, K = 6, 12288, 3072              # above 4 rows: the cluster exchanges partial maxima
+    w, wc, ws, wg = weight(N, K, seed=80)
+    x, xd = activation(M, K, 0, seed=81)
+    nvq.set_wait_limit(1)
+    try:
+        for _ in range(3):
+            nvq.nvfp4_linear_short_m(xd, wc, ws, wg, N)
+        status = nvq.device_status()
+    finally:
+        nvq.set_wait_limit(0)
+    assert status == nvq.NVQ_STATUS_TIMEOUT
+    D = nvq.nvfp4_linear_short_m(xd, wc, ws, wg, N)
+    assert nvq.device_status() == 0
+    c2, s2, g2 = nvq.nvfp4_quantize(xd)
+    D2 = nvq.block_scaled_linear("nvfp4", c2, s2, g2, wc, ws, wg, M, N, K)
+    assert torch.equal(D.view(torch.int16), D2.view(torch.int16))
