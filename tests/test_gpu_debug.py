@@ -102,7 +102,7 @@ for fmt, M, N, K, use_bias in GEMMS:
     D = gpu_linear(fmt, x, w, bias=b)              # asserts a clean status word
     check_gemm(D.float().cpu().numpy(), oracle_linear(fmt, x, w, bias=b))
 
-for M, N, K in ((1, 12288, 3072), (7, 1000, 2048)):      # one-launch short-batch linear
+for M, N, K in ((1, 12288, 3072), (7, 1000, 2048), (16, 9216, 3072)):   # one-launch short-batch linear
     x = workloads.normal(M, K, seed=M + 9)
     w = workloads.normal(N, K, seed=N + 3, std=0.05)
     wc, ws, wg = nvq.quantize_weight("nvfp4", w.cuda())

@@ -1,6 +1,7 @@
 """GPU parity of the one-launch short-batch NVFP4 linear (nvfp4_linear_short_m):
-the split-K GEMM quantizes the activation itself (every CTA takes the amax
-of the whole activation and quantizes its own share of K into its stages).
+the split-K GEMM quantizes the activation itself (each CTA quantizes its own
+share of K into its stages; the amax comes from the whole activation up to
+4 rows, and above 4 rows from partial maxima the cluster's CTAs exchange).
 
   * the output equals nvfp4_quantize + block_scaled_linear bit for bit (same
     codes, scales and global scale, same split-K order), and meets the GEMM
