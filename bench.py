@@ -836,6 +836,21 @@ def run_profile(leg, iters, device):
         if status != 0:
             raise SystemExit("device status %d" % status)
         return
+    if leg in ("short1", "short8"):
+        # the one-launch short-batch linear on the FF-up weight (1 or 8 rows)
+        w = workloads.WORKLOADS["ffup"]
+        M, N, K = (1 if leg == "short1" else 8), w.N, w.K
+        x = workloads.activation("ffup", seed=60, M=M).to(device)
+        wc, wsf, wg = nvq.quantize_weight("nvfp4", workloads.weight("ffup", seed=61).to(device))
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        for _ in range(1 + iters):
+            nvq.nvfp4_linear_short_m(x, wc, wsf, wg, N, out=out, stream=stream)
+            torch.cuda.synchronize(device)
+        status = nvq.device_status()
+        print(json.dumps({"profile": leg, "iters": iters, "M": M, "K": K, "device_status": status}), flush=True)
+        if status != 0:
+            raise SystemExit("device status %d" % status)
+        return
     name = {"ffup": "ffup", "qkv4": "qkv4", "actq": "actq", "fused": "ffup", "m1": "ffup"}[leg]
     w = workloads.WORKLOADS[name]
     M, K = (1 if leg == "m1" else w.M), w.K
@@ -887,7 +902,7 @@ def main():
     ap.add_argument("--no-ff-block", dest="ff_block", action="store_false")
     ap.add_argument("--no-act-quant", dest="act_quant", action="store_false")
     ap.add_argument("--no-qkv4", dest="qkv4", action="store_false")
-    ap.add_argument("--profile", choices=["ffup", "qkv4", "actq", "fused", "m1", "ffdown"], default=None,
+    ap.add_argument("--profile", choices=["ffup", "qkv4", "actq", "fused", "m1", "ffdown", "short1", "short8"], default=None,
                     help="run only this leg's launches (one warm-up call + --iters calls) for an ncu capture")
     ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args()

@@ -136,6 +136,28 @@ __device__ __forceinline__ uint32_t nvfp4_block_d(float d, const uint32_t (&w)[8
     return sc;
 }
 
+// Two blocks at once: both E4M3 scales from one conversion.
+__device__ __forceinline__ uint32_t nvfp4_block_pair_d(float d0, float d1, const uint32_t (&w0)[8],
+                                                       const uint32_t (&w1)[8], float g_enc, const float* rtab,
+                                                       uint32_t& lo0, uint32_t& hi0, uint32_t& lo1, uint32_t& hi1) {
+    const uint32_t pair = cvt_e4m3x2(__fmul_rn(d1, g_enc), __fmul_rn(d0, g_enc));
+    const uint32_t sc0 = pair & 0xFFu, sc1 = pair >> 8;
+    const float r0 = rtab[sc0], r1 = rtab[sc1];
+    float2 p[8], q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        p[i] = bf16x2_mul(w0[i], r0);
+        q[i] = bf16x2_mul(w1[i], r1);
+    }
+    lo0 = cvt_e2m1x8(p[0].x, p[0].y, p[1].x, p[1].y, p[2].x, p[2].y, p[3].x, p[3].y);
+    hi0 = cvt_e2m1x8(p[4].x, p[4].y, p[5].x, p[5].y, p[6].x, p[6].y, p[7].x, p[7].y);
+    lo1 = cvt_e2m1x8(q[0].x, q[0].y, q[1].x, q[1].y, q[2].x, q[2].y, q[3].x, q[3].y);
+    hi1 = cvt_e2m1x8(q[4].x, q[4].y, q[5].x, q[5].y, q[6].x, q[6].y, q[7].x, q[7].y);
+    if (sc0 == 0) lo0 = hi0 = 0;
+    if (sc1 == 0) lo1 = hi1 = 0;
+    return pair;
+}
+
 // The same block given its block max bits mb.
 __device__ __forceinline__ uint32_t nvfp4_block(uint32_t mb, const uint32_t (&w)[8], float g_enc,
                                                 const float* d6, const float* rtab, uint32_t& lo, uint32_t& hi) {
@@ -581,6 +603,7 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
             bool done = j >= gridDim.x;
             uint32_t mine = 0;
             const uint64_t t0 = globaltimer_ns();
+            uint32_t spins = 0;
             while (true) {
                 if (!done) {
                     const unsigned long long v = ld_relaxed_u64(slots + (size_t)j * kFusedSlotStride);
@@ -590,8 +613,10 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
                     }
                 }
                 if (__all_sync(0xFFFFFFFFu, done)) break;
-                int give_up = 0;                      // decided by lane 0 so the warp leaves together
-                if (lane == 0) give_up = *timeout || globaltimer_ns() - t0 > wait_ns;
+                // decided by lane 0 so the warp leaves together; the clock
+                // is read every 8th round (a round is one L2 round trip)
+                int give_up = 0;
+                if (lane == 0 && (++spins & 7u) == 0) give_up = *timeout || globaltimer_ns() - t0 > wait_ns;
                 if (__shfl_sync(0xFFFFFFFFu, give_up, 0)) {
                     if (lane == 0) *timeout = 1;
                     break;
@@ -667,9 +692,7 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
             const uint32_t w1[8] = {v[u][2].x, v[u][2].y, v[u][2].z, v[u][2].w,
                                     v[u][3].x, v[u][3].y, v[u][3].z, v[u][3].w};
             uint32_t lo0, hi0, lo1, hi1;
-            const uint32_t sc0 = nvfp4_block_d(d[u].x, w0, g_enc, rtab, lo0, hi0);
-            const uint32_t sc1 = nvfp4_block_d(d[u].y, w1, g_enc, rtab, lo1, hi1);
-            const uint32_t pair = sc0 | (sc1 << 8);
+            const uint32_t pair = nvfp4_block_pair_d(d[u].x, d[u].y, w0, w1, g_enc, rtab, lo0, hi0, lo1, hi1);
             const uint32_t next = __shfl_down_sync(0xFFFFFFFFu, pair, 1);
             if (active) {
                 if (in_bounds((uint64_t)r0 * nblk * 8 + (uint64_t)g * 16, 16, (uint64_t)rows * nblk * 8, status))
