@@ -614,9 +614,10 @@ nvfp4_quantize_fused_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint3
                 }
                 if (__all_sync(0xFFFFFFFFu, done)) break;
                 // decided by lane 0 so the warp leaves together; the clock
-                // is read every 8th round (a round is one L2 round trip)
+                // is read in the first round and every 8th after it (a round is one
+                // L2 round trip)
                 int give_up = 0;
-                if (lane == 0 && (++spins & 7u) == 0) give_up = *timeout || globaltimer_ns() - t0 > wait_ns;
+                if (lane == 0 && (spins++ & 7u) == 0) give_up = *timeout || globaltimer_ns() - t0 > wait_ns;
                 if (__shfl_sync(0xFFFFFFFFu, give_up, 0)) {
                     if (lane == 0) *timeout = 1;
                     break;
