@@ -328,9 +328,14 @@ NVQ_API int block_scaled_linear_gelu_mxfp8(int format,
  * block-scaled GEMM of block_scaled_linear, fused, for latency at short
  * batches (batch 1 of the pages' FLUX runs, page "Modelos de Difusão"; the
  * small-batch latency discussion of page "NVIDIA量化推理：5步极速优化显存+成功率
- * 翻倍").  Every CTA of the split-K GEMM takes the activation's
- * amax itself and quantizes the rows of its own share of K into its pipeline
- * stages, with the arithmetic of nvfp4_quantize, while the weight streams in.
+ * 翻倍").  Every CTA of the split-K GEMM quantizes the rows of its own share
+ * of K into its pipeline stages, with the arithmetic of nvfp4_quantize, while
+ * the weight streams in.  The amax: up to 4 rows every CTA reads the whole
+ * activation; above 4 rows each CTA takes the max over its own share and the
+ * CTAs of a cluster (whose shares cover K) exchange these partial maxima
+ * through distributed shared memory.  If that exchange's bounded wait gives
+ * up, the CTA reads the whole activation instead (the result stays exact) and
+ * NVQ_STATUS_TIMEOUT is set.
  *
  *   out = block_scaled_linear(NVQ_NVFP4, nvfp4_quantize(x), w) bit for bit:
  *   the same codes, scales and global scale, the same split-K order.
@@ -384,7 +389,7 @@ NVQ_API int nvq_set_wait_limit(uint64_t limit_ns);
 
 /*
  * nvfp4_quantize_noalloc -- nvfp4_quantize for callers that cannot allocate
- * device memory.  The paper has no counterpart to this entry point.
+ * device memory.  The pages have no counterpart to this entry point.
  *
  * Some callers cannot call cudaMalloc, nor hand the library a workspace:
  * code that runs inside a host framework which owns all device memory and
