@@ -388,6 +388,14 @@ NVQ_API const char* nvq_status_string(int code);
 NVQ_API int nvq_set_wait_limit(uint64_t limit_ns);
 
 /*
+ * nvq_wait_limit -- the limit nvq_set_wait_limit last set (0: the defaults).
+ * Its initial value comes from the environment variable NVQ_WAIT_LIMIT_NS
+ * (decimal nanoseconds, at most 4e9), read once when the library loads; an
+ * unset, malformed or larger value leaves the defaults.  No device needed.
+ */
+NVQ_API uint64_t nvq_wait_limit(void);
+
+/*
  * nvfp4_quantize_noalloc -- nvfp4_quantize for callers that cannot allocate
  * device memory.  The pages have no counterpart to this entry point.
  *

@@ -92,6 +92,8 @@ _lib.nvq_probe_bounds.restype = ctypes.c_int
 _lib.nvq_probe_bounds.argtypes = [_vp]
 _lib.nvq_set_wait_limit.restype = ctypes.c_int
 _lib.nvq_set_wait_limit.argtypes = [ctypes.c_uint64]
+_lib.nvq_wait_limit.restype = ctypes.c_uint64
+_lib.nvq_wait_limit.argtypes = []
 _lib.nvq_workspace_init.restype = ctypes.c_int
 _lib.nvq_workspace_init.argtypes = [_vp, _vp]
 _lib.nvq_gemm_plan_host.restype = ctypes.c_int
@@ -103,7 +105,7 @@ EXPORTED = ("nvq_codes_bytes", "nvq_scale_bytes", "nvq_workspace_bytes", "nvfp4_
             "nvq_device_status", "nvq_status_string", "nvq_probe_convert", "nvfp4_quantize_noalloc",
             "block_scaled_linear_gelu_mxfp8", "nvq_probe_gelu", "nvq_probe_wait", "nvq_gemm_plan",
             "nvq_gemm_plan_host", "nvq_set_wait_limit", "nvq_workspace_init", "nvq_debug_build",
-            "nvq_probe_bounds", "nvfp4_linear_short_m")
+            "nvq_probe_bounds", "nvfp4_linear_short_m", "nvq_wait_limit")
 
 DEBUG_BUILD = bool(_lib.nvq_debug_build())
 
@@ -485,6 +487,12 @@ def set_wait_limit(limit_ns):
     """Test hook: limit (ns) of the kernels' pipeline waits for later launches
     in this process; 0 restores the defaults (nvq_set_wait_limit)."""
     _check(_lib.nvq_set_wait_limit(int(limit_ns)), "nvq_set_wait_limit")
+
+
+def wait_limit():
+    """The current limit (ns) of the kernels' pipeline waits; 0 = the defaults.
+    Starts from NVQ_WAIT_LIMIT_NS in the environment (nvq_wait_limit)."""
+    return int(_lib.nvq_wait_limit())
 
 
 def probe_wait(limit_ns, device=None, stream=None):

@@ -169,7 +169,17 @@ uint32_t quant_grid(uint64_t units, int num_sms) {
 
 // Limit of the kernels' pipeline waits set by nvq_set_wait_limit (0: the
 // defaults, 4 s in the GEMMs and 2 s in the one-pass quantizer's barrier).
-std::atomic<uint64_t> g_wait_limit_ns{0};
+// NVQ_WAIT_LIMIT_NS in the environment sets its initial value (decimal
+// nanoseconds, at most the 4 s default; anything else is ignored).
+uint64_t wait_limit_from_env() {
+    const char* e = getenv("NVQ_WAIT_LIMIT_NS");
+    if (!e || !*e) return 0;
+    char* end = nullptr;
+    const unsigned long long v = strtoull(e, &end, 10);
+    if (*end != '\0' || v > kWaitLimitNs) return 0;
+    return (uint64_t)v;
+}
+std::atomic<uint64_t> g_wait_limit_ns{wait_limit_from_env()};
 
 uint64_t pipeline_wait_ns(uint64_t dflt) {
     const uint64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
@@ -1039,6 +1049,8 @@ int nvq_set_wait_limit(uint64_t limit_ns) {
     g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
     return NVQ_OK;
 }
+
+uint64_t nvq_wait_limit(void) { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 int nvq_workspace_init(void* workspace, nvq_stream_t stream) {
     if (!workspace) return NVQ_ERR_NULL;

@@ -239,3 +239,23 @@ def test_linear_short_m_rejects_bad_arguments():
     assert ls(gb=NULL) == -1
     assert ls(out=P_ODD) == -3
     assert ls(M=0) == 0                       # empty batch: nothing to do
+
+
+def test_wait_limit_starts_from_the_environment():
+    # NVQ_WAIT_LIMIT_NS sets the initial limit when the library loads; a
+    # malformed or too large value leaves the defaults (0).  Host only.
+    import subprocess
+    import sys
+    code = ("import sys; sys.path.insert(0, %r); import microscaling_quantized_linear_b200 as n; "
+            "print(n.wait_limit())" % os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    got = {}
+    for val in ("12345", "4000000000", "4000000001", "12x", ""):
+        env = dict(os.environ, NVQ_WAIT_LIMIT_NS=val)
+        out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+        assert out.returncode == 0, out.stderr[-2000:]
+        got[val] = int(out.stdout.strip().splitlines()[-1])
+    assert got == {"12345": 12345, "4000000000": 4000000000, "4000000001": 0, "12x": 0, "": 0}
+    assert L.nvq_set_wait_limit(777) == 0
+    assert nvq.wait_limit() == 777
+    assert L.nvq_set_wait_limit(0) == 0
+    assert nvq.wait_limit() == 0
