@@ -35,6 +35,8 @@ WORKLOAD = "ffup"
 ROTATE = 4                    # input sets cycled through so a step's inputs are not L2-resident
 FP4_OVER_BF16 = 4.0           # nominal dense FP4 / BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
 ACT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # BF16 read, E2M1 codes + E4M3 scale written
+WORKLOAD_DESC = ("NVFP4 W4A4 FF-up linear, FLUX-like: A BF16 [4608,3072] N(0,1) 0.5% x50 outliers, "
+                 "W BF16 [12288,3072] N(0,0.02), out BF16 [4608,12288]; dynamic per-tensor activation scale")
 
 
 # DRAM traffic of the roofline kernel per launch on this workload, from one
@@ -323,8 +325,7 @@ def run_ours(args, rank, world, device):
         "dtype": "e2m1",
         "data": "synthetic",
         "config": {
-            "workload": "NVFP4 W4A4 FF-up linear, FLUX-like: A BF16 [4608,3072] N(0,1) 0.5% x50 outliers, "
-                        "W BF16 [12288,3072] N(0,0.02), out BF16 [4608,12288]; dynamic per-tensor activation scale",
+            "workload": WORKLOAD_DESC,
             "M": M, "N": N, "K": K,
             "parallelism": "replicas" if world > 1 else "single-gpu",
             "l2": "inputs rotated over %d activation+weight sets (%.0f MB) plus a %.0f MB output write per step, "
@@ -804,8 +805,8 @@ def run_reference(args):
     return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(full * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": "NVFP4 W4A4 FF-up linear, FLUX-like, 4608x12288x3072 (CPU oracle)",
-                       "M": M, "N": N, "K": K},
+            "config": {"workload": WORKLOAD_DESC, "M": M, "N": N, "K": K, "parallelism": "single-gpu",
+                       "l2": "not applicable: the oracle runs on the host cores from host memory"},
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
