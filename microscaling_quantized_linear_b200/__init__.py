@@ -7,8 +7,12 @@ allocates output tensors with torch when the caller does not pass them, and
 raises ``NvqError`` on a non-zero return code.  There is no fallback: if the
 shared library is missing, importing this package fails.
 
-Names follow the C ABI: ``nvfp4_quantize``, ``mxfp8_quantize``,
-``quantize_weight``, ``block_scaled_linear``, plus the size helpers.
+Names follow the C ABI: ``nvfp4_quantize`` (and ``nvfp4_quantize_noalloc``),
+``mxfp8_quantize``, ``quantize_weight``, ``block_scaled_linear``,
+``block_scaled_linear_gelu_mxfp8``, ``nvfp4_linear_short_m``, plus the size
+helpers, the status word and the test hooks.  ``QuantizedLinear`` sequences
+them for a caller: weight quantized once, then per call the activation's
+quantization and the GEMM (one launch for NVFP4 batches of at most 8 rows).
 
 With NVQ_DEBUG=1 in the environment at import, the debug build
 ``libnvq_debug.so`` (bounds-checked kernels, see ``build.py``) is loaded
